@@ -1,0 +1,104 @@
+"""Pins for the BenQ oracle (CPU only).
+
+Each test ties ``oracle.benq`` to something other than itself: a worked
+example derived by hand from the BenQ card's definitions, an exhaustive
+bijection with the (independent) generator packing, torch's gather (the card
+defines decode as ``lut.gather(1, codes)``), or exact rational arithmetic.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import benq as ob
+
+
+def _f32_of_bf16(bits):
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def test_unpack_matches_hand_worked_stream(golden):
+    g = golden("benq_pack_example.txt")
+    codes = np.array([int(c) for c in g["codes"]])
+    packed = np.array([[int(b, 16) for b in g["bytes"]]], dtype=np.uint8)
+    assert ob.unpack_codes(packed, 8).tolist() == [codes.tolist()]
+
+
+def test_generator_pack_matches_hand_worked_stream(golden):
+    g = golden("benq_pack_example.txt")
+    codes = np.array([[int(c) for c in g["codes"]]], dtype=np.uint8)
+    assert synth.pack_codes(codes).tolist() == [[int(b, 16) for b in g["bytes"]]]
+
+
+def test_pack_unpack_bijection_all_code_groups():
+    # every one of the 64^4 groups of four codes survives pack -> unpack
+    c = np.arange(64 ** 4, dtype=np.int64)
+    groups = np.stack([(c >> (6 * j)) & 63 for j in range(4)], axis=1).astype(np.uint8)
+    packed = synth.pack_codes(groups.reshape(1, -1))
+    back = ob.unpack_codes(packed, groups.size).reshape(-1, 4)
+    assert np.array_equal(back, groups)
+
+
+def test_unpack_pack_bijection_all_byte_triples():
+    # every one of the 2^24 three-byte strings survives unpack -> pack
+    v = np.arange(1 << 24, dtype=np.uint32)
+    triples = np.stack([(v >> 8 * j) & 255 for j in range(3)], axis=1).astype(np.uint8)
+    codes = ob.unpack_codes(triples.reshape(1, -1), 4 * (1 << 24))
+    again = synth.pack_codes(codes.astype(np.uint8))
+    assert np.array_equal(again.reshape(-1, 3), triples)
+
+
+def test_unpack_ignores_bytes_past_the_row():
+    rng = np.random.default_rng(0)
+    packed = rng.integers(0, 256, size=(3, 24), dtype=np.uint8)
+    wide = np.concatenate([packed, rng.integers(0, 256, size=(3, 16), dtype=np.uint8)], axis=1)
+    assert np.array_equal(ob.unpack_codes(packed, 32), ob.unpack_codes(wide, 32))
+
+
+def test_dequant_is_torch_gather():
+    rng = np.random.default_rng(1)
+    N, K = 37, 96
+    codes = rng.integers(0, 64, size=(N, K), dtype=np.uint8)
+    lut = rng.integers(0, 1 << 16, size=(N, 64), dtype=np.uint16)
+    packed = synth.pack_codes(codes)
+    ref = torch.gather(torch.from_numpy(lut.astype(np.int32)), 1, torch.from_numpy(codes.astype(np.int64)))
+    assert np.array_equal(ob.dequant_bits(packed, lut, K), ref.numpy().astype(np.uint16))
+
+
+def test_linear_hand_worked_example(golden):
+    g = golden("benq_linear_example.txt")
+    c = np.array([[int(v) for v in g["codes0"]], [int(v) for v in g["codes1"]]], dtype=np.uint8)
+    lut0 = np.array([(2 * k - 63) / 32 for k in range(64)], dtype=np.float32)
+    lut1 = np.array([-(2 * k - 63) / 64 for k in range(64)], dtype=np.float32)
+    lut = synth.f32_to_bf16_bits(np.stack([lut0, lut1]))
+    assert np.array_equal(_f32_of_bf16(lut), np.stack([lut0, lut1]))    # exact in bf16
+    x = synth.f32_to_bf16_bits(np.array([[float(v) for v in g["x"]]], dtype=np.float32))
+    y = ob.linear(synth.pack_codes(c), lut, x, 4)
+    assert y.tolist() == [[float(v) for v in g["y"]]]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_linear_exact_rational_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    N, K, B = 3, 8, 2
+    codes = rng.integers(0, 64, size=(N, K), dtype=np.uint8)
+    lut = synth.f32_to_bf16_bits(rng.standard_normal((N, 64)).astype(np.float32))
+    x = synth.f32_to_bf16_bits(rng.standard_normal((B, K)).astype(np.float32))
+    y = ob.linear(synth.pack_codes(codes), lut, x, K)
+    L = _f32_of_bf16(lut)
+    X = _f32_of_bf16(x)
+    for b in range(B):
+        for n in range(N):
+            exact = sum(Fraction(float(L[n, codes[n, k]])) * Fraction(float(X[b, k])) for k in range(K))
+            bound = sum(abs(Fraction(float(L[n, codes[n, k]])) * Fraction(float(X[b, k]))) for k in range(K))
+            assert abs(Fraction(y[b, n]) - exact) <= bound * Fraction(K, 2 ** 52)
+
+
+def test_linear_row_subset_matches_full():
+    w = synth.benq_weights(64, 128, seed=7)
+    x = synth.activations(3, 128, seed=8)
+    full = ob.linear(w.codes, w.lut, x, 128)
+    rows = np.array([0, 5, 63, 17])
+    assert np.array_equal(ob.linear(w.codes, w.lut, x, 128, rows=rows), full[:, rows])

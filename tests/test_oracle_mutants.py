@@ -1,0 +1,107 @@
+"""Planted mistakes in the oracle must each fail at least one pin (CPU only).
+
+Each mutant replaces one oracle function with a plausible wrong version (bit
+order, sign convention, dropped envelope term, transposed operand, off-by-one
+in the accounting) and re-runs the pins; a mutant that no pin catches would
+mean the pins do not actually constrain that part of the oracle.
+"""
+import numpy as np
+import pytest
+
+import tests.test_oracle_accounting as ta
+import tests.test_oracle_benq as tb
+import tests.test_oracle_mdbf as tm
+from oracle import accounting as acc
+from oracle import benq as ob
+from oracle import mdbf as om
+from tests.conftest import read_golden
+
+_orig_unpack_codes = ob.unpack_codes
+_orig_unpack_signs = om.unpack_signs
+_orig_envelope = om.envelope
+
+
+def _unpack_msb_first(packed, K):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    bits = np.unpackbits(packed[:, :6 * K // 8], axis=1, bitorder="little")
+    fields = bits.reshape(packed.shape[0], K, 6).astype(np.int64)
+    return fields @ np.array([32, 16, 8, 4, 2, 1])
+
+
+def _unpack_big_endian_bytes(packed, K):
+    p = np.ascontiguousarray(packed, dtype=np.uint8)[:, :3 * K // 4]
+    p = p.reshape(p.shape[0], -1, 3)[:, :, ::-1].reshape(p.shape[0], -1)
+    return _orig_unpack_codes(p, K)
+
+
+def _dequant_reversed_table(packed, lut_bits, K):
+    return np.take_along_axis(np.asarray(lut_bits, np.uint16), 63 - _orig_unpack_codes(packed, K), axis=1)
+
+
+def _signs_flipped(packed, cols):
+    return (-_orig_unpack_signs(packed, cols)).astype(np.int8)
+
+
+def _signs_msb_first(packed, cols):
+    bits = np.unpackbits(np.ascontiguousarray(packed, np.uint8), axis=1, bitorder="big")
+    return (bits[:, :cols].astype(np.int8) * 2 - 1).astype(np.int8)
+
+
+def _envelope_first_term_only(L, R):
+    return _orig_envelope(L[:, :1], R[:, :1])
+
+
+def _envelope_reversed_columns(L, R):
+    return _orig_envelope(L, R[:, ::-1])
+
+
+def _factors_swapped_qu_qv(path, n, m, r):
+    F = (_orig_unpack_signs(path.S_A, r) * _orig_envelope(path.A_amp, path.Q_V)).astype(np.float32)
+    G = (_orig_unpack_signs(path.S_B, m) * _orig_envelope(path.Q_U, path.B_amp)).astype(np.float32)
+    return F, G
+
+
+def _b_eff_without_2r(n, m, r, P, l, scale_bits=16):
+    from fractions import Fraction
+    return Fraction(P * (r * (n + m) + scale_bits * l * (n + m)), n * m)
+
+
+BENQ_PINS = [
+    lambda: tb.test_unpack_matches_hand_worked_stream(read_golden),
+    lambda: tb.test_linear_hand_worked_example(read_golden),
+    tb.test_pack_unpack_bijection_all_code_groups,
+    tb.test_dequant_is_torch_gather,
+]
+MDBF_PINS = [
+    lambda: tm.test_sign_unpack_hand_worked(read_golden),
+    lambda: tm.test_dequant_and_linear_hand_worked(read_golden),
+    lambda: tm.test_dequant_exact_rational_dyadic((3, 4, 2, 2, 1)),
+    lambda: tm.test_dequant_exact_rational_dyadic((2, 5, 3, 2, 2)),
+]
+ACC_PINS = [ta.test_square_layer_rank_2000_is_one_bit, ta.test_mlp_layers_at_one_and_a_half_bits,
+            ta.test_b_max_is_b_eff_at_full_rank,
+            lambda: ta.test_stored_bits_of_generated_layer_equal_b_eff((64, 96, 40, 2, 1))]
+
+MUTANTS = [
+    ("benq: 6-bit field read MSB first", ob, "unpack_codes", _unpack_msb_first, BENQ_PINS),
+    ("benq: 3-byte group read big-endian", ob, "unpack_codes", _unpack_big_endian_bytes, BENQ_PINS),
+    ("benq: table indexed from the top", ob, "dequant_bits", _dequant_reversed_table, BENQ_PINS),
+    ("mdbf: bit 1 read as -1", om, "unpack_signs", _signs_flipped, MDBF_PINS),
+    ("mdbf: signs packed MSB first", om, "unpack_signs", _signs_msb_first, MDBF_PINS),
+    ("mdbf: envelope keeps only its first term", om, "envelope", _envelope_first_term_only, MDBF_PINS),
+    ("mdbf: envelope columns misaligned", om, "envelope", _envelope_reversed_columns, MDBF_PINS),
+    ("mdbf: Q_U and Q_V swapped", om, "factors", _factors_swapped_qu_qv, MDBF_PINS),
+    ("accounting: b_eff without the 2r envelope term", acc, "mdbf_b_eff", _b_eff_without_2r, ACC_PINS),
+]
+
+
+@pytest.mark.parametrize("name,mod,attr,fn,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(monkeypatch, name, mod, attr, fn, pins):
+    monkeypatch.setattr(mod, attr, fn)
+    caught = 0
+    for pin in pins:
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError):
+            caught += 1
+    assert caught >= 1, f"no pin catches: {name}"
