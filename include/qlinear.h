@@ -1,0 +1,179 @@
+/*
+ * qlinear.h -- C ABI of libqlinear.so: forward pass y = W x of a weight-only
+ * low-bit quantized linear layer whose W stays compressed in device memory and
+ * is decoded on the fly by sm_100a (B200) kernels.
+ *
+ * Two weight formats:
+ *
+ *  BenQ 6-bit ("Qwen3.8-27B -- BenQ 6-bit", section "What BenQ stores"):
+ *    every weight is a 6-bit code (1 sign bit + 5 magnitude-tier bits) indexing
+ *    its output row's own table of 64 signed bf16 magnitudes; decode is exactly
+ *    lut.gather(1, codes).  Codes are packed 4 per 3 bytes (the card's
+ *    "packing to 6-bit" remark made concrete): code k of a row occupies bits
+ *    [6k, 6k+6) of the row's little-endian bitstream, bit q of the stream being
+ *    bit q%8 of byte q/8.  W is N x K (out x in).
+ *
+ *  MDBF ("MDBF (Multi-Envelope Double Binary Factorization)", section
+ *    "Algorithm"): W ~= sum_p F_p G_p with F = S_A (.) (A_amp Q_U^T) and
+ *    G = S_B (.) (Q_V B_amp^T); S_A (n x r) and S_B (r x m) are +-1 matrices
+ *    stored one bit per element (LSB first along each row, bit 1 = +1, rows
+ *    padded to a byte stride; padding bits are ignored), the four envelopes are
+ *    fp16.  W is n x m (out x in).
+ *
+ * Conventions shared by every entry point
+ *  - Pointers named as device pointers are caller-owned device memory.  The
+ *    library never allocates, frees or keeps them.  Host pointers are read
+ *    during the call only.
+ *  - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t;
+ *    NULL is the legacy default stream).  No call synchronizes the device.
+ *  - Activations x are bf16, row-major [B][K] (BenQ) or [B][m] (MDBF).  Outputs
+ *    y are row-major [B][N] / [B][n], fp32 or bf16 (round-to-nearest-even of the
+ *    fp32 result) as chosen by `y_dtype`; accumulation is always fp32.
+ *  - Argument errors are detected on the host before any launch and return
+ *    QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED or QL_ERR_ALIGNMENT with nothing
+ *    launched; a failed launch returns QL_ERR_CUDA.  ql_last_error() gives a
+ *    message for the calling thread's last non-OK status.
+ *  - Device-side waits in the pipelined kernels are bounded.  A wait that runs
+ *    out sets a device-side flag and the kernel returns early (its output is
+ *    then undefined); ql_check() reports it as QL_ERR_TIMEOUT.
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QL_API __attribute__((visibility("default")))
+#else
+#define QL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ql_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1, /* null pointer, non-positive or inconsistent size */
+  QL_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement    */
+  QL_ERR_ALIGNMENT = 3,   /* a pointer or stride breaks a stated alignment    */
+  QL_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed             */
+  QL_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out               */
+} ql_status;
+
+typedef enum { QL_OUT_F32 = 0, QL_OUT_BF16 = 1 } ql_out_dtype;
+
+/* ---------------------------------------------------------------- BenQ ----- */
+
+/*
+ * benq_linear -- y[b][n] = sum_k lut[n][code(n,k)] * x[b][k]
+ *   ("What BenQ stores": decode is lut.gather(1, codes), fused here into the
+ *   contraction so the decoded W is never written to memory).
+ *
+ *   codes  device, uint8 [N][3K/4]: packed codes, row stride exactly 3K/4 bytes.
+ *   lut    device, bf16 bits [N][64]: row n's table; entry c is the value of code c.
+ *   x      device, bf16 bits [B][K].
+ *   y      device, [B][N] of y_dtype; fully overwritten.
+ *   B, N, K  batch rows, output features, input features.  K % 4 == 0.
+ *
+ *   B <= 16 runs the decode GEMV (one pass over the codes, bandwidth bound);
+ *   B > 16 runs the tensor-core GEMM (tcgen05, W tiles decoded into shared
+ *   memory), which needs K % 64 == 0 and N % 16 == 0 (else QL_ERR_UNSUPPORTED).
+ *   Alignment: codes, lut, x, y 16-byte aligned (QL_ERR_ALIGNMENT otherwise).
+ */
+QL_API ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
+                      ql_out_dtype y_dtype, int B, int N, int K, ql_stream_t stream);
+
+/*
+ * benq_dequant_debug -- W[n][k] = lut[n][code(n,k)] as bf16 bits, row-major
+ *   [N][K].  Bit-exact by construction; meant for checking, not speed.
+ *   Same codes / lut layout as benq_linear; K % 4 == 0.
+ */
+QL_API ql_status benq_dequant_debug(const uint8_t *codes, const uint16_t *lut, uint16_t *W, int N,
+                             int K, ql_stream_t stream);
+
+/* Storage cost of one BenQ layer: 6 code bits + 64*16/K table bits per weight
+ * (the card's bits/weight table).  Host only. */
+QL_API double benq_bits_per_weight(int K);
+
+/* ---------------------------------------------------------------- MDBF ----- */
+
+/* One residual path.  Every pointer is device memory; the struct itself is host memory. */
+typedef struct {
+  const uint8_t *S_A;     /* [n][ldSA] packed signs of the n x r matrix S_A */
+  const uint8_t *S_B;     /* [r][ldSB] packed signs of the r x m matrix S_B */
+  size_t ldSA, ldSB;      /* row strides in bytes, >= ceil(r/8), >= ceil(m/8) */
+  const uint16_t *A_amp;  /* fp16 bits [n][l] */
+  const uint16_t *B_amp;  /* fp16 bits [m][l] */
+  const uint16_t *Q_U;    /* fp16 bits [r][l] */
+  const uint16_t *Q_V;    /* fp16 bits [r][l] */
+} mdbf_path;
+
+/* Bytes of device workspace mdbf_linear needs for these sizes (0 on invalid sizes). */
+QL_API size_t mdbf_workspace_bytes(int P, int n, int m, int r, int l, int B);
+
+/*
+ * mdbf_linear -- y[b][a] = sum_p sum_j (F_p G_p)[a][j] x[b][j], evaluated
+ *   without forming W, as two sign-matrix products per path
+ *   ("Algorithm": F = S_A (.) (A_amp Q_U^T), G = S_B (.) (Q_V B_amp^T)):
+ *     t[k][b]   = sum_i Q_V[k][i] * sum_j S_B[k][j] * (B_amp[j][i] * x[b][j])
+ *     y[b][a]  += sum_i A_amp[a][i] * sum_k S_A[a][k] * (Q_U[k][i] * t[k][b]).
+ *
+ *   paths      host array of P paths (device pointers inside).
+ *   P, n, m, r, l  paths, out features, in features, rank, envelope rank;
+ *              1 <= r <= min(n, m) (the page's rank clamp), l >= 1.
+ *   x          device, bf16 bits [B][m].
+ *   y          device, [B][n] of y_dtype; fully overwritten.
+ *   workspace  device scratch of ws_bytes >= mdbf_workspace_bytes(...), 256-byte
+ *              aligned; contents on entry are ignored and on return undefined.
+ *   Limits: l * B <= 64 (else QL_ERR_UNSUPPORTED).
+ */
+QL_API ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r, int l,
+                      const uint16_t *x, void *y, ql_out_dtype y_dtype, int B, void *workspace,
+                      size_t ws_bytes, ql_stream_t stream);
+
+/*
+ * mdbf_dequant_debug -- materialises W (and optionally the factors) in fp32:
+ *   F[p][a][k] = s_A[a][k] * fp32(sum_i A_amp[a][i] Q_U[k][i])   (i ascending),
+ *   G[p][k][j] = s_B[k][j] * fp32(sum_i Q_V[k][i] B_amp[j][i])   (i ascending),
+ *   W[a][j]    = fp32( sum_p sum_k F[p][a][k] * G[p][k][j] ), the sum taken in
+ *                fp64, p outer and k ascending, so the result is reproducible
+ *                bit for bit.
+ *   W  device fp32 [n][m] (required); F device fp32 [P][n][r] or NULL;
+ *   G  device fp32 [P][r][m] or NULL.  O(P n m r) fp64 work: for checking only.
+ */
+QL_API ql_status mdbf_dequant_debug(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W,
+                             float *F, float *G, ql_stream_t stream);
+
+/* Effective bits per weight of an MDBF layer ("Bit-width and rank"):
+ *   b_eff = P [ r (n+m) + scale_bits * l (n + m + 2r) ] / (n m).  Host only. */
+QL_API double mdbf_effective_bits(int n, int m, int r, int P, int l, int scale_bits);
+
+/*
+ * mdbf_select_rank -- rank for a target bits/weight by inverting b_eff
+ *   ("Bit-width and rank"), rounded down, then clamped to min(n, m) ("The
+ *   matrix shape caps the reachable BPW").  *r_out receives the rank and
+ *   *clamped 1 when the target exceeded b_max (the layer then lands below the
+ *   request).  Returns QL_ERR_INVALID_ARG when even rank 1 exceeds the target.
+ *   Host only.
+ */
+QL_API ql_status mdbf_select_rank(int n, int m, int P, int l, int scale_bits, double target_bits,
+                           int *r_out, int *clamped);
+
+/* ---------------------------------------------------------------- misc ----- */
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+QL_API const char *ql_last_error(void);
+
+/* Waits for `stream`, then reports (and clears) a device-side timeout flag:
+ * QL_OK, QL_ERR_TIMEOUT, or QL_ERR_CUDA if the stream itself failed. */
+QL_API ql_status ql_check(ql_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLINEAR_H */

@@ -1,0 +1,195 @@
+"""Python binding of libqlinear.so: BenQ 6-bit and MDBF weight-only quantized linear layers on B200.
+
+Argument marshalling only: every function here takes torch tensors (device
+memory the caller owns), checks dtypes and shapes, passes raw pointers and the
+current CUDA stream to the C ABI declared in ``include/qlinear.h``, and raises
+``QLinearError`` on a non-OK status.  All arithmetic runs in the library's
+sm_100a kernels; there is no fallback.  If ``libqlinear.so`` is missing, import
+fails -- build it with ``python -m quantized_linear_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlinear.so")
+
+_lib = None
+
+QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_ALIGNMENT, QL_ERR_CUDA, QL_ERR_TIMEOUT = range(6)
+QL_OUT_F32, QL_OUT_BF16 = 0, 1
+STATUS_NAMES = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED", 3: "QL_ERR_ALIGNMENT",
+                4: "QL_ERR_CUDA", 5: "QL_ERR_TIMEOUT"}
+
+_vp, _i, _sz, _d = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_double
+
+
+class MDBFPathC(ctypes.Structure):
+    _fields_ = [("S_A", _vp), ("S_B", _vp), ("ldSA", _sz), ("ldSB", _sz),
+                ("A_amp", _vp), ("B_amp", _vp), ("Q_U", _vp), ("Q_V", _vp)]
+
+
+_SIGNATURES = {
+    "benq_linear": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "benq_dequant_debug": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
+    "benq_bits_per_weight": (_d, [_i]),
+    "mdbf_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "mdbf_linear": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _sz, _vp]),
+    "mdbf_dequant_debug": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "mdbf_effective_bits": (_d, [_i, _i, _i, _i, _i, _i]),
+    "mdbf_select_rank": (_i, [_i, _i, _i, _i, _i, _d, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "ql_last_error": (ctypes.c_char_p, []),
+    "ql_check": (_i, [_vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libqlinear.so (loaded on first use; raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m quantized_linear_b200.build` first")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _c(name):
+    return getattr(lib(), name)
+
+EXPORTS = ["benq_linear", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
+           "mdbf_dequant_debug", "mdbf_effective_bits", "mdbf_select_rank", "ql_last_error", "ql_check"]
+
+
+class QLinearError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _check(status: int):
+    if status != QL_OK:
+        raise QLinearError(status, (_c("ql_last_error")() or b"").decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _want(t, dtype, what):
+    if t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+
+
+def _ydt(y):
+    if y.dtype == torch.float32:
+        return QL_OUT_F32
+    if y.dtype == torch.bfloat16:
+        return QL_OUT_BF16
+    raise TypeError("y must be float32 or bfloat16")
+
+
+# ----------------------------------------------------------------------------------------------- BenQ
+
+def benq_linear(codes, lut, x, y, stream=None):
+    """y[B, N] = x[B, K] @ W^T with W[n, k] = lut[n, code(n, k)].
+
+    codes uint8 [N, 3K/4]; lut bf16 (or int16 bit patterns) [N, 64]; x bf16 [B, K];
+    y float32 or bf16 [B, N] (overwritten)."""
+    N = codes.shape[0]
+    B, K = x.shape
+    _want(codes, torch.uint8, "codes")
+    if codes.shape[1] != 3 * K // 4:
+        raise ValueError("codes must be [N, 3K/4]")
+    if lut.dtype not in (torch.bfloat16, torch.int16) or tuple(lut.shape) != (N, 64) or not lut.is_contiguous():
+        raise TypeError("lut must be a contiguous bf16 [N, 64] tensor")
+    _want(x, torch.bfloat16, "x")
+    if tuple(y.shape) != (B, N) or not y.is_contiguous():
+        raise ValueError("y must be contiguous [B, N]")
+    _check(_c("benq_linear")(_ptr(codes), _ptr(lut), _ptr(x), _ptr(y), _ydt(y), B, N, K, _stream(stream)))
+    return y
+
+
+def benq_dequant_debug(codes, lut, W, stream=None):
+    """W[n, k] = lut[n, code(n, k)] as bf16 [N, K]."""
+    N, K = W.shape
+    if codes.shape != (N, 3 * K // 4):
+        raise ValueError("codes must be [N, 3K/4]")
+    _check(_c("benq_dequant_debug")(_ptr(codes), _ptr(lut), _ptr(W), N, K, _stream(stream)))
+    return W
+
+
+def benq_bits_per_weight(K: int) -> float:
+    return float(_c("benq_bits_per_weight")(int(K)))
+
+
+# ----------------------------------------------------------------------------------------------- MDBF
+
+def mdbf_paths_c(paths):
+    """ctypes array of mdbf_path from a list of dicts / objects with S_A, S_B, A_amp, B_amp, Q_U, Q_V tensors
+    (S_A, S_B uint8 [rows, ld]; envelopes fp16 [*, l])."""
+    arr = (MDBFPathC * len(paths))()
+    for i, p in enumerate(paths):
+        g = (lambda k: p[k]) if isinstance(p, dict) else (lambda k: getattr(p, k))
+        arr[i] = MDBFPathC(_ptr(g("S_A")), _ptr(g("S_B")), g("S_A").shape[1], g("S_B").shape[1],
+                           _ptr(g("A_amp")), _ptr(g("B_amp")), _ptr(g("Q_U")), _ptr(g("Q_V")))
+    return arr
+
+
+def mdbf_workspace_bytes(P, n, m, r, l, B) -> int:
+    return int(_c("mdbf_workspace_bytes")(P, n, m, r, l, B))
+
+
+def mdbf_linear(paths, n, m, r, l, x, y, workspace, stream=None):
+    """y[B, n] = x[B, m] @ (sum_p F_p G_p)^T without forming W.  workspace: uint8 CUDA tensor of at least
+    mdbf_workspace_bytes(...) bytes, 256-byte aligned."""
+    _want(x, torch.bfloat16, "x")
+    B = x.shape[0]
+    if x.shape[1] != m or tuple(y.shape) != (B, n) or not y.is_contiguous():
+        raise ValueError("x must be [B, m] and y [B, n]")
+    arr = paths if isinstance(paths, ctypes.Array) else mdbf_paths_c(paths)
+    _check(_c("mdbf_linear")(arr, len(arr), n, m, r, l, _ptr(x), _ptr(y), _ydt(y), B, _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return y
+
+
+def mdbf_dequant_debug(paths, n, m, r, l, W, F=None, G=None, stream=None):
+    """W [n, m] fp32 (and optionally F [P, n, r], G [P, r, m]) materialised bit-reproducibly."""
+    arr = paths if isinstance(paths, ctypes.Array) else mdbf_paths_c(paths)
+    _check(_c("mdbf_dequant_debug")(arr, len(arr), n, m, r, l, _ptr(W), _ptr(F), _ptr(G), _stream(stream)))
+    return W
+
+
+def mdbf_effective_bits(n, m, r, P, l, scale_bits=16) -> float:
+    return float(_c("mdbf_effective_bits")(n, m, r, P, l, scale_bits))
+
+
+def mdbf_select_rank(n, m, P, l, scale_bits, target_bits):
+    """(rank, clamped) for a target bits/weight; raises QLinearError when even rank 1 is too big."""
+    r, c = _i(0), _i(0)
+    _check(_c("mdbf_select_rank")(n, m, P, l, scale_bits, float(target_bits), ctypes.byref(r), ctypes.byref(c)))
+    return r.value, bool(c.value)
+
+
+def ql_check(stream=None):
+    """Waits for the stream and raises QLinearError(QL_ERR_TIMEOUT) if a bounded device wait ran out."""
+    _check(_c("ql_check")(_stream(stream)))

@@ -1,0 +1,169 @@
+// libqlinear C ABI: argument validation, dispatch, status reporting and host-only accounting.
+// The kernels live in benq_gemv.cu, benq_gemm_sm100.cu and mdbf.cu.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+
+#include "ql_internal.cuh"
+
+namespace {
+thread_local char g_msg[512] = "";
+}
+
+namespace ql {
+
+ql_status fail(ql_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+ql_status launch_status(const char *what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(QL_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  return QL_OK;
+}
+
+int sm_count() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+}  // namespace ql
+
+using ql::aligned;
+using ql::fail;
+
+extern "C" {
+
+const char *ql_last_error(void) { return g_msg; }
+
+ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype y_dtype,
+                      int B, int N, int K, ql_stream_t stream) {
+  g_msg[0] = 0;
+  if (!codes || !lut || !x || !y) return fail(QL_ERR_INVALID_ARG, "benq_linear: null pointer");
+  if (B <= 0 || N <= 0 || K <= 0) return fail(QL_ERR_INVALID_ARG, "benq_linear: B, N, K must be positive");
+  if (K % 4) return fail(QL_ERR_INVALID_ARG, "benq_linear: K = %d is not a multiple of 4", K);
+  if (y_dtype != QL_OUT_F32 && y_dtype != QL_OUT_BF16) return fail(QL_ERR_INVALID_ARG, "benq_linear: bad y_dtype");
+  if (!aligned(codes, 16) || !aligned(lut, 16) || !aligned(x, 16) || !aligned(y, 16))
+    return fail(QL_ERR_ALIGNMENT, "benq_linear: codes, lut, x and y must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B <= 16) return ql::benq_gemv_launch(codes, lut, x, y, y_dtype, B, N, K, s);
+  if (K % 64 || N % 16)
+    return fail(QL_ERR_UNSUPPORTED, "benq_linear: batch %d > 16 needs K %% 64 == 0 and N %% 16 == 0", B);
+  return ql::benq_gemm_launch(codes, lut, x, y, y_dtype, B, N, K, s);
+}
+
+ql_status benq_dequant_debug(const uint8_t *codes, const uint16_t *lut, uint16_t *W, int N, int K,
+                             ql_stream_t stream) {
+  g_msg[0] = 0;
+  if (!codes || !lut || !W) return fail(QL_ERR_INVALID_ARG, "benq_dequant_debug: null pointer");
+  if (N <= 0 || K <= 0) return fail(QL_ERR_INVALID_ARG, "benq_dequant_debug: N, K must be positive");
+  if (K % 4) return fail(QL_ERR_INVALID_ARG, "benq_dequant_debug: K = %d is not a multiple of 4", K);
+  if (!aligned(lut, 2) || !aligned(W, 2)) return fail(QL_ERR_ALIGNMENT, "benq_dequant_debug: lut and W must be 2-byte aligned");
+  return ql::benq_dequant_launch(codes, lut, W, N, K, reinterpret_cast<cudaStream_t>(stream));
+}
+
+double benq_bits_per_weight(int K) { return K > 0 ? 6.0 + 64.0 * 16.0 / K : 0.0; }
+
+static ql_status check_paths(const char *who, const mdbf_path *paths, int P, int n, int m, int r, int l) {
+  if (!paths) return fail(QL_ERR_INVALID_ARG, "%s: null paths", who);
+  if (P <= 0 || n <= 0 || m <= 0 || r <= 0 || l <= 0)
+    return fail(QL_ERR_INVALID_ARG, "%s: P, n, m, r, l must be positive", who);
+  if (r > (n < m ? n : m)) return fail(QL_ERR_INVALID_ARG, "%s: rank %d exceeds min(n, m)", who, r);
+  for (int p = 0; p < P; ++p) {
+    const mdbf_path &q = paths[p];
+    if (!q.S_A || !q.S_B || !q.A_amp || !q.B_amp || !q.Q_U || !q.Q_V)
+      return fail(QL_ERR_INVALID_ARG, "%s: path %d has a null pointer", who, p);
+    if (q.ldSA < (size_t)(r + 7) / 8 || q.ldSB < (size_t)(m + 7) / 8)
+      return fail(QL_ERR_INVALID_ARG, "%s: path %d row stride too small", who, p);
+    if (q.ldSA % 4 || q.ldSB % 4 || !aligned(q.S_A, 4) || !aligned(q.S_B, 4))
+      return fail(QL_ERR_ALIGNMENT, "%s: path %d sign rows must be 4-byte aligned (stride %% 4 == 0)", who, p);
+    if (!aligned(q.A_amp, 2) || !aligned(q.B_amp, 2) || !aligned(q.Q_U, 2) || !aligned(q.Q_V, 2))
+      return fail(QL_ERR_ALIGNMENT, "%s: path %d envelopes must be 2-byte aligned", who, p);
+  }
+  return QL_OK;
+}
+
+size_t mdbf_workspace_bytes(int P, int n, int m, int r, int l, int B) {
+  if (P <= 0 || n <= 0 || m <= 0 || r <= 0 || l <= 0 || B <= 0) return 0;
+  return ql::mdbf_workspace_size(P, n, m, r, l, B);
+}
+
+ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x, void *y,
+                      ql_out_dtype y_dtype, int B, void *workspace, size_t ws_bytes, ql_stream_t stream) {
+  g_msg[0] = 0;
+  ql_status st = check_paths("mdbf_linear", paths, P, n, m, r, l);
+  if (st != QL_OK) return st;
+  if (!x || !y || !workspace) return fail(QL_ERR_INVALID_ARG, "mdbf_linear: null x, y or workspace");
+  if (B <= 0) return fail(QL_ERR_INVALID_ARG, "mdbf_linear: B must be positive");
+  if (y_dtype != QL_OUT_F32 && y_dtype != QL_OUT_BF16) return fail(QL_ERR_INVALID_ARG, "mdbf_linear: bad y_dtype");
+  if (!aligned(x, 2) || !aligned(y, 4) || !aligned(workspace, 256))
+    return fail(QL_ERR_ALIGNMENT, "mdbf_linear: x 2-, y 4- and workspace 256-byte alignment required");
+  const size_t need = ql::mdbf_workspace_size(P, n, m, r, l, B);
+  if (ws_bytes < need) return fail(QL_ERR_INVALID_ARG, "mdbf_linear: workspace %zu < %zu bytes", ws_bytes, need);
+  return ql::mdbf_linear_launch(paths, P, n, m, r, l, x, y, y_dtype, B, workspace,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+ql_status mdbf_dequant_debug(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W, float *F, float *G,
+                             ql_stream_t stream) {
+  g_msg[0] = 0;
+  ql_status st = check_paths("mdbf_dequant_debug", paths, P, n, m, r, l);
+  if (st != QL_OK) return st;
+  if (!W) return fail(QL_ERR_INVALID_ARG, "mdbf_dequant_debug: null W");
+  return ql::mdbf_dequant_launch(paths, P, n, m, r, l, W, F, G, reinterpret_cast<cudaStream_t>(stream));
+}
+
+double mdbf_effective_bits(int n, int m, int r, int P, int l, int scale_bits) {
+  if (n <= 0 || m <= 0 || r <= 0 || P <= 0 || l <= 0 || scale_bits < 0) return 0.0;
+  const double num = (double)P * ((double)r * (n + m) + (double)scale_bits * l * ((double)n + m + 2.0 * r));
+  return num / ((double)n * m);
+}
+
+ql_status mdbf_select_rank(int n, int m, int P, int l, int scale_bits, double target_bits, int *r_out, int *clamped) {
+  g_msg[0] = 0;
+  if (!r_out || !clamped) return fail(QL_ERR_INVALID_ARG, "mdbf_select_rank: null output");
+  if (n <= 0 || m <= 0 || P <= 0 || l <= 0 || scale_bits < 0 || !(target_bits > 0.0))
+    return fail(QL_ERR_INVALID_ARG, "mdbf_select_rank: bad arguments");
+  const int s = n < m ? n : m;
+  // r = (b n m / P - sb l (n+m)) / ((n+m) + 2 sb l), exactly as a quotient of two products
+  const long double num = (long double)target_bits * n * m / P - (long double)scale_bits * l * ((long double)n + m);
+  const long double den = (long double)n + m + 2.0L * scale_bits * l;
+  const long double rr = num / den;
+  *clamped = 0;
+  if (rr > (long double)s) {
+    *r_out = s;
+    *clamped = 1;
+    return QL_OK;
+  }
+  const long double f = floorl(rr);
+  if (f < 1.0L) return fail(QL_ERR_INVALID_ARG, "mdbf_select_rank: target %.6f bpw is below rank 1", target_bits);
+  *r_out = (int)f;
+  return QL_OK;
+}
+
+ql_status ql_check(ql_stream_t stream) {
+  g_msg[0] = 0;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QL_ERR_CUDA, "ql_check: %s", cudaGetErrorString(e));
+  int flag = 0;
+  ql_status st = ql::benq_gemm_read_timeout(&flag);
+  if (st != QL_OK) return st;
+  if (flag) return fail(QL_ERR_TIMEOUT, "a bounded device-side wait ran out (code %d)", flag);
+  return QL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,355 @@
+// BenQ 6-bit per-row LUT layer: debug dequantizer and the decode GEMV (batch <= 16).
+//
+// Format ("Qwen3.8-27B -- BenQ 6-bit", "What BenQ stores"): code k of row n is
+// bits [6k, 6k+6) of the row's little-endian bitstream (4 codes per 3 bytes);
+// its value is lut[n][code], a bf16 from the row's own 64-entry table.
+//
+// Decode GEMV design (bandwidth bound: 0.75 B of codes per weight):
+//  * One CTA = C warps, C = ceil(K / 1024).  Lane l of warp w owns the same 32
+//    consecutive codes [1024 w + 32 l, +32) of every row (24 bytes, read with
+//    three 8-byte loads), so at batch 1 its 32 activations live in registers
+//    for the whole kernel and the inner loop reads nothing but codes.
+//  * The CTA walks blocks of R rows (grid-stride).  The R tables (128 B of
+//    bf16 each) sit in shared memory, double-buffered; a lookup is a 16-bit
+//    shared load at byte offset 2*code.  One table spans exactly the 32 banks
+//    (two entries per 32-bit word) and all lanes read the same table, so a
+//    lookup is never a bank conflict (lanes hitting one word are a broadcast).
+//  * Per code: one shift (a funnel shift for codes straddling two words), one
+//    AND to form 2*code, the lookup, and one mixed-precision FMA
+//    (fma.rn.f32.bf16: bf16 x bf16 product, exact, added into fp32).
+//  * Lane partial sums go to shared memory; after one barrier per row block
+//    the C x 32 partials of each output are summed in a fixed order
+//    (deterministic), and the next block's codes and tables are already in flight.
+#include <algorithm>
+
+#include "ql_internal.cuh"
+
+namespace {
+
+constexpr int LANE_CODES = 32;
+constexpr int WARP_CODES = 32 * LANE_CODES;
+constexpr int MAX_WARPS = 20;  // K <= 20480 on the fast path (keeps ~100 registers per thread)
+
+// ------------------------------------------------------------------------------------------
+// Debug dequantizer: one thread per 3-byte group, 4 bf16 outputs.
+// ------------------------------------------------------------------------------------------
+__global__ void benq_dequant_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ lut,
+                                    uint16_t *__restrict__ W, int N, int K) {
+  const int64_t gpr = K / 4;
+  const int64_t total = (int64_t)N * gpr;
+  const int64_t rowbytes = 3LL * K / 4;
+  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = g / gpr;
+    const int64_t q = g - n * gpr;
+    const uint8_t *p = codes + n * rowbytes + 3 * q;
+    const uint32_t v = uint32_t(p[0]) | (uint32_t(p[1]) << 8) | (uint32_t(p[2]) << 16);
+    const uint16_t *t = lut + n * 64;
+    uint16_t *w = W + n * (int64_t)K + 4 * q;
+    w[0] = t[v & 63];
+    w[1] = t[(v >> 6) & 63];
+    w[2] = t[(v >> 12) & 63];
+    w[3] = t[(v >> 18) & 63];
+  }
+}
+
+__device__ __forceinline__ uint2 ldg_u2(const uint8_t *p) {
+  uint2 v;
+  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ldg_u4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// 2*code of code j (0..31) of a lane's 6-word (192-bit) slice: the byte offset of its table entry.
+template <int J>
+__device__ __forceinline__ uint32_t entry_offset(const uint32_t (&w)[6]) {
+  constexpr int s = 6 * J, q = s >> 5, h = s & 31;
+  if constexpr (h == 0) {
+    return (w[q] << 1) & 0x7Eu;
+  } else if constexpr (h <= 26) {
+    return (w[q] >> (h - 1)) & 0x7Eu;
+  } else {
+    return __funnelshift_r(w[q], w[q + 1], h - 1) & 0x7Eu;
+  }
+}
+
+__device__ __forceinline__ uint16_t lds_u16(uint32_t saddr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
+  return v;
+}
+
+template <int J>
+struct DecodeRow {
+  template <int BM>
+  static __device__ __forceinline__ void dot(const uint32_t (&w)[6], uint32_t tbl, const uint16_t (&xr)[32],
+                                             float &acc) {
+    DecodeRow<J - 1>::template dot<BM>(w, tbl, xr, acc);
+    acc = qld::fma_bf16(lds_u16(tbl + entry_offset<J - 1>(w)), xr[J - 1], acc);
+  }
+  static __device__ __forceinline__ void decode(const uint32_t (&w)[6], uint32_t tbl, uint16_t (&out)[32]) {
+    DecodeRow<J - 1>::decode(w, tbl, out);
+    out[J - 1] = lds_u16(tbl + entry_offset<J - 1>(w));
+  }
+};
+template <>
+struct DecodeRow<0> {
+  template <int BM>
+  static __device__ __forceinline__ void dot(const uint32_t (&)[6], uint32_t, const uint16_t (&)[32], float &) {}
+  static __device__ __forceinline__ void decode(const uint32_t (&)[6], uint32_t, uint16_t (&)[32]) {}
+};
+
+__device__ __forceinline__ void unpack_x(const uint4 (&v)[4], uint16_t (&xr)[32]) {
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t u[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      xr[8 * t + 2 * e] = uint16_t(u[e] & 0xFFFFu);
+      xr[8 * t + 2 * e + 1] = uint16_t(u[e] >> 16);
+    }
+  }
+}
+
+template <int R, int BMAX>
+__global__ void __launch_bounds__(MAX_WARPS * 32)
+    benq_gemv_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ lut,
+                     const uint16_t *__restrict__ x, void *__restrict__ y, int ydt, int B, int N, int K) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint16_t *lut_s = reinterpret_cast<uint16_t *>(smem);             // [2][R][64]
+  float *part = reinterpret_cast<float *>(smem + 2 * R * 128);      // [2][C][R*BMAX][32]
+  const int C = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kc = warp * WARP_CODES + lane * LANE_CODES;
+  const bool active = kc < K;
+  const int64_t rowbytes = 3LL * K / 4;
+  const uint8_t *cbase = codes + 3LL * kc / 4;
+  const int nblk = (N + R - 1) / R;
+  int blk = blockIdx.x;
+  if (blk >= nblk) return;
+
+  uint16_t xr[32];
+  if constexpr (BMAX == 1) {
+    uint4 v[4] = {};
+    if (active) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) v[t] = ldg_u4(x + kc + 8 * t);
+    }
+    unpack_x(v, xr);
+  }
+
+  auto load_codes = [&](int b, uint32_t (&w)[R][6]) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int n = b * R + r;
+      if (active && n < N) {
+        const uint8_t *p = cbase + n * rowbytes;
+        const uint2 a = ldg_u2(p), c = ldg_u2(p + 8), d = ldg_u2(p + 16);
+        w[r][0] = a.x; w[r][1] = a.y; w[r][2] = c.x; w[r][3] = c.y; w[r][4] = d.x; w[r][5] = d.y;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 6; ++q) w[r][q] = 0;
+      }
+    }
+  };
+  // tables: threads 0 .. 8R-1 each move 16 bytes of the R x 128-byte block
+  auto load_lut = [&](int b, uint4 &v) {
+    v = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x < 8 * R) {
+      const int n = b * R + (threadIdx.x >> 3);
+      if (n < N) v = ldg_u4(lut + (int64_t)n * 64 + (threadIdx.x & 7) * 8);
+    }
+  };
+  auto store_lut = [&](int buf, const uint4 &v) {
+    if (threadIdx.x < 8 * R) reinterpret_cast<uint4 *>(lut_s + buf * R * 64)[threadIdx.x] = v;
+  };
+
+  uint32_t cur[R][6];
+  {
+    uint4 lv;
+    load_lut(blk, lv);
+    store_lut(0, lv);
+    load_codes(blk, cur);
+  }
+  __syncthreads();
+
+  const uint32_t lut_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(lut_s));
+  for (int it = 0;; ++it) {
+    const int buf = it & 1;
+    const int nxt = blk + gridDim.x;
+    const bool has_next = nxt < nblk;
+    uint32_t nc[R][6];
+    uint4 lv;
+    if (has_next) {
+      load_codes(nxt, nc);
+      load_lut(nxt, lv);
+    }
+
+    float acc[R][BMAX];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) acc[r][b] = 0.f;
+
+    if (active) {
+      if constexpr (BMAX == 1) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint32_t tbl = lut_saddr + (buf * R + r) * 128;
+          DecodeRow<32>::dot<1>(cur[r], tbl, xr, acc[r][0]);
+        }
+      } else {
+        uint16_t wv[R][32];
+#pragma unroll
+        for (int r = 0; r < R; ++r) DecodeRow<32>::decode(cur[r], lut_saddr + (buf * R + r) * 128, wv[r]);
+#pragma unroll
+        for (int b = 0; b < BMAX; ++b) {
+          if (b < B) {
+            uint4 v[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) v[t] = ldg_u4(x + (int64_t)b * K + kc + 8 * t);
+            unpack_x(v, xr);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              float a = acc[r][b];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) a = qld::fma_bf16(wv[r][j], xr[j], a);
+              acc[r][b] = a;
+            }
+          }
+        }
+      }
+    }
+
+    float *pb = part + (size_t)buf * C * R * BMAX * 32;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) pb[((size_t)warp * R * BMAX + r * BMAX + b) * 32 + lane] = acc[r][b];
+    if (has_next) store_lut(buf ^ 1, lv);
+    __syncthreads();
+
+    // sum the C x 32 partials of each output in a fixed order
+    for (int o = warp; o < R * BMAX; o += C) {
+      const int r = o / BMAX, b = o - r * BMAX;
+      const int n = blk * R + r;
+      if (b >= B || n >= N) continue;
+      float s = 0.f;
+      for (int c = 0; c < C; ++c) s += pb[((size_t)c * R * BMAX + o) * 32 + lane];
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
+      if (lane == 0) {
+        if (ydt == QL_OUT_F32)
+          static_cast<float *>(y)[(int64_t)b * N + n] = s;
+        else
+          static_cast<uint16_t *>(y)[(int64_t)b * N + n] = qld::f32_to_bf16_rn(s);
+      }
+    }
+    if (!has_next) break;
+    blk = nxt;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int q = 0; q < 6; ++q) cur[r][q] = nc[r][q];
+  }
+}
+
+// Any K % 4 == 0: one warp per row, lanes over 3-byte groups, table read from global memory.
+__global__ void benq_gemv_generic_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ lut,
+                                         const uint16_t *__restrict__ x, void *__restrict__ y, int ydt, int B,
+                                         int N, int K) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rowbytes = 3LL * K / 4;
+  for (int64_t n = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; n < N;
+       n += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    float acc[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) acc[b] = 0.f;
+    const uint8_t *row = codes + n * rowbytes;
+    const uint16_t *t = lut + n * 64;
+    for (int q = lane; q < K / 4; q += 32) {
+      const uint32_t v = uint32_t(row[3 * q]) | (uint32_t(row[3 * q + 1]) << 8) | (uint32_t(row[3 * q + 2]) << 16);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint16_t wv = t[(v >> (6 * e)) & 63];
+#pragma unroll
+        for (int b = 0; b < 16; ++b)
+          if (b < B) acc[b] = qld::fma_bf16(wv, x[(int64_t)b * K + 4 * q + e], acc[b]);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < 16; ++b) {
+      if (b >= B) break;
+      float s = acc[b];
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
+      if (lane == 0) {
+        if (ydt == QL_OUT_F32)
+          static_cast<float *>(y)[(int64_t)b * N + n] = s;
+        else
+          static_cast<uint16_t *>(y)[(int64_t)b * N + n] = qld::f32_to_bf16_rn(s);
+      }
+    }
+  }
+}
+
+template <int R, int BMAX>
+ql_status launch_fast(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype ydt,
+                      int B, int N, int K, cudaStream_t s) {
+  const int C = (K + WARP_CODES - 1) / WARP_CODES;
+  const int threads = C * 32;
+  const size_t smem = 2 * R * 128 + (size_t)2 * C * R * BMAX * 32 * sizeof(float);
+  auto kern = benq_gemv_kernel<R, BMAX>;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return ql::fail(QL_ERR_CUDA, "benq_linear: cannot reserve %zu bytes of shared memory", smem);
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1)
+    return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
+  const int nblk = (N + R - 1) / R;
+  const int grid = std::min(nblk, per_sm * ql::sm_count());
+  kern<<<grid, threads, smem, s>>>(codes, lut, x, y, (int)ydt, B, N, K);
+  return ql::launch_status("benq_linear (decode GEMV)");
+}
+
+}  // namespace
+
+namespace ql {
+
+ql_status benq_dequant_launch(const uint8_t *codes, const uint16_t *lut, uint16_t *W, int N, int K,
+                              cudaStream_t s) {
+  const int64_t total = (int64_t)N * (K / 4);
+  const int threads = 256;
+  const int64_t want = (total + threads - 1) / threads;
+  const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count() * 8);
+  benq_dequant_kernel<<<grid, threads, 0, s>>>(codes, lut, W, N, K);
+  return launch_status("benq_dequant_debug");
+}
+
+ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
+                           ql_out_dtype ydt, int B, int N, int K, cudaStream_t s) {
+  const bool fast = (K % LANE_CODES == 0) && K <= MAX_WARPS * WARP_CODES && aligned(codes, 16) &&
+                    aligned(x, 16);
+  if (fast) {
+    if (B == 1) return launch_fast<4, 1>(codes, lut, x, y, ydt, B, N, K, s);
+    if (B <= 2) return launch_fast<2, 2>(codes, lut, x, y, ydt, B, N, K, s);
+    if (B <= 4) return launch_fast<2, 4>(codes, lut, x, y, ydt, B, N, K, s);
+    if (B <= 8) return launch_fast<2, 8>(codes, lut, x, y, ydt, B, N, K, s);
+    return launch_fast<1, 16>(codes, lut, x, y, ydt, B, N, K, s);
+  }
+  const int threads = 256;
+  const int64_t want = ((int64_t)N * 32 + threads - 1) / threads;
+  const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count() * 8);
+  benq_gemv_generic_kernel<<<grid, threads, 0, s>>>(codes, lut, x, y, (int)ydt, B, N, K);
+  return launch_status("benq_linear (generic GEMV)");
+}
+
+}  // namespace ql

@@ -1,0 +1,61 @@
+// Internal helpers shared by the libqlinear translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qlinear.h"
+
+namespace ql {
+
+// Records a message for ql_last_error() and returns `s`.
+ql_status fail(ql_status s, const char *fmt, ...);
+// Converts the launch state of the last kernel into a status (QL_ERR_CUDA on failure).
+ql_status launch_status(const char *what);
+// Multiprocessor count of the current device (cached per device).
+int sm_count();
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---- entry points implemented by the kernel translation units (arguments already validated) ----
+ql_status benq_dequant_launch(const uint8_t *codes, const uint16_t *lut, uint16_t *W, int N, int K,
+                              cudaStream_t s);
+ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
+                           ql_out_dtype ydt, int B, int N, int K, cudaStream_t s);
+ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
+                           ql_out_dtype ydt, int M, int N, int K, cudaStream_t s);
+ql_status benq_gemm_read_timeout(int *flag);  // reads and clears the GEMM's bounded-wait flag
+
+size_t mdbf_workspace_size(int P, int n, int m, int r, int l, int B);
+ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r, int l,
+                             const uint16_t *x, void *y, ql_out_dtype ydt, int B, void *ws,
+                             cudaStream_t s);
+ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W,
+                              float *F, float *G, cudaStream_t s);
+
+}  // namespace ql
+
+// ---- device helpers ----
+namespace qld {
+
+__device__ __forceinline__ float bf16_to_f32(uint32_t h16) { return __uint_as_float(h16 << 16); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
+  uint16_t h;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(f));
+  return h;
+}
+
+__device__ __forceinline__ float f16_to_f32(uint16_t h) {
+  float f;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
+  return f;
+}
+
+// acc + a * b with bf16 a, b and fp32 accumulate; the product is exact in fp32.
+__device__ __forceinline__ float fma_bf16(uint16_t a, uint16_t b, float acc) {
+  asm("fma.rn.f32.bf16 %0, %1, %2, %0;" : "+f"(acc) : "h"(a), "h"(b));
+  return acc;
+}
+
+}  // namespace qld

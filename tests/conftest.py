@@ -30,3 +30,12 @@ def read_golden(name):
 @pytest.fixture
 def golden():
     return read_golden
+
+
+@pytest.fixture(scope="session")
+def ql():
+    """The quantized_linear_b200 binding, building libqlinear.so first if it is missing or stale."""
+    from quantized_linear_b200 import build as qlbuild
+    qlbuild.build()
+    import quantized_linear_b200
+    return quantized_linear_b200

@@ -1,0 +1,117 @@
+"""BenQ parity on the GPU: the C ABI against the CPU oracle on the same seeded inputs.
+
+Debug dequantization must be bit-exact; benq_linear must be within 2e-3
+(max |y - y_ref| / max |y_ref| per batch row, fp32 output) of the oracle's
+fp64 result, and its bf16 output must be the round-to-nearest-even of its own
+fp32 output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import benq as ob
+from tests.qlhelpers import BENQ_TOL, bf16, bits16, dev, f32_to_bf16_rne, max_rel
+
+pytestmark = pytest.mark.gpu
+
+
+def _linear(ql, w, xbits, ydtype=torch.float32):
+    B = xbits.shape[0]
+    y = torch.empty(B, w.N, dtype=ydtype, device="cuda")
+    ql.benq_linear(dev(w.codes), bits16(w.lut), bf16(xbits), y)
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("N,K", [(256, 512), (1, 4), (3, 8), (5, 100), (77, 1028), (40, 5120)])
+def test_dequant_bit_exact(ql, N, K):
+    w = synth.benq_weights(N, K, seed=N * 7 + K)
+    W = torch.empty(N, K, dtype=torch.int16, device="cuda")
+    ql.benq_dequant_debug(dev(w.codes), bits16(w.lut), W)
+    torch.cuda.synchronize()
+    assert np.array_equal(W.cpu().numpy().view(np.uint16), ob.dequant_bits(w.codes, w.lut, K))
+
+
+def test_dequant_arbitrary_tables_bit_exact(ql):
+    # tables need not be sorted or symmetric: random bit patterns (NaN/Inf included) must pass through
+    rng = np.random.default_rng(3)
+    N, K = 64, 256
+    codes = rng.integers(0, 64, size=(N, K), dtype=np.uint8)
+    lut = rng.integers(0, 1 << 16, size=(N, 64), dtype=np.uint16)
+    packed = synth.pack_codes(codes)
+    W = torch.empty(N, K, dtype=torch.int16, device="cuda")
+    ql.benq_dequant_debug(dev(packed), bits16(lut), W)
+    torch.cuda.synchronize()
+    assert np.array_equal(W.cpu().numpy().view(np.uint16), ob.dequant_bits(packed, lut, K))
+
+
+def test_dequant_full_size_sampled_rows(ql):
+    N, K = 17408, 5120
+    w = synth.benq_weights(N, K, seed=1001)
+    W = torch.empty(N, K, dtype=torch.int16, device="cuda")
+    ql.benq_dequant_debug(dev(w.codes), bits16(w.lut), W)
+    torch.cuda.synchronize()
+    rows = np.r_[np.random.default_rng(0).choice(N, 96, replace=False), N - 1]
+    got = W[torch.from_numpy(rows).cuda()].cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, ob.dequant_bits(w.codes[rows], w.lut[rows], K))
+
+
+@pytest.mark.parametrize("B", [1, 8])
+def test_linear_small_layer(ql, B):
+    # 256 out x 512 in, the small seeded layer
+    w = synth.benq_weights(256, 512, seed=0)
+    x = synth.activations(B, 512, seed=1)
+    y = _linear(ql, w, x).cpu().numpy()
+    assert max_rel(y, ob.linear(w.codes, w.lut, x, 512)) <= BENQ_TOL
+    yb = _linear(ql, w, x, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(yb, f32_to_bf16_rne(y))
+
+
+@pytest.mark.parametrize("N,K,B", [(7, 32, 1), (33, 1056, 3), (100, 2048, 16), (250, 5120, 2), (13, 96, 5),
+                                   (129, 3072, 4), (65, 4096, 8), (31, 20480, 1), (2, 64, 16)])
+def test_linear_fast_path_shapes(ql, N, K, B):
+    w = synth.benq_weights(N, K, seed=N + K + B)
+    x = synth.activations(B, K, seed=B)
+    y = _linear(ql, w, x).cpu().numpy()
+    assert max_rel(y, ob.linear(w.codes, w.lut, x, K)) <= BENQ_TOL
+
+
+@pytest.mark.parametrize("N,K,B", [(1, 4, 1), (10, 100, 1), (9, 36, 4), (17, 20484, 2), (5, 1000, 16)])
+def test_linear_generic_path_shapes(ql, N, K, B):
+    w = synth.benq_weights(N, K, seed=N * K + B)
+    x = synth.activations(B, K, seed=B + 10)
+    y = _linear(ql, w, x).cpu().numpy()
+    assert max_rel(y, ob.linear(w.codes, w.lut, x, K)) <= BENQ_TOL
+
+
+@pytest.mark.parametrize("N,K", [(17408, 5120), (5120, 17408)])
+def test_linear_decode_shapes_full_size(ql, N, K):
+    # the 27B-class gate/up and down projections at batch 1, sampled rows against the oracle
+    w = synth.benq_weights(N, K, seed=1000 + N // 1024)
+    x = synth.activations(1, K, seed=1100)
+    y = _linear(ql, w, x).cpu().numpy()
+    rows = np.r_[np.random.default_rng(1).choice(N, 512, replace=False), 0, N - 1]
+    ref = ob.linear(w.codes, w.lut, x, K, rows=rows)
+    assert max_rel(y[:, rows], ref) <= BENQ_TOL
+
+
+def test_linear_is_deterministic(ql):
+    w = synth.benq_weights(5120, 5120, seed=5)
+    x = synth.activations(1, 5120, seed=6)
+    a = _linear(ql, w, x)
+    b = _linear(ql, w, x)
+    assert torch.equal(a, b)
+
+
+def test_linear_argument_errors(ql):
+    w = synth.benq_weights(8, 64, seed=0)
+    x = bf16(synth.activations(1, 64, seed=0))
+    y = torch.empty(1, 8, device="cuda")
+    codes, lut = dev(w.codes), bits16(w.lut)
+    raw = ql.lib().benq_linear
+    s = torch.cuda.current_stream().cuda_stream
+    assert raw(codes.data_ptr(), lut.data_ptr(), x.data_ptr() + 2, y.data_ptr(), 0, 1, 8, 64, s) == ql.QL_ERR_ALIGNMENT
+    assert raw(codes.data_ptr(), lut.data_ptr(), x.data_ptr(), y.data_ptr(), 0, 1, 8, 62, s) == ql.QL_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        ql.benq_linear(codes, lut, x, torch.empty(2, 8, device="cuda"))

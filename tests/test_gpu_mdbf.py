@@ -1,0 +1,104 @@
+"""MDBF parity on the GPU: the C ABI against the CPU oracle on the same seeded inputs.
+
+mdbf_dequant_debug must reproduce the oracle's W, F and G bit for bit;
+mdbf_linear must be within 5e-3 (max |y - y_ref| / max |y_ref| per batch row,
+fp32 output) of the oracle's fp64 result, and its bf16 output must be the
+round-to-nearest-even of its own fp32 output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import mdbf as om
+from tests.qlhelpers import MDBF_TOL, bf16, dev, f32_to_bf16_rne, max_rel, mdbf_dev_paths
+
+pytestmark = pytest.mark.gpu
+
+
+def _linear(ql, paths, n, m, r, l, xbits, ydtype=torch.float32):
+    B = xbits.shape[0]
+    dp = mdbf_dev_paths(paths)
+    ws = torch.empty(ql.mdbf_workspace_bytes(len(paths), n, m, r, l, B), dtype=torch.uint8, device="cuda")
+    y = torch.empty(B, n, dtype=ydtype, device="cuda")
+    ql.mdbf_linear(dp, n, m, r, l, bf16(xbits), y, ws)
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("n,m,r,l,P", [(40, 24, 20, 4, 2), (64, 96, 33, 3, 2), (100, 37, 29, 1, 1),
+                                       (128, 128, 64, 2, 1), (17, 300, 17, 2, 3), (512, 256, 200, 4, 2)])
+def test_dequant_bit_exact(ql, n, m, r, l, P):
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=n + m + r)
+    dp = mdbf_dev_paths(paths)
+    W = torch.empty(n, m, device="cuda")
+    F = torch.empty(P, n, r, device="cuda")
+    G = torch.empty(P, r, m, device="cuda")
+    ql.mdbf_dequant_debug(dp, n, m, r, l, W, F, G)
+    torch.cuda.synchronize()
+    assert np.array_equal(W.cpu().numpy().view(np.uint32), om.dequant(paths, n, m, r).view(np.uint32))
+    for p in range(P):
+        Fo, Go = om.factors(paths[p], n, m, r)
+        assert np.array_equal(F[p].cpu().numpy().view(np.uint32), Fo.view(np.uint32))
+        assert np.array_equal(G[p].cpu().numpy().view(np.uint32), Go.view(np.uint32))
+
+
+def test_dequant_hand_worked_example(ql, golden):
+    g = golden("mdbf_example.txt")
+    f16 = lambda v: np.array([float(t) for t in v], dtype=np.float16).view(np.uint16)
+    S_A = np.zeros((2, 4), np.uint8)
+    S_A[:, 0] = [int(b, 16) for b in g["S_A_bytes"]]
+    S_B = np.zeros((2, 4), np.uint8)
+    S_B[:, 0] = [int(b, 16) for b in g["S_B_bytes"]]
+    path = synth.MDBFPath(S_A=S_A, S_B=S_B, A_amp=f16(g["A_amp"]).reshape(2, 2), B_amp=f16(g["B_amp"]).reshape(3, 2),
+                          Q_U=f16(g["Q_U"]).reshape(2, 2), Q_V=f16(g["Q_V"]).reshape(2, 2))
+    W = torch.empty(2, 3, device="cuda")
+    ql.mdbf_dequant_debug(mdbf_dev_paths([path]), 2, 3, 2, 2, W)
+    x = synth.f32_to_bf16_bits(np.array([[float(v) for v in g["x"]]], dtype=np.float32))
+    y = _linear(ql, [path], 2, 3, 2, 2, x)
+    assert W.cpu().numpy().ravel().tolist() == [float(v) for v in g["W"]]
+    assert np.allclose(y.cpu().numpy().ravel(), [float(v) for v in g["y"]], rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("n,m,r,l,P,B", [(5, 7, 3, 1, 1, 1), (33, 65, 31, 2, 2, 3), (100, 40, 40, 4, 2, 16),
+                                         (64, 64, 64, 8, 1, 8), (70, 90, 50, 3, 3, 5), (300, 200, 100, 1, 2, 1),
+                                         (96, 1000, 95, 2, 1, 32), (1, 1, 1, 1, 1, 1)])
+def test_linear_shapes(ql, n, m, r, l, P, B):
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=3 * n + m)
+    x = synth.activations(B, m, seed=B)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+    yd = om.linear_dense(paths, n, m, r, x)
+    assert max_rel(y, yd) <= MDBF_TOL
+    yb = _linear(ql, paths, n, m, r, l, x, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(yb, f32_to_bf16_rne(y))
+
+
+@pytest.mark.parametrize("B", [1, 16])
+def test_linear_square_one_bit_layer(ql, B):
+    # n = m = 4096, P = 1, l = 2, r = 2000 (b_eff ~ 1.0)
+    n = m = 4096
+    r, l = 2000, 2
+    paths = synth.mdbf_paths(1, n, m, r, l, seed=3000)
+    x = synth.activations(B, m, seed=3100 + B)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+
+
+@pytest.mark.parametrize("n,m", [(17408, 5120), (5120, 17408)])
+def test_linear_mlp_shapes_sampled_rows(ql, n, m):
+    # 27B-class gate/up and down at 1.5 bits/weight: P = 2, l = 4, r = 2886
+    r, l, P = 2886, 4, 2
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=4000 + n // 1024)
+    x = synth.activations(1, m, seed=4100)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    rows = np.r_[np.random.default_rng(2).choice(n, 256, replace=False), 0, n - 1]
+    assert max_rel(y[:, rows], om.linear_factored(paths, n, m, r, x, rows=rows)) <= MDBF_TOL
+
+
+def test_linear_is_deterministic(ql):
+    paths = synth.mdbf_paths(2, 1024, 768, 300, 4, seed=8)
+    x = synth.activations(2, 768, seed=9)
+    a = _linear(ql, paths, 1024, 768, 300, 4, x)
+    b = _linear(ql, paths, 1024, 768, 300, 4, x)
+    assert torch.equal(a, b)
