@@ -300,6 +300,171 @@ __global__ void benq_gemv_generic_kernel(const uint8_t *__restrict__ codes, cons
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// Batch-1 kernel for whole tiles (K % 1024 == 0, N % B1_T == 0).  Same lane layout as above,
+// with the instruction count per code cut to: one shift, one AND|OR forming the 32-bit shared
+// address of the table entry (tables are 128-byte aligned so the OR is an add), one 16-bit
+// shared load, one integer multiply placing the bf16 in the top half (an fp32), and half of a
+// packed fp32x2 FMA.  Two row groups of B1_R rows ping-pong in registers so the next group's
+// codes are in flight while one is decoded; one barrier per tile of B1_T rows.
+// ------------------------------------------------------------------------------------------
+constexpr int B1_R = 2, B1_T = 4;
+
+struct B1Tables {
+  uint16_t lut[2][B1_T][64];
+};
+
+__device__ __forceinline__ uint32_t lds_u16_32(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(saddr));
+  return v;
+}
+
+__device__ __forceinline__ float bf16_hi(uint32_t v16) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, 65536, 0;" : "=r"(r) : "r"(v16));
+  return __uint_as_float(r);
+}
+
+// (a0, a1) += (w0, w1) * (x0, x1) as one packed fp32x2 FMA
+__device__ __forceinline__ void ffma2(float &a0, float &a1, float w0, float w1, float x0, float x1) {
+  unsigned long long acc, w, x;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(acc) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(w) : "f"(w0), "f"(w1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(w), "l"(x));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+}
+
+template <int J0>
+__device__ __forceinline__ void dot_pair(const uint32_t (&w)[6], uint32_t tbl, const float (&xf)[32], float &a0,
+                                         float &a1) {
+  const float w0 = bf16_hi(lds_u16_32(entry_offset<J0>(w) | tbl));
+  const float w1 = bf16_hi(lds_u16_32(entry_offset<J0 + 1>(w) | tbl));
+  ffma2(a0, a1, w0, w1, xf[J0], xf[J0 + 1]);
+}
+
+template <int J>
+struct DotB1 {
+  static __device__ __forceinline__ void run(const uint32_t (&w)[6], uint32_t tbl, const float (&xf)[32], float &a0,
+                                             float &a1) {
+    DotB1<J - 2>::run(w, tbl, xf, a0, a1);
+    dot_pair<J - 2>(w, tbl, xf, a0, a1);
+  }
+};
+template <>
+struct DotB1<0> {
+  static __device__ __forceinline__ void run(const uint32_t (&)[6], uint32_t, const float (&)[32], float &, float &) {}
+};
+
+__global__ void __launch_bounds__(MAX_WARPS * 32)
+    benq_gemv_b1_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ lut,
+                        const uint16_t *__restrict__ x, void *__restrict__ y, int ydt, int N, int K) {
+  __shared__ __align__(128) B1Tables tb;
+  extern __shared__ __align__(16) float b1part[];  // [2][C][B1_T][32]
+  const int C = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kc = warp * WARP_CODES + lane * LANE_CODES;
+  const uint32_t rowbytes = 3u * K / 4;
+  const uint8_t *cbase = codes + 3u * kc / 4;
+  const int ntile = N / B1_T;
+  int tile = blockIdx.x;
+  if (tile >= ntile) return;
+
+  float xf[32];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint4 v = ldg_u4(x + kc + 8 * t);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      xf[8 * t + 2 * e] = __uint_as_float(u[e] << 16);
+      xf[8 * t + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    }
+  }
+  auto load_rows = [&](int n0, uint32_t (&w)[B1_R][6]) {
+    const uint8_t *p = cbase + (size_t)n0 * rowbytes;
+#pragma unroll
+    for (int r = 0; r < B1_R; ++r) {
+      const uint2 a = ldg_u2(p + r * rowbytes), c = ldg_u2(p + r * rowbytes + 8), d = ldg_u2(p + r * rowbytes + 16);
+      w[r][0] = a.x; w[r][1] = a.y; w[r][2] = c.x; w[r][3] = c.y; w[r][4] = d.x; w[r][5] = d.y;
+    }
+  };
+  auto load_lut = [&](int t, uint4 &v) {
+    if (threadIdx.x < 8 * B1_T) v = ldg_u4(lut + ((size_t)t * B1_T + (threadIdx.x >> 3)) * 64 + (threadIdx.x & 7) * 8);
+  };
+  auto store_lut = [&](int buf, const uint4 &v) {
+    if (threadIdx.x < 8 * B1_T) reinterpret_cast<uint4 *>(&tb.lut[buf][0][0])[threadIdx.x] = v;
+  };
+  auto row_dot = [&](const uint32_t (&w)[6], uint32_t tbl) {
+    float a0 = 0.f, a1 = 0.f;
+    DotB1<32>::run(w, tbl, xf, a0, a1);
+    return a0 + a1;
+  };
+
+  uint4 lv = make_uint4(0, 0, 0, 0);
+  load_lut(tile, lv);
+  store_lut(0, lv);
+  uint32_t ga[B1_R][6], gb[B1_R][6];
+  load_rows(tile * B1_T, ga);
+  __syncthreads();
+  const uint32_t lut0 = static_cast<uint32_t>(__cvta_generic_to_shared(&tb.lut[0][0][0]));
+  float *mypart = b1part + (size_t)warp * B1_T * 32 + lane;
+  constexpr int GP = B1_T / B1_R;  // even
+  for (int buf = 0;; buf ^= 1) {
+    const int nxt = tile + gridDim.x;
+    const bool has_next = nxt < ntile;
+    if (has_next) load_lut(nxt, lv);
+    float *pb = mypart + (size_t)buf * C * B1_T * 32;
+    const uint32_t tbase = lut0 + buf * B1_T * 128;
+#pragma unroll
+    for (int g = 0; g < GP; g += 2) {
+      load_rows(tile * B1_T + (g + 1) * B1_R, gb);
+#pragma unroll
+      for (int r = 0; r < B1_R; ++r) pb[(g * B1_R + r) * 32] = row_dot(ga[r], tbase + (g * B1_R + r) * 128);
+      if (g + 2 < GP)
+        load_rows(tile * B1_T + (g + 2) * B1_R, ga);
+      else if (has_next)
+        load_rows(nxt * B1_T, ga);
+#pragma unroll
+      for (int r = 0; r < B1_R; ++r)
+        pb[((g + 1) * B1_R + r) * 32] = row_dot(gb[r], tbase + ((g + 1) * B1_R + r) * 128);
+    }
+    if (has_next) store_lut(buf ^ 1, lv);
+    __syncthreads();
+    const float *pr = b1part + (size_t)buf * C * B1_T * 32;
+    for (int o = warp; o < B1_T; o += C) {
+      float s = 0.f;
+      for (int c = 0; c < C; ++c) s += pr[(c * B1_T + o) * 32 + lane];
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
+      if (lane == 0) {
+        const int n = tile * B1_T + o;
+        if (ydt == QL_OUT_F32)
+          static_cast<float *>(y)[n] = s;
+        else
+          static_cast<uint16_t *>(y)[n] = qld::f32_to_bf16_rn(s);
+      }
+    }
+    if (!has_next) break;
+    tile = nxt;
+  }
+}
+
+ql_status launch_b1(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype ydt, int N,
+                    int K, cudaStream_t s) {
+  const int C = K / WARP_CODES;
+  const int threads = C * 32;
+  const size_t smem = (size_t)2 * C * B1_T * 32 * sizeof(float);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, benq_gemv_b1_kernel, threads, smem) != cudaSuccess ||
+      per_sm < 1)
+    return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
+  const int grid = std::min(N / B1_T, per_sm * ql::sm_count());
+  benq_gemv_b1_kernel<<<grid, threads, smem, s>>>(codes, lut, x, y, (int)ydt, N, K);
+  return ql::launch_status("benq_linear (batch-1 GEMV)");
+}
+
 template <int R, int BMAX>
 ql_status launch_fast(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype ydt,
                       int B, int N, int K, cudaStream_t s) {
@@ -339,6 +504,7 @@ ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint
   const bool fast = (K % LANE_CODES == 0) && K <= MAX_WARPS * WARP_CODES && aligned(codes, 16) &&
                     aligned(x, 16);
   if (fast) {
+    if (B == 1 && K % WARP_CODES == 0 && N % B1_T == 0) return launch_b1(codes, lut, x, y, ydt, N, K, s);
     if (B == 1) return launch_fast<4, 1>(codes, lut, x, y, ydt, B, N, K, s);
     if (B <= 2) return launch_fast<2, 2>(codes, lut, x, y, ydt, B, N, K, s);
     if (B <= 4) return launch_fast<2, 4>(codes, lut, x, y, ydt, B, N, K, s);

@@ -68,7 +68,7 @@ def test_linear_small_layer(ql, B):
     assert np.array_equal(yb, f32_to_bf16_rne(y))
 
 
-@pytest.mark.parametrize("N,K,B", [(7, 32, 1), (33, 1056, 3), (100, 2048, 16), (250, 5120, 2), (13, 96, 5),
+@pytest.mark.parametrize("N,K,B", [(8, 1024, 1), (64, 3072, 1), (40, 20480, 1), (7, 32, 1), (33, 1056, 3), (100, 2048, 16), (250, 5120, 2), (13, 96, 5),
                                    (129, 3072, 4), (65, 4096, 8), (31, 20480, 1), (2, 64, 16)])
 def test_linear_fast_path_shapes(ql, N, K, B):
     w = synth.benq_weights(N, K, seed=N + K + B)
