@@ -81,7 +81,7 @@ typedef enum { QL_OUT_F32 = 0, QL_OUT_BF16 = 1 } ql_out_dtype;
  *
  *   B <= 16 runs the decode GEMV (one pass over the codes, bandwidth bound);
  *   B > 16 runs the tensor-core GEMM (tcgen05, W tiles decoded into shared
- *   memory), which needs K % 64 == 0 and N % 16 == 0 (else QL_ERR_UNSUPPORTED).
+ *   memory), which needs K % 64 == 0 and N % 256 == 0 (else QL_ERR_UNSUPPORTED).
  *   Alignment: codes, lut, x, y 16-byte aligned (QL_ERR_ALIGNMENT otherwise).
  */
 QL_API ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,

@@ -61,8 +61,8 @@ ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t 
     return fail(QL_ERR_ALIGNMENT, "benq_linear: codes, lut, x and y must be 16-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (B <= 16) return ql::benq_gemv_launch(codes, lut, x, y, y_dtype, B, N, K, s);
-  if (K % 64 || N % 16)
-    return fail(QL_ERR_UNSUPPORTED, "benq_linear: batch %d > 16 needs K %% 64 == 0 and N %% 16 == 0", B);
+  if (K % 64 || N % 256)
+    return fail(QL_ERR_UNSUPPORTED, "benq_linear: batch %d > 16 needs K %% 64 == 0 and N %% 256 == 0", B);
   return ql::benq_gemm_launch(codes, lut, x, y, y_dtype, B, N, K, s);
 }
 

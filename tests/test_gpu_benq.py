@@ -115,3 +115,26 @@ def test_linear_argument_errors(ql):
     assert raw(codes.data_ptr(), lut.data_ptr(), x.data_ptr(), y.data_ptr(), 0, 1, 8, 62, s) == ql.QL_ERR_INVALID_ARG
     with pytest.raises(ValueError):
         ql.benq_linear(codes, lut, x, torch.empty(2, 8, device="cuda"))
+
+
+@pytest.mark.parametrize("M,N,K", [(17, 256, 64), (32, 512, 320), (300, 256, 1024), (256, 768, 5120), (513, 1024, 2048)])
+def test_gemm_shapes(ql, M, N, K):
+    w = synth.benq_weights(N, K, seed=M + N + K)
+    x = synth.activations(M, K, seed=M)
+    y = _linear(ql, w, x).cpu().numpy()
+    assert max_rel(y, ob.linear(w.codes, w.lut, x, K)) <= BENQ_TOL
+    yb = _linear(ql, w, x, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(yb, f32_to_bf16_rne(y))
+
+
+@pytest.mark.parametrize("N,K", [(17408, 5120), (5120, 17408)])
+def test_gemm_prefill_shapes_sampled_columns(ql, N, K):
+    # 2048-token prefill through the 27B-class gate/up and down projections, bf16 output
+    w = synth.benq_weights(N, K, seed=2000 + N // 1024)
+    x = synth.activations(2048, K, seed=2100)
+    y32 = _linear(ql, w, x).cpu().numpy()
+    yb = _linear(ql, w, x, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16)
+    cols = np.r_[np.random.default_rng(3).choice(N, 96, replace=False), 0, N - 1]
+    ref = ob.linear(w.codes, w.lut, x, K, rows=cols)
+    assert max_rel(y32[:, cols], ref) <= BENQ_TOL
+    assert np.array_equal(yb, f32_to_bf16_rne(y32))
