@@ -3,10 +3,11 @@
 // W is never written to global memory ("Qwen3.8-27B -- BenQ 6-bit", "What BenQ stores": the
 // gather lut[n][code] is fused into the GEMM).  One persistent CTA per SM walks 256 x 256 output
 // tiles; per 64-wide K block:
-//   * warp 0 (TMA producer) loads the X tile (256 x 64 bf16, 128-byte swizzle) and the packed
-//     code tile (256 rows x 48 bytes) with tensor copies, plus the 256 row tables of the tile
-//     (32 KB, once per tile) with a bulk copy;
-//   * warps 2..5 (decoders) expand the code tile through the row tables into the bf16 W tile,
+//   * warp 0 loads the X tile (256 x 64 bf16, 128-byte swizzle) with tensor copies into a
+//     3-stage ring released by the MMA; warp 2 loads the packed code tile (256 rows x 48 bytes)
+//     into a 2-stage ring released as soon as the decoders have read it, plus the 256 row
+//     tables of the tile (32 KB, once per tile) with a bulk copy;
+//   * warps 3..18 (decoders) expand the code tile through the row tables into the bf16 W tile,
 //     written directly in the K-major 128-byte-swizzled layout the tensor core reads, then fence
 //     the writes for the async proxy;
 //   * warp 1, one thread, issues tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32 accumulate in
@@ -27,31 +28,33 @@
 namespace {
 
 constexpr int BM = 256, BN = 256, BK = 64;        // CTA tile; BK = one 128-byte swizzle row of bf16
-constexpr int STAGES = 2;
+constexpr int SA = 3, SB = 2, SC = 2;             // stages: activations, decoded W, codes
 constexpr int A_BYTES = BM * BK * 2;              // 32 KB
 constexpr int B_BYTES = BN * BK * 2;              // 32 KB
 constexpr int C_ROW = BK * 6 / 8;                 // 48 code bytes per row per K block
 constexpr int C_BYTES = BN * C_ROW;               // 12 KB
 constexpr int LUT_BYTES = BN * 128;               // 32 KB
 constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_LUT = OFF_C + STAGES * C_BYTES + 128;   // 128 bytes of slack after the code tiles
+constexpr int OFF_B = OFF_A + SA * A_BYTES;
+constexpr int OFF_C = OFF_B + SB * B_BYTES;
+constexpr int OFF_LUT = OFF_C + SC * C_BYTES + 128;   // 128 bytes of slack after the code tiles
 constexpr int OFF_BAR = OFF_LUT + LUT_BYTES;
-constexpr int NBAR = 3 * STAGES + 4;
+constexpr int NBAR = 2 * (SA + SB + SC) + 4;
 constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;          // + alignment slack
-constexpr int THREADS = 6 * 32;
+constexpr int NDEC = 16;                                 // decoder / epilogue warps (multiple of 8)
+constexpr int THREADS = (3 + NDEC) * 32;   // A producer, MMA issuer, code producer, decoders
 constexpr long long WAIT_BUDGET = 4000000000LL;           // clock cycles (~2 s)
 constexpr uint32_t IDESC = sm100::idesc_bf16_f32(128, BN);
 
 __device__ int g_gemm_timeout = 0;
 
 struct Bars {
-  uint32_t full_ac, full_b, empty, lut_full, lut_empty, acc_full, acc_empty;
+  uint32_t full_a, empty_a, full_b, empty_b, full_c, empty_c, lut_full, lut_empty, acc_full, acc_empty;
   __device__ Bars(uint32_t base)
-      : full_ac(base), full_b(base + 8 * STAGES), empty(base + 16 * STAGES), lut_full(base + 24 * STAGES),
-        lut_empty(base + 24 * STAGES + 8), acc_full(base + 24 * STAGES + 16), acc_empty(base + 24 * STAGES + 24) {}
+      : full_a(base), empty_a(full_a + 8 * SA), full_b(empty_a + 8 * SA), empty_b(full_b + 8 * SB),
+        full_c(empty_b + 8 * SB), empty_c(full_c + 8 * SC), lut_full(empty_c + 8 * SC), lut_empty(lut_full + 8),
+        acc_full(lut_empty + 8), acc_empty(acc_full + 8) {}
 };
 
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
@@ -81,15 +84,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   bool ok = true;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      sm100::mbar_init(bar.full_ac + 8 * s, 1);
-      sm100::mbar_init(bar.full_b + 8 * s, 4);
-      sm100::mbar_init(bar.empty + 8 * s, 1);
+    for (int s = 0; s < SA; ++s) {
+      sm100::mbar_init(bar.full_a + 8 * s, 1);
+      sm100::mbar_init(bar.empty_a + 8 * s, 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      sm100::mbar_init(bar.full_b + 8 * s, NDEC);
+      sm100::mbar_init(bar.empty_b + 8 * s, 1);
+    }
+    for (int s = 0; s < SC; ++s) {
+      sm100::mbar_init(bar.full_c + 8 * s, 1);
+      sm100::mbar_init(bar.empty_c + 8 * s, NDEC);
     }
     sm100::mbar_init(bar.lut_full, 1);
-    sm100::mbar_init(bar.lut_empty, 4);
+    sm100::mbar_init(bar.lut_empty, NDEC);
     sm100::mbar_init(bar.acc_full, 1);
-    sm100::mbar_init(bar.acc_empty, 4);
+    sm100::mbar_init(bar.acc_empty, NDEC);
     sm100::fence_barrier_init();
     sm100::prefetch_tensormap(&map_x);
     sm100::prefetch_tensormap(&map_codes);
@@ -104,23 +114,39 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem_raw + (tmem_slot - raw));
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ activation producer (TMA)
+    if (lane == 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const int m0 = (t % mt) * BM;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % SA;
+          if (it >= SA && !sm100::mbar_wait(bar.empty_a + 8 * s, ((it / SA) & 1) ^ 1, WAIT_BUDGET)) {
+            ok = false;
+            break;
+          }
+          sm100::mbar_arrive_expect_tx(bar.full_a + 8 * s, A_BYTES);
+          sm100::tma_load_2d(sbase + OFF_A + s * A_BYTES, &map_x, kb * BK, m0, bar.full_a + 8 * s);
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ code and table producer (TMA)
     if (lane == 0) {
       int it = 0, tl = 0;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tl) {
-        const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
+        const int n0 = (t / mt) * BN;
         if (tl > 0 && !sm100::mbar_wait(bar.lut_empty, (tl - 1) & 1, WAIT_BUDGET)) { ok = false; break; }
         sm100::mbar_arrive_expect_tx(bar.lut_full, LUT_BYTES);
         sm100::bulk_g2s(sbase + OFF_LUT, lut + (size_t)n0 * 64, LUT_BYTES, bar.lut_full);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (it >= STAGES && !sm100::mbar_wait(bar.empty + 8 * s, ((it / STAGES) & 1) ^ 1, WAIT_BUDGET)) {
+          const int s = it % SC;
+          if (it >= SC && !sm100::mbar_wait(bar.empty_c + 8 * s, ((it / SC) & 1) ^ 1, WAIT_BUDGET)) {
             ok = false;
             break;
           }
-          sm100::mbar_arrive_expect_tx(bar.full_ac + 8 * s, A_BYTES + C_BYTES);
-          sm100::tma_load_2d(sbase + OFF_A + s * A_BYTES, &map_x, kb * BK, m0, bar.full_ac + 8 * s);
-          sm100::tma_load_2d(sbase + OFF_C + s * C_BYTES, &map_codes, kb * C_ROW, n0, bar.full_ac + 8 * s);
+          sm100::mbar_arrive_expect_tx(bar.full_c + 8 * s, C_BYTES);
+          sm100::tma_load_2d(sbase + OFF_C + s * C_BYTES, &map_codes, kb * C_ROW, n0, bar.full_c + 8 * s);
         }
       }
     }
@@ -132,15 +158,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (tl > 0 && !sm100::mbar_wait(bar.acc_empty, (tl - 1) & 1, WAIT_BUDGET)) { ok = false; break; }
         sm100::tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!sm100::mbar_wait(bar.full_ac + 8 * s, ph, WAIT_BUDGET) ||
-              !sm100::mbar_wait(bar.full_b + 8 * s, ph, WAIT_BUDGET)) {
+          const int sa = it % SA, sb = it % SB;
+          if (!sm100::mbar_wait(bar.full_a + 8 * sa, (it / SA) & 1, WAIT_BUDGET) ||
+              !sm100::mbar_wait(bar.full_b + 8 * sb, (it / SB) & 1, WAIT_BUDGET)) {
             ok = false;
             break;
           }
           sm100::tc_fence_after();
-          const uint32_t a = sbase + OFF_A + s * A_BYTES, b = sbase + OFF_B + s * B_BYTES;
+          const uint32_t a = sbase + OFF_A + sa * A_BYTES, b = sbase + OFF_B + sb * B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t bdesc = sm100::sw128_kmajor_desc(b + kk * 32);
@@ -150,7 +175,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               sm100::mma_bf16(tmem + h * BN, adesc, bdesc, IDESC, (kb | kk) ? 1u : 0u);
             }
           }
-          sm100::mma_commit(bar.empty + 8 * s);
+          sm100::mma_commit(bar.empty_a + 8 * sa);
+          sm100::mma_commit(bar.empty_b + 8 * sb);
         }
         if (!ok) break;
         sm100::mma_commit(bar.acc_full);
@@ -158,38 +184,46 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ decoders, then epilogue
-    const int dw = warp - 2;            // 0..3: decoder index
+    const int dw = warp - 3;            // decoder index 0 .. NDEC-1
     const int q = warp & 3;             // tensor-memory lane quarter this warp may read
+    const int ch = dw >> 2;             // which NDEC/4-th of the 256 accumulator columns it drains
     int it = 0, tl = 0;
     // lane l expands codes 2l, 2l+1 of a row's 64-code block: bits [12l, 12l+12) of its 48 bytes
     const int wq = (12 * lane) >> 5, wsh = (12 * lane) & 31;
     const int chunk = lane >> 2, inner = (lane & 3) * 4;
+    // swizzled position of codes 2*lane, 2*lane+1 within row r = dw (mod 8) of a K block
+    const uint32_t dst_lane = (dw >> 3) * 1024 + (dw & 7) * 128 + ((chunk ^ (dw & 7)) << 4) + inner;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tl) {
       const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
       if (!sm100::mbar_wait(bar.lut_full, tl & 1, WAIT_BUDGET)) { ok = false; break; }
-      const uint32_t lutb = sbase + OFF_LUT;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        if ((it >= STAGES && !sm100::mbar_wait(bar.empty + 8 * s, ph ^ 1, WAIT_BUDGET)) ||
-            !sm100::mbar_wait(bar.full_ac + 8 * s, ph, WAIT_BUDGET)) {
+        const int sb = it % SB, sc = it % SC;
+        if ((it >= SB && !sm100::mbar_wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, WAIT_BUDGET)) ||
+            !sm100::mbar_wait(bar.full_c + 8 * sc, (it / SC) & 1, WAIT_BUDGET)) {
           ok = false;
           break;
         }
-        const uint32_t cb = sbase + OFF_C + s * C_BYTES, bb = sbase + OFF_B + s * B_BYTES;
-        for (int r = dw; r < BN; r += 4) {
-          const uint32_t w0 = lds32(cb + r * C_ROW + 4 * wq);
-          const uint32_t w1 = lds32(cb + r * C_ROW + 4 * wq + 4);   // may read the next row: unused bits
+        // rows r = dw + NDEC*i: r & 7 == dw & 7 is fixed per warp, so every address below is
+        // a per-warp base plus a compile-time multiple of the row step
+        const uint32_t cb = sbase + OFF_C + sc * C_BYTES + dw * C_ROW + 4 * wq;
+        const uint32_t bb = sbase + OFF_B + sb * B_BYTES + dst_lane;
+        const uint32_t tb = sbase + OFF_LUT + dw * 128;
+#pragma unroll 4
+        for (int i = 0; i < BN / NDEC; ++i) {
+          const uint32_t w0 = lds32(cb + i * NDEC * C_ROW);
+          const uint32_t w1 = lds32(cb + i * NDEC * C_ROW + 4);   // may read the next row: unused bits
           const uint32_t v = __funnelshift_r(w0, w1, wsh);
-          const uint32_t tbl = lutb + r * 128;
+          const uint32_t tbl = tb + i * NDEC * 128;
           const uint32_t e0 = lds_u16(((v << 1) & 0x7Eu) | tbl);
           const uint32_t e1 = lds_u16(((v >> 5) & 0x7Eu) | tbl);
-          const uint32_t dst = bb + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4) + inner;
-          sts32(dst, __byte_perm(e0, e1, 0x5410));
+          sts32(bb + i * (NDEC / 8) * 1024, __byte_perm(e0, e1, 0x5410));
         }
         sm100::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) sm100::mbar_arrive(bar.full_b + 8 * s);
+        if (lane == 0) {
+          sm100::mbar_arrive(bar.full_b + 8 * sb);
+          sm100::mbar_arrive(bar.empty_c + 8 * sc);
+        }
       }
       if (!ok) break;
       __syncwarp();
@@ -201,7 +235,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int h = 0; h < 2; ++h) {
         const int row = m0 + h * 128 + 32 * q + lane;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = ch * (BN / 32) / (NDEC / 4); c < (ch + 1) * (BN / 32) / (NDEC / 4); ++c) {
           uint32_t v[32];
           sm100::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + h * BN + c * 32, v);
           sm100::tmem_wait_ld();
