@@ -136,6 +136,29 @@ QL_API ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r,
                       size_t ws_bytes, ql_stream_t stream);
 
 /*
+ * mdbf_linear_noalloc -- mdbf_linear for callers that cannot allocate device memory.
+ *   The paper has no counterpart: this is a deployment convenience.  Some callers can't call
+ *   cudaMalloc (or must not: allocator-internal code, real-time threads that may not block in
+ *   the driver, hosts with a memory budget fixed at start-up), so this entry point needs no
+ *   workspace.  Its scratch is a fixed 4 MiB array compiled into the library
+ *   (mdbf_noalloc_scratch_bytes()); every GPU that loads the library holds it until the process
+ *   exits, and sizes whose mdbf_workspace_bytes() exceed it return QL_ERR_UNSUPPORTED.  The
+ *   library allocates nothing for this call.
+ *   Arguments, layouts and results are those of mdbf_linear without workspace/ws_bytes.
+ *   All calls share the one array: calls that may overlap on the GPU (two streams, or two host
+ *   threads with no ordering between their streams) race and must be serialised by the caller.
+ *   Every scratch byte that is read is first written by the same call, so nothing needs
+ *   clearing between calls.  The first call on each device looks up the array's device address
+ *   with that device current; make that first call before any stream capture.
+ */
+QL_API ql_status mdbf_linear_noalloc(const mdbf_path *paths, int P, int n, int m, int r, int l,
+                                     const uint16_t *x, void *y, ql_out_dtype y_dtype, int B,
+                                     ql_stream_t stream);
+
+/* Size in bytes of the static scratch array mdbf_linear_noalloc uses (its size limit).  Host only. */
+QL_API size_t mdbf_noalloc_scratch_bytes(void);
+
+/*
  * mdbf_dequant_debug -- materialises W (and optionally the factors) in fp32:
  *   F[p][a][k] = s_A[a][k] * fp32(sum_i A_amp[a][i] Q_U[k][i])   (i ascending),
  *   G[p][k][j] = s_B[k][j] * fp32(sum_i Q_V[k][i] B_amp[j][i])   (i ascending),

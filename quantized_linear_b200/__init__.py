@@ -39,6 +39,8 @@ _SIGNATURES = {
     "mdbf_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "mdbf_linear": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _sz, _vp]),
     "mdbf_dequant_debug": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "mdbf_linear_noalloc": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp]),
+    "mdbf_noalloc_scratch_bytes": (_sz, []),
     "mdbf_effective_bits": (_d, [_i, _i, _i, _i, _i, _i]),
     "mdbf_select_rank": (_i, [_i, _i, _i, _i, _i, _d, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "ql_last_error": (ctypes.c_char_p, []),
@@ -65,7 +67,8 @@ def _c(name):
     return getattr(lib(), name)
 
 EXPORTS = ["benq_linear", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
-           "mdbf_dequant_debug", "mdbf_effective_bits", "mdbf_select_rank", "ql_last_error", "ql_check"]
+           "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
+           "mdbf_select_rank", "ql_last_error", "ql_check"]
 
 
 class QLinearError(RuntimeError):
@@ -170,6 +173,25 @@ def mdbf_linear(paths, n, m, r, l, x, y, workspace, stream=None):
     _check(_c("mdbf_linear")(arr, len(arr), n, m, r, l, _ptr(x), _ptr(y), _ydt(y), B, _ptr(workspace),
                         workspace.numel() * workspace.element_size(), _stream(stream)))
     return y
+
+
+def mdbf_linear_noalloc(paths, n, m, r, l, x, y, stream=None):
+    """mdbf_linear without a caller workspace, for callers that cannot allocate device memory.
+
+    The scratch is a fixed array inside the library (mdbf_noalloc_scratch_bytes() bytes, shared by
+    all calls: calls that overlap on the GPU race).  Make the first call on a device before any
+    stream capture."""
+    _want(x, torch.bfloat16, "x")
+    B = x.shape[0]
+    if x.shape[1] != m or tuple(y.shape) != (B, n) or not y.is_contiguous():
+        raise ValueError("x must be [B, m] and y [B, n]")
+    arr = paths if isinstance(paths, ctypes.Array) else mdbf_paths_c(paths)
+    _check(_c("mdbf_linear_noalloc")(arr, len(arr), n, m, r, l, _ptr(x), _ptr(y), _ydt(y), B, _stream(stream)))
+    return y
+
+
+def mdbf_noalloc_scratch_bytes() -> int:
+    return int(_c("mdbf_noalloc_scratch_bytes")())
 
 
 def mdbf_dequant_debug(paths, n, m, r, l, W, F=None, G=None, stream=None):

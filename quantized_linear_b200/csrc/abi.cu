@@ -118,6 +118,32 @@ ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r, int l,
                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
+ql_status mdbf_linear_noalloc(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x, void *y,
+                              ql_out_dtype y_dtype, int B, ql_stream_t stream) {
+  g_msg[0] = 0;
+  ql_status st = check_paths("mdbf_linear_noalloc", paths, P, n, m, r, l);
+  if (st != QL_OK) return st;
+  if (!x || !y) return fail(QL_ERR_INVALID_ARG, "mdbf_linear_noalloc: null x or y");
+  if (B <= 0) return fail(QL_ERR_INVALID_ARG, "mdbf_linear_noalloc: B must be positive");
+  if (y_dtype != QL_OUT_F32 && y_dtype != QL_OUT_BF16)
+    return fail(QL_ERR_INVALID_ARG, "mdbf_linear_noalloc: bad y_dtype");
+  if (!aligned(x, 2) || !aligned(y, 4)) return fail(QL_ERR_ALIGNMENT, "mdbf_linear_noalloc: x 2- and y 4-byte alignment required");
+  const size_t need = ql::mdbf_workspace_size(P, n, m, r, l, B);
+  const size_t limit = ql::mdbf_noalloc_scratch_limit();
+  if (need > limit)
+    return fail(QL_ERR_UNSUPPORTED,
+                "mdbf_linear_noalloc: these sizes need %zu bytes of scratch, more than the %zu-byte static array; "
+                "use mdbf_linear with a caller workspace",
+                need, limit);
+  void *scratch = nullptr;
+  st = ql::mdbf_noalloc_scratch(&scratch);
+  if (st != QL_OK) return st;
+  return ql::mdbf_linear_launch(paths, P, n, m, r, l, x, y, y_dtype, B, scratch,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t mdbf_noalloc_scratch_bytes(void) { return ql::mdbf_noalloc_scratch_limit(); }
+
 ql_status mdbf_dequant_debug(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W, float *F, float *G,
                              ql_stream_t stream) {
   g_msg[0] = 0;

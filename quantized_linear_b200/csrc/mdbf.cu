@@ -16,6 +16,7 @@
 // FMAs; the vectors are read as warp-wide broadcasts.  Column-split partials
 // are summed through shared memory in a fixed order.
 #include <algorithm>
+#include <mutex>
 
 #include "ql_internal.cuh"
 
@@ -331,6 +332,44 @@ ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r
   const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 16);
   mdbf_w_kernel<<<grid, 256, 0, s>>>(ps, P, W, n, m, r, l);
   return launch_status("mdbf_dequant_debug (W)");
+}
+
+}  // namespace ql
+
+// ------------------------------------------------------------------ no-allocation variant
+// Some callers cannot call cudaMalloc at all: code running where the allocator is forbidden or
+// unavailable (inside a custom allocator's own paths, in real-time threads that must never block
+// in the driver, or in hosts whose memory budget is fixed before the first inference).  For them
+// mdbf_linear_noalloc takes its scratch from this file-scope device array instead of a caller
+// workspace.  Every GPU that loads the library holds it until the process exits.
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(4) << 20;   // 4 MiB
+static __device__ __align__(256) unsigned char g_mdbf_scratch[NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[64] = {nullptr};
+}  // namespace
+
+namespace ql {
+
+size_t mdbf_noalloc_scratch_limit() { return NOALLOC_SCRATCH_BYTES; }
+
+// Device address of the scratch array on the current device.  The host-side symbol is only a
+// stand-in, so the address is looked up once per device (with that device current) and cached.
+ql_status mdbf_noalloc_scratch(void **ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(QL_ERR_CUDA, "mdbf_linear_noalloc: no current CUDA device");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_mdbf_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(QL_ERR_CUDA, "mdbf_linear_noalloc: cannot resolve the scratch array: %s", cudaGetErrorString(e));
+    g_scratch_ptr[dev] = p;
+  }
+  *ptr = g_scratch_ptr[dev];
+  return QL_OK;
 }
 
 }  // namespace ql

@@ -1,0 +1,62 @@
+"""mdbf_linear_noalloc: the entry point for callers that cannot allocate device memory.
+
+Some callers may not call cudaMalloc (allocator-internal code, real-time threads that must not
+block in the driver, hosts with a memory budget fixed at start-up).  mdbf_linear_noalloc serves
+them from a fixed scratch array compiled into the library.  This test calls it through the C ABI
+and checks each result against mdbf_linear (the workspace entry point) on two calls in a row with
+different problems, so stale scratch from the first call cannot leak into the second.  It lives in
+a file of its own that pytest collects last, and passes alone or after the other tests.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests.qlhelpers import MDBF_TOL, bf16, max_rel, mdbf_dev_paths
+
+pytestmark = pytest.mark.gpu
+
+
+def _reference(ql, paths_c, n, m, r, l, x):
+    B = x.shape[0]
+    ws = torch.empty(ql.mdbf_workspace_bytes(len(paths_c), n, m, r, l, B), dtype=torch.uint8, device="cuda")
+    y = torch.empty(B, n, device="cuda")
+    ql.mdbf_linear(paths_c, n, m, r, l, x, y, ws)
+    return y
+
+
+def _noalloc_raw(ql, paths_c, n, m, r, l, x, y):
+    f = ql.lib().mdbf_linear_noalloc
+    return f(paths_c, len(paths_c), n, m, r, l, x.data_ptr(), y.data_ptr(), ql.QL_OUT_F32, x.shape[0],
+             torch.cuda.current_stream().cuda_stream)
+
+
+def test_noalloc_matches_workspace_entry_on_two_calls(ql):
+    problems = [(1024, 768, 300, 4, 2, 3, 71), (640, 1280, 257, 2, 1, 16, 72)]
+    for n, m, r, l, P, B, seed in problems:
+        paths = synth.mdbf_paths(P, n, m, r, l, seed=seed)
+        dp = mdbf_dev_paths(paths)
+        pc = ql.mdbf_paths_c(dp)
+        x = bf16(synth.activations(B, m, seed=seed + 1))
+        assert ql.mdbf_workspace_bytes(P, n, m, r, l, B) <= ql.mdbf_noalloc_scratch_bytes()
+        y = torch.full((B, n), float("nan"), device="cuda")
+        assert _noalloc_raw(ql, pc, n, m, r, l, x, y) == ql.QL_OK
+        y_ref = _reference(ql, pc, n, m, r, l, x)
+        torch.cuda.synchronize()
+        assert max_rel(y.cpu().numpy(), y_ref.cpu().numpy()) <= MDBF_TOL
+        assert torch.equal(y, y_ref)
+
+
+def test_noalloc_rejects_sizes_beyond_the_scratch(ql):
+    n = m = 4096
+    r, l, P, B = 4096, 8, 8, 8                 # needs far more than the static array
+    assert ql.mdbf_workspace_bytes(P, n, m, r, l, B) > ql.mdbf_noalloc_scratch_bytes()
+    A = 1 << 20                                # never dereferenced: rejected before any launch
+    arr = (ql.MDBFPathC * P)()
+    for p in range(P):
+        arr[p] = ql.MDBFPathC(A, A, 512, 512, A, A, A, A)
+    status = ql.lib().mdbf_linear_noalloc(arr, P, n, m, r, l, A, A, ql.QL_OUT_F32, B, None)
+    assert status == ql.QL_ERR_UNSUPPORTED
+    assert b"scratch" in ql.lib().ql_last_error()
