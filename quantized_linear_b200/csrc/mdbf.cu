@@ -6,15 +6,16 @@
 //   (G x)_k = sum_i Q_V[k,i] * sum_j S_B[k,j] * (B_amp[j,i] x_j)
 //   (F t)_a = sum_i A_amp[a,i] * sum_k S_A[a,k] * (Q_U[k,i] t_k)
 // so each path is two products of a packed +-1 matrix with l*B dense vectors:
-//   prologue  z[p][j][b*l+i] = B_amp[j,i] * x[b,j]                (exact in fp32)
+//   prologue  z[p][j][b*l+i] = B_amp[j,i] * x[b,j]                (exact in fp32, packed as
+//             bf16 high + low MMA fragments)
 //   G stage   u = S_B z;   t[k][b] = sum_i Q_V[k,i] u[k][b*l+i];
 //             w[p][k][b*l+i] = Q_U[k,i] * t[k][b]                  (epilogue, fused)
 //   F stage   v = S_A w;   y[b][a] = sum_p sum_i A_amp[a,i] v[a][b*l+i]   (epilogue, fused;
 //             the path sum is taken inside one launch, in p order)
-// Sign products: lane = matrix row, warps split the columns; each sign bit
-// becomes +-1.0f (two integer ops) and multiplies the l*B vector values with
-// FMAs; the vectors are read as warp-wide broadcasts.  Column-split partials
-// are summed through shared memory in a fixed order.
+// The sign products run on the warp MMA (see "Sign products on the warp MMA"
+// below); column-split partials are summed through shared memory in a fixed
+// order, so results are deterministic.  Launches per call: pack z, G stage,
+// pack w, F stage.
 #include <algorithm>
 #include <mutex>
 
@@ -33,165 +34,234 @@ struct Paths {
 };
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
-__host__ __device__ inline int vpad(int vb) { return (vb + 3) & ~3; }
 
-__device__ __forceinline__ uint32_t ldg_u32(const uint8_t *p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ float4 ldg_f4(const float *p) {
-  float4 v;
-  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
-  return v;
+// ------------------------------------------------------------------------------------------
+// Sign products on the warp MMA.
+//
+// OUT[rows][v] = sum_c s[row][c] * VEC[c][v] is an (rows x cols) x (cols x V) product with a +-1
+// left operand.  Each sign bit becomes a bf16 +-1 (exact) straight in the A fragment of
+// mma.m16n8k16 (bf16 in, fp32 accumulate); the dense right operand VEC (fp32) is split into a
+// bf16 high part and a bf16 low part (relative error ~2^-16) and laid out once, in a prologue,
+// as ready-made B fragments.  The K ordering inside one 32-column sign word is permuted so that
+// the two bits of every A register sit 16 bit positions apart: one shift and one masked XOR
+// build a register, i.e. one integer op per sign bit.  Logical K pairs of MMA h (h = 0, 1) map
+// to physical columns (c, c + 16) with c = 8h + q (pair 2q, 2q+1) and c = 8h + 4 + q (pair
+// 2q+8, 2q+9), q = lane % 4; the B fragments are packed with the same map.
+// B fragment columns: n < V hold the high parts of vector n, V <= n < 2V the low parts, the
+// rest zero; NB = ceil(2V / 8) MMAs cover them.  Columns past `cols` pack as zero, so the
+// padding bits of the last sign word contribute nothing.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// z[p][j][v] = B_amp[j][i] * x[b][j] for v = b*l + i (zero padding up to a multiple of 4).
-__global__ void mdbf_prologue_kernel(Paths ps, const uint16_t *__restrict__ x, float *__restrict__ Z, int m, int l,
-                                     int B) {
+// bf16 pair {+-1 from bit (15 - s) of w, +-1 from bit (31 - s)}: bit 1 -> +1.0, bit 0 -> -1.0
+__device__ __forceinline__ uint32_t sign_pair(uint32_t w, int s) {
+  return ((w << s) & 0x80008000u) ^ 0xBF80BF80u;
+}
+
+__device__ __forceinline__ uint32_t bf16_rn_bits(float f) { return qld::f32_to_bf16_rn(f); }
+
+// value of B-fragment column n at physical column c: high / low bf16 part of VEC[c][v]
+template <typename Get>
+__device__ __forceinline__ uint32_t frag_value(Get get, int c, int n, int cols, int V) {
+  if (c >= cols || n >= 2 * V) return 0u;
+  const float v = get(c, n < V ? n : n - V);
+  const uint32_t hi = bf16_rn_bits(v);
+  if (n < V) return hi;
+  return bf16_rn_bits(v - __uint_as_float(hi << 16));
+}
+
+// packed B fragments: VB[qw][nb][h][lane] as uint2, for one path
+template <typename Get>
+__device__ __forceinline__ uint2 pack_fragment(Get get, int qw, int nb, int h, int lane, int cols, int V) {
+  const int g = lane >> 2, q = lane & 3, n = 8 * nb + g;
+  const int ca = 32 * qw + 8 * h + q, cb = ca + 4;
+  uint2 r;
+  r.x = frag_value(get, ca, n, cols, V) | (frag_value(get, ca + 16, n, cols, V) << 16);
+  r.y = frag_value(get, cb, n, cols, V) | (frag_value(get, cb + 16, n, cols, V) << 16);
+  return r;
+}
+
+// G-stage B fragments from z[j][b*l+i] = B_amp[j][i] * x[b][j] (exact in fp32)
+__global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uint2 *__restrict__ out, int m, int l,
+                                   int B, int NB) {
   const int p = blockIdx.y;
-  const int vb = l * B, vp = vpad(vb);
-  const int64_t total = (int64_t)m * vp;
-  float *zp = Z + (int64_t)p * total;
+  const int QW = (m + 31) / 32, V = l * B;
+  const int64_t total = (int64_t)QW * NB * 2 * 32;
+  const uint16_t *bm = ps.Bm[p];
+  auto get = [&](int c, int v) {
+    const int b = v / l, i = v - b * l;
+    return qld::f16_to_f32(bm[(int64_t)c * l + i]) * qld::bf16_to_f32(x[(int64_t)b * m + c]);
+  };
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t j = e / vp;
-    const int v = int(e - j * vp);
-    float z = 0.f;
-    if (v < vb) {
-      const int b = v / l, i = v - b * l;
-      z = qld::f16_to_f32(ps.Bm[p][j * l + i]) * qld::bf16_to_f32(x[(int64_t)b * m + j]);
-    }
-    zp[e] = z;
+    const int lane = int(e & 31);
+    const int64_t f = e >> 5;
+    const int h = int(f & 1);
+    const int64_t f2 = f >> 1;
+    const int nb = int(f2 % NB);
+    const int qw = int(f2 / NB);
+    out[(int64_t)p * total + e] = pack_fragment(get, qw, nb, h, lane, m, V);
   }
 }
 
-// acc[v] += sum over this warp's columns of s[row][col] * vec[col][v]
-template <int VMAX>
-__device__ __forceinline__ void sign_dot(const uint8_t *row_bits, bool row_ok, const float *__restrict__ vec,
-                                         int vp, int cols, int q0, int q1, float (&acc)[VMAX]) {
-  for (int q = q0; q < q1; ++q) {
-    const uint32_t bits = row_ok ? ldg_u32(row_bits + 4 * q) : 0u;
-    const int jmax = min(32, cols - 32 * q);
-    const float *vq = vec + (int64_t)32 * q * vp;
-#pragma unroll 4
-    for (int jj = 0; jj < 32; ++jj) {
-      if (jj >= jmax) break;
-      const float s = __uint_as_float(0xBF800000u ^ ((bits << (31 - jj)) & 0x80000000u));
-      const float *vj = vq + (int64_t)jj * vp;
-#pragma unroll
-      for (int v4 = 0; v4 < VMAX / 4; ++v4) {
-        if (4 * v4 < vp) {
-          const float4 z = ldg_f4(vj + 4 * v4);
-          acc[4 * v4 + 0] = fmaf(s, z.x, acc[4 * v4 + 0]);
-          acc[4 * v4 + 1] = fmaf(s, z.y, acc[4 * v4 + 1]);
-          acc[4 * v4 + 2] = fmaf(s, z.z, acc[4 * v4 + 2]);
-          acc[4 * v4 + 3] = fmaf(s, z.w, acc[4 * v4 + 3]);
-        }
-      }
-    }
-  }
-}
-
-// Sums the per-warp partials (part[KS][VMAX][32]) into warp 0's acc, fixed order.
-template <int VMAX>
-__device__ __forceinline__ void reduce_warps(float *part, int vp, float (&acc)[VMAX]) {
-  const int warp = threadIdx.y, lane = threadIdx.x, KS = blockDim.y;
-#pragma unroll
-  for (int v = 0; v < VMAX; ++v)
-    if (v < vp) part[(warp * VMAX + v) * 32 + lane] = acc[v];
-  __syncthreads();
-  if (warp == 0) {
-#pragma unroll
-    for (int v = 0; v < VMAX; ++v) {
-      if (v < vp) {
-        float s = part[v * 32 + lane];
-        for (int w = 1; w < KS; ++w) s += part[(w * VMAX + v) * 32 + lane];
-        acc[v] = s;
-      }
-    }
-  }
-}
-
-template <int VMAX>
-__global__ void mdbf_g_stage_kernel(Paths ps, const float *__restrict__ Z, float *__restrict__ Wv, int m, int r,
-                                    int l, int B) {
-  extern __shared__ float part[];  // [KS][VMAX][32]
+// F-stage B fragments from w[p][k][v] (fp32, written by the G stage)
+__global__ void mdbf_pack_w_kernel(const float *__restrict__ w, uint2 *__restrict__ out, int r, int V, int NB) {
   const int p = blockIdx.y;
-  const int lane = threadIdx.x, warp = threadIdx.y, KS = blockDim.y;
-  const int k = blockIdx.x * 32 + lane;
-  const bool ok = k < r;
-  const int vb = l * B, vp = vpad(vb);
-  const int nq = (m + 31) / 32;
-  const int q0 = (int)((int64_t)nq * warp / KS), q1 = (int)((int64_t)nq * (warp + 1) / KS);
-  float acc[VMAX];
+  const int QW = (r + 31) / 32;
+  const int64_t total = (int64_t)QW * NB * 2 * 32;
+  const float *wp = w + (int64_t)p * r * V;
+  auto get = [&](int c, int v) { return wp[(int64_t)c * V + v]; };
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int lane = int(e & 31);
+    const int64_t f = e >> 5;
+    const int h = int(f & 1);
+    const int64_t f2 = f >> 1;
+    const int nb = int(f2 % NB);
+    const int qw = int(f2 / NB);
+    out[(int64_t)p * total + e] = pack_fragment(get, qw, nb, h, lane, r, V);
+  }
+}
+
+constexpr int SP_WARPS = 8;
+
+// Accumulates one warp's share of words into acc for RT row tiles of 16 rows starting at row0.
+template <int NB, int RT>
+__device__ __forceinline__ void sign_mma_rows(const uint8_t *__restrict__ S, size_t ld, int rows, int row0,
+                                              const uint2 *__restrict__ vb, int w0, int w1,
+                                              float (&acc)[RT][NB][4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const uint8_t *rp[RT][2];
+  bool ok[RT][2];
 #pragma unroll
-  for (int v = 0; v < VMAX; ++v) acc[v] = 0.f;
-  sign_dot<VMAX>(ps.SB[p] + (int64_t)(ok ? k : 0) * ps.ldSB[p], ok, Z + (int64_t)p * m * vp, vp, m, q0, q1, acc);
-  reduce_warps<VMAX>(part, vp, acc);
-  if (warp == 0 && ok) {
-    float *out = Wv + ((int64_t)p * r + k) * vp;
-    const uint16_t *qv = ps.QV[p] + (int64_t)k * l;
-    const uint16_t *qu = ps.QU[p] + (int64_t)k * l;
+  for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-    for (int v = 0; v < VMAX; ++v)
-      if (v >= vb && v < vp) out[v] = 0.f;
-    for (int b = 0; b < B; ++b) {
-      float t = 0.f;
+    for (int hh = 0; hh < 2; ++hh) {
+      const int row = row0 + 16 * rt + g + 8 * hh;
+      ok[rt][hh] = row < rows;
+      rp[rt][hh] = S + (size_t)(ok[rt][hh] ? row : 0) * ld;
+    }
+  for (int qw = w0; qw < w1; ++qw) {
+    uint2 bf[NB][2];
 #pragma unroll
-      for (int v = 0; v < VMAX; ++v)
-        if (v >= b * l && v < (b + 1) * l) t = fmaf(qld::f16_to_f32(qv[v - b * l]), acc[v], t);
+    for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-      for (int v = 0; v < VMAX; ++v)
-        if (v >= b * l && v < (b + 1) * l) out[v] = qld::f16_to_f32(qu[v - b * l]) * t;
+      for (int h = 0; h < 2; ++h) bf[nb][h] = __ldg(vb + (((size_t)qw * NB + nb) * 2 + h) * 32 + lane);
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt) {
+      const uint32_t s0 = ok[rt][0] ? __ldg(reinterpret_cast<const uint32_t *>(rp[rt][0]) + qw) : 0u;
+      const uint32_t s1 = ok[rt][1] ? __ldg(reinterpret_cast<const uint32_t *>(rp[rt][1]) + qw) : 0u;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int sa = 15 - 8 * h - q, sb = 11 - 8 * h - q;
+        const uint32_t a0 = sign_pair(s0, sa), a1 = sign_pair(s1, sa);
+        const uint32_t a2 = sign_pair(s0, sb), a3 = sign_pair(s1, sb);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) mma16816(acc[rt][nb], a0, a1, a2, a3, bf[nb][h].x, bf[nb][h].y);
+      }
     }
   }
 }
 
-template <int VMAX>
-__global__ void mdbf_f_stage_kernel(Paths ps, int P, const float *__restrict__ Wv, void *__restrict__ y, int ydt,
-                                    int n, int r, int l, int B) {
-  extern __shared__ float part[];  // [KS][VMAX][32]
-  const int lane = threadIdx.x, warp = threadIdx.y, KS = blockDim.y;
-  const int a = blockIdx.x * 32 + lane;
-  const bool ok = a < n;
-  const int vb = l * B, vp = vpad(vb);
-  const int nq = (r + 31) / 32;
-  const int q0 = (int)((int64_t)nq * warp / KS), q1 = (int)((int64_t)nq * (warp + 1) / KS);
-  float yacc[VMAX];
+// Sums the warps' fragments into D[rt][16][8 NB] (fp32, shared), fixed order.
+template <int NB, int RT>
+__device__ __forceinline__ void reduce_fragments(float *red, float *D, const float (&acc)[RT][NB][4]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int PER = RT * NB * 4 * 32;
 #pragma unroll
-  for (int v = 0; v < VMAX; ++v) yacc[v] = 0.f;
-  for (int p = 0; p < P; ++p) {
-    float acc[VMAX];
+  for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-    for (int v = 0; v < VMAX; ++v) acc[v] = 0.f;
-    sign_dot<VMAX>(ps.SA[p] + (int64_t)(ok ? a : 0) * ps.ldSA[p], ok, Wv + (int64_t)p * r * vp, vp, r, q0, q1, acc);
-    if (p > 0) __syncthreads();  // previous path's reduction has finished reading `part`
-    reduce_warps<VMAX>(part, vp, acc);
-    if (warp == 0 && ok) {
-      const uint16_t *am = ps.A[p] + (int64_t)a * l;
+    for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-      for (int v = 0; v < VMAX; ++v) {
-        if (v < vb) {
-          const int b = v / l;
-          const float av = qld::f16_to_f32(am[v - b * l]);
-          // yacc[b] += A[a][i] * v[b*l+i], i ascending within each path
-#pragma unroll
-          for (int bb = 0; bb < VMAX; ++bb)
-            if (bb == b) yacc[bb] = fmaf(av, acc[v], yacc[bb]);
-        }
-      }
-    }
+      for (int i = 0; i < 4; ++i) red[warp * PER + ((rt * NB + nb) * 4 + i) * 32 + lane] = acc[rt][nb][i];
+  __syncthreads();
+  for (int e = threadIdx.x; e < PER; e += blockDim.x) {
+    float s = red[e];
+    for (int w = 1; w < SP_WARPS; ++w) s += red[w * PER + e];
+    const int ln = e & 31, i = (e >> 5) & 3, nb = (e >> 7) % NB, rt = (e >> 7) / NB;
+    const int row = (ln >> 2) + 8 * (i >> 1), n = 8 * nb + 2 * (ln & 3) + (i & 1);
+    D[(rt * 16 + row) * (8 * NB) + n] = s;
   }
-  if (warp == 0 && ok) {
+  __syncthreads();
+}
+
+// G stage: t[k][b] = sum_i Q_V[k][i] u[k][b*l+i],  w[p][k][b*l+i] = Q_U[k][i] t[k][b]
+template <int NB, int RT>
+__global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_mma_kernel(Paths ps, const uint2 *__restrict__ zpk,
+                                                                     float *__restrict__ wout, int m, int r, int l,
+                                                                     int B) {
+  extern __shared__ float sm[];
+  float *red = sm, *D = sm + SP_WARPS * RT * NB * 128;
+  const int p = blockIdx.y, warp = threadIdx.x >> 5;
+  const int QW = (m + 31) / 32, V = l * B;
+  const int row0 = blockIdx.x * 16 * RT;
+  float acc[RT][NB][4];
 #pragma unroll
-    for (int b = 0; b < VMAX; ++b) {
-      if (b < B) {
-        if (ydt == QL_OUT_F32)
-          static_cast<float *>(y)[(int64_t)b * n + a] = yacc[b];
-        else
-          static_cast<uint16_t *>(y)[(int64_t)b * n + a] = qld::f32_to_bf16_rn(yacc[b]);
-      }
+  for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
+  const int w0 = (int)((int64_t)QW * warp / SP_WARPS), w1 = (int)((int64_t)QW * (warp + 1) / SP_WARPS);
+  sign_mma_rows<NB, RT>(ps.SB[p], ps.ldSB[p], r, row0, zpk + (size_t)p * QW * NB * 64, w0, w1, acc);
+  reduce_fragments<NB, RT>(red, D, acc);
+  for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) {
+    const int rr = e / B, b = e - rr * B, k = row0 + rr;
+    if (k >= r) continue;
+    const float *Dr = D + rr * (8 * NB);
+    const uint16_t *qv = ps.QV[p] + (int64_t)k * l, *qu = ps.QU[p] + (int64_t)k * l;
+    float t = 0.f;
+    for (int i = 0; i < l; ++i) t = fmaf(qld::f16_to_f32(qv[i]), Dr[b * l + i] + Dr[V + b * l + i], t);
+    float *wo = wout + ((int64_t)p * r + k) * V + b * l;
+    for (int i = 0; i < l; ++i) wo[i] = qld::f16_to_f32(qu[i]) * t;
+  }
+}
+
+// F stage: y[b][a] = sum_p sum_i A_amp[a][i] v_p[a][b*l+i], paths summed in p order
+template <int NB, int RT>
+__global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int P, const uint2 *__restrict__ wpk,
+                                                                     void *__restrict__ y, int ydt, int n, int r, int l,
+                                                                     int B) {
+  extern __shared__ float sm[];
+  float *red = sm, *D = sm + SP_WARPS * RT * NB * 128, *yacc = D + RT * 16 * 8 * NB;
+  const int warp = threadIdx.x >> 5;
+  const int QW = (r + 31) / 32, V = l * B;
+  const int row0 = blockIdx.x * 16 * RT;
+  for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) yacc[e] = 0.f;
+  const int w0 = (int)((int64_t)QW * warp / SP_WARPS), w1 = (int)((int64_t)QW * (warp + 1) / SP_WARPS);
+  for (int p = 0; p < P; ++p) {
+    float acc[RT][NB][4];
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
+    sign_mma_rows<NB, RT>(ps.SA[p], ps.ldSA[p], n, row0, wpk + (size_t)p * QW * NB * 64, w0, w1, acc);
+    reduce_fragments<NB, RT>(red, D, acc);
+    for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) {
+      const int rr = e / B, b = e - rr * B, a = row0 + rr;
+      if (a >= n) continue;
+      const float *Dr = D + rr * (8 * NB);
+      const uint16_t *am = ps.A[p] + (int64_t)a * l;
+      float s = yacc[e];
+      for (int i = 0; i < l; ++i) s = fmaf(qld::f16_to_f32(am[i]), Dr[b * l + i] + Dr[V + b * l + i], s);
+      yacc[e] = s;
     }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) {
+    const int rr = e / B, b = e - rr * B, a = row0 + rr;
+    if (a >= n) continue;
+    if (ydt == QL_OUT_F32)
+      static_cast<float *>(y)[(int64_t)b * n + a] = yacc[e];
+    else
+      static_cast<uint16_t *>(y)[(int64_t)b * n + a] = qld::f32_to_bf16_rn(yacc[e]);
   }
 }
 
@@ -260,28 +330,57 @@ Paths pack_paths(const mdbf_path *paths, int P) {
   return ps;
 }
 
-template <int VMAX>
-ql_status run_stages(const Paths &ps, int P, int n, int m, int r, int l, int B, float *Z, float *Wv,
-                     void *y, ql_out_dtype ydt, cudaStream_t s) {
-  constexpr int KSG = 8, KSF = 4;
-  const size_t smg = (size_t)KSG * VMAX * 32 * sizeof(float), smf = (size_t)KSF * VMAX * 32 * sizeof(float);
-  if (smg > 48 * 1024 &&
-      cudaFuncSetAttribute(mdbf_g_stage_kernel<VMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg) != cudaSuccess)
+int nb_for(int V) {
+  const int need = (2 * V + 7) / 8;
+  int nb = 1;
+  while (nb < need) nb *= 2;
+  return nb;
+}
+
+template <int NB, int RTG, int RTF>
+ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint2 *zpk,
+                         float *wf, uint2 *wpk, void *y, ql_out_dtype ydt, cudaStream_t s) {
+  const int V = l * B;
+  const size_t smg = (size_t)(SP_WARPS * RTG * NB * 128 + RTG * 16 * 8 * NB) * sizeof(float);
+  const size_t smf = (size_t)(SP_WARPS * RTF * NB * 128 + RTF * 16 * 8 * NB + RTF * 16 * B) * sizeof(float);
+  auto kg = mdbf_g_mma_kernel<NB, RTG>;
+  auto kf = mdbf_f_mma_kernel<NB, RTF>;
+  if (cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg) != cudaSuccess ||
+      cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf) != cudaSuccess)
     return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-  if (smf > 48 * 1024 &&
-      cudaFuncSetAttribute(mdbf_f_stage_kernel<VMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf) != cudaSuccess)
-    return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
+  const int sms = ql::sm_count();
   {
-    const dim3 block(32, KSG), grid((r + 31) / 32, P);
-    mdbf_g_stage_kernel<VMAX><<<grid, block, smg, s>>>(ps, Z, Wv, m, r, l, B);
-    ql_status st = ql::launch_status("mdbf_linear (G stage)");
+    const int64_t total = (int64_t)((m + 31) / 32) * NB * 64;
+    const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sms * 4);
+    mdbf_pack_z_kernel<<<dim3(grid, P), 256, 0, s>>>(ps, x, zpk, m, l, B, NB);
+    ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
+  kg<<<dim3((r + 16 * RTG - 1) / (16 * RTG), P), SP_WARPS * 32, smg, s>>>(ps, zpk, wf, m, r, l, B);
+  ql_status st = ql::launch_status("mdbf_linear (G stage)");
+  if (st != QL_OK) return st;
   {
-    const dim3 block(32, KSF), grid((n + 31) / 32);
-    mdbf_f_stage_kernel<VMAX><<<grid, block, smf, s>>>(ps, P, Wv, y, (int)ydt, n, r, l, B);
-    return ql::launch_status("mdbf_linear (F stage)");
+    const int64_t total = (int64_t)((r + 31) / 32) * NB * 64;
+    const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sms * 4);
+    mdbf_pack_w_kernel<<<dim3(grid, P), 256, 0, s>>>(wf, wpk, r, V, NB);
+    st = ql::launch_status("mdbf_linear (pack w)");
+    if (st != QL_OK) return st;
   }
+  kf<<<(n + 16 * RTF - 1) / (16 * RTF), SP_WARPS * 32, smf, s>>>(ps, P, wpk, y, (int)ydt, n, r, l, B);
+  return ql::launch_status("mdbf_linear (F stage)");
+}
+
+struct WsLayout {
+  size_t zpk, wf, wpk, total;
+};
+WsLayout ws_layout(int P, int m, int r, int l, int B) {
+  const int NB = nb_for(l * B);
+  WsLayout L;
+  L.zpk = 0;
+  L.wf = align256((size_t)P * ((m + 31) / 32) * NB * 64 * sizeof(uint2));
+  L.wpk = L.wf + align256((size_t)P * r * l * B * sizeof(float));
+  L.total = L.wpk + align256((size_t)P * ((r + 31) / 32) * NB * 64 * sizeof(uint2));
+  return L;
 }
 
 }  // namespace
@@ -290,8 +389,7 @@ namespace ql {
 
 size_t mdbf_workspace_size(int P, int n, int m, int r, int l, int B) {
   (void)n;
-  const size_t vp = (size_t)vpad(l * B);
-  return align256((size_t)P * m * vp * sizeof(float)) + align256((size_t)P * r * vp * sizeof(float));
+  return ws_layout(P, m, r, l, B).total;
 }
 
 ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x,
@@ -299,22 +397,18 @@ ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r,
   if (P > PMAX) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: P = %d exceeds %d paths", P, PMAX);
   if (l * B > VLIM) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: l*B = %d exceeds %d", l * B, VLIM);
   const Paths ps = pack_paths(paths, P);
-  const int vp = vpad(l * B);
-  float *Z = static_cast<float *>(ws);
-  float *Wv = reinterpret_cast<float *>(static_cast<char *>(ws) + align256((size_t)P * m * vp * sizeof(float)));
-  {
-    const int64_t total = (int64_t)m * vp;
-    const int threads = 256;
-    const int grid = (int)std::min<int64_t>((total + threads - 1) / threads, (int64_t)sm_count() * 4);
-    mdbf_prologue_kernel<<<dim3(grid, P), threads, 0, s>>>(ps, x, Z, m, l, B);
-    ql_status st = launch_status("mdbf_linear (prologue)");
-    if (st != QL_OK) return st;
+  const WsLayout L = ws_layout(P, m, r, l, B);
+  char *base = static_cast<char *>(ws);
+  uint2 *zpk = reinterpret_cast<uint2 *>(base + L.zpk);
+  float *wf = reinterpret_cast<float *>(base + L.wf);
+  uint2 *wpk = reinterpret_cast<uint2 *>(base + L.wpk);
+  switch (nb_for(l * B)) {
+    case 1: return run_mma_stages<1, 1, 4>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
+    case 2: return run_mma_stages<2, 1, 2>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
+    case 4: return run_mma_stages<4, 1, 1>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
+    case 8: return run_mma_stages<8, 1, 1>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
+    default: return run_mma_stages<16, 1, 1>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
   }
-  if (vp <= 4) return run_stages<4>(ps, P, n, m, r, l, B, Z, Wv, y, ydt, s);
-  if (vp <= 8) return run_stages<8>(ps, P, n, m, r, l, B, Z, Wv, y, ydt, s);
-  if (vp <= 16) return run_stages<16>(ps, P, n, m, r, l, B, Z, Wv, y, ydt, s);
-  if (vp <= 32) return run_stages<32>(ps, P, n, m, r, l, B, Z, Wv, y, ydt, s);
-  return run_stages<64>(ps, P, n, m, r, l, B, Z, Wv, y, ydt, s);
 }
 
 ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W, float *F,
