@@ -14,8 +14,8 @@
 //             the path sum is taken inside one launch, in p order)
 // The sign products run on the warp MMA (see "Sign products on the warp MMA"
 // below); column-split partials are summed through shared memory in a fixed
-// order, so results are deterministic.  Launches per call: pack z, G stage,
-// pack w, F stage.
+// order, so results are deterministic.  Launches per call: pack z, G stage
+// (which also packs w for the F stage), F stage.
 #include <algorithm>
 #include <mutex>
 
@@ -77,23 +77,26 @@ __device__ __forceinline__ uint32_t frag_value(Get get, int c, int n, int cols, 
   return bf16_rn_bits(v - __uint_as_float(hi << 16));
 }
 
-// packed B fragments: VB[qw][nb][h][lane] as uint2, for one path
+// packed B fragments of one 32-column word, VB[qw][nb][lane] as uint4 = {MMA 0 regs, MMA 1 regs}
 template <typename Get>
-__device__ __forceinline__ uint2 pack_fragment(Get get, int qw, int nb, int h, int lane, int cols, int V) {
+__device__ __forceinline__ uint4 pack_fragment(Get get, int qw, int nb, int lane, int cols, int V) {
   const int g = lane >> 2, q = lane & 3, n = 8 * nb + g;
-  const int ca = 32 * qw + 8 * h + q, cb = ca + 4;
-  uint2 r;
-  r.x = frag_value(get, ca, n, cols, V) | (frag_value(get, ca + 16, n, cols, V) << 16);
-  r.y = frag_value(get, cb, n, cols, V) | (frag_value(get, cb + 16, n, cols, V) << 16);
-  return r;
+  uint32_t o[4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int ca = 32 * qw + 8 * h + q, cb = ca + 4;
+    o[2 * h] = frag_value(get, ca, n, cols, V) | (frag_value(get, ca + 16, n, cols, V) << 16);
+    o[2 * h + 1] = frag_value(get, cb, n, cols, V) | (frag_value(get, cb + 16, n, cols, V) << 16);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // G-stage B fragments from z[j][b*l+i] = B_amp[j][i] * x[b][j] (exact in fp32)
-__global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uint2 *__restrict__ out, int m, int l,
+__global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uint4 *__restrict__ out, int m, int l,
                                    int B, int NB) {
   const int p = blockIdx.y;
   const int QW = (m + 31) / 32, V = l * B;
-  const int64_t total = (int64_t)QW * NB * 2 * 32;
+  const int64_t total = (int64_t)QW * NB * 32;
   const uint16_t *bm = ps.Bm[p];
   auto get = [&](int c, int v) {
     const int b = v / l, i = v - b * l;
@@ -102,41 +105,21 @@ __global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uin
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
     const int lane = int(e & 31);
     const int64_t f = e >> 5;
-    const int h = int(f & 1);
-    const int64_t f2 = f >> 1;
-    const int nb = int(f2 % NB);
-    const int qw = int(f2 / NB);
-    out[(int64_t)p * total + e] = pack_fragment(get, qw, nb, h, lane, m, V);
-  }
-}
-
-// F-stage B fragments from w[p][k][v] (fp32, written by the G stage)
-__global__ void mdbf_pack_w_kernel(const float *__restrict__ w, uint2 *__restrict__ out, int r, int V, int NB) {
-  const int p = blockIdx.y;
-  const int QW = (r + 31) / 32;
-  const int64_t total = (int64_t)QW * NB * 2 * 32;
-  const float *wp = w + (int64_t)p * r * V;
-  auto get = [&](int c, int v) { return wp[(int64_t)c * V + v]; };
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int lane = int(e & 31);
-    const int64_t f = e >> 5;
-    const int h = int(f & 1);
-    const int64_t f2 = f >> 1;
-    const int nb = int(f2 % NB);
-    const int qw = int(f2 / NB);
-    out[(int64_t)p * total + e] = pack_fragment(get, qw, nb, h, lane, r, V);
+    out[(int64_t)p * total + e] = pack_fragment(get, int(f / NB), int(f % NB), lane, m, V);
   }
 }
 
 constexpr int SP_WARPS = 8;
+constexpr int SP_U = 4;   // sign words per load group (one 16-byte load per row when rows are 16-byte aligned)
 
-// Accumulates one warp's share of words into acc for RT row tiles of 16 rows starting at row0.
-template <int NB, int RT>
+// Accumulates one warp's share of words [w0, w1) into acc for RT row tiles of 16 rows at row0.
+// w0 is a multiple of SP_U.  VEC16: sign rows are 16-byte aligned, so SP_U words load at once.
+template <int NB, int RT, bool VEC16>
 __device__ __forceinline__ void sign_mma_rows(const uint8_t *__restrict__ S, size_t ld, int rows, int row0,
-                                              const uint2 *__restrict__ vb, int w0, int w1,
+                                              const uint4 *__restrict__ vb, int w0, int w1,
                                               float (&acc)[RT][NB][4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-  const uint8_t *rp[RT][2];
+  const uint32_t *rp[RT][2];
   bool ok[RT][2];
 #pragma unroll
   for (int rt = 0; rt < RT; ++rt)
@@ -144,28 +127,61 @@ __device__ __forceinline__ void sign_mma_rows(const uint8_t *__restrict__ S, siz
     for (int hh = 0; hh < 2; ++hh) {
       const int row = row0 + 16 * rt + g + 8 * hh;
       ok[rt][hh] = row < rows;
-      rp[rt][hh] = S + (size_t)(ok[rt][hh] ? row : 0) * ld;
+      rp[rt][hh] = reinterpret_cast<const uint32_t *>(S + (size_t)(ok[rt][hh] ? row : 0) * ld);
     }
-  for (int qw = w0; qw < w1; ++qw) {
-    uint2 bf[NB][2];
+  for (int qw0 = w0; qw0 < w1; qw0 += SP_U) {
+    uint32_t sw[SP_U][RT][2];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
+    for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) bf[nb][h] = __ldg(vb + (((size_t)qw * NB + nb) * 2 + h) * 32 + lane);
+      for (int hh = 0; hh < 2; ++hh) {
+        if constexpr (VEC16) {
+          const uint4 v = ok[rt][hh] ? __ldg(reinterpret_cast<const uint4 *>(rp[rt][hh] + qw0)) : make_uint4(0, 0, 0, 0);
+          sw[0][rt][hh] = v.x; sw[1][rt][hh] = v.y; sw[2][rt][hh] = v.z; sw[3][rt][hh] = v.w;
+        } else {
 #pragma unroll
-    for (int rt = 0; rt < RT; ++rt) {
-      const uint32_t s0 = ok[rt][0] ? __ldg(reinterpret_cast<const uint32_t *>(rp[rt][0]) + qw) : 0u;
-      const uint32_t s1 = ok[rt][1] ? __ldg(reinterpret_cast<const uint32_t *>(rp[rt][1]) + qw) : 0u;
+          for (int u = 0; u < SP_U; ++u)
+            sw[u][rt][hh] = (ok[rt][hh] && qw0 + u < w1) ? __ldg(rp[rt][hh] + qw0 + u) : 0u;
+        }
+      }
+    // fragments: all SP_U words up front when they are few registers, else one word at a time
+    constexpr int UB = NB <= 2 ? SP_U : 1;
+    uint4 bf[UB][NB];
+    auto load_frags = [&](int slot, int qw) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int sa = 15 - 8 * h - q, sb = 11 - 8 * h - q;
-        const uint32_t a0 = sign_pair(s0, sa), a1 = sign_pair(s1, sa);
-        const uint32_t a2 = sign_pair(s0, sb), a3 = sign_pair(s1, sb);
+      for (int nb = 0; nb < NB; ++nb)
+        bf[slot][nb] = (qw < w1) ? __ldg(vb + ((size_t)qw * NB + nb) * 32 + lane) : make_uint4(0, 0, 0, 0);
+    };
+    if constexpr (UB == SP_U) {
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) mma16816(acc[rt][nb], a0, a1, a2, a3, bf[nb][h].x, bf[nb][h].y);
+      for (int u = 0; u < SP_U; ++u) load_frags(u, qw0 + u);
+    }
+#pragma unroll
+    for (int u = 0; u < SP_U; ++u) {
+      const int slot = UB == SP_U ? u : 0;
+      if constexpr (UB != SP_U) load_frags(0, qw0 + u);
+#pragma unroll
+      for (int rt = 0; rt < RT; ++rt) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int sa = 15 - 8 * h - q, sb = 11 - 8 * h - q;
+          const uint32_t a0 = sign_pair(sw[u][rt][0], sa), a1 = sign_pair(sw[u][rt][1], sa);
+          const uint32_t a2 = sign_pair(sw[u][rt][0], sb), a3 = sign_pair(sw[u][rt][1], sb);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const uint32_t b0 = h ? bf[slot][nb].z : bf[slot][nb].x, b1 = h ? bf[slot][nb].w : bf[slot][nb].y;
+            mma16816(acc[rt][nb], a0, a1, a2, a3, b0, b1);
+          }
+        }
       }
     }
   }
+}
+
+__device__ __forceinline__ void warp_words(int QW, int warp, int &w0, int &w1) {
+  const int groups = (QW + SP_U - 1) / SP_U;
+  w0 = SP_U * (int)((int64_t)groups * warp / SP_WARPS);
+  w1 = min(QW, SP_U * (int)((int64_t)groups * (warp + 1) / SP_WARPS));
 }
 
 // Sums the warps' fragments into D[rt][16][8 NB] (fp32, shared), fixed order.
@@ -190,41 +206,52 @@ __device__ __forceinline__ void reduce_fragments(float *red, float *D, const flo
   __syncthreads();
 }
 
-// G stage: t[k][b] = sum_i Q_V[k][i] u[k][b*l+i],  w[p][k][b*l+i] = Q_U[k][i] t[k][b]
-template <int NB, int RT>
-__global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_mma_kernel(Paths ps, const uint2 *__restrict__ zpk,
-                                                                     float *__restrict__ wout, int m, int r, int l,
+// G stage over 32 rows k (one word of the F stage):
+//   t[k][b] = sum_i Q_V[k][i] u[k][b*l+i],  w[k][b*l+i] = Q_U[k][i] t[k][b],
+// and w is written straight out as the F stage's packed B fragments for that word.
+template <int NB, bool VEC16>
+__global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_mma_kernel(Paths ps, const uint4 *__restrict__ zpk,
+                                                                     uint4 *__restrict__ wpk, int m, int r, int l,
                                                                      int B) {
   extern __shared__ float sm[];
-  float *red = sm, *D = sm + SP_WARPS * RT * NB * 128;
+  float *red = sm, *D = sm + SP_WARPS * 2 * NB * 128, *Ws = D + 32 * 8 * NB;
   const int p = blockIdx.y, warp = threadIdx.x >> 5;
   const int QW = (m + 31) / 32, V = l * B;
-  const int row0 = blockIdx.x * 16 * RT;
-  float acc[RT][NB][4];
+  const int row0 = blockIdx.x * 32;
+  float acc[2][NB][4];
 #pragma unroll
-  for (int rt = 0; rt < RT; ++rt)
+  for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
-  const int w0 = (int)((int64_t)QW * warp / SP_WARPS), w1 = (int)((int64_t)QW * (warp + 1) / SP_WARPS);
-  sign_mma_rows<NB, RT>(ps.SB[p], ps.ldSB[p], r, row0, zpk + (size_t)p * QW * NB * 64, w0, w1, acc);
-  reduce_fragments<NB, RT>(red, D, acc);
-  for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) {
+  int w0, w1;
+  warp_words(QW, warp, w0, w1);
+  sign_mma_rows<NB, 2, VEC16>(ps.SB[p], ps.ldSB[p], r, row0, zpk + (size_t)p * QW * NB * 32, w0, w1, acc);
+  reduce_fragments<NB, 2>(red, D, acc);
+  for (int e = threadIdx.x; e < 32 * B; e += blockDim.x) {
     const int rr = e / B, b = e - rr * B, k = row0 + rr;
-    if (k >= r) continue;
+    float *wo = Ws + rr * V + b * l;
+    if (k >= r) {
+      for (int i = 0; i < l; ++i) wo[i] = 0.f;
+      continue;
+    }
     const float *Dr = D + rr * (8 * NB);
     const uint16_t *qv = ps.QV[p] + (int64_t)k * l, *qu = ps.QU[p] + (int64_t)k * l;
     float t = 0.f;
     for (int i = 0; i < l; ++i) t = fmaf(qld::f16_to_f32(qv[i]), Dr[b * l + i] + Dr[V + b * l + i], t);
-    float *wo = wout + ((int64_t)p * r + k) * V + b * l;
     for (int i = 0; i < l; ++i) wo[i] = qld::f16_to_f32(qu[i]) * t;
   }
+  __syncthreads();
+  const int qw = blockIdx.x, QWr = (r + 31) / 32;
+  auto get = [&](int c, int v) { return Ws[(c - 32 * qw) * V + v]; };
+  for (int e = threadIdx.x; e < NB * 32; e += blockDim.x)
+    wpk[((size_t)p * QWr + qw) * NB * 32 + e] = pack_fragment(get, qw, e >> 5, e & 31, r, V);
 }
 
 // F stage: y[b][a] = sum_p sum_i A_amp[a][i] v_p[a][b*l+i], paths summed in p order
-template <int NB, int RT>
-__global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int P, const uint2 *__restrict__ wpk,
+template <int NB, int RT, bool VEC16>
+__global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int P, const uint4 *__restrict__ wpk,
                                                                      void *__restrict__ y, int ydt, int n, int r, int l,
                                                                      int B) {
   extern __shared__ float sm[];
@@ -233,7 +260,8 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int
   const int QW = (r + 31) / 32, V = l * B;
   const int row0 = blockIdx.x * 16 * RT;
   for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) yacc[e] = 0.f;
-  const int w0 = (int)((int64_t)QW * warp / SP_WARPS), w1 = (int)((int64_t)QW * (warp + 1) / SP_WARPS);
+  int w0, w1;
+  warp_words(QW, warp, w0, w1);
   for (int p = 0; p < P; ++p) {
     float acc[RT][NB][4];
 #pragma unroll
@@ -242,7 +270,7 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int
       for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
-    sign_mma_rows<NB, RT>(ps.SA[p], ps.ldSA[p], n, row0, wpk + (size_t)p * QW * NB * 64, w0, w1, acc);
+    sign_mma_rows<NB, RT, VEC16>(ps.SA[p], ps.ldSA[p], n, row0, wpk + (size_t)p * QW * NB * 32, w0, w1, acc);
     reduce_fragments<NB, RT>(red, D, acc);
     for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) {
       const int rr = e / B, b = e - rr * B, a = row0 + rr;
@@ -337,49 +365,60 @@ int nb_for(int V) {
   return nb;
 }
 
-template <int NB, int RTG, int RTF>
-ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint2 *zpk,
-                         float *wf, uint2 *wpk, void *y, ql_out_dtype ydt, cudaStream_t s) {
-  const int V = l * B;
-  const size_t smg = (size_t)(SP_WARPS * RTG * NB * 128 + RTG * 16 * 8 * NB) * sizeof(float);
+template <int NB, int RTF, bool VEC16>
+ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk,
+                         uint4 *wpk, void *y, ql_out_dtype ydt, cudaStream_t s) {
+  const size_t smg = (size_t)(SP_WARPS * 2 * NB * 128 + 32 * 8 * NB + 32 * l * B) * sizeof(float);
   const size_t smf = (size_t)(SP_WARPS * RTF * NB * 128 + RTF * 16 * 8 * NB + RTF * 16 * B) * sizeof(float);
-  auto kg = mdbf_g_mma_kernel<NB, RTG>;
-  auto kf = mdbf_f_mma_kernel<NB, RTF>;
+  auto kg = mdbf_g_mma_kernel<NB, VEC16>;
+  auto kf = mdbf_f_mma_kernel<NB, RTF, VEC16>;
   if (cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg) != cudaSuccess ||
       cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf) != cudaSuccess)
     return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-  const int sms = ql::sm_count();
   {
-    const int64_t total = (int64_t)((m + 31) / 32) * NB * 64;
-    const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sms * 4);
+    const int64_t total = (int64_t)((m + 31) / 32) * NB * 32;
+    const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)ql::sm_count() * 4);
     mdbf_pack_z_kernel<<<dim3(grid, P), 256, 0, s>>>(ps, x, zpk, m, l, B, NB);
     ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
-  kg<<<dim3((r + 16 * RTG - 1) / (16 * RTG), P), SP_WARPS * 32, smg, s>>>(ps, zpk, wf, m, r, l, B);
+  kg<<<dim3((r + 31) / 32, P), SP_WARPS * 32, smg, s>>>(ps, zpk, wpk, m, r, l, B);
   ql_status st = ql::launch_status("mdbf_linear (G stage)");
   if (st != QL_OK) return st;
-  {
-    const int64_t total = (int64_t)((r + 31) / 32) * NB * 64;
-    const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sms * 4);
-    mdbf_pack_w_kernel<<<dim3(grid, P), 256, 0, s>>>(wf, wpk, r, V, NB);
-    st = ql::launch_status("mdbf_linear (pack w)");
-    if (st != QL_OK) return st;
-  }
   kf<<<(n + 16 * RTF - 1) / (16 * RTF), SP_WARPS * 32, smf, s>>>(ps, P, wpk, y, (int)ydt, n, r, l, B);
   return ql::launch_status("mdbf_linear (F stage)");
 }
 
+template <int NB, bool VEC16>
+ql_status run_nb(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk, uint4 *wpk,
+                 void *y, ql_out_dtype ydt, cudaStream_t s) {
+  // two 16-row tiles per F block once there are enough rows to fill the machine twice over
+  if (NB == 1 && n >= 16 * 2 * 4 * ql::sm_count())
+    return run_mma_stages<NB, 2, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+  return run_mma_stages<NB, 1, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+}
+
+template <bool VEC16>
+ql_status run_vec(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk,
+                  uint4 *wpk, void *y, ql_out_dtype ydt, cudaStream_t s) {
+  switch (nb_for(l * B)) {
+    case 1: return run_nb<1, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+    case 2: return run_nb<2, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+    case 4: return run_nb<4, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+    case 8: return run_nb<8, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+    default: return run_nb<16, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+  }
+}
+
 struct WsLayout {
-  size_t zpk, wf, wpk, total;
+  size_t zpk, wpk, total;
 };
 WsLayout ws_layout(int P, int m, int r, int l, int B) {
   const int NB = nb_for(l * B);
   WsLayout L;
   L.zpk = 0;
-  L.wf = align256((size_t)P * ((m + 31) / 32) * NB * 64 * sizeof(uint2));
-  L.wpk = L.wf + align256((size_t)P * r * l * B * sizeof(float));
-  L.total = L.wpk + align256((size_t)P * ((r + 31) / 32) * NB * 64 * sizeof(uint2));
+  L.wpk = align256((size_t)P * ((m + 31) / 32) * NB * 32 * sizeof(uint4));
+  L.total = L.wpk + align256((size_t)P * ((r + 31) / 32) * NB * 32 * sizeof(uint4));
   return L;
 }
 
@@ -399,16 +438,14 @@ ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r,
   const Paths ps = pack_paths(paths, P);
   const WsLayout L = ws_layout(P, m, r, l, B);
   char *base = static_cast<char *>(ws);
-  uint2 *zpk = reinterpret_cast<uint2 *>(base + L.zpk);
-  float *wf = reinterpret_cast<float *>(base + L.wf);
-  uint2 *wpk = reinterpret_cast<uint2 *>(base + L.wpk);
-  switch (nb_for(l * B)) {
-    case 1: return run_mma_stages<1, 1, 4>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
-    case 2: return run_mma_stages<2, 1, 2>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
-    case 4: return run_mma_stages<4, 1, 1>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
-    case 8: return run_mma_stages<8, 1, 1>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
-    default: return run_mma_stages<16, 1, 1>(ps, P, n, m, r, l, B, x, zpk, wf, wpk, y, ydt, s);
-  }
+  uint4 *zpk = reinterpret_cast<uint4 *>(base + L.zpk);
+  uint4 *wpk = reinterpret_cast<uint4 *>(base + L.wpk);
+  bool vec16 = true;
+  for (int p = 0; p < P; ++p)
+    vec16 = vec16 && paths[p].ldSA % 16 == 0 && paths[p].ldSB % 16 == 0 && aligned(paths[p].S_A, 16) &&
+            aligned(paths[p].S_B, 16);
+  if (vec16) return run_vec<true>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+  return run_vec<false>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
 }
 
 ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W, float *F,
