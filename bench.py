@@ -334,41 +334,61 @@ def main():
         step(i)
     torch.cuda.synchronize()
 
-    # per-kernel durations, measured live on the launching stream over the timed region
+    # A decode step is launch-bound at this size, so it is replayed as a CUDA graph: one graph
+    # per rotating weight copy, kernels chained by programmatic dependent launch.
     dom = [L for L in wl.layers if L["kind"] == ("benq" if args.workload in ("decode", "prefill", "layer") else "mdbf")]
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in dom]
-          for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+
+    def capture(layers, copies):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for c in copies:
+                for L in layers:
+                    wl.run_layer(L, c)
+        return g
+
+    # one graph per rotation cycle (steps on copies 0 .. ncopy-1), as a model graph holds many
+    # layers; single-step graphs cover a remainder so that exactly `steps` steps run
+    def graph_set(layers):
+        return {"cycle": capture(layers, range(ncopy)), "one": [capture(layers, [c]) for c in range(ncopy)]}
+
+    graphs = graph_set(wl.layers)
+    dom_graphs = graphs if len(dom) == len(wl.layers) else graph_set(dom)
+
+    def replay(gs, steps):
+        for _ in range(steps // ncopy):
+            gs["cycle"].replay()
+        for c in range(steps % ncopy):
+            gs["one"][c].replay()
+
+    def timed(gs, steps):
+        """Replays `steps` steps between two events on the launching stream; returns
+        milliseconds, the max over ranks."""
+        replay(gs, max(args.warmup, ncopy))
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         start.record(stream)
-        for i in range(args.steps):
-            c = i % ncopy
-            j = 0
-            for L in wl.layers:
-                if L in dom:
-                    ev[i][j][0].record(stream)
-                    wl.run_layer(L, c)
-                    ev[i][j][1].record(stream)
-                    j += 1
-                else:
-                    wl.run_layer(L, c)
+        replay(gs, steps)
         stop.record(stream)
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        if world > 1:
+            dist.barrier()
+        t_ms = start.elapsed_time(stop)
+        if world > 1:
+            t = torch.tensor([t_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            t_ms = float(t.item())
+        return t_ms
+
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms = timed(graphs, args.steps)
+        # the dominant kernel's average duration: its own launches back to back, in the same
+        # graphs when the step holds nothing else
+        dom_ms = ms if dom_graphs is graphs else timed(dom_graphs, args.steps)
     ms_per_step = ms / args.steps
     step_bytes = wl.step_bytes()
     value = world * step_bytes * args.steps / (ms / 1e3) / 1e9
-
-    dom_ms = sum(a.elapsed_time(b) for row in ev for (a, b) in row)
     dom_launches = len(dom) * args.steps
     peaks = _peaks()
     if args.workload == "prefill":
@@ -431,13 +451,16 @@ def main():
                        "tflops": (wl.step_flops() * args.steps / (ms / 1e3) / 1e12) if wl.step_flops() else None,
                        "l2": f"inputs larger than L2: {ncopy} rotating weight copies, "
                              f"{wl.working_set / 2**20:.0f} MiB working set vs 126 MiB L2",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}",
+                       "launch": f"CUDA graphs of {ncopy} steps (one weight-copy rotation), kernels chained "
+                                 "by programmatic dependent launch; e2e uses eager calls"},
             "roofline": roof, "e2e": e2e, "gpu_launches": wl.launches_per_step() * args.steps,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graphs, dom_graphs
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -195,6 +195,20 @@ QL_API const char *ql_last_error(void);
  * QL_OK, QL_ERR_TIMEOUT, or QL_ERR_CUDA if the stream itself failed. */
 QL_API ql_status ql_check(ql_stream_t stream);
 
+/* Launch overlap (programmatic dependent launch).  No counterpart in the pages:
+ * this is launch plumbing.  When enabled (the default; the environment variable
+ * QL_PDL=0 at load time disables it), every kernel is launched so that it may
+ * start while the kernel before it in the same stream is still finishing.  Each
+ * kernel reads its WEIGHTS (codes, tables, sign bits, envelopes) before it has
+ * waited for that predecessor, and reads activations / workspace and writes
+ * outputs only after the wait.  Weights are therefore treated as constants: a
+ * caller that writes weights with a kernel and then calls a linear entry point on
+ * the same stream right after it must either disable overlap or put a host
+ * synchronisation, an event wait or a copy between the two.  The setting is
+ * process-wide and takes effect at the next launch.  Returns the previous
+ * setting (1 enabled, 0 disabled). */
+QL_API int ql_set_pdl(int enable);
+
 #ifdef __cplusplus
 }
 #endif

@@ -45,6 +45,7 @@ _SIGNATURES = {
     "mdbf_select_rank": (_i, [_i, _i, _i, _i, _i, _d, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "ql_last_error": (ctypes.c_char_p, []),
     "ql_check": (_i, [_vp]),
+    "ql_set_pdl": (_i, [_i]),
 }
 
 
@@ -68,7 +69,7 @@ def _c(name):
 
 EXPORTS = ["benq_linear", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
            "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
-           "mdbf_select_rank", "ql_last_error", "ql_check"]
+           "mdbf_select_rank", "ql_last_error", "ql_check", "ql_set_pdl"]
 
 
 class QLinearError(RuntimeError):
@@ -215,3 +216,10 @@ def mdbf_select_rank(n, m, P, l, scale_bits, target_bits):
 def ql_check(stream=None):
     """Waits for the stream and raises QLinearError(QL_ERR_TIMEOUT) if a bounded device wait ran out."""
     _check(_c("ql_check")(_stream(stream)))
+
+
+def ql_set_pdl(enable: bool) -> bool:
+    """Enables or disables launch overlap (programmatic dependent launch) for every later call;
+    returns the previous setting.  With overlap on, weights are read before the preceding kernel
+    in the stream has finished, so they must not be written by that kernel."""
+    return bool(_c("ql_set_pdl")(1 if enable else 0))

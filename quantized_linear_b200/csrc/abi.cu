@@ -1,15 +1,24 @@
 // libqlinear C ABI: argument validation, dispatch, status reporting and host-only accounting.
 // The kernels live in benq_gemv.cu, benq_gemm_sm100.cu and mdbf.cu.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "ql_internal.cuh"
 
 namespace {
 thread_local char g_msg[512] = "";
+
+int pdl_default() {
+  const char *e = std::getenv("QL_PDL");
+  return (e && std::strcmp(e, "0") == 0) ? 0 : 1;
 }
+std::atomic<int> g_pdl{pdl_default()};
+}  // namespace
 
 namespace ql {
 
@@ -26,6 +35,8 @@ ql_status launch_status(const char *what) {
   if (e != cudaSuccess) return fail(QL_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
   return QL_OK;
 }
+
+bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
 
 int sm_count() {
   static std::mutex mu;
@@ -49,6 +60,8 @@ using ql::fail;
 extern "C" {
 
 const char *ql_last_error(void) { return g_msg; }
+
+int ql_set_pdl(int enable) { return g_pdl.exchange(enable ? 1 : 0); }
 
 ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype y_dtype,
                       int B, int N, int K, ql_stream_t stream) {

@@ -112,10 +112,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem_raw + (tmem_slot - raw));
+  // codes and tables are weights: their producer starts at once; activations are read and y is
+  // written only after the preceding kernel in the stream has completed
+  qld::pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ activation producer (TMA)
     if (lane == 0) {
+      qld::pdl_wait();
       int it = 0;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const int m0 = (t % mt) * BM;
@@ -230,6 +234,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) sm100::mbar_arrive(bar.lut_empty);
       // epilogue: this warp drains lanes [32q, 32q+32) of both 128-row accumulators
       if (!sm100::mbar_wait(bar.acc_full, tl & 1, WAIT_BUDGET)) { ok = false; break; }
+      qld::pdl_wait();
       sm100::tc_fence_after();
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
@@ -333,7 +338,7 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
   if (attr_err != cudaSuccess) return fail(QL_ERR_CUDA, "benq_linear: cannot reserve GEMM shared memory");
   const int ntiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = std::min(ntiles, sm_count());
-  benq_gemm_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mx, mc, lut, y, (int)ydt, M, N, K);
+  launch(benq_gemm_kernel, grid, THREADS, SMEM_BYTES, s, mx, mc, lut, y, (int)ydt, M, N, K);
   return launch_status("benq_linear (tensor-core GEMM)");
 }
 

@@ -38,6 +38,8 @@ __global__ void benq_dequant_kernel(const uint8_t *__restrict__ codes, const uin
   const int64_t gpr = K / 4;
   const int64_t total = (int64_t)N * gpr;
   const int64_t rowbytes = 3LL * K / 4;
+  qld::pdl_trigger();
+  qld::pdl_wait();
   for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total;
        g += (int64_t)gridDim.x * blockDim.x) {
     const int64_t n = g / gpr;
@@ -135,16 +137,6 @@ __global__ void __launch_bounds__(MAX_WARPS * 32)
   int blk = blockIdx.x;
   if (blk >= nblk) return;
 
-  uint16_t xr[32];
-  if constexpr (BMAX == 1) {
-    uint4 v[4] = {};
-    if (active) {
-#pragma unroll
-      for (int t = 0; t < 4; ++t) v[t] = ldg_u4(x + kc + 8 * t);
-    }
-    unpack_x(v, xr);
-  }
-
   auto load_codes = [&](int b, uint32_t (&w)[R][6]) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -171,12 +163,25 @@ __global__ void __launch_bounds__(MAX_WARPS * 32)
     if (threadIdx.x < 8 * R) reinterpret_cast<uint4 *>(lut_s + buf * R * 64)[threadIdx.x] = v;
   };
 
+  // the first block's weights do not depend on the preceding kernel: fetch them before waiting
   uint32_t cur[R][6];
   {
     uint4 lv;
     load_lut(blk, lv);
     store_lut(0, lv);
     load_codes(blk, cur);
+  }
+  qld::pdl_trigger();
+  qld::pdl_wait();
+
+  uint16_t xr[32];
+  if constexpr (BMAX == 1) {
+    uint4 v[4] = {};
+    if (active) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) v[t] = ldg_u4(x + kc + 8 * t);
+    }
+    unpack_x(v, xr);
   }
   __syncthreads();
 
@@ -267,6 +272,8 @@ __global__ void benq_gemv_generic_kernel(const uint8_t *__restrict__ codes, cons
                                          int N, int K) {
   const int lane = threadIdx.x & 31;
   const int64_t rowbytes = 3LL * K / 4;
+  qld::pdl_trigger();
+  qld::pdl_wait();
   for (int64_t n = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; n < N;
        n += ((int64_t)gridDim.x * blockDim.x) >> 5) {
     float acc[16];
@@ -302,11 +309,13 @@ __global__ void benq_gemv_generic_kernel(const uint8_t *__restrict__ codes, cons
 
 // ------------------------------------------------------------------------------------------
 // Batch-1 kernel for whole tiles (K % 1024 == 0, N % B1_T == 0).  Same lane layout as above,
-// with the instruction count per code cut to: one shift, one AND|OR forming the 32-bit shared
-// address of the table entry (tables are 128-byte aligned so the OR is an add), one 16-bit
-// shared load, one integer multiply placing the bf16 in the top half (an fp32), and half of a
-// packed fp32x2 FMA.  Two row groups of B1_R rows ping-pong in registers so the next group's
-// codes are in flight while one is decoded; one barrier per tile of B1_T rows.
+// with the work per code cut to: one shift, one AND|OR forming the 32-bit shared address of
+// the table entry (tables are 128-byte aligned, so the OR is an add), one 16-bit shared load
+// and one mixed-precision FMA of the raw bf16 entry with the raw bf16 activation.  Two
+// accumulators per row halve the FMA dependency chain.  Two row groups of B1_R rows ping-pong
+// in registers so the next group's codes are in flight while one is decoded; one barrier per
+// tile of B1_T rows.  The table buffer index is a compile-time constant in each half of the
+// tile loop, so every table address is a constant offset from one base.
 // ------------------------------------------------------------------------------------------
 constexpr int B1_R = 2, B1_T = 4;
 
@@ -314,50 +323,26 @@ struct B1Tables {
   uint16_t lut[2][B1_T][64];
 };
 
-__device__ __forceinline__ uint32_t lds_u16_32(uint32_t saddr) {
-  uint32_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(saddr));
-  return v;
-}
-
-__device__ __forceinline__ float bf16_hi(uint32_t v16) {
-  uint32_t r;
-  asm("mad.lo.u32 %0, %1, 65536, 0;" : "=r"(r) : "r"(v16));
-  return __uint_as_float(r);
-}
-
-// (a0, a1) += (w0, w1) * (x0, x1) as one packed fp32x2 FMA
-__device__ __forceinline__ void ffma2(float &a0, float &a1, float w0, float w1, float x0, float x1) {
-  unsigned long long acc, w, x;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(acc) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(w) : "f"(w0), "f"(w1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(w), "l"(x));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
-}
-
-template <int J0>
-__device__ __forceinline__ void dot_pair(const uint32_t (&w)[6], uint32_t tbl, const float (&xf)[32], float &a0,
-                                         float &a1) {
-  const float w0 = bf16_hi(lds_u16_32(entry_offset<J0>(w) | tbl));
-  const float w1 = bf16_hi(lds_u16_32(entry_offset<J0 + 1>(w) | tbl));
-  ffma2(a0, a1, w0, w1, xf[J0], xf[J0 + 1]);
-}
-
-template <int J>
-struct DotB1 {
-  static __device__ __forceinline__ void run(const uint32_t (&w)[6], uint32_t tbl, const float (&xf)[32], float &a0,
-                                             float &a1) {
-    DotB1<J - 2>::run(w, tbl, xf, a0, a1);
-    dot_pair<J - 2>(w, tbl, xf, a0, a1);
+// Byte offsets of the table entries of codes J and J + 1 (J even), as compile-time selections.
+__device__ __forceinline__ void pair_offsets(const uint32_t (&w)[6], int j, uint32_t &o0, uint32_t &o1) {
+  switch (j) {
+#define QL_PAIR(J)                \
+  case J:                         \
+    o0 = entry_offset<J>(w);      \
+    o1 = entry_offset<J + 1>(w);  \
+    break;
+    QL_PAIR(0) QL_PAIR(2) QL_PAIR(4) QL_PAIR(6) QL_PAIR(8) QL_PAIR(10) QL_PAIR(12) QL_PAIR(14)
+    QL_PAIR(16) QL_PAIR(18) QL_PAIR(20) QL_PAIR(22) QL_PAIR(24) QL_PAIR(26) QL_PAIR(28) QL_PAIR(30)
+#undef QL_PAIR
   }
-};
-template <>
-struct DotB1<0> {
-  static __device__ __forceinline__ void run(const uint32_t (&)[6], uint32_t, const float (&)[32], float &, float &) {}
+}
+
+template <int V>
+struct IntC {
+  static constexpr int value = V;
 };
 
-__global__ void __launch_bounds__(MAX_WARPS * 32)
+__global__ void __launch_bounds__(MAX_WARPS * 32, 1)
     benq_gemv_b1_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ lut,
                         const uint16_t *__restrict__ x, void *__restrict__ y, int ydt, int N, int K) {
   __shared__ __align__(128) B1Tables tb;
@@ -370,16 +355,28 @@ __global__ void __launch_bounds__(MAX_WARPS * 32)
   const int ntile = N / B1_T;
   int tile = blockIdx.x;
   if (tile >= ntile) return;
-
-  float xf[32];
+  // Before waiting on the preceding kernel, pull this CTA's first tile of weights (codes and
+  // tables) toward L2; prefetches hold no registers, so the loop below is compiled as if they
+  // were absent.  Activations are loaded first after the wait: loading them after the codes
+  // made the compiler schedule the decode loop far worse.
+  {
+    const uint8_t *p = cbase + (size_t)tile * B1_T * rowbytes;
+#pragma unroll
+    for (int r = 0; r < B1_T; ++r) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (size_t)r * rowbytes));
+    if (threadIdx.x < B1_T)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(lut + ((size_t)tile * B1_T + threadIdx.x) * 64));
+  }
+  qld::pdl_trigger();
+  qld::pdl_wait();
+  uint16_t xh[32];
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
     const uint4 v = ldg_u4(x + kc + 8 * t);
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      xf[8 * t + 2 * e] = __uint_as_float(u[e] << 16);
-      xf[8 * t + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      xh[8 * t + 2 * e] = u[e] & 0xFFFF;
+      xh[8 * t + 2 * e + 1] = u[e] >> 16;
     }
   }
   auto load_rows = [&](int n0, uint32_t (&w)[B1_R][6]) {
@@ -396,43 +393,50 @@ __global__ void __launch_bounds__(MAX_WARPS * 32)
   auto store_lut = [&](int buf, const uint4 &v) {
     if (threadIdx.x < 8 * B1_T) reinterpret_cast<uint4 *>(&tb.lut[buf][0][0])[threadIdx.x] = v;
   };
-  auto row_dot = [&](const uint32_t (&w)[6], uint32_t tbl) {
+  auto dot = [&](const uint32_t (&w)[6], const uint16_t *tp) -> float {
+    const uint32_t tbs = (uint32_t)__cvta_generic_to_shared(tp);
     float a0 = 0.f, a1 = 0.f;
-    DotB1<32>::run(w, tbl, xf, a0, a1);
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      uint32_t o0, o1;
+      pair_offsets(w, j, o0, o1);
+      a0 = qld::fma_bf16(lds_u16(o0 | tbs), xh[j], a0);
+      a1 = qld::fma_bf16(lds_u16(o1 | tbs), xh[j + 1], a1);
+    }
     return a0 + a1;
   };
-
   uint4 lv = make_uint4(0, 0, 0, 0);
   load_lut(tile, lv);
   store_lut(0, lv);
   uint32_t ga[B1_R][6], gb[B1_R][6];
   load_rows(tile * B1_T, ga);
   __syncthreads();
-  const uint32_t lut0 = static_cast<uint32_t>(__cvta_generic_to_shared(&tb.lut[0][0][0]));
-  float *mypart = b1part + (size_t)warp * B1_T * 32 + lane;
+  float *mypart = b1part + (warp * B1_T) * 32 + lane;
   constexpr int GP = B1_T / B1_R;  // even
-  for (int buf = 0;; buf ^= 1) {
-    const int nxt = tile + gridDim.x;
+
+  // One tile with table buffer BUF.  On entry ga holds the tile's first row group; on exit it
+  // holds the next tile's first group.  Returns whether there is a next tile.
+  auto do_tile = [&](auto bufc, int nxt) {
+    constexpr int BUF = decltype(bufc)::value;
     const bool has_next = nxt < ntile;
     if (has_next) load_lut(nxt, lv);
-    float *pb = mypart + (size_t)buf * C * B1_T * 32;
-    const uint32_t tbase = lut0 + buf * B1_T * 128;
+    float *pb = mypart + BUF * C * B1_T * 32;
 #pragma unroll
     for (int g = 0; g < GP; g += 2) {
       load_rows(tile * B1_T + (g + 1) * B1_R, gb);
 #pragma unroll
-      for (int r = 0; r < B1_R; ++r) pb[(g * B1_R + r) * 32] = row_dot(ga[r], tbase + (g * B1_R + r) * 128);
+      for (int r = 0; r < B1_R; ++r) pb[(g * B1_R + r) * 32] = dot(ga[r], &tb.lut[BUF][g * B1_R + r][0]);
       if (g + 2 < GP)
         load_rows(tile * B1_T + (g + 2) * B1_R, ga);
       else if (has_next)
         load_rows(nxt * B1_T, ga);
 #pragma unroll
       for (int r = 0; r < B1_R; ++r)
-        pb[((g + 1) * B1_R + r) * 32] = row_dot(gb[r], tbase + ((g + 1) * B1_R + r) * 128);
+        pb[((g + 1) * B1_R + r) * 32] = dot(gb[r], &tb.lut[BUF][(g + 1) * B1_R + r][0]);
     }
-    if (has_next) store_lut(buf ^ 1, lv);
+    if (has_next) store_lut(BUF ^ 1, lv);
     __syncthreads();
-    const float *pr = b1part + (size_t)buf * C * B1_T * 32;
+    const float *pr = b1part + BUF * C * B1_T * 32;
     for (int o = warp; o < B1_T; o += C) {
       float s = 0.f;
       for (int c = 0; c < C; ++c) s += pr[(c * B1_T + o) * 32 + lane];
@@ -446,8 +450,12 @@ __global__ void __launch_bounds__(MAX_WARPS * 32)
           static_cast<uint16_t *>(y)[n] = qld::f32_to_bf16_rn(s);
       }
     }
-    if (!has_next) break;
     tile = nxt;
+    return has_next;
+  };
+  while (true) {
+    if (!do_tile(IntC<0>{}, tile + gridDim.x)) break;
+    if (!do_tile(IntC<1>{}, tile + gridDim.x)) break;
   }
 }
 
@@ -461,7 +469,7 @@ ql_status launch_b1(const uint8_t *codes, const uint16_t *lut, const uint16_t *x
       per_sm < 1)
     return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
   const int grid = std::min(N / B1_T, per_sm * ql::sm_count());
-  benq_gemv_b1_kernel<<<grid, threads, smem, s>>>(codes, lut, x, y, (int)ydt, N, K);
+  ql::launch(benq_gemv_b1_kernel, grid, threads, smem, s, codes, lut, x, y, (int)ydt, N, K);
   return ql::launch_status("benq_linear (batch-1 GEMV)");
 }
 
@@ -481,7 +489,7 @@ ql_status launch_fast(const uint8_t *codes, const uint16_t *lut, const uint16_t 
     return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
   const int nblk = (N + R - 1) / R;
   const int grid = std::min(nblk, per_sm * ql::sm_count());
-  kern<<<grid, threads, smem, s>>>(codes, lut, x, y, (int)ydt, B, N, K);
+  ql::launch(kern, grid, threads, smem, s, codes, lut, x, y, (int)ydt, B, N, K);
   return ql::launch_status("benq_linear (decode GEMV)");
 }
 
@@ -495,7 +503,7 @@ ql_status benq_dequant_launch(const uint8_t *codes, const uint16_t *lut, uint16_
   const int threads = 256;
   const int64_t want = (total + threads - 1) / threads;
   const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count() * 8);
-  benq_dequant_kernel<<<grid, threads, 0, s>>>(codes, lut, W, N, K);
+  launch(benq_dequant_kernel, grid, threads, 0, s, codes, lut, W, N, K);
   return launch_status("benq_dequant_debug");
 }
 
@@ -514,7 +522,7 @@ ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint
   const int threads = 256;
   const int64_t want = ((int64_t)N * 32 + threads - 1) / threads;
   const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count() * 8);
-  benq_gemv_generic_kernel<<<grid, threads, 0, s>>>(codes, lut, x, y, (int)ydt, B, N, K);
+  launch(benq_gemv_generic_kernel, grid, threads, 0, s, codes, lut, x, y, (int)ydt, B, N, K);
   return launch_status("benq_linear (generic GEMV)");
 }
 

@@ -98,6 +98,8 @@ __global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uin
   const int QW = (m + 31) / 32, V = l * B;
   const int64_t total = (int64_t)QW * NB * 32;
   const uint16_t *bm = ps.Bm[p];
+  qld::pdl_trigger();
+  qld::pdl_wait();
   auto get = [&](int c, int v) {
     const int b = v / l, i = v - b * l;
     return qld::f16_to_f32(bm[(int64_t)c * l + i]) * qld::bf16_to_f32(x[(int64_t)b * m + c]);
@@ -106,6 +108,16 @@ __global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uin
     const int lane = int(e & 31);
     const int64_t f = e >> 5;
     out[(int64_t)p * total + e] = pack_fragment(get, int(f / NB), int(f % NB), lane, m, V);
+  }
+}
+
+// Pulls rows [row0, row0 + nrows) of a sign matrix toward L2.  Sign bits are weights, so this
+// may run before the wait on the preceding kernel; every address stays inside its row.
+__device__ __forceinline__ void prefetch_sign_rows(const uint8_t *S, size_t ld, int row0, int nrows, int rows) {
+  const int lines = (int)((ld + 127) / 128);
+  for (int e = threadIdx.x; e < nrows * lines; e += blockDim.x) {
+    const int rr = e / lines, c = e - rr * lines;
+    if (row0 + rr < rows) asm volatile("prefetch.global.L2 [%0];" ::"l"(S + (size_t)(row0 + rr) * ld + 128 * c));
   }
 }
 
@@ -218,6 +230,9 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_mma_kernel(Paths ps, con
   const int p = blockIdx.y, warp = threadIdx.x >> 5;
   const int QW = (m + 31) / 32, V = l * B;
   const int row0 = blockIdx.x * 32;
+  prefetch_sign_rows(ps.SB[p], ps.ldSB[p], row0, 32, r);
+  qld::pdl_trigger();
+  qld::pdl_wait();
   float acc[2][NB][4];
 #pragma unroll
   for (int rt = 0; rt < 2; ++rt)
@@ -259,6 +274,9 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int
   const int warp = threadIdx.x >> 5;
   const int QW = (r + 31) / 32, V = l * B;
   const int row0 = blockIdx.x * 16 * RT;
+  prefetch_sign_rows(ps.SA[0], ps.ldSA[0], row0, 16 * RT, n);
+  qld::pdl_trigger();
+  qld::pdl_wait();
   for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) yacc[e] = 0.f;
   int w0, w1;
   warp_words(QW, warp, w0, w1);
@@ -307,6 +325,8 @@ __global__ void mdbf_factors_kernel(Paths ps, float *__restrict__ F, float *__re
                                     int l) {
   const int p = blockIdx.y;
   const int64_t nF = (int64_t)n * r, nG = (int64_t)r * m;
+  qld::pdl_trigger();
+  qld::pdl_wait();
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < nF + nG; e += (int64_t)gridDim.x * blockDim.x) {
     if (e < nF) {
       if (!F) continue;
@@ -325,6 +345,8 @@ __global__ void mdbf_factors_kernel(Paths ps, float *__restrict__ F, float *__re
 
 __global__ void mdbf_w_kernel(Paths ps, int P, float *__restrict__ W, int n, int m, int r, int l) {
   const int64_t total = (int64_t)n * m;
+  qld::pdl_trigger();
+  qld::pdl_wait();
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t a = e / m;
     const int j = int(e - a * m);
@@ -378,14 +400,15 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
   {
     const int64_t total = (int64_t)((m + 31) / 32) * NB * 32;
     const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)ql::sm_count() * 4);
-    mdbf_pack_z_kernel<<<dim3(grid, P), 256, 0, s>>>(ps, x, zpk, m, l, B, NB);
+    ql::launch(mdbf_pack_z_kernel, dim3(grid, P), 256, 0, s, ps, x, zpk, m, l, B, NB);
     ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
-  kg<<<dim3((r + 31) / 32, P), SP_WARPS * 32, smg, s>>>(ps, zpk, wpk, m, r, l, B);
+  ql::launch(kg, dim3((r + 31) / 32, P), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
   ql_status st = ql::launch_status("mdbf_linear (G stage)");
   if (st != QL_OK) return st;
-  kf<<<(n + 16 * RTF - 1) / (16 * RTF), SP_WARPS * 32, smf, s>>>(ps, P, wpk, y, (int)ydt, n, r, l, B);
+  ql::launch(kf, (n + 16 * RTF - 1) / (16 * RTF), SP_WARPS * 32, smf, s, ps, P, (const uint4 *)wpk, y, (int)ydt, n,
+             r, l, B);
   return ql::launch_status("mdbf_linear (F stage)");
 }
 
@@ -455,13 +478,13 @@ ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r
   if (F || G) {
     const int64_t total = (int64_t)n * r + (int64_t)r * m;
     const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8);
-    mdbf_factors_kernel<<<dim3(grid, P), 256, 0, s>>>(ps, F, G, n, m, r, l);
+    launch(mdbf_factors_kernel, dim3(grid, P), 256, 0, s, ps, F, G, n, m, r, l);
     ql_status st = launch_status("mdbf_dequant_debug (factors)");
     if (st != QL_OK) return st;
   }
   const int64_t total = (int64_t)n * m;
   const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 16);
-  mdbf_w_kernel<<<grid, 256, 0, s>>>(ps, P, W, n, m, r, l);
+  launch(mdbf_w_kernel, grid, 256, 0, s, ps, P, W, n, m, r, l);
   return launch_status("mdbf_dequant_debug (W)");
 }
 

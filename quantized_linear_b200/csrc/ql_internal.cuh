@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "qlinear.h"
 
 namespace ql {
@@ -16,6 +18,27 @@ ql_status launch_status(const char *what);
 int sm_count();
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Whether kernels are launched with programmatic dependent launch (ql_set_pdl).
+bool pdl_enabled();
+
+// Launches `k` on `s`, allowed to overlap the tail of the preceding kernel in the stream when
+// overlap is enabled.  Every kernel launched this way calls qld::pdl_wait() before it reads
+// anything but weights and before its first global store.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
 
 // ---- entry points implemented by the kernel translation units (arguments already validated) ----
 ql_status benq_dequant_launch(const uint8_t *codes, const uint16_t *lut, uint16_t *W, int N, int K,
@@ -53,6 +76,12 @@ __device__ __forceinline__ float f16_to_f32(uint16_t h) {
   asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
   return f;
 }
+
+// Programmatic dependent launch: wait until the preceding grid in the stream has completed and
+// its writes are visible (a no-op when the kernel was launched without overlap), and allow the
+// next grid to be scheduled (it still waits for this one to complete before touching its data).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // acc + a * b with bf16 a, b and fp32 accumulate; the product is exact in fp32.
 __device__ __forceinline__ float fma_bf16(uint16_t a, uint16_t b, float acc) {
