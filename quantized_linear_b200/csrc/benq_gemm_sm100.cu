@@ -1,22 +1,28 @@
 // BenQ prefill GEMM on sm_100a tensor cores: Y[M][N] = X[M][K] * W[N][K]^T, W decoded on the fly.
 //
 // W is never written to global memory ("Qwen3.8-27B -- BenQ 6-bit", "What BenQ stores": the
-// gather lut[n][code] is fused into the GEMM).  One persistent CTA per SM walks 256 x 256 output
-// tiles; per 64-wide K block:
-//   * warp 0 loads the X tile (256 x 64 bf16, 128-byte swizzle) with tensor copies into a
-//     3-stage ring released by the MMA; warp 2 loads the packed code tile (256 rows x 48 bytes)
-//     into a 2-stage ring released as soon as the decoders have read it, plus the 256 row
-//     tables of the tile (32 KB, once per tile) with a bulk copy;
-//   * warps 3..18 (decoders) expand the code tile through the row tables into the bf16 W tile,
-//     written directly in the K-major 128-byte-swizzled layout the tensor core reads, then fence
-//     the writes for the async proxy;
-//   * warp 1, one thread, issues tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32 accumulate in
-//     tensor memory): two M halves share each decoded W tile, so each decoded weight feeds 256
-//     rows of X;
-//   * after the last K block the decoder warps drain the 2 x 128 x 256 fp32 accumulators from
-//     tensor memory (tcgen05.ld), round to bf16 (or keep fp32) and store Y.
-// Stages are handed over with mbarriers; every wait gives up after a fixed clock budget, sets a
-// device flag read by ql_check(), and the CTA winds down (tensor memory is freed on every path).
+// gather lut[n][code] is fused into the GEMM).  The work unit is a CTA pair (a cluster of two
+// CTAs on two SMs) and a 512 x 256 output tile: CTA r of the pair owns X rows [256 r, 256 r + 256)
+// of the tile and decodes W rows [128 r, 128 r + 128) of it.  Pair MMAs (tcgen05.mma.cta_group::2,
+// M = 256, N = 256, K = 16) read A from each CTA's own shared memory and B from both, so every
+// decoded weight feeds all 512 rows of X while each SM decodes only half of the W tile and each
+// SM's tensor core reads only its half of B.  Per 64-wide K block, in each CTA:
+//   * warp 0 loads its X tile (256 x 64 bf16, 128-byte swizzle) with tensor copies into a 3-stage
+//     ring; completion is counted on the even CTA's barrier, whose MMA thread consumes both;
+//   * warp 2 loads its packed codes for 4 K blocks at a time (128 rows x 192 bytes: narrow rows
+//     make slow tensor copies) into a 2-stage ring, plus the 128 row tables of the tile (16 KB,
+//     once per tile) with a bulk copy;
+//   * warps 3..18 (decoders) expand the code tile through the row tables into the bf16 W half
+//     tile, written directly in the K-major 128-byte-swizzled layout the tensor core reads, fence
+//     the writes for the async proxy and arrive on the even CTA's barrier;
+//   * in the even CTA only, warp 1 (one thread) issues the pair MMAs (two M halves share each
+//     decoded W tile) into both CTAs' tensor memory (2 x 128 x 256 fp32 per CTA) and signals
+//     stage release to both CTAs with a multicast commit;
+//   * after the last K block the decoder warps of each CTA drain their own accumulators
+//     (tcgen05.ld), round to bf16 (or keep fp32) and store Y.
+// No tensor or bulk load is multicast.  Every wait gives up after a fixed clock budget or as soon
+// as another wait of the pair has given up, sets a device flag read by ql_check(), and the CTA
+// winds down; both CTAs meet at a cluster barrier before tensor memory is freed and they exit.
 #include <cuda.h>
 
 #include <algorithm>
@@ -27,29 +33,41 @@
 
 namespace {
 
-constexpr int BM = 256, BN = 256, BK = 64;        // CTA tile; BK = one 128-byte swizzle row of bf16
-constexpr int SA = 3, SB = 2, SC = 2;             // stages: activations, decoded W, codes
+constexpr int BM = 256;                           // X rows per CTA (two 128-row MMA halves)
+constexpr int PM = 2 * BM;                        // X rows per pair tile
+constexpr int BN = 256;                           // W rows per pair tile (the MMA's N)
+constexpr int BNH = BN / 2;                       // W rows decoded by each CTA
+constexpr int BK = 64;                            // one 128-byte swizzle row of bf16
+constexpr int SA = 3, SB = 4, SC = 2;             // stages: activations, decoded W, codes
 constexpr int A_BYTES = BM * BK * 2;              // 32 KB
-constexpr int B_BYTES = BN * BK * 2;              // 32 KB
+constexpr int B_BYTES = BNH * BK * 2;             // 16 KB
 constexpr int C_ROW = BK * 6 / 8;                 // 48 code bytes per row per K block
-constexpr int C_BYTES = BN * C_ROW;               // 12 KB
-constexpr int LUT_BYTES = BN * 128;               // 32 KB
+constexpr int CKB = 4;                            // K blocks per code stage (one copy of 192-byte rows)
+constexpr int C_SROW = CKB * C_ROW;               // 192 code bytes per row per code stage
+constexpr int C_BYTES = BNH * C_SROW;             // 24 KB
+constexpr int LUT_BYTES = BNH * 128;              // 16 KB
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + SA * A_BYTES;
 constexpr int OFF_C = OFF_B + SB * B_BYTES;
-constexpr int OFF_LUT = OFF_C + SC * C_BYTES + 128;   // 128 bytes of slack after the code tiles
+constexpr int OFF_LUT = OFF_C + SC * C_BYTES + 128;   // 128 bytes of slack: the last row's second code word
 constexpr int OFF_BAR = OFF_LUT + LUT_BYTES;
 constexpr int NBAR = 2 * (SA + SB + SC) + 4;
-constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
-constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;          // + alignment slack
-constexpr int NDEC = 16;                                 // decoder / epilogue warps (multiple of 8)
-constexpr int THREADS = (3 + NDEC) * 32;   // A producer, MMA issuer, code producer, decoders
-constexpr long long WAIT_BUDGET = 4000000000LL;           // clock cycles (~2 s)
-constexpr uint32_t IDESC = sm100::idesc_bf16_f32(128, BN);
+constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;          // tensor-memory address, then the abort flag
+constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;      // + alignment slack
+constexpr int NDEC = 16;                              // decoder / epilogue warps (multiple of 8)
+constexpr int THREADS = (3 + NDEC) * 32;              // A producer, MMA issuer, code producer, decoders
+constexpr long long WAIT_BUDGET = 4000000000LL;       // clock cycles (~2 s)
+constexpr uint32_t IDESC = sm100::idesc_bf16_f32(2 * 128, BN);   // pair MMA: M = 256 over two CTAs
+constexpr uint16_t PAIR = 0x3;                        // both CTAs of the cluster
+static_assert(OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
+static_assert(OFF_LUT % 128 == 0 && OFF_BAR % 8 == 0, "alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 __device__ int g_gemm_timeout = 0;
 
 struct Bars {
+  // full_a, full_b and acc_empty are used in the even CTA only (both CTAs arrive on them);
+  // the others are local to each CTA.
   uint32_t full_a, empty_a, full_b, empty_b, full_c, empty_c, lut_full, lut_empty, acc_full, acc_empty;
   __device__ Bars(uint32_t base)
       : full_a(base), empty_a(full_a + 8 * SA), full_b(empty_a + 8 * SA), empty_b(full_b + 8 * SB),
@@ -70,8 +88,38 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
 __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t ld_volatile_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
 
-__global__ void __launch_bounds__(THREADS, 1)
+// Bounded wait shared by all roles.  Gives up when the budget runs out or when the pair's abort
+// flag is set; a thread that runs out sets the flag in both CTAs so that the others stop at once.
+struct Waiter {
+  uint32_t abort_local, abort_peer;
+  __device__ bool wait(uint32_t bar, uint32_t parity, bool cluster_scope) const {
+    auto probe = [&] {
+      return cluster_scope ? sm100::mbar_try_wait_cluster(bar, parity) : sm100::mbar_try_wait(bar, parity);
+    };
+    if (probe()) return true;
+    const long long t0 = clock64();
+    while (!probe()) {
+      if (ld_volatile_u32(abort_local) != 0) return false;
+      if (clock64() - t0 > WAIT_BUDGET) {
+        sts32(abort_local, 1);
+        st_cluster_u32(abort_peer, 1);
+        return false;
+      }
+    }
+    return true;
+  }
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     benq_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
                      const uint16_t *__restrict__ lut, void *__restrict__ y, int ydt, int M, int N, int K) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -79,8 +127,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   const Bars bar(sbase + OFF_BAR);
   const uint32_t tmem_slot = sbase + OFF_TMEM;
+  const uint32_t rank = sm100::cluster_ctarank();        // 0: the even CTA, which issues the MMAs
+  const bool lead = rank == 0;
+  const Waiter wt{tmem_slot + 4, sm100::mapa_shared(tmem_slot + 4, rank ^ 1u)};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = (M + BM - 1) / BM, nt = N / BN, ntiles = mt * nt, nkb = K / BK;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int mt = (M + PM - 1) / PM, nt = N / BN, ntiles = mt * nt, nkb = K / BK;
   bool ok = true;
 
   if (threadIdx.x == 0) {
@@ -89,7 +141,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       sm100::mbar_init(bar.empty_a + 8 * s, 1);
     }
     for (int s = 0; s < SB; ++s) {
-      sm100::mbar_init(bar.full_b + 8 * s, NDEC);
+      sm100::mbar_init(bar.full_b + 8 * s, 2 * NDEC);
       sm100::mbar_init(bar.empty_b + 8 * s, 1);
     }
     for (int s = 0; s < SC; ++s) {
@@ -99,17 +151,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     sm100::mbar_init(bar.lut_full, 1);
     sm100::mbar_init(bar.lut_empty, NDEC);
     sm100::mbar_init(bar.acc_full, 1);
-    sm100::mbar_init(bar.acc_empty, NDEC);
+    sm100::mbar_init(bar.acc_empty, 2 * NDEC);
+    sts32(tmem_slot + 4, 0);
     sm100::fence_barrier_init();
     sm100::prefetch_tensormap(&map_x);
     sm100::prefetch_tensormap(&map_codes);
   }
   if (warp == 1) {
-    sm100::tmem_alloc(tmem_slot, 512);
-    sm100::tmem_relinquish();
+    __syncwarp();
+    sm100::tmem_alloc_pair(tmem_slot, 512);
+    sm100::tmem_relinquish_pair();
   }
   sm100::tc_fence_before();
-  __syncthreads();
+  sm100::cluster_sync();   // both CTAs' barriers initialised and tensor memory allocated
   sm100::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem_raw + (tmem_slot - raw));
   // codes and tables are weights: their producer starts at once; activations are read and y is
@@ -117,54 +171,56 @@ __global__ void __launch_bounds__(THREADS, 1)
   qld::pdl_trigger();
 
   if (warp == 0) {
-    // ------------------------------------------------------------ activation producer (TMA)
+    // ------------------------------------------------------------ activation producer (tensor copies)
     if (lane == 0) {
       qld::pdl_wait();
+      const uint32_t lead_full_a = sm100::mapa_shared(bar.full_a, 0);
       int it = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const int m0 = (t % mt) * BM;
+      for (int t = pair; t < ntiles && ok; t += npairs) {
+        const int m0 = (t % mt) * PM + (int)rank * BM;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % SA;
-          if (it >= SA && !sm100::mbar_wait(bar.empty_a + 8 * s, ((it / SA) & 1) ^ 1, WAIT_BUDGET)) {
+          if (it >= SA && !wt.wait(bar.empty_a + 8 * s, ((it / SA) & 1) ^ 1, true)) {
             ok = false;
             break;
           }
-          sm100::mbar_arrive_expect_tx(bar.full_a + 8 * s, A_BYTES);
-          sm100::tma_load_2d(sbase + OFF_A + s * A_BYTES, &map_x, kb * BK, m0, bar.full_a + 8 * s);
+          if (lead) sm100::mbar_arrive_expect_tx(bar.full_a + 8 * s, 2 * A_BYTES);
+          sm100::tma_load_2d_pair(sbase + OFF_A + s * A_BYTES, &map_x, kb * BK, m0, lead_full_a + 8 * s);
         }
       }
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------------ code and table producer (TMA)
+    // ------------------------------------------------------------ code and table producer (local)
     if (lane == 0) {
-      int it = 0, tl = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tl) {
-        const int n0 = (t / mt) * BN;
-        if (tl > 0 && !sm100::mbar_wait(bar.lut_empty, (tl - 1) & 1, WAIT_BUDGET)) { ok = false; break; }
+      const int ncs = (nkb + CKB - 1) / CKB;   // code stages per tile; a ragged last one reads zeros
+      int ic = 0, tl = 0;
+      for (int t = pair; t < ntiles && ok; t += npairs, ++tl) {
+        const int n0 = (t / mt) * BN + (int)rank * BNH;
+        if (tl > 0 && !wt.wait(bar.lut_empty, (tl - 1) & 1, false)) { ok = false; break; }
         sm100::mbar_arrive_expect_tx(bar.lut_full, LUT_BYTES);
         sm100::bulk_g2s(sbase + OFF_LUT, lut + (size_t)n0 * 64, LUT_BYTES, bar.lut_full);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % SC;
-          if (it >= SC && !sm100::mbar_wait(bar.empty_c + 8 * s, ((it / SC) & 1) ^ 1, WAIT_BUDGET)) {
+        for (int cs = 0; cs < ncs; ++cs, ++ic) {
+          const int s = ic % SC;
+          if (ic >= SC && !wt.wait(bar.empty_c + 8 * s, ((ic / SC) & 1) ^ 1, false)) {
             ok = false;
             break;
           }
           sm100::mbar_arrive_expect_tx(bar.full_c + 8 * s, C_BYTES);
-          sm100::tma_load_2d(sbase + OFF_C + s * C_BYTES, &map_codes, kb * C_ROW, n0, bar.full_c + 8 * s);
+          sm100::tma_load_2d(sbase + OFF_C + s * C_BYTES, &map_codes, cs * C_SROW, n0, bar.full_c + 8 * s);
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ pair MMA issuer (even CTA)
+    if (lead && lane == 0) {
       int it = 0, tl = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tl) {
-        if (tl > 0 && !sm100::mbar_wait(bar.acc_empty, (tl - 1) & 1, WAIT_BUDGET)) { ok = false; break; }
+      for (int t = pair; t < ntiles && ok; t += npairs, ++tl) {
+        if (tl > 0 && !wt.wait(bar.acc_empty, (tl - 1) & 1, true)) { ok = false; break; }
         sm100::tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int sa = it % SA, sb = it % SB;
-          if (!sm100::mbar_wait(bar.full_a + 8 * sa, (it / SA) & 1, WAIT_BUDGET) ||
-              !sm100::mbar_wait(bar.full_b + 8 * sb, (it / SB) & 1, WAIT_BUDGET)) {
+          if (!wt.wait(bar.full_a + 8 * sa, (it / SA) & 1, true) ||
+              !wt.wait(bar.full_b + 8 * sb, (it / SB) & 1, true)) {
             ok = false;
             break;
           }
@@ -176,14 +232,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint64_t adesc = sm100::sw128_kmajor_desc(a + h * (A_BYTES / 2) + kk * 32);
-              sm100::mma_bf16(tmem + h * BN, adesc, bdesc, IDESC, (kb | kk) ? 1u : 0u);
+              sm100::mma_bf16_pair(tmem + h * BN, adesc, bdesc, IDESC, (kb | kk) ? 1u : 0u);
             }
           }
-          sm100::mma_commit(bar.empty_a + 8 * sa);
-          sm100::mma_commit(bar.empty_b + 8 * sb);
+          sm100::mma_commit_pair(bar.empty_a + 8 * sa, PAIR);
+          sm100::mma_commit_pair(bar.empty_b + 8 * sb, PAIR);
         }
         if (!ok) break;
-        sm100::mma_commit(bar.acc_full);
+        sm100::mma_commit_pair(bar.acc_full, PAIR);
       }
     }
   } else {
@@ -191,49 +247,59 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int dw = warp - 3;            // decoder index 0 .. NDEC-1
     const int q = warp & 3;             // tensor-memory lane quarter this warp may read
     const int ch = dw >> 2;             // which NDEC/4-th of the 256 accumulator columns it drains
-    int it = 0, tl = 0;
+    const uint32_t lead_full_b = sm100::mapa_shared(bar.full_b, 0);
+    const uint32_t lead_acc_empty = sm100::mapa_shared(bar.acc_empty, 0);
+    int it = 0, tl = 0, ic = 0;
     // lane l expands codes 2l, 2l+1 of a row's 64-code block: bits [12l, 12l+12) of its 48 bytes
     const int wq = (12 * lane) >> 5, wsh = (12 * lane) & 31;
     const int chunk = lane >> 2, inner = (lane & 3) * 4;
     // swizzled position of codes 2*lane, 2*lane+1 within row r = dw (mod 8) of a K block
     const uint32_t dst_lane = (dw >> 3) * 1024 + (dw & 7) * 128 + ((chunk ^ (dw & 7)) << 4) + inner;
-    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tl) {
-      const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
-      if (!sm100::mbar_wait(bar.lut_full, tl & 1, WAIT_BUDGET)) { ok = false; break; }
+    for (int t = pair; t < ntiles && ok; t += npairs, ++tl) {
+      const int m0 = (t % mt) * PM + (int)rank * BM, n0 = (t / mt) * BN;
+      if (!wt.wait(bar.lut_full, tl & 1, false)) { ok = false; break; }
       for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int sb = it % SB, sc = it % SC;
-        if ((it >= SB && !sm100::mbar_wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, WAIT_BUDGET)) ||
-            !sm100::mbar_wait(bar.full_c + 8 * sc, (it / SC) & 1, WAIT_BUDGET)) {
+        const int sb = it % SB, sc = ic % SC, sub = kb % CKB;
+        if ((it >= SB && !wt.wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, true)) ||
+            (sub == 0 && !wt.wait(bar.full_c + 8 * sc, (ic / SC) & 1, false))) {
           ok = false;
           break;
         }
         // rows r = dw + NDEC*i: r & 7 == dw & 7 is fixed per warp, so every address below is
-        // a per-warp base plus a compile-time multiple of the row step
-        const uint32_t cb = sbase + OFF_C + sc * C_BYTES + dw * C_ROW + 4 * wq;
+        // a per-warp base plus a compile-time multiple of the row step.  All code words of the
+        // warp's rows are loaded before the first lookup.
+        const uint32_t cb = sbase + OFF_C + sc * C_BYTES + dw * C_SROW + sub * C_ROW + 4 * wq;
         const uint32_t bb = sbase + OFF_B + sb * B_BYTES + dst_lane;
         const uint32_t tb = sbase + OFF_LUT + dw * 128;
-#pragma unroll 4
-        for (int i = 0; i < BN / NDEC; ++i) {
-          const uint32_t w0 = lds32(cb + i * NDEC * C_ROW);
-          const uint32_t w1 = lds32(cb + i * NDEC * C_ROW + 4);   // may read the next row: unused bits
-          const uint32_t v = __funnelshift_r(w0, w1, wsh);
+        constexpr int RPW = BNH / NDEC;   // rows per decoder warp per K block
+        uint32_t v[RPW];
+#pragma unroll
+        for (int i = 0; i < RPW; ++i) {
+          const uint32_t w0 = lds32(cb + i * NDEC * C_SROW);
+          const uint32_t w1 = lds32(cb + i * NDEC * C_SROW + 4);   // may read past the row: unused bits
+          v[i] = __funnelshift_r(w0, w1, wsh);
+        }
+#pragma unroll
+        for (int i = 0; i < RPW; ++i) {
           const uint32_t tbl = tb + i * NDEC * 128;
-          const uint32_t e0 = lds_u16(((v << 1) & 0x7Eu) | tbl);
-          const uint32_t e1 = lds_u16(((v >> 5) & 0x7Eu) | tbl);
+          const uint32_t e0 = lds_u16(((v[i] << 1) & 0x7Eu) | tbl);
+          const uint32_t e1 = lds_u16(((v[i] >> 5) & 0x7Eu) | tbl);
           sts32(bb + i * (NDEC / 8) * 1024, __byte_perm(e0, e1, 0x5410));
         }
         sm100::fence_proxy_async_smem();
         __syncwarp();
+        const bool stage_done = sub == CKB - 1 || kb == nkb - 1;
         if (lane == 0) {
-          sm100::mbar_arrive(bar.full_b + 8 * sb);
-          sm100::mbar_arrive(bar.empty_c + 8 * sc);
+          sm100::mbar_arrive_cluster(lead_full_b + 8 * sb);
+          if (stage_done) sm100::mbar_arrive(bar.empty_c + 8 * sc);
         }
+        if (stage_done) ++ic;
       }
       if (!ok) break;
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(bar.lut_empty);
       // epilogue: this warp drains lanes [32q, 32q+32) of both 128-row accumulators
-      if (!sm100::mbar_wait(bar.acc_full, tl & 1, WAIT_BUDGET)) { ok = false; break; }
+      if (!wt.wait(bar.acc_full, tl & 1, true)) { ok = false; break; }
       qld::pdl_wait();
       sm100::tc_fence_after();
 #pragma unroll 1
@@ -268,16 +334,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(bar.acc_empty);
+      if (lane == 0) sm100::mbar_arrive_cluster(lead_acc_empty);
     }
   }
 
   if (!ok) atomicExch(&g_gemm_timeout, 1);
+  // neither CTA leaves while its peer may still arrive on its barriers, read its shared memory
+  // through a pair MMA or write its tensor memory
   sm100::tc_fence_before();
-  __syncthreads();
+  sm100::cluster_sync();
   if (warp == 1) {
+    __syncwarp();
     sm100::tc_fence_after();
-    sm100::tmem_dealloc(tmem, 512);
+    sm100::tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -297,6 +366,28 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   });
   return fn;
+}
+
+// CTA pairs that can be resident at once on the current device (cached per device).
+int resident_pairs() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (ql::sm_count() / 2));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, benq_gemm_kernel, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = ql::sm_count() / 2;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
 }
 
 }  // namespace
@@ -323,7 +414,7 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
     const cuuint64_t rowbytes = (cuuint64_t)K * 3 / 4;
     const cuuint64_t dims[2] = {rowbytes, (cuuint64_t)N};
     const cuuint64_t strides[1] = {rowbytes};
-    const cuuint32_t box[2] = {C_ROW, BN};
+    const cuuint32_t box[2] = {C_SROW, BNH};
     const cuuint32_t es[2] = {1, 1};
     if (enc(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -336,9 +427,9 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
     attr_err = cudaFuncSetAttribute(benq_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return fail(QL_ERR_CUDA, "benq_linear: cannot reserve GEMM shared memory");
-  const int ntiles = ((M + BM - 1) / BM) * (N / BN);
-  const int grid = std::min(ntiles, sm_count());
-  launch(benq_gemm_kernel, grid, THREADS, SMEM_BYTES, s, mx, mc, lut, y, (int)ydt, M, N, K);
+  const int ntiles = ((M + PM - 1) / PM) * (N / BN);
+  const int pairs = std::min(ntiles, resident_pairs());
+  launch(benq_gemm_kernel, 2 * pairs, THREADS, SMEM_BYTES, s, mx, mc, lut, y, (int)ydt, M, N, K);
   return launch_status("benq_linear (tensor-core GEMM)");
 }
 
