@@ -140,7 +140,9 @@ class Workload:
             x_h = synth.activations(B, K, seed=seed + 500)
             x = bf16(x_h)
             y = torch.empty(B, N, dtype=out_dtype, device=cuda)
-            return dict(kind="benq", N=N, K=K, B=B, codes=[codes], lut=[lut], x=x, x_h=x_h, y=y,
+            nws = ql.benq_linear_workspace_bytes(B, N, K)
+            ws = torch.empty(nws, dtype=torch.uint8, device=cuda) if nws else None
+            return dict(kind="benq", N=N, K=K, B=B, codes=[codes], lut=[lut], x=x, x_h=x_h, y=y, ws=ws,
                         wbytes=codes.numel() + lut.numel() * 2, label=label or f"benq_{K}x{N}_b{B}")
 
         def mdbf_layer(n, m, B, seed, label=None):
@@ -206,7 +208,7 @@ class Workload:
     def run_layer(self, L, c):
         ql = self.ql
         if L["kind"] == "benq":
-            ql.benq_linear(L["codes"][c], L["lut"][c], L["x"], L["y"])
+            ql.benq_linear(L["codes"][c], L["lut"][c], L["x"], L["y"], workspace=L["ws"])
         else:
             ql.mdbf_linear(L["paths"][c], L["n"], L["m"], MLP_R, MLP_L, L["x"], L["y"], L["ws"])
 

@@ -88,6 +88,31 @@ QL_API ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const ui
                       ql_out_dtype y_dtype, int B, int N, int K, ql_stream_t stream);
 
 /*
+ * benq_linear_ws -- benq_linear with a caller workspace for the GEMM's last
+ *   wave.  No counterpart in the pages: this is scheduling.  The GEMM runs whole
+ *   output tiles in waves over the SM pairs; when the last wave would leave at
+ *   least half of them idle, it splits each of its tiles into up to 8 K ranges,
+ *   writes fp32 partials to `workspace` and sums them in a fixed order (results
+ *   are deterministic and, for a given device, independent of the stream).
+ *   Results equal benq_linear's up to fp32 summation order.
+ *
+ *   workspace  device, 256-byte aligned, ws_bytes >= benq_linear_workspace_bytes
+ *              (B, N, K) to enable the split; NULL with ws_bytes == 0 runs exactly
+ *              benq_linear.  A smaller non-NULL workspace also runs without the
+ *              split.  Owned by the caller; must not be used by another call
+ *              running at the same time.  Other arguments as benq_linear.
+ *   Errors: QL_ERR_INVALID_ARG if only one of workspace / ws_bytes is set,
+ *   QL_ERR_ALIGNMENT if the workspace is not 256-byte aligned.
+ */
+QL_API ql_status benq_linear_ws(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
+                                ql_out_dtype y_dtype, int B, int N, int K, void *workspace, size_t ws_bytes,
+                                ql_stream_t stream);
+
+/* Workspace bytes benq_linear_ws uses for these sizes on the current device
+ * (0 when B <= 16 or when no split applies).  Needs a CUDA device. */
+QL_API size_t benq_linear_workspace_bytes(int B, int N, int K);
+
+/*
  * benq_dequant_debug -- W[n][k] = lut[n][code(n,k)] as bf16 bits, row-major
  *   [N][K].  Bit-exact by construction; meant for checking, not speed.
  *   Same codes / lut layout as benq_linear; K % 4 == 0.

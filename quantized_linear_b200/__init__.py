@@ -34,6 +34,8 @@ class MDBFPathC(ctypes.Structure):
 
 _SIGNATURES = {
     "benq_linear": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "benq_linear_ws": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "benq_linear_workspace_bytes": (_sz, [_i, _i, _i]),
     "benq_dequant_debug": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
     "benq_bits_per_weight": (_d, [_i]),
     "mdbf_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -67,7 +69,7 @@ def lib() -> ctypes.CDLL:
 def _c(name):
     return getattr(lib(), name)
 
-EXPORTS = ["benq_linear", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
+EXPORTS = ["benq_linear", "benq_linear_ws", "benq_linear_workspace_bytes", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
            "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
            "mdbf_select_rank", "ql_last_error", "ql_check", "ql_set_pdl"]
 
@@ -114,11 +116,13 @@ def _ydt(y):
 
 # ----------------------------------------------------------------------------------------------- BenQ
 
-def benq_linear(codes, lut, x, y, stream=None):
+def benq_linear(codes, lut, x, y, stream=None, workspace=None):
     """y[B, N] = x[B, K] @ W^T with W[n, k] = lut[n, code(n, k)].
 
     codes uint8 [N, 3K/4]; lut bf16 (or int16 bit patterns) [N, 64]; x bf16 [B, K];
-    y float32 or bf16 [B, N] (overwritten)."""
+    y float32 or bf16 [B, N] (overwritten).  With a uint8 device `workspace` of at least
+    benq_linear_workspace_bytes(B, N, K) bytes the GEMM splits its last wave along K
+    (benq_linear_ws)."""
     N = codes.shape[0]
     B, K = x.shape
     _want(codes, torch.uint8, "codes")
@@ -129,8 +133,18 @@ def benq_linear(codes, lut, x, y, stream=None):
     _want(x, torch.bfloat16, "x")
     if tuple(y.shape) != (B, N) or not y.is_contiguous():
         raise ValueError("y must be contiguous [B, N]")
-    _check(_c("benq_linear")(_ptr(codes), _ptr(lut), _ptr(x), _ptr(y), _ydt(y), B, N, K, _stream(stream)))
+    if workspace is None:
+        _check(_c("benq_linear")(_ptr(codes), _ptr(lut), _ptr(x), _ptr(y), _ydt(y), B, N, K, _stream(stream)))
+    else:
+        nbytes = workspace.numel() * workspace.element_size()
+        _check(_c("benq_linear_ws")(_ptr(codes), _ptr(lut), _ptr(x), _ptr(y), _ydt(y), B, N, K, _ptr(workspace),
+                                    nbytes, _stream(stream)))
     return y
+
+
+def benq_linear_workspace_bytes(B: int, N: int, K: int) -> int:
+    """Bytes of workspace the GEMM's split last wave uses for these sizes on the current device."""
+    return int(_c("benq_linear_workspace_bytes")(B, N, K))
 
 
 def benq_dequant_debug(codes, lut, W, stream=None):

@@ -63,10 +63,23 @@ const char *ql_last_error(void) { return g_msg; }
 
 int ql_set_pdl(int enable) { return g_pdl.exchange(enable ? 1 : 0); }
 
+size_t benq_linear_workspace_bytes(int B, int N, int K) {
+  if (B <= 16) return 0;
+  return ql::benq_gemm_workspace_size(B, N, K);
+}
+
 ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype y_dtype,
                       int B, int N, int K, ql_stream_t stream) {
+  return benq_linear_ws(codes, lut, x, y, y_dtype, B, N, K, nullptr, 0, stream);
+}
+
+ql_status benq_linear_ws(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype y_dtype,
+                         int B, int N, int K, void *workspace, size_t ws_bytes, ql_stream_t stream) {
   g_msg[0] = 0;
   if (!codes || !lut || !x || !y) return fail(QL_ERR_INVALID_ARG, "benq_linear: null pointer");
+  if ((workspace == nullptr) != (ws_bytes == 0))
+    return fail(QL_ERR_INVALID_ARG, "benq_linear_ws: workspace and ws_bytes must both be set or both be empty");
+  if (workspace && !aligned(workspace, 256)) return fail(QL_ERR_ALIGNMENT, "benq_linear_ws: workspace must be 256-byte aligned");
   if (B <= 0 || N <= 0 || K <= 0) return fail(QL_ERR_INVALID_ARG, "benq_linear: B, N, K must be positive");
   if (K % 4) return fail(QL_ERR_INVALID_ARG, "benq_linear: K = %d is not a multiple of 4", K);
   if (y_dtype != QL_OUT_F32 && y_dtype != QL_OUT_BF16) return fail(QL_ERR_INVALID_ARG, "benq_linear: bad y_dtype");
@@ -76,7 +89,7 @@ ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t 
   if (B <= 16) return ql::benq_gemv_launch(codes, lut, x, y, y_dtype, B, N, K, s);
   if (K % 64 || N % 256)
     return fail(QL_ERR_UNSUPPORTED, "benq_linear: batch %d > 16 needs K %% 64 == 0 and N %% 256 == 0", B);
-  return ql::benq_gemm_launch(codes, lut, x, y, y_dtype, B, N, K, s);
+  return ql::benq_gemm_launch(codes, lut, x, y, y_dtype, B, N, K, workspace, ws_bytes, s);
 }
 
 ql_status benq_dequant_debug(const uint8_t *codes, const uint16_t *lut, uint16_t *W, int N, int K,

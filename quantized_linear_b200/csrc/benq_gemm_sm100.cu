@@ -51,8 +51,8 @@ constexpr int OFF_B = OFF_A + SA * A_BYTES;
 constexpr int OFF_C = OFF_B + SB * B_BYTES;
 constexpr int OFF_LUT = OFF_C + SC * C_BYTES + 128;   // 128 bytes of slack: the last row's second code word
 constexpr int OFF_BAR = OFF_LUT + LUT_BYTES;
-constexpr int NBAR = 2 * (SA + SB + SC) + 4;
-constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;          // tensor-memory address, then the abort flag
+constexpr int NBAR = 2 * (SA + SB + SC) + 6;
+constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;          // tensor-memory address, abort flag, last-part flag
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;      // + alignment slack
 constexpr int NDEC = 16;                              // decoder / epilogue warps (multiple of 8)
 constexpr int THREADS = (3 + NDEC) * 32;              // A producer, MMA issuer, code producer, decoders
@@ -68,11 +68,12 @@ __device__ int g_gemm_timeout = 0;
 struct Bars {
   // full_a, full_b and acc_empty are used in the even CTA only (both CTAs arrive on them);
   // the others are local to each CTA.
-  uint32_t full_a, empty_a, full_b, empty_b, full_c, empty_c, lut_full, lut_empty, acc_full, acc_empty;
+  uint32_t full_a, empty_a, full_b, empty_b, full_c, empty_c, lut_full, lut_empty, acc_full, acc_empty, split_done,
+      split_go;
   __device__ Bars(uint32_t base)
       : full_a(base), empty_a(full_a + 8 * SA), full_b(empty_a + 8 * SA), empty_b(full_b + 8 * SB),
         full_c(empty_b + 8 * SB), empty_c(full_c + 8 * SC), lut_full(empty_c + 8 * SC), lut_empty(lut_full + 8),
-        acc_full(lut_empty + 8), acc_empty(acc_full + 8) {}
+        acc_full(lut_empty + 8), acc_empty(acc_full + 8), split_done(acc_empty + 8), split_go(split_done + 8) {}
 };
 
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
@@ -119,9 +120,22 @@ struct Waiter {
   }
 };
 
+// Work items: pair tiles 0 .. full-1 whole, then each of the remaining tiles (the last, partial
+// wave) split into `parts` K ranges so that the otherwise idle pairs share it.  A split item
+// writes an fp32 partial; the last CTA to finish a tile sums the partials in part order.
+struct Item {
+  int tile, kb0, kb1, part;   // part < 0: whole tile
+};
+__device__ __forceinline__ Item item_of(int i, int full, int parts, int nkb) {
+  if (i < full) return {i, 0, nkb, -1};
+  const int u = i - full, j = u / parts, q = u - j * parts;
+  return {full + j, (int)((int64_t)q * nkb / parts), (int)((int64_t)(q + 1) * nkb / parts), q};
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     benq_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
-                     const uint16_t *__restrict__ lut, void *__restrict__ y, int ydt, int M, int N, int K) {
+                     const uint16_t *__restrict__ lut, void *__restrict__ y, int ydt, int M, int N, int K,
+                     float *__restrict__ part_ws, unsigned *__restrict__ part_cnt, int full, int parts) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -133,6 +147,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int mt = (M + PM - 1) / PM, nt = N / BN, ntiles = mt * nt, nkb = K / BK;
+  const int nitems = full + (ntiles - full) * parts;
   bool ok = true;
 
   if (threadIdx.x == 0) {
@@ -152,6 +167,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     sm100::mbar_init(bar.lut_empty, NDEC);
     sm100::mbar_init(bar.acc_full, 1);
     sm100::mbar_init(bar.acc_empty, 2 * NDEC);
+    sm100::mbar_init(bar.split_done, NDEC);
+    sm100::mbar_init(bar.split_go, 1);
     sts32(tmem_slot + 4, 0);
     sm100::fence_barrier_init();
     sm100::prefetch_tensormap(&map_x);
@@ -176,9 +193,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       qld::pdl_wait();
       const uint32_t lead_full_a = sm100::mapa_shared(bar.full_a, 0);
       int it = 0;
-      for (int t = pair; t < ntiles && ok; t += npairs) {
-        const int m0 = (t % mt) * PM + (int)rank * BM;
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+      for (int wi = pair; wi < nitems && ok; wi += npairs) {
+        const Item w = item_of(wi, full, parts, nkb);
+        const int m0 = (w.tile % mt) * PM + (int)rank * BM;
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % SA;
           if (it >= SA && !wt.wait(bar.empty_a + 8 * s, ((it / SA) & 1) ^ 1, true)) {
             ok = false;
@@ -192,10 +210,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ code and table producer (local)
     if (lane == 0) {
-      const int ncs = (nkb + CKB - 1) / CKB;   // code stages per tile; a ragged last one reads zeros
       int ic = 0, tl = 0;
-      for (int t = pair; t < ntiles && ok; t += npairs, ++tl) {
-        const int n0 = (t / mt) * BN + (int)rank * BNH;
+      for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
+        const Item w = item_of(wi, full, parts, nkb);
+        const int n0 = (w.tile / mt) * BN + (int)rank * BNH;
+        const int ncs = (w.kb1 - w.kb0 + CKB - 1) / CKB;   // code stages; a ragged last one reads zeros
         if (tl > 0 && !wt.wait(bar.lut_empty, (tl - 1) & 1, false)) { ok = false; break; }
         sm100::mbar_arrive_expect_tx(bar.lut_full, LUT_BYTES);
         sm100::bulk_g2s(sbase + OFF_LUT, lut + (size_t)n0 * 64, LUT_BYTES, bar.lut_full);
@@ -206,7 +225,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             break;
           }
           sm100::mbar_arrive_expect_tx(bar.full_c + 8 * s, C_BYTES);
-          sm100::tma_load_2d(sbase + OFF_C + s * C_BYTES, &map_codes, cs * C_SROW, n0, bar.full_c + 8 * s);
+          sm100::tma_load_2d(sbase + OFF_C + s * C_BYTES, &map_codes, (w.kb0 + cs * CKB) * C_ROW, n0,
+                             bar.full_c + 8 * s);
         }
       }
     }
@@ -214,10 +234,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ pair MMA issuer (even CTA)
     if (lead && lane == 0) {
       int it = 0, tl = 0;
-      for (int t = pair; t < ntiles && ok; t += npairs, ++tl) {
+      for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
+        const Item w = item_of(wi, full, parts, nkb);
         if (tl > 0 && !wt.wait(bar.acc_empty, (tl - 1) & 1, true)) { ok = false; break; }
         sm100::tc_fence_after();
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int sa = it % SA, sb = it % SB;
           if (!wt.wait(bar.full_a + 8 * sa, (it / SA) & 1, true) ||
               !wt.wait(bar.full_b + 8 * sb, (it / SB) & 1, true)) {
@@ -232,7 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint64_t adesc = sm100::sw128_kmajor_desc(a + h * (A_BYTES / 2) + kk * 32);
-              sm100::mma_bf16_pair(tmem + h * BN, adesc, bdesc, IDESC, (kb | kk) ? 1u : 0u);
+              sm100::mma_bf16_pair(tmem + h * BN, adesc, bdesc, IDESC, (kb > w.kb0 || kk > 0) ? 1u : 0u);
             }
           }
           sm100::mma_commit_pair(bar.empty_a + 8 * sa, PAIR);
@@ -249,17 +270,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int ch = dw >> 2;             // which NDEC/4-th of the 256 accumulator columns it drains
     const uint32_t lead_full_b = sm100::mapa_shared(bar.full_b, 0);
     const uint32_t lead_acc_empty = sm100::mapa_shared(bar.acc_empty, 0);
-    int it = 0, tl = 0, ic = 0;
+    int it = 0, tl = 0, ic = 0, ns = 0;
     // lane l expands codes 2l, 2l+1 of a row's 64-code block: bits [12l, 12l+12) of its 48 bytes
     const int wq = (12 * lane) >> 5, wsh = (12 * lane) & 31;
     const int chunk = lane >> 2, inner = (lane & 3) * 4;
     // swizzled position of codes 2*lane, 2*lane+1 within row r = dw (mod 8) of a K block
     const uint32_t dst_lane = (dw >> 3) * 1024 + (dw & 7) * 128 + ((chunk ^ (dw & 7)) << 4) + inner;
-    for (int t = pair; t < ntiles && ok; t += npairs, ++tl) {
-      const int m0 = (t % mt) * PM + (int)rank * BM, n0 = (t / mt) * BN;
+    for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
+      const Item w = item_of(wi, full, parts, nkb);
+      const int m0 = (w.tile % mt) * PM + (int)rank * BM, n0 = (w.tile / mt) * BN;
       if (!wt.wait(bar.lut_full, tl & 1, false)) { ok = false; break; }
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int sb = it % SB, sc = ic % SC, sub = kb % CKB;
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+        const int sb = it % SB, sc = ic % SC, sub = (kb - w.kb0) % CKB;
         if ((it >= SB && !wt.wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, true)) ||
             (sub == 0 && !wt.wait(bar.full_c + 8 * sc, (ic / SC) & 1, false))) {
           ok = false;
@@ -288,7 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         sm100::fence_proxy_async_smem();
         __syncwarp();
-        const bool stage_done = sub == CKB - 1 || kb == nkb - 1;
+        const bool stage_done = sub == CKB - 1 || kb == w.kb1 - 1;
         if (lane == 0) {
           sm100::mbar_arrive_cluster(lead_full_b + 8 * sb);
           if (stage_done) sm100::mbar_arrive(bar.empty_c + 8 * sc);
@@ -302,15 +324,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (!wt.wait(bar.acc_full, tl & 1, true)) { ok = false; break; }
       qld::pdl_wait();
       sm100::tc_fence_after();
+      const bool split = w.part >= 0;
+      // fp32 partials of a split tile: [tile - full][part][rank][BM rows][BN columns]
+      float *const slot =
+          split ? part_ws + ((size_t)((w.tile - full) * parts + w.part) * 2 + rank) * (size_t)(BM * BN) : nullptr;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        const int row = m0 + h * 128 + 32 * q + lane;
+        const int lr = h * 128 + 32 * q + lane, row = m0 + lr;
 #pragma unroll 1
         for (int c = ch * (BN / 32) / (NDEC / 4); c < (ch + 1) * (BN / 32) / (NDEC / 4); ++c) {
           uint32_t v[32];
           sm100::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + h * BN + c * 32, v);
           sm100::tmem_wait_ld();
-          if (row < M) {
+          if (split) {
+            float4 *dst = reinterpret_cast<float4 *>(slot + (size_t)lr * BN + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          } else if (row < M) {
             if (ydt == QL_OUT_F32) {
               float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(y) + (size_t)row * N + n0 + c * 32);
 #pragma unroll
@@ -335,6 +367,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive_cluster(lead_acc_empty);
+      if (split) {
+        // The last of the tile's parts to finish (per CTA half) sums all parts in part order.
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(bar.split_done);
+        const uint32_t last_flag = tmem_slot + 8;
+        if (dw == 0) {
+          if (!wt.wait(bar.split_done, ns & 1, false)) { ok = false; break; }
+          if (lane == 0) {
+            __threadfence();
+            unsigned *cnt = part_cnt + (w.tile - full) * 2 + rank;
+            const bool last = atomicAdd(cnt, 1u) == (unsigned)parts - 1;
+            if (last) {
+              atomicExch(cnt, 0u);   // ready for the next call
+              __threadfence();
+            }
+            sts32(last_flag, last ? 1u : 0u);
+            sm100::mbar_arrive(bar.split_go);
+          }
+          __syncwarp();
+        }
+        if (!wt.wait(bar.split_go, ns & 1, false)) { ok = false; break; }
+        ++ns;
+        if (lds32(last_flag)) {
+          const float *p0 = part_ws + ((size_t)(w.tile - full) * parts * 2 + rank) * (size_t)(BM * BN);
+          const size_t pstride = (size_t)2 * BM * BN;
+          for (int e = (dw * 32 + lane) * 4; e < BM * BN; e += NDEC * 32 * 4) {
+            const int row = m0 + e / BN, col = n0 + e % BN;
+            float4 a = __ldcg(reinterpret_cast<const float4 *>(p0 + e));
+            for (int pq = 1; pq < parts; ++pq) {
+              const float4 b = __ldcg(reinterpret_cast<const float4 *>(p0 + pq * pstride + e));
+              a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+            }
+            if (row >= M) continue;
+            if (ydt == QL_OUT_F32) {
+              *reinterpret_cast<float4 *>(static_cast<float *>(y) + (size_t)row * N + col) = a;
+            } else {
+              const uint32_t lo = uint32_t(qld::f32_to_bf16_rn(a.x)) | (uint32_t(qld::f32_to_bf16_rn(a.y)) << 16);
+              const uint32_t hi = uint32_t(qld::f32_to_bf16_rn(a.z)) | (uint32_t(qld::f32_to_bf16_rn(a.w)) << 16);
+              *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(y) + (size_t)row * N + col) = make_uint2(lo, hi);
+            }
+          }
+        }
+      }
     }
   }
 
@@ -390,12 +466,43 @@ int resident_pairs() {
   return cache[dev];
 }
 
+constexpr int SPLIT_MAX = 8;   // K ranges per tile of the last wave
+
+// Whole tiles run in full waves of `pairs` CTA pairs; when the last wave would leave at least
+// half of the pairs idle, its L tiles are split into `parts` K ranges each (L * parts <= pairs).
+struct SplitPlan {
+  int full, parts, leftover;
+  size_t partial_bytes, counter_bytes;
+};
+SplitPlan split_plan(int M, int N, int K, int pairs) {
+  const int ntiles = ((M + PM - 1) / PM) * (N / BN), nkb = K / BK;
+  SplitPlan p{ntiles, 1, 0, 0, 0};
+  const int full = (ntiles / pairs) * pairs, left = ntiles - full;
+  if (left > 0 && 2 * left <= pairs) {
+    const int parts = std::min(std::min(pairs / left, SPLIT_MAX), nkb);
+    if (parts >= 2) {
+      p.full = full;
+      p.parts = parts;
+      p.leftover = left;
+      p.partial_bytes = (size_t)left * parts * 2 * BM * BN * sizeof(float);
+      p.counter_bytes = ((size_t)left * 2 * sizeof(unsigned) + 255) / 256 * 256;
+    }
+  }
+  return p;
+}
+
 }  // namespace
 
 namespace ql {
 
+size_t benq_gemm_workspace_size(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0 || N % BN || K % BK) return 0;
+  const SplitPlan p = split_plan(M, N, K, resident_pairs());
+  return p.partial_bytes + p.counter_bytes;
+}
+
 ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype ydt,
-                           int M, int N, int K, cudaStream_t s) {
+                           int M, int N, int K, void *ws, size_t ws_bytes, cudaStream_t s) {
   if (N % BN || K % BK) return fail(QL_ERR_UNSUPPORTED, "benq_linear: batch > 16 needs N %% 256 == 0 and K %% 64 == 0");
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(QL_ERR_CUDA, "benq_linear: cuTensorMapEncodeTiled is unavailable");
@@ -428,8 +535,22 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
   });
   if (attr_err != cudaSuccess) return fail(QL_ERR_CUDA, "benq_linear: cannot reserve GEMM shared memory");
   const int ntiles = ((M + PM - 1) / PM) * (N / BN);
-  const int pairs = std::min(ntiles, resident_pairs());
-  launch(benq_gemm_kernel, 2 * pairs, THREADS, SMEM_BYTES, s, mx, mc, lut, y, (int)ydt, M, N, K);
+  const int resident = resident_pairs();
+  SplitPlan plan = split_plan(M, N, K, resident);
+  float *part_ws = nullptr;
+  unsigned *part_cnt = nullptr;
+  if (plan.parts > 1 && ws != nullptr && ws_bytes >= plan.partial_bytes + plan.counter_bytes) {
+    part_ws = static_cast<float *>(ws);
+    part_cnt = reinterpret_cast<unsigned *>(static_cast<char *>(ws) + plan.partial_bytes);
+    if (cudaMemsetAsync(part_cnt, 0, plan.counter_bytes, s) != cudaSuccess)
+      return fail(QL_ERR_CUDA, "benq_linear: cannot clear the split-tile counters");
+  } else {
+    plan = SplitPlan{ntiles, 1, 0, 0, 0};   // no (or too small a) workspace: whole tiles only
+  }
+  const int nitems = plan.full + plan.leftover * plan.parts;
+  const int pairs = std::min(nitems, resident);
+  launch(benq_gemm_kernel, 2 * pairs, THREADS, SMEM_BYTES, s, mx, mc, lut, y, (int)ydt, M, N, K, part_ws, part_cnt,
+         plan.full, plan.parts);
   return launch_status("benq_linear (tensor-core GEMM)");
 }
 

@@ -138,3 +138,72 @@ def test_gemm_prefill_shapes_sampled_columns(ql, N, K):
     ref = ob.linear(w.codes, w.lut, x, K, rows=cols)
     assert max_rel(y32[:, cols], ref) <= BENQ_TOL
     assert np.array_equal(yb, f32_to_bf16_rne(y32))
+
+
+def _linear_ws(ql, w, xbits, ydtype=torch.float32):
+    B = xbits.shape[0]
+    nbytes = ql.benq_linear_workspace_bytes(B, w.N, xbits.shape[1])
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device="cuda") if nbytes else None
+    y = torch.empty(B, w.N, dtype=ydtype, device="cuda")
+    ql.benq_linear(dev(w.codes), bits16(w.lut), bf16(xbits), y, workspace=ws)
+    torch.cuda.synchronize()
+    return y, nbytes
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 1024, 1024), (1024, 768, 704), (2048, 512, 256)])
+def test_gemm_split_last_wave(ql, M, N, K):
+    # a single partial wave of pair tiles: every tile is split along K across idle SM pairs
+    w = synth.benq_weights(N, K, seed=M + 3 * N + K)
+    x = synth.activations(M, K, seed=M + 1)
+    y, nbytes = _linear_ws(ql, w, x)
+    assert nbytes > 0
+    y = y.cpu().numpy()
+    assert max_rel(y, ob.linear(w.codes, w.lut, x, K)) <= BENQ_TOL
+    y_plain = _linear(ql, w, x).cpu().numpy()
+    assert np.max(np.abs(y - y_plain)) <= 1e-5 * np.max(np.abs(y_plain))   # only the fp32 summation order differs
+    yb, _ = _linear_ws(ql, w, x, torch.bfloat16)
+    assert np.array_equal(yb.cpu().view(torch.int16).numpy().view(np.uint16), f32_to_bf16_rne(y))
+
+
+def test_gemm_split_repeated_calls_are_identical(ql):
+    # the per-tile counters are reset by the last part, so back-to-back calls on one workspace agree bit for bit
+    M, N, K = 600, 1024, 2048
+    w = synth.benq_weights(N, K, seed=77)
+    xb = bf16(synth.activations(M, K, seed=78))
+    codes, lut = dev(w.codes), bits16(w.lut)
+    ws = torch.empty(ql.benq_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    ys = [torch.empty(M, N, device="cuda") for _ in range(4)]
+    for y in ys:
+        ql.benq_linear(codes, lut, xb, y, workspace=ws)
+    torch.cuda.synchronize()
+    ql.ql_check()
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
+
+
+def test_gemm_down_projection_split_sampled_columns(ql):
+    # 2048 x 17408 -> 5120: 80 pair tiles, the last partial wave split along K
+    N, K = 5120, 17408
+    w = synth.benq_weights(N, K, seed=2000 + N // 1024)
+    x = synth.activations(2048, K, seed=2100)
+    y, nbytes = _linear_ws(ql, w, x)
+    y = y.cpu().numpy()
+    cols = np.r_[np.random.default_rng(5).choice(N, 64, replace=False), 0, N - 1]
+    assert max_rel(y[:, cols], ob.linear(w.codes, w.lut, x, K, rows=cols)) <= BENQ_TOL
+
+
+def test_workspace_arguments(ql):
+    assert ql.benq_linear_workspace_bytes(16, 1024, 1024) == 0      # GEMV: no workspace
+    codes = torch.zeros(256, 48, dtype=torch.uint8, device="cuda")
+    lut = torch.zeros(256, 64, dtype=torch.int16, device="cuda")
+    x = torch.zeros(32, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(32, 256, device="cuda")
+    ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    raw = ql.lib().benq_linear_ws
+    s = torch.cuda.current_stream().cuda_stream
+    args = (codes.data_ptr(), lut.data_ptr(), x.data_ptr(), y.data_ptr(), 0, 32, 256, 64)
+    assert raw(*args, ws.data_ptr(), 0, s) == ql.QL_ERR_INVALID_ARG
+    assert raw(*args, None, 4096, s) == ql.QL_ERR_INVALID_ARG
+    assert raw(*args, ws.data_ptr() + 16, 1024, s) == ql.QL_ERR_ALIGNMENT
+    assert raw(*args, ws.data_ptr(), 4096, s) == ql.QL_OK     # too small for a split: whole tiles
+    torch.cuda.synchronize()
