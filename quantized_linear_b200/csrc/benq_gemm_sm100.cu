@@ -444,6 +444,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Opts the GEMM kernel into its dynamic shared memory (once per process).
+cudaError_t smem_attr() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(benq_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  return err;
+}
+
 // CTA pairs that can be resident at once on the current device (cached per device).
 int resident_pairs() {
   static std::mutex mu;
@@ -452,6 +462,7 @@ int resident_pairs() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
   std::lock_guard<std::mutex> lock(mu);
   if (cache[dev] == 0) {
+    (void)smem_attr();   // the occupancy query needs the kernel's shared-memory opt-in
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (ql::sm_count() / 2));
     cfg.blockDim = dim3(THREADS);
@@ -528,12 +539,7 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return fail(QL_ERR_CUDA, "benq_linear: cannot encode the code tensor map");
   }
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(benq_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
-  if (attr_err != cudaSuccess) return fail(QL_ERR_CUDA, "benq_linear: cannot reserve GEMM shared memory");
+  if (smem_attr() != cudaSuccess) return fail(QL_ERR_CUDA, "benq_linear: cannot reserve GEMM shared memory");
   const int ntiles = ((M + PM - 1) / PM) * (N / BN);
   const int resident = resident_pairs();
   SplitPlan plan = split_plan(M, N, K, resident);
