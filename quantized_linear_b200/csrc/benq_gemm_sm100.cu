@@ -13,8 +13,8 @@
 //     make slow tensor copies) into a 2-stage ring, plus the 128 row tables of the tile (16 KB,
 //     once per tile) with a bulk copy;
 //   * warps 3..18 (decoders) expand the code tile through the row tables into the bf16 W half
-//     tile, written directly in the K-major 128-byte-swizzled layout the tensor core reads, fence
-//     the writes for the async proxy and arrive on the even CTA's barrier;
+//     tile, two K blocks per pass, written directly in the K-major 128-byte-swizzled layout the
+//     tensor core reads, fence the writes for the async proxy and arrive on the even CTA's barrier;
 //   * in the even CTA only, warp 1 (one thread) issues the pair MMAs (two M halves share each
 //     decoded W tile) into both CTAs' tensor memory (2 x 128 x 256 fp32 per CTA) and signals
 //     stage release to both CTAs with a multicast commit;
@@ -88,6 +88,9 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
 }
 __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t lo, uint32_t hi) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(lo), "r"(hi) : "memory");
 }
 __device__ __forceinline__ uint32_t ld_volatile_u32(uint32_t a) {
   uint32_t v;
@@ -271,18 +274,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t lead_full_b = sm100::mapa_shared(bar.full_b, 0);
     const uint32_t lead_acc_empty = sm100::mapa_shared(bar.acc_empty, 0);
     int it = 0, tl = 0, ic = 0, ns = 0;
-    // lane l expands codes 2l, 2l+1 of a row's 64-code block: bits [12l, 12l+12) of its 48 bytes
-    const int wq = (12 * lane) >> 5, wsh = (12 * lane) & 31;
-    const int chunk = lane >> 2, inner = (lane & 3) * 4;
-    // swizzled position of codes 2*lane, 2*lane+1 within row r = dw (mod 8) of a K block
-    const uint32_t dst_lane = (dw >> 3) * 1024 + (dw & 7) * 128 + ((chunk ^ (dw & 7)) << 4) + inner;
+    // A pass decodes two K blocks: lanes 0-15 the first, 16-31 the second.  Lane l expands the 4
+    // codes in bytes [3l, 3l + 3) of the two blocks' 96 code bytes of a row (codes 4(l&15) ..
+    // 4(l&15)+3 of its block), so two 32-bit loads serve 4 codes and its output is 8 bytes.
+    const int half = lane >> 4;
+    const int cwo = 4 * ((3 * lane) >> 2), csh = 8 * ((3 * lane) & 3);
+    // swizzled position of those 4 codes within row r = dw (mod 8) of a K block
+    const uint32_t dst_lane =
+        (dw >> 3) * 1024 + (dw & 7) * 128 + ((((lane & 15) >> 1) ^ (dw & 7)) << 4) + (lane & 1) * 8;
     for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
       const Item w = item_of(wi, full, parts, nkb);
       const int m0 = (w.tile % mt) * PM + (int)rank * BM, n0 = (w.tile / mt) * BN;
       if (!wt.wait(bar.lut_full, tl & 1, false)) { ok = false; break; }
-      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
-        const int sb = it % SB, sc = ic % SC, sub = (kb - w.kb0) % CKB;
-        if ((it >= SB && !wt.wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, true)) ||
+      for (int kb = w.kb0; kb < w.kb1;) {
+        const bool two = kb + 1 < w.kb1;
+        const int sb0 = it % SB, sb1 = (it + 1) % SB, sc = ic % SC, sub = (kb - w.kb0) % CKB;   // sub is 0 or 2
+        if ((it >= SB && !wt.wait(bar.empty_b + 8 * sb0, ((it / SB) & 1) ^ 1, true)) ||
+            (two && it + 1 >= SB && !wt.wait(bar.empty_b + 8 * sb1, (((it + 1) / SB) & 1) ^ 1, true)) ||
             (sub == 0 && !wt.wait(bar.full_c + 8 * sc, (ic / SC) & 1, false))) {
           ok = false;
           break;
@@ -290,8 +298,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // rows r = dw + NDEC*i: r & 7 == dw & 7 is fixed per warp, so every address below is
         // a per-warp base plus a compile-time multiple of the row step.  All code words of the
         // warp's rows are loaded before the first lookup.
-        const uint32_t cb = sbase + OFF_C + sc * C_BYTES + dw * C_SROW + sub * C_ROW + 4 * wq;
-        const uint32_t bb = sbase + OFF_B + sb * B_BYTES + dst_lane;
+        const uint32_t cb = sbase + OFF_C + sc * C_BYTES + dw * C_SROW + sub * C_ROW + cwo;
+        const uint32_t bb = sbase + OFF_B + (half ? sb1 : sb0) * B_BYTES + dst_lane;
         const uint32_t tb = sbase + OFF_LUT + dw * 128;
         constexpr int RPW = BNH / NDEC;   // rows per decoder warp per K block
         uint32_t v[RPW];
@@ -299,23 +307,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int i = 0; i < RPW; ++i) {
           const uint32_t w0 = lds32(cb + i * NDEC * C_SROW);
           const uint32_t w1 = lds32(cb + i * NDEC * C_SROW + 4);   // may read past the row: unused bits
-          v[i] = __funnelshift_r(w0, w1, wsh);
+          v[i] = __funnelshift_r(w0, w1, csh);
         }
+        const bool store = half == 0 || two;
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
           const uint32_t tbl = tb + i * NDEC * 128;
           const uint32_t e0 = lds_u16(((v[i] << 1) & 0x7Eu) | tbl);
           const uint32_t e1 = lds_u16(((v[i] >> 5) & 0x7Eu) | tbl);
-          sts32(bb + i * (NDEC / 8) * 1024, __byte_perm(e0, e1, 0x5410));
+          const uint32_t e2 = lds_u16(((v[i] >> 11) & 0x7Eu) | tbl);
+          const uint32_t e3 = lds_u16(((v[i] >> 17) & 0x7Eu) | tbl);
+          if (store) sts64(bb + i * (NDEC / 8) * 1024, __byte_perm(e0, e1, 0x5410), __byte_perm(e2, e3, 0x5410));
         }
         sm100::fence_proxy_async_smem();
         __syncwarp();
-        const bool stage_done = sub == CKB - 1 || kb == w.kb1 - 1;
+        const int step = two ? 2 : 1;
+        const bool stage_done = sub + step >= CKB || kb + step == w.kb1;
         if (lane == 0) {
-          sm100::mbar_arrive_cluster(lead_full_b + 8 * sb);
+          sm100::mbar_arrive_cluster(lead_full_b + 8 * sb0);
+          if (two) sm100::mbar_arrive_cluster(lead_full_b + 8 * sb1);
           if (stage_done) sm100::mbar_arrive(bar.empty_c + 8 * sc);
         }
         if (stage_done) ++ic;
+        kb += step;
+        it += step;
       }
       if (!ok) break;
       __syncwarp();
