@@ -216,10 +216,18 @@ class Workload:
         return sum(1 if L["kind"] == "benq" else 3 for L in self.layers)
 
 
-def _kernel_source_sha():
+# the sources each kernel's DRAM-traffic figure depends on
+_KERNEL_SOURCES = {
+    "benq_gemv": ["benq_gemv.cu", "ql_internal.cuh"],
+    "benq_gemm": ["benq_gemm_sm100.cu", "sm100_ptx.cuh", "ql_internal.cuh"],
+    "mdbf_linear": ["mdbf.cu", "ql_internal.cuh"],
+}
+
+
+def _kernel_source_sha(kernel_key):
     h = hashlib.sha256()
     d = os.path.join(ROOT, "quantized_linear_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in _KERNEL_SOURCES[kernel_key]:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -233,7 +241,7 @@ def _traffic(kernel_key):
     with open(path) as f:
         d = json.load(f)
     e = d.get(kernel_key)
-    if not e or e.get("source_sha") != _kernel_source_sha():
+    if not e or e.get("source_sha") != _kernel_source_sha(kernel_key):
         return None
     return e.get("dram_bytes_per_launch")
 
