@@ -20,6 +20,7 @@
 #include <mutex>
 
 #include "ql_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace {
 
@@ -91,23 +92,53 @@ __device__ __forceinline__ uint4 pack_fragment(Get get, int qw, int nb, int lane
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// G-stage B fragments from z[j][b*l+i] = B_amp[j][i] * x[b][j] (exact in fp32)
+// G-stage B fragments from z[j][b*l+i] = B_amp[j][i] * x[b][j] (exact in fp32).  One thread per
+// fragment register set (word qw, n block nb, lane): its 8 columns' B_amp and x values are all
+// loaded before any is used, and the weights (B_amp) are pulled toward L2 before the wait on
+// the preceding kernel.
 __global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uint4 *__restrict__ out, int m, int l,
                                    int B, int NB) {
   const int p = blockIdx.y;
   const int QW = (m + 31) / 32, V = l * B;
   const int64_t total = (int64_t)QW * NB * 32;
   const uint16_t *bm = ps.Bm[p];
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x)
+    if ((e & 31) == 0) {
+      const int64_t c0 = std::min<int64_t>(32 * ((e >> 5) / NB), m - 1);   // first column of the word, in bounds
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(bm + c0 * l));
+    }
   qld::pdl_trigger();
   qld::pdl_wait();
-  auto get = [&](int c, int v) {
-    const int b = v / l, i = v - b * l;
-    return qld::f16_to_f32(bm[(int64_t)c * l + i]) * qld::bf16_to_f32(x[(int64_t)b * m + c]);
-  };
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int lane = int(e & 31);
+    const int lane = int(e & 31), g = lane >> 2, q = lane & 3;
     const int64_t f = e >> 5;
-    out[(int64_t)p * total + e] = pack_fragment(get, int(f / NB), int(f % NB), lane, m, V);
+    const int qw = int(f / NB), nb = int(f % NB), nn = 8 * nb + g;
+    // the 8 physical columns of this lane's registers (see "Sign products on the warp MMA")
+    int col[8];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int ca = 32 * qw + 8 * h + q, cb = ca + 4;
+      col[4 * h] = ca; col[4 * h + 1] = ca + 16; col[4 * h + 2] = cb; col[4 * h + 3] = cb + 16;
+    }
+    const bool live = nn < 2 * V;
+    const int v = nn < V ? nn : nn - V, b = live ? v / l : 0, i = live ? v - b * l : 0;
+    float z[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const bool in = live && col[t] < m;
+      const int c = in ? col[t] : 0;
+      const float bv = qld::f16_to_f32(bm[(int64_t)c * l + i]);
+      const float xv = qld::bf16_to_f32(x[(int64_t)b * m + c]);
+      z[t] = in ? bv * xv : 0.f;
+    }
+    uint32_t o[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const uint32_t hi = bf16_rn_bits(z[t]);
+      o[t] = nn < V ? hi : bf16_rn_bits(z[t] - __uint_as_float(hi << 16));
+      if (!live) o[t] = 0u;
+    }
+    out[(int64_t)p * total + e] = make_uint4(o[0] | (o[1] << 16), o[2] | (o[3] << 16), o[4] | (o[5] << 16), o[6] | (o[7] << 16));
   }
 }
 
@@ -264,6 +295,134 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_mma_kernel(Paths ps, con
     wpk[((size_t)p * QWr + qw) * NB * 32 + e] = pack_fragment(get, qw, e >> 5, e & 31, r, V);
 }
 
+// G stage as above, with the CTA's 32 sign rows staged in shared memory by one bulk copy issued
+// before the wait on the preceding kernel (the rows are contiguous: ldSB apart).  Warps split
+// the K words as mdbf_g_mma_kernel does and load the next word group's fragments while the
+// current one is multiplied.  Rows past r read stale shared memory; their results are dropped.
+// set when a bounded wait of an MDBF kernel runs out; read and cleared by ql_check()
+__device__ int g_mdbf_timeout = 0;
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32s(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+
+constexpr long long G_WAIT_BUDGET = 4000000000LL;   // clock cycles (~2 s)
+
+template <int NB>
+__global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, const uint4 *__restrict__ zpk,
+                                                                      uint4 *__restrict__ wpk, int m, int r, int l,
+                                                                      int B, uint32_t sign_bytes) {
+  extern __shared__ __align__(128) unsigned char gsm[];
+  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(gsm));
+  float *red = reinterpret_cast<float *>(gsm + sign_bytes + 128), *D = red + SP_WARPS * 2 * NB * 128,
+        *Ws = D + 32 * 8 * NB;
+  const int p = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int QW = (m + 31) / 32, V = l * B;
+  const int row0 = blockIdx.x * 32, rows = min(32, r - row0);
+  const uint32_t ld = (uint32_t)ps.ldSB[p], bar = sbase + sign_bytes;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(bar, 1);
+    sm100::fence_barrier_init();
+    sm100::mbar_arrive_expect_tx(bar, rows * ld);
+    sm100::bulk_g2s(sbase, ps.SB[p] + (size_t)row0 * ld, rows * ld, bar);
+  }
+  qld::pdl_trigger();
+  qld::pdl_wait();
+  __syncthreads();
+  const bool ok = sm100::mbar_wait(bar, 0, G_WAIT_BUDGET);
+  if (!ok && threadIdx.x == 0) atomicExch(&g_mdbf_timeout, 1);
+
+  float acc[2][NB][4];
+#pragma unroll
+  for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
+  int w0, w1;
+  warp_words(QW, warp, w0, w1);
+  const uint4 *vb = zpk + (size_t)p * QW * NB * 32;
+  uint32_t rowaddr[2][2];
+#pragma unroll
+  for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) rowaddr[rt][hh] = sbase + (16 * rt + g + 8 * hh) * ld;
+  constexpr int UB = NB <= 2 ? SP_U : 1;   // words of fragments held per group
+  auto load_frags = [&](uint4 (&bf)[UB][NB], int qwb) {
+#pragma unroll
+    for (int u = 0; u < UB; ++u)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+        bf[u][nb] = (qwb + u < w1) ? __ldg(vb + ((size_t)(qwb + u) * NB + nb) * 32 + lane) : make_uint4(0, 0, 0, 0);
+  };
+  uint4 cur[UB][NB], nxt[UB][NB];
+  if (ok && w0 < w1) load_frags(cur, w0);
+  for (int qw0 = w0; ok && qw0 < w1; qw0 += SP_U) {
+    uint32_t sw[SP_U][2][2];
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint4 v = lds128(rowaddr[rt][hh] + 4 * qw0);
+        sw[0][rt][hh] = v.x; sw[1][rt][hh] = v.y; sw[2][rt][hh] = v.z; sw[3][rt][hh] = v.w;
+      }
+    if constexpr (UB == SP_U) {
+      if (qw0 + SP_U < w1) load_frags(nxt, qw0 + SP_U);
+    }
+#pragma unroll
+    for (int u = 0; u < SP_U; ++u) {
+      if constexpr (UB != SP_U) load_frags(cur, qw0 + u);
+      const int slot = UB == SP_U ? u : 0;
+#pragma unroll
+      for (int rt = 0; rt < 2; ++rt) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int sa = 15 - 8 * h - q, sb = 11 - 8 * h - q;
+          const uint32_t a0 = sign_pair(sw[u][rt][0], sa), a1 = sign_pair(sw[u][rt][1], sa);
+          const uint32_t a2 = sign_pair(sw[u][rt][0], sb), a3 = sign_pair(sw[u][rt][1], sb);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const uint32_t b0 = h ? cur[slot][nb].z : cur[slot][nb].x, b1 = h ? cur[slot][nb].w : cur[slot][nb].y;
+            mma16816(acc[rt][nb], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      }
+    }
+    if constexpr (UB == SP_U) {
+#pragma unroll
+      for (int u = 0; u < UB; ++u)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) cur[u][nb] = nxt[u][nb];
+    }
+  }
+  reduce_fragments<NB, 2>(red, D, acc);
+  for (int e = threadIdx.x; e < 32 * B; e += blockDim.x) {
+    const int rr = e / B, b = e - rr * B, k = row0 + rr;
+    float *wo = Ws + rr * V + b * l;
+    if (k >= r) {
+      for (int i = 0; i < l; ++i) wo[i] = 0.f;
+      continue;
+    }
+    const float *Dr = D + rr * (8 * NB);
+    const uint16_t *qv = ps.QV[p] + (int64_t)k * l, *qu = ps.QU[p] + (int64_t)k * l;
+    float t = 0.f;
+    for (int i = 0; i < l; ++i) t = fmaf(qld::f16_to_f32(qv[i]), Dr[b * l + i] + Dr[V + b * l + i], t);
+    for (int i = 0; i < l; ++i) wo[i] = qld::f16_to_f32(qu[i]) * t;
+  }
+  __syncthreads();
+  const int qw = blockIdx.x, QWr = (r + 31) / 32;
+  auto get = [&](int c, int v) { return Ws[(c - 32 * qw) * V + v]; };
+  for (int e = threadIdx.x; e < NB * 32; e += blockDim.x)
+    wpk[((size_t)p * QWr + qw) * NB * 32 + e] = pack_fragment(get, qw, e >> 5, e & 31, r, V);
+}
+
 // F stage: y[b][a] = sum_p sum_i A_amp[a][i] v_p[a][b*l+i], paths summed in p order
 template <int NB, int RT, bool VEC16>
 __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int P, const uint4 *__restrict__ wpk,
@@ -304,6 +463,158 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int
   for (int e = threadIdx.x; e < 16 * RT * B; e += blockDim.x) {
     const int rr = e / B, b = e - rr * B, a = row0 + rr;
     if (a >= n) continue;
+    if (ydt == QL_OUT_F32)
+      static_cast<float *>(y)[(int64_t)b * n + a] = yacc[e];
+    else
+      static_cast<uint16_t *>(y)[(int64_t)b * n + a] = qld::f32_to_bf16_rn(yacc[e]);
+  }
+}
+
+// ---------------------------------------------------------------- F stage, staged tiles ------
+// One CTA per 128 rows of S_A.  Each path's 128-row sign block is contiguous in memory (rows are
+// ldSA apart), so one bulk copy brings it into shared memory, issued before the wait on the G
+// stage (signs are weights); the path's packed w fragments follow after the wait.  Two stages
+// let path p + 1 (or p + 2) arrive while path p is multiplied.  Warp w owns rows
+// [16 (w % 8), +16) of the block over the K-word group w / 8 (KG groups of consecutive words);
+// the groups' partial sums are added in group order.  Paths are summed in p order.
+constexpr int FT_WARPS = 8, FT_ROWS = 16 * FT_WARPS;
+constexpr long long FT_WAIT_BUDGET = 4000000000LL;   // clock cycles (~2 s)
+
+
+struct FTileLayout {
+  uint32_t sign_bytes, frag_bytes, stage_bytes, nstage, off_bars, off_d, off_y, total;
+};
+__host__ __device__ inline FTileLayout ftile_layout(size_t ld_max, int r, int NB, int B, int nstage, int KG) {
+  FTileLayout L;
+  L.sign_bytes = (uint32_t)((FT_ROWS * ld_max + 127) / 128 * 128);
+  L.frag_bytes = (uint32_t)((r + 31) / 32) * NB * 32 * 16;
+  L.stage_bytes = L.sign_bytes + L.frag_bytes;
+  L.nstage = (uint32_t)nstage;
+  L.off_bars = L.nstage * L.stage_bytes;
+  L.off_d = L.off_bars + 128;                                   // per-warp D scratch [16][8 NB] fp32
+  L.off_y = L.off_d + KG * FT_WARPS * 16 * 8 * NB * 4;           // per-row-tile y accumulators [16][B] fp32
+  L.total = L.off_y + FT_WARPS * 16 * B * 4;
+  return L;
+}
+
+
+template <int NB, int KG>
+__global__ void __launch_bounds__(FT_WARPS * 32 * KG)
+    mdbf_f_tile_kernel(Paths ps, int P, const uint4 *__restrict__ wpk, void *__restrict__ y, int ydt, int n, int r,
+                       int l, int B, FTileLayout L) {
+  extern __shared__ __align__(128) unsigned char fsm[];
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(fsm));
+  const int QW = (r + 31) / 32, V = l * B;
+  const int row0 = blockIdx.x * FT_ROWS, rows = min(FT_ROWS, n - row0);
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int warp = wid % FT_WARPS, kg = wid / FT_WARPS;   // row tile, K-word group
+  const int qw0 = kg * QW / KG, qw1 = (kg + 1) * QW / KG;
+  const uint32_t bars = base + L.off_bars;
+  float *const dsc_all = reinterpret_cast<float *>(fsm + L.off_d);
+  float *dsc = dsc_all + wid * 16 * 8 * NB;
+  float *yacc = reinterpret_cast<float *>(fsm + L.off_y) + warp * 16 * B;
+  if (kg == 0)
+    for (int e = lane; e < 16 * B; e += 32) yacc[e] = 0.f;
+
+  // stage s receives path p's signs (weights) and w fragments (made by the G stage)
+  int issued[2] = {0, 0};   // copies issued per stage (thread 0), for the drain after a timeout
+  auto issue = [&](int p, int st, bool after_wait) {
+    const uint32_t bar = bars + 8 * st, dst = base + st * L.stage_bytes;
+    const uint32_t sbytes = (uint32_t)(rows * ps.ldSA[p]);
+    if (!after_wait) {
+      ++issued[st];
+      sm100::mbar_arrive_expect_tx(bar, sbytes + L.frag_bytes);
+      sm100::bulk_g2s(dst, ps.SA[p] + (size_t)row0 * ps.ldSA[p], sbytes, bar);
+    } else {
+      sm100::bulk_g2s(dst + L.sign_bytes, wpk + (size_t)p * QW * NB * 32, L.frag_bytes, bar);
+    }
+  };
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < (int)L.nstage; ++st) sm100::mbar_init(bars + 8 * st, 1);
+    sm100::fence_barrier_init();
+    for (int p = 0; p < P && p < (int)L.nstage; ++p) issue(p, p, false);
+    qld::pdl_trigger();
+    qld::pdl_wait();
+    for (int p = 0; p < P && p < (int)L.nstage; ++p) issue(p, p, true);
+  }
+  qld::pdl_wait();
+  __syncthreads();
+
+  bool ok = true;
+  for (int p = 0; p < P; ++p) {
+    const int st = p % (int)L.nstage;
+    if (!sm100::mbar_wait(bars + 8 * st, (p / (int)L.nstage) & 1, FT_WAIT_BUDGET)) ok = false;
+    if (ok && 16 * warp < rows) {
+      const uint32_t sbase = base + st * L.stage_bytes;
+      const uint32_t ldp = (uint32_t)ps.ldSA[p];
+      const uint32_t r0 = sbase + (16 * warp + g) * ldp, r1 = r0 + 8 * ldp;   // rows past `rows` read stale bytes: not stored
+      const uint32_t fb = sbase + L.sign_bytes + lane * 16;
+      float acc[NB][4];
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+#pragma unroll 2
+      for (int qw = qw0; qw < qw1; ++qw) {
+        const uint32_t s0 = lds32s(r0 + 4 * qw), s1 = lds32s(r1 + 4 * qw);
+        uint4 bf[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) bf[nb] = lds128(fb + (qw * NB + nb) * 512);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int sa = 15 - 8 * h - q, sb = 11 - 8 * h - q;
+          const uint32_t a0 = sign_pair(s0, sa), a1 = sign_pair(s1, sa), a2 = sign_pair(s0, sb), a3 = sign_pair(s1, sb);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb)
+            mma16816(acc[nb], a0, a1, a2, a3, h ? bf[nb].z : bf[nb].x, h ? bf[nb].w : bf[nb].y);
+        }
+      }
+      // D fragment -> per-warp scratch [16 rows][8 NB columns]
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        const int c = 8 * nb + 2 * q;
+        dsc[g * 8 * NB + c] = acc[nb][0];
+        dsc[g * 8 * NB + c + 1] = acc[nb][1];
+        dsc[(g + 8) * 8 * NB + c] = acc[nb][2];
+        dsc[(g + 8) * 8 * NB + c + 1] = acc[nb][3];
+      }
+    }
+    __syncthreads();   // every warp is done with stage st and has written its partial D
+    if (ok && kg == 0 && 16 * warp < rows) {
+      // sum the K groups' partials in group order, then the A_amp epilogue
+      for (int e = lane; e < 16 * 8 * NB; e += 32) {
+        float d = dsc_all[warp * 16 * 8 * NB + e];
+        for (int k = 1; k < KG; ++k) d += dsc_all[(k * FT_WARPS + warp) * 16 * 8 * NB + e];
+        dsc[e] = d;
+      }
+      __syncwarp();
+      for (int e = lane; e < 16 * B; e += 32) {
+        const int rr = e / B, b = e - rr * B, a = row0 + 16 * warp + rr;
+        if (a >= n) continue;
+        const float *Dr = dsc + rr * 8 * NB;
+        const uint16_t *am = ps.A[p] + (int64_t)a * l;
+        float sacc = yacc[e];
+        for (int i = 0; i < l; ++i) sacc = fmaf(qld::f16_to_f32(am[i]), Dr[b * l + i] + Dr[V + b * l + i], sacc);
+        yacc[e] = sacc;
+      }
+    }
+    __syncthreads();   // partials consumed; stage st free
+    if (threadIdx.x == 0 && p + (int)L.nstage < P && ok) {
+      issue(p + L.nstage, st, false);
+      issue(p + L.nstage, st, true);
+    }
+  }
+  if (!ok) {
+    if (threadIdx.x == 0) {
+      atomicExch(&g_mdbf_timeout, 1);
+      // leave no copy in flight: wait (bounded) for the last phase of every stage
+      for (int st = 0; st < (int)L.nstage; ++st)
+        if (issued[st] > 0) (void)sm100::mbar_wait(bars + 8 * st, (issued[st] - 1) & 1, FT_WAIT_BUDGET);
+    }
+    __syncthreads();
+    return;
+  }
+  for (int e = lane; e < 16 * B; e += 32) {
+    const int rr = e / B, b = e - rr * B, a = row0 + 16 * warp + rr;
+    if (kg != 0 || a >= n || 16 * warp >= rows) continue;
     if (ydt == QL_OUT_F32)
       static_cast<float *>(y)[(int64_t)b * n + a] = yacc[e];
     else
@@ -397,6 +708,20 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
   if (cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg) != cudaSuccess ||
       cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf) != cudaSuccess)
     return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
+  // G stage with staged signs when the 32 sign rows fit next to the reduction buffers
+  bool g_tile = false;
+  uint32_t g_sign_bytes = 0;
+  size_t smg_t = 0;
+  if constexpr (VEC16) {
+    size_t ldb = 0;
+    for (int p = 0; p < P; ++p) ldb = std::max(ldb, ps.ldSB[p]);
+    g_sign_bytes = (uint32_t)((32 * ldb + 127) / 128 * 128);
+    smg_t = g_sign_bytes + 128 + smg;
+    g_tile = smg_t <= 227 * 1024;
+    if (g_tile && cudaFuncSetAttribute(mdbf_g_tile_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smg_t) != cudaSuccess)
+      return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
+  }
   {
     const int64_t total = (int64_t)((m + 31) / 32) * NB * 32;
     const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)ql::sm_count() * 4);
@@ -404,9 +729,29 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
-  ql::launch(kg, dim3((r + 31) / 32, P), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
+  if (g_tile)
+    ql::launch(mdbf_g_tile_kernel<NB>, dim3((r + 31) / 32, P), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
+               m, r, l, B, g_sign_bytes);
+  else
+    ql::launch(kg, dim3((r + 31) / 32, P), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
   ql_status st = ql::launch_status("mdbf_linear (G stage)");
   if (st != QL_OK) return st;
+  if constexpr (VEC16) {
+    // staged-tile F stage when two (else one) path stages fit in shared memory
+    size_t ld_max = 0;
+    for (int p = 0; p < P; ++p) ld_max = std::max(ld_max, ps.ldSA[p]);
+    constexpr int KG = NB <= 4 ? 4 : NB == 8 ? 2 : 1;   // K-word groups: as many warps as the registers allow
+    FTileLayout L = ftile_layout(ld_max, r, NB, B, 2, KG);
+    if (L.total > 227 * 1024) L = ftile_layout(ld_max, r, NB, B, 1, KG);
+    if (L.total <= 227 * 1024) {
+      auto kt = mdbf_f_tile_kernel<NB, KG>;
+      if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total) != cudaSuccess)
+        return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
+      ql::launch(kt, (n + FT_ROWS - 1) / FT_ROWS, FT_WARPS * 32 * KG, L.total, s, ps, P, (const uint4 *)wpk, y,
+                 (int)ydt, n, r, l, B, L);
+      return ql::launch_status("mdbf_linear (F stage)");
+    }
+  }
   ql::launch(kf, (n + 16 * RTF - 1) / (16 * RTF), SP_WARPS * 32, smf, s, ps, P, (const uint4 *)wpk, y, (int)ydt, n,
              r, l, B);
   return ql::launch_status("mdbf_linear (F stage)");
@@ -448,6 +793,14 @@ WsLayout ws_layout(int P, int m, int r, int l, int B) {
 }  // namespace
 
 namespace ql {
+
+ql_status mdbf_read_timeout(int *flag) {
+  int zero = 0;
+  if (cudaMemcpyFromSymbol(flag, g_mdbf_timeout, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_mdbf_timeout, &zero, sizeof(int)) != cudaSuccess)
+    return fail(QL_ERR_CUDA, "ql_check: cannot read the device timeout flag");
+  return QL_OK;
+}
 
 size_t mdbf_workspace_size(int P, int n, int m, int r, int l, int B) {
   (void)n;

@@ -54,6 +54,7 @@ size_t mdbf_workspace_size(int P, int n, int m, int r, int l, int B);
 ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r, int l,
                              const uint16_t *x, void *y, ql_out_dtype ydt, int B, void *ws,
                              cudaStream_t s);
+ql_status mdbf_read_timeout(int *flag);   // reads and clears the MDBF kernels' bounded-wait flag
 size_t mdbf_noalloc_scratch_limit();
 ql_status mdbf_noalloc_scratch(void **ptr);
 ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W,
