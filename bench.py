@@ -284,6 +284,26 @@ def cpu_baseline(workload, budget_s=10.0):
             "sample": f"{len(samples)} row blocks of {rows} rows ({samples[0]} ...), {t_used:.1f} s of oracle time"}
 
 
+def max_over_ranks(value, world):
+    """The largest of the ranks' `value` (a device time in ms), every rank getting the result.
+    One rank returns its own value; otherwise an all-reduce on the process group (NCCL: a CUDA
+    tensor, gloo: a CPU one)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step, steps, ms, world):
+    """Whole-job GB/s: every rank processes bytes_per_step per step (weak scaling), timed by the
+    slowest rank's `ms` for `steps` steps."""
+    return world * bytes_per_step * steps / (ms / 1e3) / 1e9
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -384,12 +404,7 @@ def main():
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        t_ms = start.elapsed_time(stop)
-        if world > 1:
-            t = torch.tensor([t_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t_ms = float(t.item())
-        return t_ms
+        return max_over_ranks(start.elapsed_time(stop), world)
 
     with ClockSampler(torch.cuda.current_device()) as clk:
         ms = timed(graphs, args.steps)
@@ -398,7 +413,7 @@ def main():
         dom_ms = ms if dom_graphs is graphs else timed(dom_graphs, args.steps)
     ms_per_step = ms / args.steps
     step_bytes = wl.step_bytes()
-    value = world * step_bytes * args.steps / (ms / 1e3) / 1e9
+    value = job_throughput(step_bytes, args.steps, ms, world)
     dom_launches = len(dom) * args.steps
     peaks = _peaks()
     if args.workload == "prefill":
@@ -441,12 +456,8 @@ def main():
                 yh.copy_(L["y"], non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * step_bytes * args.steps / (ems / 1e3) / 1e9, "unit": "GB/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": job_throughput(step_bytes, args.steps, ems, world), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems / args.steps}
     except Exception as exc:  # pragma: no cover - reported, not hidden
         e2e = {"error": repr(exc)}
