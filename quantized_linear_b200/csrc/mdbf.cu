@@ -65,6 +65,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 __device__ __forceinline__ uint32_t sign_pair(uint32_t w, int s) {
   return ((w << s) & 0x80008000u) ^ 0xBF80BF80u;
 }
+// The same with the shift given as the multiplier 2^s: the multiply runs on the FMA pipe, which
+// the sign products leave idle, instead of the integer pipe that the mask-and-flip also needs.
+__device__ __forceinline__ uint32_t sign_pair_mul(uint32_t w, uint32_t pow2s) {
+  uint32_t t;
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(t) : "r"(w), "r"(pow2s));
+  return (t & 0x80008000u) ^ 0xBF80BF80u;
+}
 
 __device__ __forceinline__ uint32_t bf16_rn_bits(float f) { return qld::f32_to_bf16_rn(f); }
 
@@ -384,9 +391,9 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
       for (int rt = 0; rt < 2; ++rt) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int sa = 15 - 8 * h - q, sb = 11 - 8 * h - q;
-          const uint32_t a0 = sign_pair(sw[u][rt][0], sa), a1 = sign_pair(sw[u][rt][1], sa);
-          const uint32_t a2 = sign_pair(sw[u][rt][0], sb), a3 = sign_pair(sw[u][rt][1], sb);
+          const uint32_t ma = 1u << (15 - 8 * h - q), mb = 1u << (11 - 8 * h - q);
+          const uint32_t a0 = sign_pair_mul(sw[u][rt][0], ma), a1 = sign_pair_mul(sw[u][rt][1], ma);
+          const uint32_t a2 = sign_pair_mul(sw[u][rt][0], mb), a3 = sign_pair_mul(sw[u][rt][1], mb);
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb) {
             const uint32_t b0 = h ? cur[slot][nb].z : cur[slot][nb].x, b1 = h ? cur[slot][nb].w : cur[slot][nb].y;
@@ -477,44 +484,47 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int
 // let path p + 1 (or p + 2) arrive while path p is multiplied.  Warp w owns rows
 // [16 (w % 8), +16) of the block over the K-word group w / 8 (KG groups of consecutive words);
 // the groups' partial sums are added in group order.  Paths are summed in p order.
-constexpr int FT_WARPS = 8, FT_ROWS = 16 * FT_WARPS;
+constexpr int FT_WARPS = 8;   // 16-row tiles of a full-size F block
 constexpr long long FT_WAIT_BUDGET = 4000000000LL;   // clock cycles (~2 s)
 
 
 struct FTileLayout {
   uint32_t sign_bytes, frag_bytes, stage_bytes, nstage, off_bars, off_d, off_y, total;
 };
-__host__ __device__ inline FTileLayout ftile_layout(size_t ld_max, int r, int NB, int B, int nstage, int KG) {
+__host__ __device__ inline FTileLayout ftile_layout(size_t ld_max, int r, int NB, int B, int nstage, int KG,
+                                                    int tiles) {
   FTileLayout L;
-  L.sign_bytes = (uint32_t)((FT_ROWS * ld_max + 127) / 128 * 128);
+  L.sign_bytes = (uint32_t)((16 * tiles * ld_max + 127) / 128 * 128);
   L.frag_bytes = (uint32_t)((r + 31) / 32) * NB * 32 * 16;
   L.stage_bytes = L.sign_bytes + L.frag_bytes;
   L.nstage = (uint32_t)nstage;
   L.off_bars = L.nstage * L.stage_bytes;
   L.off_d = L.off_bars + 128;                                   // per-warp D scratch [16][8 NB] fp32
-  L.off_y = L.off_d + KG * FT_WARPS * 16 * 8 * NB * 4;           // per-row-tile y accumulators [16][B] fp32
-  L.total = L.off_y + FT_WARPS * 16 * B * 4;
+  L.off_y = L.off_d + KG * tiles * 16 * 8 * NB * 4;              // per-row-tile y accumulators [16][B] fp32
+  L.total = L.off_y + tiles * 16 * B * 4;
   return L;
 }
 
 
-template <int NB, int KG>
-__global__ void __launch_bounds__(FT_WARPS * 32 * KG)
+template <int NB, int KG, int RT, int NRG>
+__global__ void __launch_bounds__(NRG * 32 * KG)
     mdbf_f_tile_kernel(Paths ps, int P, const uint4 *__restrict__ wpk, void *__restrict__ y, int ydt, int n, int r,
                        int l, int B, FTileLayout L) {
+  constexpr int TILES = RT * NRG;      // 16-row tiles per CTA: NRG row groups of RT tiles
   extern __shared__ __align__(128) unsigned char fsm[];
   const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(fsm));
   const int QW = (r + 31) / 32, V = l * B;
-  const int row0 = blockIdx.x * FT_ROWS, rows = min(FT_ROWS, n - row0);
+  const int row0 = blockIdx.x * 16 * TILES, rows = min(16 * TILES, n - row0);
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-  const int warp = wid % FT_WARPS, kg = wid / FT_WARPS;   // row tile, K-word group
+  const int rg = wid % NRG, kg = wid / NRG;   // row group, K-word group
   const int qw0 = kg * QW / KG, qw1 = (kg + 1) * QW / KG;
+  const int rbase = 16 * RT * rg;             // first row of this warp's tiles within the block
   const uint32_t bars = base + L.off_bars;
-  float *const dsc_all = reinterpret_cast<float *>(fsm + L.off_d);
-  float *dsc = dsc_all + wid * 16 * 8 * NB;
-  float *yacc = reinterpret_cast<float *>(fsm + L.off_y) + warp * 16 * B;
+  float *const dsc_all = reinterpret_cast<float *>(fsm + L.off_d);    // [KG][8 tiles][16][8 NB]
+  float *const yacc_all = reinterpret_cast<float *>(fsm + L.off_y);   // [8 tiles][16][B]
+  auto dsc_of = [&](int k, int tile) { return dsc_all + ((size_t)k * TILES + tile) * 16 * 8 * NB; };
   if (kg == 0)
-    for (int e = lane; e < 16 * B; e += 32) yacc[e] = 0.f;
+    for (int e = lane; e < RT * 16 * B; e += 32) yacc_all[RT * rg * 16 * B + e] = 0.f;
 
   // stage s receives path p's signs (weights) and w fragments (made by the G stage)
   int issued[2] = {0, 0};   // copies issued per stage (thread 0), for the drain after a timeout
@@ -541,59 +551,82 @@ __global__ void __launch_bounds__(FT_WARPS * 32 * KG)
   __syncthreads();
 
   bool ok = true;
+  const bool live = rbase < rows;   // rows past `rows` read stale bytes and are never stored
   for (int p = 0; p < P; ++p) {
     const int st = p % (int)L.nstage;
     if (!sm100::mbar_wait(bars + 8 * st, (p / (int)L.nstage) & 1, FT_WAIT_BUDGET)) ok = false;
-    if (ok && 16 * warp < rows) {
-      const uint32_t sbase = base + st * L.stage_bytes;
+    if (ok && live) {
+      const uint32_t sb = base + st * L.stage_bytes;
       const uint32_t ldp = (uint32_t)ps.ldSA[p];
-      const uint32_t r0 = sbase + (16 * warp + g) * ldp, r1 = r0 + 8 * ldp;   // rows past `rows` read stale bytes: not stored
-      const uint32_t fb = sbase + L.sign_bytes + lane * 16;
-      float acc[NB][4];
+      uint32_t r0[RT];
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+      for (int t = 0; t < RT; ++t) r0[t] = sb + (rbase + 16 * t + g) * ldp;
+      const uint32_t fb = sb + L.sign_bytes + lane * 16;
+      float acc[RT][NB][4];
+#pragma unroll
+      for (int t = 0; t < RT; ++t)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) acc[t][nb][0] = acc[t][nb][1] = acc[t][nb][2] = acc[t][nb][3] = 0.f;
 #pragma unroll 2
       for (int qw = qw0; qw < qw1; ++qw) {
-        const uint32_t s0 = lds32s(r0 + 4 * qw), s1 = lds32s(r1 + 4 * qw);
+        uint32_t s0[RT], s1[RT];
+#pragma unroll
+        for (int t = 0; t < RT; ++t) {
+          s0[t] = lds32s(r0[t] + 4 * qw);
+          s1[t] = lds32s(r0[t] + 8 * ldp + 4 * qw);
+        }
         uint4 bf[NB];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) bf[nb] = lds128(fb + (qw * NB + nb) * 512);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int sa = 15 - 8 * h - q, sb = 11 - 8 * h - q;
-          const uint32_t a0 = sign_pair(s0, sa), a1 = sign_pair(s1, sa), a2 = sign_pair(s0, sb), a3 = sign_pair(s1, sb);
+          const uint32_t ma = 1u << (15 - 8 * h - q), mb = 1u << (11 - 8 * h - q);
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb)
-            mma16816(acc[nb], a0, a1, a2, a3, h ? bf[nb].z : bf[nb].x, h ? bf[nb].w : bf[nb].y);
+          for (int t = 0; t < RT; ++t) {
+            const uint32_t a0 = sign_pair_mul(s0[t], ma), a1 = sign_pair_mul(s1[t], ma),
+                           a2 = sign_pair_mul(s0[t], mb), a3 = sign_pair_mul(s1[t], mb);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+              mma16816(acc[t][nb], a0, a1, a2, a3, h ? bf[nb].z : bf[nb].x, h ? bf[nb].w : bf[nb].y);
+          }
         }
       }
-      // D fragment -> per-warp scratch [16 rows][8 NB columns]
+      // D fragments -> this K group's scratch [tile][16 rows][8 NB columns]
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const int c = 8 * nb + 2 * q;
-        dsc[g * 8 * NB + c] = acc[nb][0];
-        dsc[g * 8 * NB + c + 1] = acc[nb][1];
-        dsc[(g + 8) * 8 * NB + c] = acc[nb][2];
-        dsc[(g + 8) * 8 * NB + c + 1] = acc[nb][3];
+      for (int t = 0; t < RT; ++t) {
+        float *dsc = dsc_of(kg, RT * rg + t);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          const int c = 8 * nb + 2 * q;
+          dsc[g * 8 * NB + c] = acc[t][nb][0];
+          dsc[g * 8 * NB + c + 1] = acc[t][nb][1];
+          dsc[(g + 8) * 8 * NB + c] = acc[t][nb][2];
+          dsc[(g + 8) * 8 * NB + c + 1] = acc[t][nb][3];
+        }
       }
     }
     __syncthreads();   // every warp is done with stage st and has written its partial D
-    if (ok && kg == 0 && 16 * warp < rows) {
+    if (ok && kg == 0 && live) {
       // sum the K groups' partials in group order, then the A_amp epilogue
-      for (int e = lane; e < 16 * 8 * NB; e += 32) {
-        float d = dsc_all[warp * 16 * 8 * NB + e];
-        for (int k = 1; k < KG; ++k) d += dsc_all[(k * FT_WARPS + warp) * 16 * 8 * NB + e];
-        dsc[e] = d;
-      }
-      __syncwarp();
-      for (int e = lane; e < 16 * B; e += 32) {
-        const int rr = e / B, b = e - rr * B, a = row0 + 16 * warp + rr;
-        if (a >= n) continue;
-        const float *Dr = dsc + rr * 8 * NB;
-        const uint16_t *am = ps.A[p] + (int64_t)a * l;
-        float sacc = yacc[e];
-        for (int i = 0; i < l; ++i) sacc = fmaf(qld::f16_to_f32(am[i]), Dr[b * l + i] + Dr[V + b * l + i], sacc);
-        yacc[e] = sacc;
+      for (int t = 0; t < RT; ++t) {
+        const int tile = RT * rg + t;
+        float *dsc = dsc_of(0, tile);
+        for (int e = lane; e < 16 * 8 * NB; e += 32) {
+          float d = dsc[e];
+          for (int k = 1; k < KG; ++k) d += dsc_of(k, tile)[e];
+          dsc[e] = d;
+        }
+        __syncwarp();
+        float *yacc = yacc_all + tile * 16 * B;
+        for (int e = lane; e < 16 * B; e += 32) {
+          const int rr = e / B, b = e - rr * B, a = row0 + 16 * tile + rr;
+          if (a >= n) continue;
+          const float *Dr = dsc + rr * 8 * NB;
+          const uint16_t *am = ps.A[p] + (int64_t)a * l;
+          float sacc = yacc[e];
+          for (int i = 0; i < l; ++i) sacc = fmaf(qld::f16_to_f32(am[i]), Dr[b * l + i] + Dr[V + b * l + i], sacc);
+          yacc[e] = sacc;
+        }
       }
     }
     __syncthreads();   // partials consumed; stage st free
@@ -612,13 +645,18 @@ __global__ void __launch_bounds__(FT_WARPS * 32 * KG)
     __syncthreads();
     return;
   }
-  for (int e = lane; e < 16 * B; e += 32) {
-    const int rr = e / B, b = e - rr * B, a = row0 + 16 * warp + rr;
-    if (kg != 0 || a >= n || 16 * warp >= rows) continue;
-    if (ydt == QL_OUT_F32)
-      static_cast<float *>(y)[(int64_t)b * n + a] = yacc[e];
-    else
-      static_cast<uint16_t *>(y)[(int64_t)b * n + a] = qld::f32_to_bf16_rn(yacc[e]);
+  if (kg != 0 || !live) return;
+  for (int t = 0; t < RT; ++t) {
+    const int tile = RT * rg + t;
+    const float *yacc = yacc_all + tile * 16 * B;
+    for (int e = lane; e < 16 * B; e += 32) {
+      const int rr = e / B, b = e - rr * B, a = row0 + 16 * tile + rr;
+      if (a >= n) continue;
+      if (ydt == QL_OUT_F32)
+        static_cast<float *>(y)[(int64_t)b * n + a] = yacc[e];
+      else
+        static_cast<uint16_t *>(y)[(int64_t)b * n + a] = qld::f32_to_bf16_rn(yacc[e]);
+    }
   }
 }
 
@@ -740,14 +778,19 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     // staged-tile F stage when two (else one) path stages fit in shared memory
     size_t ld_max = 0;
     for (int p = 0; p < P; ++p) ld_max = std::max(ld_max, ps.ldSA[p]);
-    constexpr int KG = NB <= 4 ? 4 : NB == 8 ? 2 : 1;   // K-word groups: as many warps as the registers allow
-    FTileLayout L = ftile_layout(ld_max, r, NB, B, 2, KG);
-    if (L.total > 227 * 1024) L = ftile_layout(ld_max, r, NB, B, 1, KG);
+    constexpr int RT = NB <= 2 ? 2 : 1;                   // row tiles per warp, sharing each fragment load
+    constexpr int KG = NB <= 2 ? 8 : NB == 4 ? 4 : NB == 8 ? 2 : 1;   // K-word groups: as many warps as registers allow
+    // 128-row CTAs when they fill the SMs, else 32-row CTAs (RT == 2) so that small n still spreads
+    const bool small = RT == 2 && (n + 127) / 128 < ql::sm_count();
+    const int tiles = small ? RT : 8;
+    FTileLayout L = ftile_layout(ld_max, r, NB, B, small ? 1 : 2, KG, tiles);
+    if (L.total > 227 * 1024) L = ftile_layout(ld_max, r, NB, B, 1, KG, tiles);
     if (L.total <= 227 * 1024) {
-      auto kt = mdbf_f_tile_kernel<NB, KG>;
+      auto kt = small ? mdbf_f_tile_kernel<NB, KG, RT, 1> : mdbf_f_tile_kernel<NB, KG, RT, 8 / RT>;
       if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total) != cudaSuccess)
         return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-      ql::launch(kt, (n + FT_ROWS - 1) / FT_ROWS, FT_WARPS * 32 * KG, L.total, s, ps, P, (const uint4 *)wpk, y,
+      const int threads = (small ? 1 : 8 / RT) * 32 * KG;
+      ql::launch(kt, (n + 16 * tiles - 1) / (16 * tiles), threads, L.total, s, ps, P, (const uint4 *)wpk, y,
                  (int)ydt, n, r, l, B, L);
       return ql::launch_status("mdbf_linear (F stage)");
     }
