@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_f_mma_kernel(Paths ps, int
 // let path p + 1 (or p + 2) arrive while path p is multiplied.  Warp w owns rows
 // [16 (w % 8), +16) of the block over the K-word group w / 8 (KG groups of consecutive words);
 // the groups' partial sums are added in group order.  Paths are summed in p order.
-constexpr int FT_WARPS = 8;   // 16-row tiles of a full-size F block
+constexpr int FT_TILES = 8;   // 16-row tiles of a full-size (128-row) F block
 constexpr long long FT_WAIT_BUDGET = 4000000000LL;   // clock cycles (~2 s)
 
 
@@ -782,14 +782,14 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     constexpr int KG = NB <= 2 ? 8 : NB == 4 ? 4 : NB == 8 ? 2 : 1;   // K-word groups: as many warps as registers allow
     // 128-row CTAs when they fill the SMs, else 32-row CTAs (RT == 2) so that small n still spreads
     const bool small = RT == 2 && (n + 127) / 128 < ql::sm_count();
-    const int tiles = small ? RT : 8;
+    const int tiles = small ? RT : FT_TILES;
     FTileLayout L = ftile_layout(ld_max, r, NB, B, small ? 1 : 2, KG, tiles);
     if (L.total > 227 * 1024) L = ftile_layout(ld_max, r, NB, B, 1, KG, tiles);
     if (L.total <= 227 * 1024) {
-      auto kt = small ? mdbf_f_tile_kernel<NB, KG, RT, 1> : mdbf_f_tile_kernel<NB, KG, RT, 8 / RT>;
+      auto kt = small ? mdbf_f_tile_kernel<NB, KG, RT, 1> : mdbf_f_tile_kernel<NB, KG, RT, FT_TILES / RT>;
       if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total) != cudaSuccess)
         return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-      const int threads = (small ? 1 : 8 / RT) * 32 * KG;
+      const int threads = (small ? 1 : FT_TILES / RT) * 32 * KG;
       ql::launch(kt, (n + 16 * tiles - 1) / (16 * tiles), threads, L.total, s, ps, P, (const uint4 *)wpk, y,
                  (int)ydt, n, r, l, B, L);
       return ql::launch_status("mdbf_linear (F stage)");
