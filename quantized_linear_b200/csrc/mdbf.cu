@@ -302,10 +302,13 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_mma_kernel(Paths ps, con
     wpk[((size_t)p * QWr + qw) * NB * 32 + e] = pack_fragment(get, qw, e >> 5, e & 31, r, V);
 }
 
-// G stage as above, with the CTA's 32 sign rows staged in shared memory by one bulk copy issued
-// before the wait on the preceding kernel (the rows are contiguous: ldSB apart).  Warps split
-// the K words as mdbf_g_mma_kernel does and load the next word group's fragments while the
-// current one is multiplied.  Rows past r read stale shared memory; their results are dropped.
+// G stage as above, with each warp streaming its word groups through a private 4-stage ring in
+// shared memory filled by cp.async: per group of SP_U words, lane (g, q) copies 16 bytes of sign
+// row g + 8q (the 32 rows of the block) and its own 16-byte fragment register sets, three groups
+// ahead of the one being multiplied.  The first groups' signs are requested before the wait on
+// the preceding kernel.  Needs 16-byte aligned sign rows.
+constexpr int GR_STAGES = 4;
+
 // set when a bounded wait of an MDBF kernel runs out; read and cleared by ql_check()
 __device__ int g_mdbf_timeout = 0;
 
@@ -320,31 +323,56 @@ __device__ __forceinline__ uint32_t lds32s(uint32_t a) {
   return v;
 }
 
-constexpr long long G_WAIT_BUDGET = 4000000000LL;   // clock cycles (~2 s)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int NB>
+__host__ __device__ constexpr int g_ring_stage_bytes() { return 32 * 16 + SP_U * NB * 32 * 16; }
 
 template <int NB>
 __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, const uint4 *__restrict__ zpk,
                                                                       uint4 *__restrict__ wpk, int m, int r, int l,
-                                                                      int B, uint32_t sign_bytes) {
+                                                                      int B) {
+  constexpr int STAGE = g_ring_stage_bytes<NB>();
   extern __shared__ __align__(128) unsigned char gsm[];
   const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(gsm));
-  float *red = reinterpret_cast<float *>(gsm + sign_bytes + 128), *D = red + SP_WARPS * 2 * NB * 128,
+  float *red = reinterpret_cast<float *>(gsm + SP_WARPS * GR_STAGES * STAGE), *D = red + SP_WARPS * 2 * NB * 128,
         *Ws = D + 32 * 8 * NB;
   const int p = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
   const int QW = (m + 31) / 32, V = l * B;
-  const int row0 = blockIdx.x * 32, rows = min(32, r - row0);
-  const uint32_t ld = (uint32_t)ps.ldSB[p], bar = sbase + sign_bytes;
-  if (threadIdx.x == 0) {
-    sm100::mbar_init(bar, 1);
-    sm100::fence_barrier_init();
-    sm100::mbar_arrive_expect_tx(bar, rows * ld);
-    sm100::bulk_g2s(sbase, ps.SB[p] + (size_t)row0 * ld, rows * ld, bar);
-  }
+  const int row0 = blockIdx.x * 32;
+  const size_t ld = ps.ldSB[p];
+  const uint32_t ring = sbase + warp * GR_STAGES * STAGE;
+  const uint4 *vb = zpk + (size_t)p * QW * NB * 32;
+  // this lane's sign row (rows past r repeat the last row; their results are dropped)
+  const uint8_t *srow = ps.SB[p] + (size_t)min(row0 + g + 8 * q, r - 1) * ld;
+  int w0, w1;
+  warp_words(QW, warp, w0, w1);
+  const int ngroups = (w1 - w0 + SP_U - 1) / SP_U;
+  auto issue_signs = [&](int grp) {
+    const uint32_t st = ring + (grp % GR_STAGES) * STAGE;
+    cp_async16(st + (g + 8 * q) * 16, srow + 4 * (w0 + SP_U * grp));   // 16 bytes: SP_U sign words
+  };
+  auto issue_frags = [&](int grp) {
+    const uint32_t st = ring + (grp % GR_STAGES) * STAGE + 32 * 16;
+#pragma unroll
+    for (int u = 0; u < SP_U; ++u) {
+      const int qw = min(w0 + SP_U * grp + u, QW - 1);   // words past the range are loaded but multiply zero-padding... see below
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) cp_async16(st + ((u * NB + nb) * 32 + lane) * 16, vb + ((size_t)qw * NB + nb) * 32 + lane);
+    }
+  };
+  for (int grp = 0; grp < GR_STAGES - 1 && grp < ngroups; ++grp) issue_signs(grp);
   qld::pdl_trigger();
   qld::pdl_wait();
-  __syncthreads();
-  const bool ok = sm100::mbar_wait(bar, 0, G_WAIT_BUDGET);
-  if (!ok && threadIdx.x == 0) atomicExch(&g_mdbf_timeout, 1);
+  for (int grp = 0; grp < GR_STAGES - 1; ++grp) {
+    if (grp < ngroups) issue_frags(grp);
+    cp_async_commit();
+  }
 
   float acc[2][NB][4];
 #pragma unroll
@@ -353,40 +381,34 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
     for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
-  int w0, w1;
-  warp_words(QW, warp, w0, w1);
-  const uint4 *vb = zpk + (size_t)p * QW * NB * 32;
-  uint32_t rowaddr[2][2];
-#pragma unroll
-  for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) rowaddr[rt][hh] = sbase + (16 * rt + g + 8 * hh) * ld;
-  constexpr int UB = NB <= 2 ? SP_U : 1;   // words of fragments held per group
-  auto load_frags = [&](uint4 (&bf)[UB][NB], int qwb) {
-#pragma unroll
-    for (int u = 0; u < UB; ++u)
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
-        bf[u][nb] = (qwb + u < w1) ? __ldg(vb + ((size_t)(qwb + u) * NB + nb) * 32 + lane) : make_uint4(0, 0, 0, 0);
-  };
-  uint4 cur[UB][NB], nxt[UB][NB];
-  if (ok && w0 < w1) load_frags(cur, w0);
-  for (int qw0 = w0; ok && qw0 < w1; qw0 += SP_U) {
+  for (int grp = 0; grp < ngroups; ++grp) {
+    cp_async_wait<GR_STAGES - 2>();
+    __syncwarp();   // sign rows were copied by other lanes of the warp
+    const uint32_t st = ring + (grp % GR_STAGES) * STAGE;
     uint32_t sw[SP_U][2][2];
 #pragma unroll
     for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        const uint4 v = lds128(rowaddr[rt][hh] + 4 * qw0);
+        const uint4 v = lds128(st + (16 * rt + g + 8 * hh) * 16);
         sw[0][rt][hh] = v.x; sw[1][rt][hh] = v.y; sw[2][rt][hh] = v.z; sw[3][rt][hh] = v.w;
       }
-    if constexpr (UB == SP_U) {
-      if (qw0 + SP_U < w1) load_frags(nxt, qw0 + SP_U);
+    uint4 bf[SP_U][NB];
+#pragma unroll
+    for (int u = 0; u < SP_U; ++u)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) bf[u][nb] = lds128(st + 32 * 16 + ((u * NB + nb) * 32 + lane) * 16);
+    __syncwarp();   // every lane has read this stage before it is refilled
+    const int nxt = grp + GR_STAGES - 1;
+    if (nxt < ngroups) {
+      issue_signs(nxt);
+      issue_frags(nxt);
     }
+    cp_async_commit();
+    const int valid = min(SP_U, w1 - (w0 + SP_U * grp));   // words of this group inside the warp's range
 #pragma unroll
     for (int u = 0; u < SP_U; ++u) {
-      if constexpr (UB != SP_U) load_frags(cur, qw0 + u);
-      const int slot = UB == SP_U ? u : 0;
+      if (u >= valid) break;
 #pragma unroll
       for (int rt = 0; rt < 2; ++rt) {
 #pragma unroll
@@ -395,20 +417,13 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
           const uint32_t a0 = sign_pair_mul(sw[u][rt][0], ma), a1 = sign_pair_mul(sw[u][rt][1], ma);
           const uint32_t a2 = sign_pair_mul(sw[u][rt][0], mb), a3 = sign_pair_mul(sw[u][rt][1], mb);
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            const uint32_t b0 = h ? cur[slot][nb].z : cur[slot][nb].x, b1 = h ? cur[slot][nb].w : cur[slot][nb].y;
-            mma16816(acc[rt][nb], a0, a1, a2, a3, b0, b1);
-          }
+          for (int nb = 0; nb < NB; ++nb)
+            mma16816(acc[rt][nb], a0, a1, a2, a3, h ? bf[u][nb].z : bf[u][nb].x, h ? bf[u][nb].w : bf[u][nb].y);
         }
       }
     }
-    if constexpr (UB == SP_U) {
-#pragma unroll
-      for (int u = 0; u < UB; ++u)
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) cur[u][nb] = nxt[u][nb];
-    }
   }
+  cp_async_wait<0>();
   reduce_fragments<NB, 2>(red, D, acc);
   for (int e = threadIdx.x; e < 32 * B; e += blockDim.x) {
     const int rr = e / B, b = e - rr * B, k = row0 + rr;
@@ -746,18 +761,13 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
   if (cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg) != cudaSuccess ||
       cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf) != cudaSuccess)
     return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-  // G stage with staged signs when the 32 sign rows fit next to the reduction buffers
-  bool g_tile = false;
-  uint32_t g_sign_bytes = 0;
-  size_t smg_t = 0;
-  if constexpr (VEC16) {
-    size_t ldb = 0;
-    for (int p = 0; p < P; ++p) ldb = std::max(ldb, ps.ldSB[p]);
-    g_sign_bytes = (uint32_t)((32 * ldb + 127) / 128 * 128);
-    smg_t = g_sign_bytes + 128 + smg;
-    g_tile = smg_t <= 227 * 1024;
-    if (g_tile && cudaFuncSetAttribute(mdbf_g_tile_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smg_t) != cudaSuccess)
+  // G stage through per-warp cp.async rings when sign rows are 16-byte aligned and the vectors
+  // are narrow (decode batches); wider ones keep mdbf_g_mma_kernel
+  constexpr bool g_ring = VEC16 && NB <= 2;
+  const size_t smg_t = (size_t)SP_WARPS * GR_STAGES * g_ring_stage_bytes<NB>() + smg;
+  if constexpr (g_ring) {
+    if (cudaFuncSetAttribute(mdbf_g_tile_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg_t) !=
+        cudaSuccess)
       return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
   }
   {
@@ -767,9 +777,9 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
-  if (g_tile)
+  if (g_ring)
     ql::launch(mdbf_g_tile_kernel<NB>, dim3((r + 31) / 32, P), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
-               m, r, l, B, g_sign_bytes);
+               m, r, l, B);
   else
     ql::launch(kg, dim3((r + 31) / 32, P), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
   ql_status st = ql::launch_status("mdbf_linear (G stage)");
