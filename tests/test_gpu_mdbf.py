@@ -102,3 +102,36 @@ def test_linear_is_deterministic(ql):
     a = _linear(ql, paths, 1024, 768, 300, 4, x)
     b = _linear(ql, paths, 1024, 768, 300, 4, x)
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("B", [1, 2])
+def test_linear_tall_layer_full_size_blocks(ql, B):
+    # n >= 128 x 148 rows: the F stage runs 128-row blocks (smaller n runs 32-row blocks)
+    n, m, r, l, P = 20480, 1024, 256, 4, 2
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=5000 + B)
+    x = synth.activations(B, m, seed=5100 + B)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    rows = np.r_[np.random.default_rng(4).choice(n, 256, replace=False), 0, 127, 128, n - 129, n - 1]
+    assert max_rel(y[:, rows], om.linear_factored(paths, n, m, r, x, rows=rows)) <= MDBF_TOL
+
+
+@pytest.mark.parametrize("l,B", [(4, 4), (4, 8), (2, 16)])
+def test_linear_wider_vector_blocks(ql, l, B):
+    # l * B = 16, 32, 32: four and eight 8-column MMA blocks per word
+    n, m, r, P = 700, 900, 300, 2
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=5200 + l * B)
+    x = synth.activations(B, m, seed=5300 + B)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+
+
+@pytest.mark.parametrize("B", [1, 3])
+def test_linear_unaligned_sign_strides(ql, B):
+    # row strides that are multiples of 4 but not of 16 take the kernels that read signs per lane
+    n, m, r, l, P = 300, 200, 100, 2, 2
+    ldSA, ldSB = 20, 28   # >= ceil(100/8) = 13 and >= ceil(200/8) = 25
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=5400 + B, ldSA=ldSA, ldSB=ldSB)
+    assert paths[0].S_A.shape[1] == ldSA and paths[0].S_B.shape[1] == ldSB
+    x = synth.activations(B, m, seed=5500 + B)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
