@@ -790,8 +790,9 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     for (int p = 0; p < P; ++p) ld_max = std::max(ld_max, ps.ldSA[p]);
     constexpr int RT = NB <= 2 ? 2 : 1;                   // row tiles per warp, sharing each fragment load
     constexpr int KG = NB <= 2 ? 8 : NB == 4 ? 4 : NB == 8 ? 2 : 1;   // K-word groups: as many warps as registers allow
-    // 128-row CTAs when they fill the SMs, else 32-row CTAs (RT == 2) so that small n still spreads
-    const bool small = RT == 2 && (n + 127) / 128 < ql::sm_count();
+    // 32-row CTAs (RT == 2, one stage, three per SM) when 128-row ones would leave SMs idle and the
+    // 32-row ones still fit in one round; else 128-row CTAs
+    const bool small = RT == 2 && (n + 127) / 128 < ql::sm_count() && (n + 31) / 32 <= 3 * ql::sm_count();
     const int tiles = small ? RT : FT_TILES;
     FTileLayout L = ftile_layout(ld_max, r, NB, B, small ? 1 : 2, KG, tiles);
     if (L.total > 227 * 1024) L = ftile_layout(ld_max, r, NB, B, 1, KG, tiles);
