@@ -137,7 +137,10 @@ typedef struct {
   const uint16_t *Q_V;    /* fp16 bits [r][l] */
 } mdbf_path;
 
-/* Bytes of device workspace mdbf_linear needs for these sizes (0 on invalid sizes). */
+/* Bytes of device workspace mdbf_linear needs for these sizes (0 on invalid sizes).  For
+ * batches that run on the tensor cores (see mdbf_linear) the size depends on how many CTA pairs
+ * the current device holds at once: query it with the device current that will run the call
+ * (without a device it returns the size of a run that does not split the last wave). */
 QL_API size_t mdbf_workspace_bytes(int P, int n, int m, int r, int l, int B);
 
 /*
@@ -154,7 +157,14 @@ QL_API size_t mdbf_workspace_bytes(int P, int n, int m, int r, int l, int B);
  *   y          device, [B][n] of y_dtype; fully overwritten.
  *   workspace  device scratch of ws_bytes >= mdbf_workspace_bytes(...), 256-byte
  *              aligned; contents on entry are ignored and on return undefined.
- *   Limits: l * B <= 64 (else QL_ERR_UNSUPPORTED).
+ *   Execution: l * B <= 64 runs the decode kernels once (sign products on the warp MMA with
+ *   the dense operand split into bf16 high and low parts).  Larger batches with l <= 32 and
+ *   n, m, r >= 64 run as two tensor-core GEMMs, T = X G^T and y = T F^T, each factor element
+ *   rebuilt in fp16 inside the GEMM (fp32 accumulation); each token row of x is first scaled by
+ *   a power of two so that x and T fit fp16, and y is scaled back exactly.  This assumes every
+ *   factor element |F[a][k]|, |G[k][j]| is below 65504.  All other batches run through the
+ *   decode kernels floor(64 / l) rows at a time.
+ *   Limits: l <= 64 (else QL_ERR_UNSUPPORTED), P <= 8.
  */
 QL_API ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r, int l,
                       const uint16_t *x, void *y, ql_out_dtype y_dtype, int B, void *workspace,

@@ -211,13 +211,16 @@ ql_status ql_check(ql_stream_t stream) {
   g_msg[0] = 0;
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(QL_ERR_CUDA, "ql_check: %s", cudaGetErrorString(e));
-  int flag = 0, flag2 = 0;
+  int flag = 0, flag2 = 0, flag3 = 0;
   ql_status st = ql::benq_gemm_read_timeout(&flag);
   if (st != QL_OK) return st;
   st = ql::mdbf_read_timeout(&flag2);
   if (st != QL_OK) return st;
+  st = ql::mdbf_gemm_read_timeout(&flag3);
+  if (st != QL_OK) return st;
   if (flag) return fail(QL_ERR_TIMEOUT, "a bounded device-side wait of the GEMM ran out (code %d)", flag);
   if (flag2) return fail(QL_ERR_TIMEOUT, "a bounded device-side wait of the MDBF F stage ran out (code %d)", flag2);
+  if (flag3) return fail(QL_ERR_TIMEOUT, "a bounded device-side wait of the MDBF GEMM ran out (code %d)", flag3);
   return QL_OK;
 }
 

@@ -29,9 +29,12 @@
 #include <mutex>
 
 #include "ql_internal.cuh"
+#include "pair_gemm.cuh"
 #include "sm100_ptx.cuh"
 
 namespace {
+
+using namespace pairgemm;
 
 constexpr int BM = 256;                           // X rows per CTA (two 128-row MMA halves)
 constexpr int PM = 2 * BM;                        // X rows per pair tile
@@ -56,7 +59,6 @@ constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;          // tensor-memory address, 
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;      // + alignment slack
 constexpr int NDEC = 16;                              // decoder / epilogue warps (multiple of 8)
 constexpr int THREADS = (3 + NDEC) * 32;              // A producer, MMA issuer, code producer, decoders
-constexpr long long WAIT_BUDGET = 4000000000LL;       // clock cycles (~2 s)
 constexpr uint32_t IDESC = sm100::idesc_bf16_f32(2 * 128, BN);   // pair MMA: M = 256 over two CTAs
 constexpr uint16_t PAIR = 0x3;                        // both CTAs of the cluster
 static_assert(OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
@@ -75,65 +77,6 @@ struct Bars {
         full_c(empty_b + 8 * SB), empty_c(full_c + 8 * SC), lut_full(empty_c + 8 * SC), lut_empty(lut_full + 8),
         acc_full(lut_empty + 8), acc_empty(acc_full + 8), split_done(acc_empty + 8), split_go(split_done + 8) {}
 };
-
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-__device__ __forceinline__ void sts64(uint32_t a, uint32_t lo, uint32_t hi) {
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(lo), "r"(hi) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_volatile_u32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-
-// Bounded wait shared by all roles.  Gives up when the budget runs out or when the pair's abort
-// flag is set; a thread that runs out sets the flag in both CTAs so that the others stop at once.
-struct Waiter {
-  uint32_t abort_local, abort_peer;
-  __device__ bool wait(uint32_t bar, uint32_t parity, bool cluster_scope) const {
-    auto probe = [&] {
-      return cluster_scope ? sm100::mbar_try_wait_cluster(bar, parity) : sm100::mbar_try_wait(bar, parity);
-    };
-    if (probe()) return true;
-    const long long t0 = clock64();
-    while (!probe()) {
-      if (ld_volatile_u32(abort_local) != 0) return false;
-      if (clock64() - t0 > WAIT_BUDGET) {
-        sts32(abort_local, 1);
-        st_cluster_u32(abort_peer, 1);
-        return false;
-      }
-    }
-    return true;
-  }
-};
-
-// Work items: pair tiles 0 .. full-1 whole, then each of the remaining tiles (the last, partial
-// wave) split into `parts` K ranges so that the otherwise idle pairs share it.  A split item
-// writes an fp32 partial; the last CTA to finish a tile sums the partials in part order.
-struct Item {
-  int tile, kb0, kb1, part;   // part < 0: whole tile
-};
-__device__ __forceinline__ Item item_of(int i, int full, int parts, int nkb) {
-  if (i < full) return {i, 0, nkb, -1};
-  const int u = i - full, j = u / parts, q = u - j * parts;
-  return {full + j, (int)((int64_t)q * nkb / parts), (int)((int64_t)(q + 1) * nkb / parts), q};
-}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     benq_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
@@ -256,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint64_t adesc = sm100::sw128_kmajor_desc(a + h * (A_BYTES / 2) + kk * 32);
-              sm100::mma_bf16_pair(tmem + h * BN, adesc, bdesc, IDESC, (kb > w.kb0 || kk > 0) ? 1u : 0u);
+              sm100::mma_f16kind_pair(tmem + h * BN, adesc, bdesc, IDESC, (kb > w.kb0 || kk > 0) ? 1u : 0u);
             }
           }
           sm100::mma_commit_pair(bar.empty_a + 8 * sa, PAIR);
@@ -442,23 +385,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 // Opts the GEMM kernel into its dynamic shared memory (once per process).
 cudaError_t smem_attr() {
   static std::once_flag once;
@@ -492,29 +418,8 @@ int resident_pairs() {
   return cache[dev];
 }
 
-constexpr int SPLIT_MAX = 8;   // K ranges per tile of the last wave
-
-// Whole tiles run in full waves of `pairs` CTA pairs; when the last wave would leave at least
-// half of the pairs idle, its L tiles are split into `parts` K ranges each (L * parts <= pairs).
-struct SplitPlan {
-  int full, parts, leftover;
-  size_t partial_bytes, counter_bytes;
-};
 SplitPlan split_plan(int M, int N, int K, int pairs) {
-  const int ntiles = ((M + PM - 1) / PM) * (N / BN), nkb = K / BK;
-  SplitPlan p{ntiles, 1, 0, 0, 0};
-  const int full = (ntiles / pairs) * pairs, left = ntiles - full;
-  if (left > 0 && 2 * left <= pairs) {
-    const int parts = std::min(std::min(pairs / left, SPLIT_MAX), nkb);
-    if (parts >= 2) {
-      p.full = full;
-      p.parts = parts;
-      p.leftover = left;
-      p.partial_bytes = (size_t)left * parts * 2 * BM * BN * sizeof(float);
-      p.counter_bytes = ((size_t)left * 2 * sizeof(unsigned) + 255) / 256 * 256;
-    }
-  }
-  return p;
+  return pairgemm::split_plan(((M + PM - 1) / PM) * (N / BN), K / BK, pairs, (size_t)2 * BM * BN * sizeof(float));
 }
 
 }  // namespace
@@ -530,7 +435,7 @@ size_t benq_gemm_workspace_size(int M, int N, int K) {
 ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype ydt,
                            int M, int N, int K, void *ws, size_t ws_bytes, cudaStream_t s) {
   if (N % BN || K % BK) return fail(QL_ERR_UNSUPPORTED, "benq_linear: batch > 16 needs N %% 256 == 0 and K %% 64 == 0");
-  EncodeTiledFn enc = encode_fn();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return fail(QL_ERR_CUDA, "benq_linear: cuTensorMapEncodeTiled is unavailable");
   CUtensorMap mx, mc;
   {

@@ -856,15 +856,37 @@ ql_status mdbf_read_timeout(int *flag) {
   return QL_OK;
 }
 
+// Batches with l * B above VLIM run on the tensor cores (mdbf_gemm_sm100.cu) when the layer
+// qualifies (mdbf_use_gemm), otherwise through the decode kernels VLIM / l rows at a time.
 size_t mdbf_workspace_size(int P, int n, int m, int r, int l, int B) {
-  (void)n;
+  if (mdbf_use_gemm(n, m, r, l, B, VLIM)) return mdbf_gemm_workspace_size(P, n, m, r, l, B);
+  if (l * B > VLIM && l <= VLIM) B = VLIM / l;
   return ws_layout(P, m, r, l, B).total;
 }
+
+ql_status mdbf_decode_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x, void *y,
+                             ql_out_dtype ydt, int B, void *ws, cudaStream_t s);
 
 ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x,
                              void *y, ql_out_dtype ydt, int B, void *ws, cudaStream_t s) {
   if (P > PMAX) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: P = %d exceeds %d paths", P, PMAX);
-  if (l * B > VLIM) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: l*B = %d exceeds %d", l * B, VLIM);
+  if (l * B <= VLIM) return mdbf_decode_launch(paths, P, n, m, r, l, x, y, ydt, B, ws, s);
+  if (mdbf_use_gemm(n, m, r, l, B, VLIM)) return mdbf_gemm_launch(paths, P, n, m, r, l, x, y, ydt, B, ws, s);
+  if (l > VLIM) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: l = %d exceeds %d", l, VLIM);
+  const int bc = VLIM / l;
+  const size_t ysz = ydt == QL_OUT_F32 ? 4 : 2;
+  for (int b0 = 0; b0 < B; b0 += bc) {
+    const ql_status st = mdbf_decode_launch(paths, P, n, m, r, l, x + (size_t)b0 * m,
+                                            static_cast<char *>(y) + (size_t)b0 * n * ysz, ydt, std::min(bc, B - b0),
+                                            ws, s);
+    if (st != QL_OK) return st;
+  }
+  return QL_OK;
+}
+
+// The decode kernels: one pass for l * B <= VLIM token rows.
+ql_status mdbf_decode_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x, void *y,
+                             ql_out_dtype ydt, int B, void *ws, cudaStream_t s) {
   const Paths ps = pack_paths(paths, P);
   const WsLayout L = ws_layout(P, m, r, l, B);
   char *base = static_cast<char *>(ws);

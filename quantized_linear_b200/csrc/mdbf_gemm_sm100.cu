@@ -1,0 +1,789 @@
+// MDBF prefill on sm_100a tensor cores: Y[B][n] = X W^T with W = sum_p F_p G_p, W never formed.
+//
+// "MDBF (Multi-Envelope Double Binary Factorization)", section "Algorithm":
+//   F = S_A (.) (A_amp Q_U^T)   (n x r),     G = S_B (.) (Q_V B_amp^T)   (r x m).
+// For a batch of token rows the product is two dense contractions, both on the tensor cores:
+//   T = X [G_1; ..; G_P]^T            (B x P r: the paths side by side along N),
+//   Y = T [F_1 .. F_P]^T              (the paths concatenated along K, so their sum is free).
+// Neither factor is ever written to memory.  Inside the GEMM that consumes it, each factor element
+// is rebuilt from its packed sign bit and its envelope entry sum_i L[row][i] R[col][i]: the
+// envelope of a 16 x 8 block is one warp MMA (mma.sync m16n8k16, fp16 in, fp32 out; the fp16 x
+// fp16 products are exact), the sign flips the fp16 sign bit, and the element is rounded to fp16
+// straight into the tensor core's shared-memory operand tile.
+//
+// Numerics.  The tensor-core operands are fp16 (both operands of kind::f16 must share one type,
+// and fp16's 11-bit significand keeps the result well inside the parity tolerance where bf16's
+// 8 bits would not).  Activations arrive as bf16, whose range is wider than fp16's, so each token
+// row is first scaled by a power of two (exact) into X' with max|X'| in [2^-e, 2^(1-e)); e >= 0 is
+// the smallest exponent for which the envelope bound
+//   |T'[b][k]| <= m * max|X'| * beta,   beta = max_p sum_i max_k|Q_V[k][i]| * max_j|B_amp[j][i]|,
+// stays below half the fp16 maximum, so the intermediate T' = X' G^T is stored in fp16 without
+// overflow.  The last epilogue multiplies each row by the inverse power of two.  Decoded factor
+// elements are assumed to lie within fp16 range (|F|, |G| < 65504).
+//
+// Launches per call: envelope column maxima, activation prep (scale, convert, pad), GEMM 1
+// (decodes G), GEMM 2 (decodes F).  The GEMMs share the CTA-pair structure of the BenQ GEMM: CTA
+// r of a pair owns rows [256 r, 256 r + 256) of a 512 x 256 output tile and decodes operand rows
+// [128 r, 128 r + 128); pair MMAs (M = 256 over two CTAs, N = 256, K = 16) read A from each CTA and
+// B from both.  Per CTA: warp 0 loads A tiles (256 x 64 fp16, 128-byte swizzle) with tensor
+// copies, warp 1 (even CTA) issues the pair MMAs, warps 2..17 decode the factor operand and then
+// drain the accumulators.  No tensor or bulk load is multicast.  Every wait is bounded (see
+// pair_gemm.cuh); a wait that runs out sets a flag read by ql_check().
+#include <cuda.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "pair_gemm.cuh"
+#include "ql_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+using namespace pairgemm;
+
+constexpr int PMAX = 8;                           // paths per call (the ABI's limit)
+constexpr int LMAX = ql::MDBF_GEMM_LMAX;            // envelope rank handled by these kernels
+constexpr int BM = 256;                           // A rows per CTA (two 128-row MMA halves)
+constexpr int PM = 2 * BM;                        // A rows per pair tile
+constexpr int BN = 256;                           // operand rows per pair tile (the MMA's N)
+constexpr int BNH = BN / 2;                       // operand rows decoded by each CTA
+constexpr int BK = 64;                            // one 128-byte swizzle row of fp16
+constexpr int SA = 4, SB = 4;                     // stages: A tiles, decoded operand tiles
+constexpr int A_BYTES = BM * BK * 2;              // 32 KB
+constexpr int B_BYTES = BNH * BK * 2;             // 16 KB
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + SA * A_BYTES;
+constexpr int OFF_BAR = OFF_B + SB * B_BYTES;
+constexpr int NBAR = 2 * (SA + SB) + 4;
+constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // tensor-memory address, abort flag, last-part flag
+constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;  // + alignment slack
+constexpr int NDEC = 16;                          // decoder / epilogue warps: 8 row groups x 2 column halves
+constexpr int THREADS = (2 + NDEC) * 32;          // A producer, MMA issuer, decoders
+constexpr uint32_t IDESC = sm100::idesc_f16_f32(2 * 128, BN);   // pair MMA: M = 256 over two CTAs
+constexpr uint16_t PAIR = 0x3;
+// Bound the intermediate T' is kept under: half the fp16 maximum, which leaves room for the fp16
+// rounding of the decoded G and for the fp32 accumulation order.
+constexpr float T_BOUND = 32768.0f;
+static_assert(OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+
+__device__ int g_mgemm_timeout = 0;
+
+// One factor operand, as the GEMM that decodes it sees it: element (row, col) of path p is
+//   sign(bit col of S[p] row `row`) * sum_i Lrow[p][row][i] * Lcol[p][col][i].
+// For G: rows are k (r of them), columns j (m), Lrow = Q_V, Lcol = B_amp, S = S_B; the paths sit
+// side by side along the GEMM's N (path p owns rows [p seg, p seg + r)).  For F: rows are a (n),
+// columns k (r), Lrow = A_amp, Lcol = Q_U, S = S_A; the paths follow one another along K (path p
+// owns K columns [p seg, p seg + r)).  seg = r rounded up to the K block.
+struct Factor {
+  const uint8_t *S[PMAX];
+  size_t ld[PMAX];
+  const uint16_t *Lrow[PMAX];
+  const uint16_t *Lcol[PMAX];
+  int rows, cols, seg, P, l;
+  int l_vec2;   // l even and every envelope base 4-byte aligned
+};
+
+struct Bars {
+  // full_a, full_b and acc_empty are used in the even CTA only (both CTAs arrive on them).
+  uint32_t full_a, empty_a, full_b, empty_b, acc_full, acc_empty, split_done, split_go;
+  __device__ Bars(uint32_t base)
+      : full_a(base), empty_a(full_a + 8 * SA), full_b(empty_a + 8 * SA), empty_b(full_b + 8 * SB),
+        acc_full(empty_b + 8 * SB), acc_empty(acc_full + 8), split_done(acc_empty + 8), split_go(split_done + 8) {}
+};
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// {fp16(lo), fp16(hi)} rounded to nearest even, lo in the low half
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint16_t f16_rn(float f) {
+  uint16_t h;
+  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(h) : "f"(f));
+  return h;
+}
+
+// Sign-flip mask of an fp16 pair from two adjacent sign bits: bit 1 keeps the value (+1), bit 0
+// flips it (-1).  JL = 0 takes bits 0 and 1 of e, JL = 1 bits 8 and 9; the multiply copies the
+// pair to bits 15/16 and 30/31 at once, and the mask keeps 15 and 31.
+template <int JL>
+__device__ __forceinline__ uint32_t sign_flip(uint32_t e) {
+  constexpr uint32_t keep = JL == 0 ? 0x3u : 0x300u;
+  constexpr uint32_t spread = JL == 0 ? 0x40008000u : 0x00400080u;   // 2^30 + 2^15, 2^22 + 2^7
+  uint32_t t;
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(t) : "r"(e & keep), "r"(spread));
+  return ~t & 0x80008000u;
+}
+
+// Two consecutive fp16 envelope entries v[i], v[i + 1] of one row (zero past l).
+__device__ __forceinline__ uint32_t env_pair(const uint16_t *__restrict__ v, int l, int i, bool vec2) {
+  if (i >= l) return 0u;
+  if (vec2) return __ldg(reinterpret_cast<const unsigned int *>(v + i));
+  const uint32_t lo = __ldg(reinterpret_cast<const unsigned short *>(v + i));
+  const uint32_t hi = i + 1 < l ? __ldg(reinterpret_cast<const unsigned short *>(v + i + 1)) : 0u;
+  return lo | (hi << 16);
+}
+
+// The 32 sign bits of columns [c0, c0 + 32) of one packed row (c0 a multiple of 32).  Rows are
+// 4-byte aligned with strides that are multiples of 4 (checked by the ABI), so a word that starts
+// inside the row's ceil(cols / 8) bytes ends inside its stride; bits past column cols - 1 are
+// padding and meet a zero envelope.  Words past the row's bytes are not read.
+__device__ __forceinline__ uint32_t sign_word(const uint8_t *__restrict__ row, int c0, int rowbytes) {
+  const int b0 = c0 >> 3;
+  return b0 < rowbytes ? __ldg(reinterpret_cast<const unsigned int *>(row + b0)) : 0u;
+}
+
+// ------------------------------------------------------------------ envelope column maxima
+// emax[p][0][z][i] = max |Q_V[k][i]| and emax[p][1][z][i] = max |B_amp[j][i]| over row slice z of
+// NSL (grid P x 2 x NSL).  Weights are read before the wait on the preceding kernel; the store
+// comes after it.
+constexpr int NSL = 16;
+__global__ void __launch_bounds__(256) mdbf_envmax_kernel(Factor g, float *__restrict__ emax) {
+  qld::pdl_trigger();
+  const int p = blockIdx.x, which = blockIdx.y, z = blockIdx.z;
+  const unsigned short *v = reinterpret_cast<const unsigned short *>(which == 0 ? g.Lrow[p] : g.Lcol[p]);
+  const int nrow = which == 0 ? g.rows : g.cols, l = g.l;
+  const int per = (nrow + NSL - 1) / NSL, r0 = z * per, r1 = min(nrow, r0 + per);
+  __shared__ float red[8][LMAX];
+  float mx[LMAX];
+#pragma unroll
+  for (int i = 0; i < LMAX; ++i) mx[i] = 0.f;
+  for (int rr = r0 + (int)threadIdx.x; rr < r1; rr += blockDim.x) {
+#pragma unroll
+    for (int i = 0; i < LMAX; ++i)
+      if (i < l) mx[i] = fmaxf(mx[i], fabsf(qld::f16_to_f32(__ldg(v + (size_t)rr * l + i))));
+  }
+#pragma unroll
+  for (int i = 0; i < LMAX; ++i) {
+    float a = mx[i];
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5][i] = a;
+  }
+  __syncthreads();
+  qld::pdl_wait();
+  if ((int)threadIdx.x < l) {
+    float a = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) a = fmaxf(a, red[w][threadIdx.x]);
+    emax[((p * 2 + which) * NSL + z) * LMAX + threadIdx.x] = a;
+  }
+}
+
+// ------------------------------------------------------------------ activation prep
+// One CTA per token row b: X'[b][j] = fp16(x[b][j] * 2^s_b) for j < m, 0 for m <= j < mp, and
+// inv_s[b] = 2^-s_b, with s_b chosen as described at the top of this file.  CTA 0 also clears the
+// split-tile counters of both GEMMs.
+__global__ void __launch_bounds__(256) mdbf_xprep_kernel(const uint16_t *__restrict__ x, int m, int mp,
+                                                         const float *__restrict__ emax, int P, int l,
+                                                         uint16_t *__restrict__ xs, float *__restrict__ inv_s,
+                                                         unsigned *__restrict__ counters, int ncounters, int vec8) {
+  qld::pdl_trigger();
+  qld::pdl_wait();
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const uint16_t *xr = x + (size_t)b * m;
+  __shared__ float red[8];
+  __shared__ int s_exp;
+  if (b == 0)
+    for (int i = tid; i < ncounters; i += blockDim.x) counters[i] = 0u;
+  float mx = 0.f;
+  if (vec8) {
+    for (int j = tid * 8; j < m; j += blockDim.x * 8) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + j));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        mx = fmaxf(mx, fmaxf(fabsf(qld::bf16_to_f32(w[i] & 0xFFFFu)), fabsf(qld::bf16_to_f32(w[i] >> 16))));
+    }
+  } else {
+    for (int j = tid; j < m; j += blockDim.x) mx = fmaxf(mx, fabsf(qld::bf16_to_f32(xr[j])));
+  }
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  if (tid == 0) {
+    float rmax = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) rmax = fmaxf(rmax, red[w]);
+    float beta = 0.f;
+    for (int p = 0; p < P; ++p) {
+      float sp = 0.f;
+      for (int i = 0; i < l; ++i) {
+        float mq = 0.f, mb = 0.f;
+        for (int z = 0; z < NSL; ++z) {
+          mq = fmaxf(mq, emax[((p * 2) * NSL + z) * LMAX + i]);
+          mb = fmaxf(mb, emax[((p * 2 + 1) * NSL + z) * LMAX + i]);
+        }
+        sp += mq * mb;
+      }
+      beta = fmaxf(beta, sp);
+    }
+    // e: smallest e >= 0 with m * 2^(1-e) * beta <= T_BOUND
+    int e = 0;
+    const float need = 2.0f * (float)m * beta / T_BOUND;
+    if (need > 1.0f) {
+      int ex;
+      const float f = frexpf(need, &ex);   // need = f 2^ex, f in [0.5, 1)
+      e = f == 0.5f ? ex - 1 : ex;
+    }
+    int se = 0;   // scale exponent: max|x'| = rmax 2^se in [2^-e, 2^(1-e))
+    if (rmax > 0.f) {
+      int ex;
+      (void)frexpf(rmax, &ex);   // rmax in [2^(ex-1), 2^ex)
+      se = 1 - ex - e;
+    }
+    se = max(-126, min(127, se));
+    s_exp = se;
+    inv_s[b] = ldexpf(1.0f, -se);
+  }
+  __syncthreads();
+  const float s = ldexpf(1.0f, s_exp);
+  uint16_t *xo = xs + (size_t)b * mp;
+  if (vec8) {
+    for (int j = tid * 8; j < mp; j += blockDim.x * 8) {
+      uint32_t o[4] = {0u, 0u, 0u, 0u};
+      if (j < m) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + j));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          o[i] = pack_f16x2(qld::bf16_to_f32(w[i] & 0xFFFFu) * s, qld::bf16_to_f32(w[i] >> 16) * s);
+      }
+      *reinterpret_cast<uint4 *>(xo + j) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  } else {
+    for (int j = tid; j < mp; j += blockDim.x) xo[j] = j < m ? f16_rn(qld::bf16_to_f32(xr[j]) * s) : (uint16_t)0;
+  }
+}
+
+// ------------------------------------------------------------------ output stores
+// NV consecutive accumulator values of one output row, starting at column col0.
+//   G stage (FST false): T' in fp16, unscaled; Nout is a multiple of 64, so a span is either
+//   wholly inside or wholly past it, and T' rows are 16-byte aligned.
+//   F stage: y in bf16 (round to nearest even) or fp32, each value times the row's inverse scale
+//   rs (a power of two, so the product is exact); spans past n or rows that are not vector-aligned
+//   are stored element by element.
+template <bool FST, int NV>
+__device__ __forceinline__ void put_span(void *out, int ldo, bool ovec, int ydt, int row, int col0, int Nout,
+                                         const float (&v)[NV], float rs) {
+  static_assert(NV % 4 == 0, "spans of 4");
+  if (!FST) {
+    if (col0 >= Nout) return;
+    uint16_t *o = static_cast<uint16_t *>(out) + (size_t)row * ldo + col0;
+#pragma unroll
+    for (int i = 0; i < NV / 4; ++i)
+      *reinterpret_cast<uint2 *>(o + 4 * i) = make_uint2(pack_f16x2(v[4 * i], v[4 * i + 1]), pack_f16x2(v[4 * i + 2], v[4 * i + 3]));
+    return;
+  }
+  const bool whole = ovec && col0 + NV <= Nout;
+  if (ydt == QL_OUT_F32) {
+    float *o = static_cast<float *>(out) + (size_t)row * ldo + col0;
+    if (whole) {
+#pragma unroll
+      for (int i = 0; i < NV / 4; ++i)
+        *reinterpret_cast<float4 *>(o + 4 * i) = make_float4(v[4 * i] * rs, v[4 * i + 1] * rs, v[4 * i + 2] * rs, v[4 * i + 3] * rs);
+    } else {
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (col0 + i < Nout) o[i] = v[i] * rs;
+    }
+  } else {
+    uint16_t *o = static_cast<uint16_t *>(out) + (size_t)row * ldo + col0;
+    if (whole) {
+#pragma unroll
+      for (int i = 0; i < NV / 4; ++i) {
+        const uint32_t lo = uint32_t(qld::f32_to_bf16_rn(v[4 * i] * rs)) | (uint32_t(qld::f32_to_bf16_rn(v[4 * i + 1] * rs)) << 16);
+        const uint32_t hi = uint32_t(qld::f32_to_bf16_rn(v[4 * i + 2] * rs)) | (uint32_t(qld::f32_to_bf16_rn(v[4 * i + 3] * rs)) << 16);
+        *reinterpret_cast<uint2 *>(o + 4 * i) = make_uint2(lo, hi);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (col0 + i < Nout) o[i] = qld::f32_to_bf16_rn(v[i] * rs);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ the GEMM
+// C[M][Nout] = A[M][K] D[Nout][K]^T with A an fp16 array read by tensor copies (map_a) and D the
+// factor operand decoded on the fly.  FST false: D = [G_1; ..; G_P] (N = P seg), C = T' in fp16.
+// FST true: D = [F_1 .. F_P] (K = P seg), C = y scaled by row_scale.  LC: envelope chunks of 16
+// (l <= 16 LC).
+template <bool FST, int LC>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    mdbf_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ Factor fac,
+                     void *__restrict__ out, int ldo, int ovec, int ydt, const float *__restrict__ row_scale, int M,
+                     int Nout, int nkb, float *__restrict__ part_ws, unsigned *__restrict__ part_cnt, int full,
+                     int parts) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  const Bars bar(sbase + OFF_BAR);
+  const uint32_t tmem_slot = sbase + OFF_TMEM;
+  const uint32_t rank = sm100::cluster_ctarank();        // 0: the even CTA, which issues the MMAs
+  const bool lead = rank == 0;
+  const Waiter wt{tmem_slot + 4, sm100::mapa_shared(tmem_slot + 4, rank ^ 1u)};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int mt = (M + PM - 1) / PM, nt = (Nout + BN - 1) / BN, ntiles = mt * nt;
+  const int nitems = full + (ntiles - full) * parts;
+  bool ok = true;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SA; ++s) {
+      sm100::mbar_init(bar.full_a + 8 * s, 1);
+      sm100::mbar_init(bar.empty_a + 8 * s, 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      sm100::mbar_init(bar.full_b + 8 * s, 2 * NDEC);
+      sm100::mbar_init(bar.empty_b + 8 * s, 1);
+    }
+    sm100::mbar_init(bar.acc_full, 1);
+    sm100::mbar_init(bar.acc_empty, 2 * NDEC);
+    sm100::mbar_init(bar.split_done, NDEC);
+    sm100::mbar_init(bar.split_go, 1);
+    sts32(tmem_slot + 4, 0);
+    sm100::fence_barrier_init();
+    sm100::prefetch_tensormap(&map_a);
+  }
+  if (warp == 1) {
+    __syncwarp();
+    sm100::tmem_alloc_pair(tmem_slot, 512);
+    sm100::tmem_relinquish_pair();
+  }
+  sm100::tc_fence_before();
+  sm100::cluster_sync();   // both CTAs' barriers initialised and tensor memory allocated
+  sm100::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem_raw + (tmem_slot - raw));
+  // the factor operand is weights: its decoders start at once; A is read and C written only
+  // after the preceding kernel in the stream has completed
+  qld::pdl_trigger();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ A producer (tensor copies)
+    if (lane == 0) {
+      qld::pdl_wait();
+      const uint32_t lead_full_a = sm100::mapa_shared(bar.full_a, 0);
+      int it = 0;
+      for (int wi = pair; wi < nitems && ok; wi += npairs) {
+        const Item w = item_of(wi, full, parts, nkb);
+        const int m0 = (w.tile % mt) * PM + (int)rank * BM;
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int s = it % SA;
+          if (it >= SA && !wt.wait(bar.empty_a + 8 * s, ((it / SA) & 1) ^ 1, true)) {
+            ok = false;
+            break;
+          }
+          if (lead) sm100::mbar_arrive_expect_tx(bar.full_a + 8 * s, 2 * A_BYTES);
+          sm100::tma_load_2d_pair(sbase + OFF_A + s * A_BYTES, &map_a, kb * BK, m0, lead_full_a + 8 * s);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ pair MMA issuer (even CTA)
+    if (lead && lane == 0) {
+      int it = 0, tl = 0;
+      for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
+        const Item w = item_of(wi, full, parts, nkb);
+        if (tl > 0 && !wt.wait(bar.acc_empty, (tl - 1) & 1, true)) { ok = false; break; }
+        sm100::tc_fence_after();
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int sa = it % SA, sb = it % SB;
+          if (!wt.wait(bar.full_a + 8 * sa, (it / SA) & 1, true) ||
+              !wt.wait(bar.full_b + 8 * sb, (it / SB) & 1, true)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint32_t a = sbase + OFF_A + sa * A_BYTES, b = sbase + OFF_B + sb * B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bdesc = sm100::sw128_kmajor_desc(b + kk * 32);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t adesc = sm100::sw128_kmajor_desc(a + h * (A_BYTES / 2) + kk * 32);
+              sm100::mma_f16kind_pair(tmem + h * BN, adesc, bdesc, IDESC, (kb > w.kb0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          sm100::mma_commit_pair(bar.empty_a + 8 * sa, PAIR);
+          sm100::mma_commit_pair(bar.empty_b + 8 * sb, PAIR);
+        }
+        if (!ok) break;
+        sm100::mma_commit_pair(bar.acc_full, PAIR);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ decoders, then epilogue
+    // Decoder warp dw rebuilds rows [16 rg, 16 rg + 16) x columns [32 hh, 32 hh + 32) of this
+    // CTA's 128 x 64 operand block per K block: four m16n8k16 envelope MMAs (one per 8 columns,
+    // LC per 16 envelope terms), then per element pair a sign flip and one 32-bit shared store in
+    // the 128-byte-swizzled K-major layout.  Lane (g, t) = (lane / 4, lane % 4) owns rows g and
+    // g + 8 of the group and columns 8 jj + 2t, 8 jj + 2t + 1.
+    const int dw = warp - 2;            // decoder index 0 .. NDEC-1
+    const int q = warp & 3;             // tensor-memory lane quarter this warp may read
+    const int ch = dw >> 2;             // which quarter of the 256 accumulator columns it drains
+    const int rg = dw & 7, hh = dw >> 3;
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t st_off = (uint32_t)(2 * rg) * 1024u + (uint32_t)g * 128u + 4u * (uint32_t)t;
+    const uint32_t xsw = (uint32_t)((4 * hh) ^ g);
+    const uint32_t lead_full_b = sm100::mapa_shared(bar.full_b, 0);
+    const uint32_t lead_acc_empty = sm100::mapa_shared(bar.acc_empty, 0);
+    const int kbp = fac.seg / BK;                      // K blocks per path (F stage)
+    const int rowbytes = (fac.cols + 7) >> 3;
+    const bool lvec = fac.l_vec2 != 0;
+    const int l = fac.l;
+    int it = 0, tl = 0, ns = 0;
+    for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
+      const Item w = item_of(wi, full, parts, nkb);
+      const int m0 = (w.tile % mt) * PM + (int)rank * BM, n0 = (w.tile / mt) * BN;
+      // first operand row of this warp's group (along the GEMM's N); in the G stage it fixes the
+      // path, in the F stage the path follows the K block
+      const int grow = n0 + BNH * (int)rank + 16 * rg;
+      const int prow = FST ? 0 : grow / fac.seg;
+      const bool pv = FST || prow < fac.P;
+      const int ra = (FST ? grow : grow - prow * fac.seg) + g, rb = ra + 8;
+      const bool va = pv && ra < fac.rows, vb = pv && rb < fac.rows;
+      uint32_t afr[LC][4];
+      auto load_rows = [&](int p) {
+        const uint16_t *L = fac.Lrow[p];
+#pragma unroll
+        for (int c = 0; c < LC; ++c) {
+          const int k0 = 16 * c + 2 * t;
+          afr[c][0] = va ? env_pair(L + (size_t)ra * l, l, k0, lvec) : 0u;
+          afr[c][1] = vb ? env_pair(L + (size_t)rb * l, l, k0, lvec) : 0u;
+          afr[c][2] = va ? env_pair(L + (size_t)ra * l, l, k0 + 8, lvec) : 0u;
+          afr[c][3] = vb ? env_pair(L + (size_t)rb * l, l, k0 + 8, lvec) : 0u;
+        }
+      };
+      // sign words and envelope B fragments of one K block, loaded one block ahead
+      struct Pre {
+        uint32_t wa, wb, b[4][LC][2];
+      };
+      auto fetch = [&](int kb, Pre &o) {
+        const int p = FST ? kb / kbp : prow;
+        const int cw = (FST ? (kb - p * kbp) * BK : kb * BK) + 32 * hh;   // first column of the warp's half
+        o.wa = 0u;
+        o.wb = 0u;
+        if (pv) {
+          const uint8_t *S = fac.S[p];
+          const size_t ld = fac.ld[p];
+          if (va) o.wa = sign_word(S + (size_t)ra * ld, cw, rowbytes);
+          if (vb) o.wb = sign_word(S + (size_t)rb * ld, cw, rowbytes);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int col = cw + 8 * jj + g;
+          const bool vc = pv && col < fac.cols;
+          const uint16_t *C = vc ? fac.Lcol[p] + (size_t)col * l : nullptr;
+#pragma unroll
+          for (int c = 0; c < LC; ++c) {
+            o.b[jj][c][0] = vc ? env_pair(C, l, 16 * c + 2 * t, lvec) : 0u;
+            o.b[jj][c][1] = vc ? env_pair(C, l, 16 * c + 2 * t + 8, lvec) : 0u;
+          }
+        }
+      };
+      if (!FST) {
+        if (pv) {
+          load_rows(prow);
+        } else {
+#pragma unroll
+          for (int c = 0; c < LC; ++c) afr[c][0] = afr[c][1] = afr[c][2] = afr[c][3] = 0u;
+        }
+      }
+      int pcur = -1;
+      Pre cur, nxt;
+      fetch(w.kb0, cur);
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+        if (kb + 1 < w.kb1) fetch(kb + 1, nxt);
+        if (FST) {
+          const int p = kb / kbp;
+          if (p != pcur) {
+            load_rows(p);
+            pcur = p;
+          }
+        }
+        const int sb = it % SB;
+        if (it >= SB && !wt.wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, true)) {
+          ok = false;
+          break;
+        }
+        const uint32_t base = sbase + OFF_B + sb * B_BYTES + st_off;
+        const uint32_t ea = cur.wa >> (2 * t), eb = cur.wb >> (2 * t);
+        const uint32_t ea2 = ea >> 16, eb2 = eb >> 16;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < LC; ++c) mma_f16_16816(d, afr[c], cur.b[jj][c][0], cur.b[jj][c][1]);
+          const uint32_t sa_ = jj < 2 ? ea : ea2, sb_ = jj < 2 ? eb : eb2;
+          const uint32_t fa = (jj & 1) ? sign_flip<1>(sa_) : sign_flip<0>(sa_);
+          const uint32_t fb = (jj & 1) ? sign_flip<1>(sb_) : sign_flip<0>(sb_);
+          const uint32_t off = (xsw ^ (uint32_t)jj) << 4;
+          sts32(base + off, pack_f16x2(d[0], d[1]) ^ fa);
+          sts32(base + 1024u + off, pack_f16x2(d[2], d[3]) ^ fb);
+        }
+        sm100::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive_cluster(lead_full_b + 8 * sb);
+        if (kb + 1 < w.kb1) cur = nxt;
+      }
+      if (!ok) break;
+      // epilogue: this warp drains lanes [32q, 32q+32) of both 128-row accumulators
+      if (!wt.wait(bar.acc_full, tl & 1, true)) { ok = false; break; }
+      qld::pdl_wait();
+      sm100::tc_fence_after();
+      const bool split = w.part >= 0;
+      // fp32 partials of a split tile: [tile - full][part][rank][BM rows][BN columns]
+      float *const slot =
+          split ? part_ws + ((size_t)((w.tile - full) * parts + w.part) * 2 + rank) * (size_t)(BM * BN) : nullptr;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int lr = h * 128 + 32 * q + lane, row = m0 + lr;
+        const float rs = (FST && !split && row < M) ? __ldg(row_scale + row) : 1.f;
+#pragma unroll 1
+        for (int c = ch * (BN / 32) / (NDEC / 4); c < (ch + 1) * (BN / 32) / (NDEC / 4); ++c) {
+          uint32_t v[32];
+          sm100::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + h * BN + c * 32, v);
+          sm100::tmem_wait_ld();
+          if (split) {
+            float4 *dst = reinterpret_cast<float4 *>(slot + (size_t)lr * BN + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          } else if (row < M) {
+            float f[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+            put_span<FST, 32>(out, ldo, ovec != 0, ydt, row, n0 + c * 32, Nout, f, rs);
+          }
+        }
+      }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive_cluster(lead_acc_empty);
+      if (split) {
+        // The last of the tile's parts to finish (per CTA half) sums all parts in part order.
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(bar.split_done);
+        const uint32_t last_flag = tmem_slot + 8;
+        if (dw == 0) {
+          if (!wt.wait(bar.split_done, ns & 1, false)) { ok = false; break; }
+          if (lane == 0) {
+            __threadfence();
+            unsigned *cnt = part_cnt + (w.tile - full) * 2 + rank;
+            const bool last = atomicAdd(cnt, 1u) == (unsigned)parts - 1;
+            if (last) {
+              atomicExch(cnt, 0u);
+              __threadfence();
+            }
+            sts32(last_flag, last ? 1u : 0u);
+            sm100::mbar_arrive(bar.split_go);
+          }
+          __syncwarp();
+        }
+        if (!wt.wait(bar.split_go, ns & 1, false)) { ok = false; break; }
+        ++ns;
+        if (lds32(last_flag)) {
+          const float *p0 = part_ws + ((size_t)(w.tile - full) * parts * 2 + rank) * (size_t)(BM * BN);
+          const size_t pstride = (size_t)2 * BM * BN;
+          for (int e = (dw * 32 + lane) * 4; e < BM * BN; e += NDEC * 32 * 4) {
+            const int row = m0 + e / BN, col = n0 + e % BN;
+            float4 a = __ldcg(reinterpret_cast<const float4 *>(p0 + e));
+            for (int pq = 1; pq < parts; ++pq) {
+              const float4 b = __ldcg(reinterpret_cast<const float4 *>(p0 + pq * pstride + e));
+              a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+            }
+            if (row >= M) continue;
+            const float f[4] = {a.x, a.y, a.z, a.w};
+            put_span<FST, 4>(out, ldo, ovec != 0, ydt, row, col, Nout, f, FST ? __ldg(row_scale + row) : 1.f);
+          }
+        }
+      }
+    }
+  }
+
+  if (!ok) atomicExch(&g_mgemm_timeout, 1);
+  // neither CTA leaves while its peer may still arrive on its barriers, read its shared memory
+  // through a pair MMA or write its tensor memory
+  sm100::tc_fence_before();
+  sm100::cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------- host side
+template <bool FST, int LC>
+cudaError_t smem_attr_one() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(mdbf_gemm_kernel<FST, LC>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  return err;
+}
+cudaError_t smem_attr() {
+  cudaError_t e = smem_attr_one<false, 1>();
+  if (e == cudaSuccess) e = smem_attr_one<true, 1>();
+  if (e == cudaSuccess) e = smem_attr_one<false, 2>();
+  if (e == cudaSuccess) e = smem_attr_one<true, 2>();
+  return e;
+}
+
+// CTA pairs that can be resident at once on the current device (cached per device); 0 when no
+// device is usable (the split of the last wave is then not planned).
+int resident_pairs() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (smem_attr() == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (ql::sm_count() / 2));
+      cfg.blockDim = dim3(THREADS);
+      cfg.dynamicSmemBytes = SMEM_BYTES;
+      if (cudaOccupancyMaxActiveClusters(&n, mdbf_gemm_kernel<false, 1>, &cfg) != cudaSuccess || n <= 0) n = 0;
+    }
+    if (n <= 0) {
+      (void)cudaGetLastError();
+      n = ql::sm_count() / 2;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Workspace of one call: envelope maxima, inverse row scales, X' [B][mp] fp16, T' [B][P seg]
+// fp16, the split counters of both GEMMs, and one region of fp32 partials that GEMM 1 and then
+// GEMM 2 use in turn.
+struct GemmWs {
+  int mp, seg;
+  SplitPlan g1, g2;
+  size_t emax, inv_s, xs, ts, cnt, part, total;
+};
+GemmWs gemm_ws(int P, int n, int m, int r, int B, int pairs) {
+  GemmWs L;
+  L.mp = (m + BK - 1) / BK * BK;
+  L.seg = (r + BK - 1) / BK * BK;
+  const int mt = (B + PM - 1) / PM;
+  const size_t tile_bytes = (size_t)2 * BM * BN * sizeof(float);
+  L.g1 = split_plan(mt * ((P * L.seg + BN - 1) / BN), L.mp / BK, pairs, tile_bytes);
+  L.g2 = split_plan(mt * ((n + BN - 1) / BN), P * L.seg / BK, pairs, tile_bytes);
+  L.emax = 0;
+  L.inv_s = L.emax + align256((size_t)P * 2 * NSL * LMAX * sizeof(float));
+  L.xs = L.inv_s + align256((size_t)B * sizeof(float));
+  L.ts = L.xs + align256((size_t)B * L.mp * 2);
+  L.cnt = L.ts + align256((size_t)B * P * L.seg * 2);
+  L.part = L.cnt + L.g1.counter_bytes + L.g2.counter_bytes;
+  L.total = L.part + std::max(L.g1.partial_bytes, L.g2.partial_bytes);
+  return L;
+}
+
+Factor make_factor(const mdbf_path *paths, int P, bool f_stage, int n, int m, int r, int l, int seg) {
+  Factor f = {};
+  bool l2 = l % 2 == 0;
+  for (int p = 0; p < P; ++p) {
+    const mdbf_path &q = paths[p];
+    f.S[p] = f_stage ? q.S_A : q.S_B;
+    f.ld[p] = f_stage ? q.ldSA : q.ldSB;
+    f.Lrow[p] = f_stage ? q.A_amp : q.Q_V;
+    f.Lcol[p] = f_stage ? q.Q_U : q.B_amp;
+    l2 = l2 && ql::aligned(f.Lrow[p], 4) && ql::aligned(f.Lcol[p], 4);
+  }
+  f.rows = f_stage ? n : r;
+  f.cols = f_stage ? r : m;
+  f.seg = seg;
+  f.P = P;
+  f.l = l;
+  f.l_vec2 = l2 ? 1 : 0;
+  return f;
+}
+
+template <int LC>
+void launch_gemms(const CUtensorMap &mx, const CUtensorMap &mt_, const Factor &fg, const Factor &ff, const GemmWs &L,
+                  char *base, void *y, int ydt, bool yvec, int B, int P, int n, int resident, cudaStream_t s) {
+  float *part = reinterpret_cast<float *>(base + L.part);
+  unsigned *cnt1 = reinterpret_cast<unsigned *>(base + L.cnt);
+  unsigned *cnt2 = reinterpret_cast<unsigned *>(base + L.cnt + L.g1.counter_bytes);
+  const int items1 = L.g1.full + L.g1.leftover * L.g1.parts, items2 = L.g2.full + L.g2.leftover * L.g2.parts;
+  ql::launch(mdbf_gemm_kernel<false, LC>, 2 * std::min(items1, resident), THREADS, SMEM_BYTES, s, mx, fg,
+             static_cast<void *>(base + L.ts), P * L.seg, 1, 0, static_cast<const float *>(nullptr), B, P * L.seg,
+             L.mp / BK, part, cnt1, L.g1.full, L.g1.parts);
+  ql::launch(mdbf_gemm_kernel<true, LC>, 2 * std::min(items2, resident), THREADS, SMEM_BYTES, s, mt_, ff, y, n,
+             yvec ? 1 : 0, ydt, reinterpret_cast<const float *>(base + L.inv_s), B, n, P * L.seg / BK, part, cnt2,
+             L.g2.full, L.g2.parts);
+}
+
+}  // namespace
+
+namespace ql {
+
+size_t mdbf_gemm_workspace_size(int P, int n, int m, int r, int l, int B) {
+  if (P <= 0 || n <= 0 || m <= 0 || r <= 0 || l <= 0 || l > LMAX || B <= 0) return 0;
+  return gemm_ws(P, n, m, r, B, resident_pairs()).total;
+}
+
+ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x, void *y,
+                           ql_out_dtype ydt, int B, void *ws, cudaStream_t s) {
+  if (P > PMAX) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: P = %d exceeds %d paths", P, PMAX);
+  if (l > LMAX) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: the batched path takes l <= %d (got %d)", LMAX, l);
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return fail(QL_ERR_CUDA, "mdbf_linear: cuTensorMapEncodeTiled is unavailable");
+  if (smem_attr() != cudaSuccess) return fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve GEMM shared memory");
+  const int resident = std::max(1, resident_pairs());
+  const GemmWs L = gemm_ws(P, n, m, r, B, resident);
+  char *base = static_cast<char *>(ws);
+  CUtensorMap mx, mtm;
+  if (!encode_rows_sw128(enc, &mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + L.xs, B, L.mp, L.mp, BM) ||
+      !encode_rows_sw128(enc, &mtm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + L.ts, B, (uint64_t)P * L.seg,
+                         (uint64_t)P * L.seg, BM))
+    return fail(QL_ERR_CUDA, "mdbf_linear: cannot encode the activation tensor maps");
+  const Factor fg = make_factor(paths, P, false, n, m, r, l, L.seg);
+  const Factor ff = make_factor(paths, P, true, n, m, r, l, L.seg);
+  float *emax = reinterpret_cast<float *>(base + L.emax);
+  launch(mdbf_envmax_kernel, dim3(P, 2, NSL), 256, 0, s, fg, emax);
+  ql_status st = launch_status("mdbf_linear (envelope maxima)");
+  if (st != QL_OK) return st;
+  const bool xvec = m % 8 == 0 && aligned(x, 16);
+  const int ncnt = (int)((L.g1.counter_bytes + L.g2.counter_bytes) / sizeof(unsigned));
+  launch(mdbf_xprep_kernel, B, 256, 0, s, x, m, L.mp, static_cast<const float *>(emax), P, l,
+         reinterpret_cast<uint16_t *>(base + L.xs), reinterpret_cast<float *>(base + L.inv_s),
+         reinterpret_cast<unsigned *>(base + L.cnt), ncnt, xvec ? 1 : 0);
+  st = launch_status("mdbf_linear (activation prep)");
+  if (st != QL_OK) return st;
+  const bool yvec = aligned(y, 16) && (ydt == QL_OUT_F32 ? n % 4 == 0 : n % 8 == 0);
+  if (l <= 16)
+    launch_gemms<1>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+  else
+    launch_gemms<2>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+  return launch_status("mdbf_linear (tensor-core GEMMs)");
+}
+
+ql_status mdbf_gemm_read_timeout(int *flag) {
+  int zero = 0;
+  if (cudaMemcpyFromSymbol(flag, g_mgemm_timeout, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_mgemm_timeout, &zero, sizeof(int)) != cudaSuccess)
+    return fail(QL_ERR_CUDA, "ql_check: cannot read the device timeout flag");
+  return QL_OK;
+}
+
+}  // namespace ql

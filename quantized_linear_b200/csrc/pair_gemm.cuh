@@ -1,0 +1,133 @@
+// Scaffolding shared by the tensor-core GEMMs that run on CTA pairs (benq_gemm_sm100.cu and
+// mdbf_gemm_sm100.cu): shared-memory accessors, the bounded wait, work items with a split last
+// wave, and the host-side split plan.  Not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "sm100_ptx.cuh"
+
+namespace pairgemm {
+
+constexpr long long WAIT_BUDGET = 4000000000LL;   // clock cycles (~2 s)
+constexpr int SPLIT_MAX = 8;                      // K ranges per tile of the last wave
+
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t lo, uint32_t hi) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(lo), "r"(hi) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_volatile_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Bounded wait shared by all roles.  Gives up when the budget runs out or when the pair's abort
+// flag is set; a thread that runs out sets the flag in both CTAs so that the others stop at once.
+struct Waiter {
+  uint32_t abort_local, abort_peer;
+  __device__ bool wait(uint32_t bar, uint32_t parity, bool cluster_scope) const {
+    auto probe = [&] {
+      return cluster_scope ? sm100::mbar_try_wait_cluster(bar, parity) : sm100::mbar_try_wait(bar, parity);
+    };
+    if (probe()) return true;
+    const long long t0 = clock64();
+    while (!probe()) {
+      if (ld_volatile_u32(abort_local) != 0) return false;
+      if (clock64() - t0 > WAIT_BUDGET) {
+        sts32(abort_local, 1);
+        st_cluster_u32(abort_peer, 1);
+        return false;
+      }
+    }
+    return true;
+  }
+};
+
+// Work items: pair tiles 0 .. full-1 whole, then each of the remaining tiles (the last, partial
+// wave) split into `parts` K ranges so that the otherwise idle pairs share it.  A split item
+// writes an fp32 partial; the last CTA to finish a tile sums the partials in part order.
+struct Item {
+  int tile, kb0, kb1, part;   // part < 0: whole tile
+};
+__device__ __forceinline__ Item item_of(int i, int full, int parts, int nkb) {
+  if (i < full) return {i, 0, nkb, -1};
+  const int u = i - full, j = u / parts, q = u - j * parts;
+  return {full + j, (int)((int64_t)q * nkb / parts), (int)((int64_t)(q + 1) * nkb / parts), q};
+}
+
+// Whole tiles run in full waves of `pairs` CTA pairs; when the last wave would leave at least
+// half of the pairs idle, its L tiles are split into `parts` K ranges each (L * parts <= pairs).
+// `pair_tile_bytes` is the size of one fp32 partial of a pair tile (both CTAs).
+struct SplitPlan {
+  int full, parts, leftover;
+  size_t partial_bytes, counter_bytes;
+};
+inline SplitPlan split_plan(int ntiles, int nkb, int pairs, size_t pair_tile_bytes) {
+  SplitPlan p{ntiles, 1, 0, 0, 0};
+  if (pairs <= 0) return p;
+  const int full = (ntiles / pairs) * pairs, left = ntiles - full;
+  if (left > 0 && 2 * left <= pairs) {
+    const int parts = std::min(std::min(pairs / left, SPLIT_MAX), nkb);
+    if (parts >= 2) {
+      p.full = full;
+      p.parts = parts;
+      p.leftover = left;
+      p.partial_bytes = (size_t)left * parts * pair_tile_bytes;
+      p.counter_bytes = ((size_t)left * 2 * sizeof(unsigned) + 255) / 256 * 256;
+    }
+  }
+  return p;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+inline EncodeTiledFn encode_tiled_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map of a row-major 2-D array [rows][cols] of 2-byte elements (row stride ld elements)
+// read in boxes of box_rows x 64 elements with the 128-byte swizzle the tensor core expects.
+inline bool encode_rows_sw128(EncodeTiledFn enc, CUtensorMap *map, CUtensorMapDataType dt, const void *base,
+                              uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace pairgemm

@@ -55,6 +55,20 @@ ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r,
                              const uint16_t *x, void *y, ql_out_dtype ydt, int B, void *ws,
                              cudaStream_t s);
 ql_status mdbf_read_timeout(int *flag);   // reads and clears the MDBF kernels' bounded-wait flag
+// batched MDBF (l * B above the decode kernels' limit) on the tensor cores, mdbf_gemm_sm100.cu:
+// envelope ranks up to MDBF_GEMM_LMAX and layers whose n, m and r are all at least
+// MDBF_GEMM_MIN.  Smaller layers would leave most of each 512 x 256 tile idle, and with only a
+// handful of outputs or of rank terms per row a row's largest output can be a small remainder of
+// cancelling terms, where fp16 factors are too coarse; those run through the decode kernels.
+constexpr int MDBF_GEMM_LMAX = 32;
+constexpr int MDBF_GEMM_MIN = 64;
+inline bool mdbf_use_gemm(int n, int m, int r, int l, int B, int vlim) {
+  return l * B > vlim && l <= MDBF_GEMM_LMAX && n >= MDBF_GEMM_MIN && m >= MDBF_GEMM_MIN && r >= MDBF_GEMM_MIN;
+}
+size_t mdbf_gemm_workspace_size(int P, int n, int m, int r, int l, int B);
+ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x,
+                           void *y, ql_out_dtype ydt, int B, void *ws, cudaStream_t s);
+ql_status mdbf_gemm_read_timeout(int *flag);
 size_t mdbf_noalloc_scratch_limit();
 ql_status mdbf_noalloc_scratch(void **ptr);
 ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W,

@@ -1,6 +1,6 @@
 // Thin wrappers over the sm_100a PTX used by the tensor-core kernels: mbarriers, bulk and tensor
 // (TMA) copies, tcgen05 (TMEM allocation, MMA, commit, loads) for one CTA and for a CTA pair,
-// and the shared-memory matrix descriptor of a K-major, 128-byte-swizzled bf16 operand.  No
+// and the shared-memory matrix descriptor of a K-major, 128-byte-swizzled 16-bit operand.  No
 // tensor or bulk load uses a multicast form; only the MMA completion signal (tcgen05.commit) is
 // multicast to the two CTAs of a pair.
 #pragma once
@@ -159,8 +159,9 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
 }
 // Pair MMA issued by the even CTA: A rows come from each CTA's shared memory (M/2 each), B
-// columns likewise (N/2 each), and each CTA's tensor memory receives its M/2 rows x N.
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// columns likewise (N/2 each), and each CTA's tensor memory receives its M/2 rows x N.  kind::f16:
+// the operand type (fp16 or bf16, the same for A and B) comes from the instruction descriptor.
+__device__ __forceinline__ void mma_f16kind_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                               uint32_t accumulate) {
   asm volatile(
       "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
@@ -182,6 +183,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                     // D format: f32
          | (1u << 7)                   // A format: bf16
          | (1u << 10)                  // B format: bf16
+         | (uint32_t(N >> 3) << 17)    // N / 8
+         | (uint32_t(M >> 4) << 24);   // M / 16
+}
+
+// The same with fp16 A and B (format code 0 in both fields).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                     // D format: f32
          | (uint32_t(N >> 3) << 17)    // N / 8
          | (uint32_t(M >> 4) << 24);   // M / 16
 }

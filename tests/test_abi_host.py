@@ -115,8 +115,13 @@ def test_mdbf_argument_errors_are_caught_on_the_host(ql):
     assert f(ok, 1, 64, 64, 32, 2, A, A, 0, 1, A + 16, ws, None) == ql.QL_ERR_ALIGNMENT     # workspace 256
     assert f(_fake_paths(ql, 1, ldSA=2), 1, 64, 64, 32, 2, A, A, 0, 1, A, ws, None) == ql.QL_ERR_INVALID_ARG
     assert f(_fake_paths(ql, 1, ldSB=10), 1, 64, 64, 32, 2, A, A, 0, 1, A, ws, None) == ql.QL_ERR_ALIGNMENT
-    big = ql.mdbf_workspace_bytes(1, 64, 64, 32, 8, 9)
-    assert f(ok, 1, 64, 64, 32, 8, A, A, 0, 9, A, big, None) == ql.QL_ERR_UNSUPPORTED      # l * B > 64
+    # l * B > 64 runs on the tensor cores: its workspace holds at least X' and T' in fp16
+    # (B x m and B x r rounded up to 64 columns)
+    big = ql.mdbf_workspace_bytes(1, 64, 64, 64, 8, 9)
+    assert big >= 9 * 64 * 2 * 2 and big > ws
+    assert f(ok, 1, 64, 64, 64, 8, A, A, 0, 9, A, big - 1, None) == ql.QL_ERR_INVALID_ARG  # workspace
+    ws65 = ql.mdbf_workspace_bytes(1, 64, 64, 32, 65, 1)
+    assert f(ok, 1, 64, 64, 32, 65, A, A, 0, 1, A, ws65, None) == ql.QL_ERR_UNSUPPORTED    # l > 64
     g = _raw(ql, "mdbf_dequant_debug")
     assert g(ok, 1, 64, 64, 32, 2, None, None, None, None) == ql.QL_ERR_INVALID_ARG
 
