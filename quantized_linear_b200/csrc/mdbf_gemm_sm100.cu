@@ -26,8 +26,8 @@
 // r of a pair owns rows [256 r, 256 r + 256) of a 512 x 256 output tile and decodes operand rows
 // [128 r, 128 r + 128); pair MMAs (M = 256 over two CTAs, N = 256, K = 16) read A from each CTA and
 // B from both.  Per CTA: warp 0 loads A tiles (256 x 64 fp16, 128-byte swizzle) with tensor
-// copies, warp 1 (even CTA) issues the pair MMAs, warps 2..17 decode the factor operand and then
-// drain the accumulators.  No tensor or bulk load is multicast.  Every wait is bounded (see
+// copies, warp 1 issues the pair MMAs (even CTA) or relays the odd CTA's decoded blocks to them,
+// warps 2..17 decode the factor operand and then drain the accumulators.  No tensor or bulk load is multicast.  Every wait is bounded (see
 // pair_gemm.cuh); a wait that runs out sets a flag read by ql_check().
 #include <cuda.h>
 
@@ -55,7 +55,7 @@ constexpr int B_BYTES = BNH * BK * 2;             // 16 KB
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + SA * A_BYTES;
 constexpr int OFF_BAR = OFF_B + SB * B_BYTES;
-constexpr int NBAR = 2 * (SA + SB) + 4;
+constexpr int NBAR = 2 * SA + 3 * SB + 4;
 constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // tensor-memory address, abort flag, last-part flag
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;  // + alignment slack
 constexpr int NDEC = 16;                          // decoder / epilogue warps: 8 row groups x 2 column halves
@@ -86,11 +86,13 @@ struct Factor {
 };
 
 struct Bars {
-  // full_a, full_b and acc_empty are used in the even CTA only (both CTAs arrive on them).
-  uint32_t full_a, empty_a, full_b, empty_b, acc_full, acc_empty, split_done, split_go;
+  // full_a, peer_b and acc_empty are used in the even CTA only (both CTAs arrive on full_a and
+  // acc_empty; the odd CTA's forwarder on peer_b).  dec_done collects this CTA's decoder warps.
+  uint32_t full_a, empty_a, dec_done, peer_b, empty_b, acc_full, acc_empty, split_done, split_go;
   __device__ Bars(uint32_t base)
-      : full_a(base), empty_a(full_a + 8 * SA), full_b(empty_a + 8 * SA), empty_b(full_b + 8 * SB),
-        acc_full(empty_b + 8 * SB), acc_empty(acc_full + 8), split_done(acc_empty + 8), split_go(split_done + 8) {}
+      : full_a(base), empty_a(full_a + 8 * SA), dec_done(empty_a + 8 * SA), peer_b(dec_done + 8 * SB),
+        empty_b(peer_b + 8 * SB), acc_full(empty_b + 8 * SB), acc_empty(acc_full + 8), split_done(acc_empty + 8),
+        split_go(split_done + 8) {}
 };
 
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -132,15 +134,6 @@ __device__ __forceinline__ uint32_t env_pair(const uint16_t *__restrict__ v, int
   const uint32_t lo = __ldg(reinterpret_cast<const unsigned short *>(v + i));
   const uint32_t hi = i + 1 < l ? __ldg(reinterpret_cast<const unsigned short *>(v + i + 1)) : 0u;
   return lo | (hi << 16);
-}
-
-// The 32 sign bits of columns [c0, c0 + 32) of one packed row (c0 a multiple of 32).  Rows are
-// 4-byte aligned with strides that are multiples of 4 (checked by the ABI), so a word that starts
-// inside the row's ceil(cols / 8) bytes ends inside its stride; bits past column cols - 1 are
-// padding and meet a zero envelope.  Words past the row's bytes are not read.
-__device__ __forceinline__ uint32_t sign_word(const uint8_t *__restrict__ row, int c0, int rowbytes) {
-  const int b0 = c0 >> 3;
-  return b0 < rowbytes ? __ldg(reinterpret_cast<const unsigned int *>(row + b0)) : 0u;
 }
 
 // ------------------------------------------------------------------ envelope column maxima
@@ -314,9 +307,9 @@ __device__ __forceinline__ void put_span(void *out, int ldo, bool ovec, int ydt,
 // ------------------------------------------------------------------ the GEMM
 // C[M][Nout] = A[M][K] D[Nout][K]^T with A an fp16 array read by tensor copies (map_a) and D the
 // factor operand decoded on the fly.  FST false: D = [G_1; ..; G_P] (N = P seg), C = T' in fp16.
-// FST true: D = [F_1 .. F_P] (K = P seg), C = y scaled by row_scale.  LC: envelope chunks of 16
-// (l <= 16 LC).
-template <bool FST, int LC>
+// FST true: D = [F_1 .. F_P] (K = P seg), C = y scaled by row_scale.  LK: envelope terms the
+// warp MMAs cover (8, 16 or 32; l <= LK), in LC chunks of 16.
+template <bool FST, int LK, int LC = (LK + 15) / 16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     mdbf_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ Factor fac,
                      void *__restrict__ out, int ldo, int ovec, int ydt, const float *__restrict__ row_scale, int M,
@@ -342,7 +335,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       sm100::mbar_init(bar.empty_a + 8 * s, 1);
     }
     for (int s = 0; s < SB; ++s) {
-      sm100::mbar_init(bar.full_b + 8 * s, 2 * NDEC);
+      sm100::mbar_init(bar.dec_done + 8 * s, NDEC);
+      sm100::mbar_init(bar.peer_b + 8 * s, 1);
       sm100::mbar_init(bar.empty_b + 8 * s, 1);
     }
     sm100::mbar_init(bar.acc_full, 1);
@@ -397,7 +391,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int sa = it % SA, sb = it % SB;
           if (!wt.wait(bar.full_a + 8 * sa, (it / SA) & 1, true) ||
-              !wt.wait(bar.full_b + 8 * sb, (it / SB) & 1, true)) {
+              !wt.wait(bar.dec_done + 8 * sb, (it / SB) & 1, false) ||
+              !wt.wait(bar.peer_b + 8 * sb, (it / SB) & 1, true)) {
             ok = false;
             break;
           }
@@ -418,14 +413,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (!ok) break;
         sm100::mma_commit_pair(bar.acc_full, PAIR);
       }
+    } else if (!lead && lane == 0) {
+      // ---------------------------------------------------------- forwarder (odd CTA)
+      // relays each decoded block of this CTA to the even CTA's MMA thread: one cluster-scope
+      // release per block instead of one per decoder warp
+      const uint32_t lead_peer_b = sm100::mapa_shared(bar.peer_b, 0);
+      int it = 0;
+      for (int wi = pair; wi < nitems && ok; wi += npairs) {
+        const Item w = item_of(wi, full, parts, nkb);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int sb = it % SB;
+          if (!wt.wait(bar.dec_done + 8 * sb, (it / SB) & 1, false)) {
+            ok = false;
+            break;
+          }
+          sm100::mbar_arrive_cluster(lead_peer_b + 8 * sb);
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------ decoders, then epilogue
     // Decoder warp dw rebuilds rows [16 rg, 16 rg + 16) x columns [32 hh, 32 hh + 32) of this
     // CTA's 128 x 64 operand block per K block: four m16n8k16 envelope MMAs (one per 8 columns,
-    // LC per 16 envelope terms), then per element pair a sign flip and one 32-bit shared store in
-    // the 128-byte-swizzled K-major layout.  Lane (g, t) = (lane / 4, lane % 4) owns rows g and
-    // g + 8 of the group and columns 8 jj + 2t, 8 jj + 2t + 1.
+    // one per 16 envelope terms), then per element pair a sign flip and one 32-bit shared store
+    // in the 128-byte-swizzled K-major layout.  Lane (g, t) = (lane / 4, lane % 4) owns rows g and
+    // g + 8 of the group and columns 8 jj + 2t, 8 jj + 2t + 1.  The sign words and column
+    // envelopes of the next K block are loaded while this one is decoded; pointers advance by a
+    // fixed stride per block, and only a block that reaches past the last column tests columns.
     const int dw = warp - 2;            // decoder index 0 .. NDEC-1
     const int q = warp & 3;             // tensor-memory lane quarter this warp may read
     const int ch = dw >> 2;             // which quarter of the 256 accumulator columns it drains
@@ -433,12 +447,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int g = lane >> 2, t = lane & 3;
     const uint32_t st_off = (uint32_t)(2 * rg) * 1024u + (uint32_t)g * 128u + 4u * (uint32_t)t;
     const uint32_t xsw = (uint32_t)((4 * hh) ^ g);
-    const uint32_t lead_full_b = sm100::mapa_shared(bar.full_b, 0);
     const uint32_t lead_acc_empty = sm100::mapa_shared(bar.acc_empty, 0);
     const int kbp = fac.seg / BK;                      // K blocks per path (F stage)
-    const int rowbytes = (fac.cols + 7) >> 3;
+    const int l = fac.l, cols = fac.cols;
     const bool lvec = fac.l_vec2 != 0;
-    const int l = fac.l;
+    const size_t lblk = (size_t)BK * l;                // column-envelope elements per K block
+    const int l8 = 8 * l;
+    // this lane's envelope terms: 16c + 2t, +1 (k0) and 16c + 2t + 8, +1 (k1) of chunk c
+    bool k0v[LC], k1v[LC];
+#pragma unroll
+    for (int c = 0; c < LC; ++c) {
+      k0v[c] = 16 * c + 2 * t < l;
+      k1v[c] = LK > 8 && 16 * c + 2 * t + 8 < l;
+    }
     int it = 0, tl = 0, ns = 0;
     for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
       const Item w = item_of(wi, full, parts, nkb);
@@ -458,56 +479,73 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const int k0 = 16 * c + 2 * t;
           afr[c][0] = va ? env_pair(L + (size_t)ra * l, l, k0, lvec) : 0u;
           afr[c][1] = vb ? env_pair(L + (size_t)rb * l, l, k0, lvec) : 0u;
-          afr[c][2] = va ? env_pair(L + (size_t)ra * l, l, k0 + 8, lvec) : 0u;
-          afr[c][3] = vb ? env_pair(L + (size_t)rb * l, l, k0 + 8, lvec) : 0u;
+          afr[c][2] = (LK > 8 && va) ? env_pair(L + (size_t)ra * l, l, k0 + 8, lvec) : 0u;
+          afr[c][3] = (LK > 8 && vb) ? env_pair(L + (size_t)rb * l, l, k0 + 8, lvec) : 0u;
         }
       };
-      // sign words and envelope B fragments of one K block, loaded one block ahead
+      // fetch state: path fp and path-local K block fkl of the next block to load
+      int fp = FST ? w.kb0 / kbp : prow;
+      int fkl = FST ? w.kb0 - fp * kbp : w.kb0;
+      const uint8_t *sga = nullptr, *sgb = nullptr;   // sign rows ra, rb from the warp's column half
+      const uint16_t *lcp = nullptr;                 // column envelope of column 32 hh + g
+      auto set_path = [&](int p) {
+        const size_t ld = fac.ld[p];
+        sga = fac.S[p] + (size_t)ra * ld + 4 * hh;
+        sgb = sga + 8 * ld;
+        lcp = fac.Lcol[p] + (size_t)(32 * hh + g) * l;
+      };
+      if (pv) set_path(fp);
       struct Pre {
         uint32_t wa, wb, b[4][LC][2];
       };
-      auto fetch = [&](int kb, Pre &o) {
-        const int p = FST ? kb / kbp : prow;
-        const int cw = (FST ? (kb - p * kbp) * BK : kb * BK) + 32 * hh;   // first column of the warp's half
-        o.wa = 0u;
-        o.wb = 0u;
-        if (pv) {
-          const uint8_t *S = fac.S[p];
-          const size_t ld = fac.ld[p];
-          if (va) o.wa = sign_word(S + (size_t)ra * ld, cw, rowbytes);
-          if (vb) o.wb = sign_word(S + (size_t)rb * ld, cw, rowbytes);
-        }
+      auto fetch = [&](Pre &o) {
+        const int kc = fkl * BK + 32 * hh;           // first column of the warp's half in the path
+        // The 32 sign bits of the half's columns: rows are 4-byte aligned with strides that are
+        // multiples of 4 (checked by the ABI), so a word that starts inside the row's
+        // ceil(cols / 8) bytes ends inside its stride; bits past the last column are padding and
+        // meet a zero column envelope.
+        const bool win = pv && kc < cols;            // the half starts inside the row
+        const int lim = win ? cols - kc - g : 0;     // column 8 jj + g of the half is in range iff 8 jj < lim
+        o.wa = (va && win) ? __ldg(reinterpret_cast<const unsigned int *>(sga + 8 * fkl)) : 0u;
+        o.wb = (vb && win) ? __ldg(reinterpret_cast<const unsigned int *>(sgb + 8 * fkl)) : 0u;
+        const uint16_t *cp = lcp + (size_t)fkl * lblk;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          const int col = cw + 8 * jj + g;
-          const bool vc = pv && col < fac.cols;
-          const uint16_t *C = vc ? fac.Lcol[p] + (size_t)col * l : nullptr;
+          const bool okc = 8 * jj < lim;
 #pragma unroll
           for (int c = 0; c < LC; ++c) {
-            o.b[jj][c][0] = vc ? env_pair(C, l, 16 * c + 2 * t, lvec) : 0u;
-            o.b[jj][c][1] = vc ? env_pair(C, l, 16 * c + 2 * t + 8, lvec) : 0u;
+            if (lvec) {
+              const unsigned int *v = reinterpret_cast<const unsigned int *>(cp + jj * l8 + 16 * c + 2 * t);
+              o.b[jj][c][0] = (okc && k0v[c]) ? __ldg(v) : 0u;
+              o.b[jj][c][1] = (okc && k1v[c]) ? __ldg(v + 4) : 0u;
+            } else {
+              o.b[jj][c][0] = okc ? env_pair(cp + jj * l8, l, 16 * c + 2 * t, false) : 0u;
+              o.b[jj][c][1] = (LK > 8 && okc) ? env_pair(cp + jj * l8, l, 16 * c + 2 * t + 8, false) : 0u;
+            }
           }
+        }
+        if (FST && ++fkl == kbp) {
+          fkl = 0;
+          if (++fp < fac.P) set_path(fp);
+        } else if (!FST) {
+          ++fkl;
         }
       };
-      if (!FST) {
-        if (pv) {
-          load_rows(prow);
-        } else {
+      // path and path-local K block of the block being decoded (F stage)
+      int pc = FST ? w.kb0 / kbp : prow, kcl = FST ? w.kb0 - pc * kbp : 0;
+      if (FST || pv) {
+        load_rows(pc);
+      } else {
 #pragma unroll
-          for (int c = 0; c < LC; ++c) afr[c][0] = afr[c][1] = afr[c][2] = afr[c][3] = 0u;
-        }
+        for (int c = 0; c < LC; ++c) afr[c][0] = afr[c][1] = afr[c][2] = afr[c][3] = 0u;
       }
-      int pcur = -1;
       Pre cur, nxt;
-      fetch(w.kb0, cur);
+      fetch(cur);
       for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
-        if (kb + 1 < w.kb1) fetch(kb + 1, nxt);
-        if (FST) {
-          const int p = kb / kbp;
-          if (p != pcur) {
-            load_rows(p);
-            pcur = p;
-          }
+        if (kb + 1 < w.kb1) fetch(nxt);
+        if (FST && kcl == kbp) {
+          kcl = 0;
+          load_rows(++pc);
         }
         const int sb = it % SB;
         if (it >= SB && !wt.wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, true)) {
@@ -529,9 +567,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           sts32(base + off, pack_f16x2(d[0], d[1]) ^ fa);
           sts32(base + 1024u + off, pack_f16x2(d[2], d[3]) ^ fb);
         }
+        // the block is handed to this CTA's MMA side through a CTA-scope barrier: the even CTA's
+        // MMA thread waits on it directly, the odd CTA's forwarder relays it at cluster scope
         sm100::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) sm100::mbar_arrive_cluster(lead_full_b + 8 * sb);
+        if (lane == 0) sm100::mbar_arrive(bar.dec_done + 8 * sb);
+        if (FST) ++kcl;
         if (kb + 1 < w.kb1) cur = nxt;
       }
       if (!ok) break;
@@ -624,20 +665,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------- host side
-template <bool FST, int LC>
+template <bool FST, int LK>
 cudaError_t smem_attr_one() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
-    err = cudaFuncSetAttribute(mdbf_gemm_kernel<FST, LC>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    err = cudaFuncSetAttribute(mdbf_gemm_kernel<FST, LK>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   });
   return err;
 }
 cudaError_t smem_attr() {
-  cudaError_t e = smem_attr_one<false, 1>();
-  if (e == cudaSuccess) e = smem_attr_one<true, 1>();
-  if (e == cudaSuccess) e = smem_attr_one<false, 2>();
-  if (e == cudaSuccess) e = smem_attr_one<true, 2>();
+  cudaError_t e = cudaSuccess;
+  for (cudaError_t r : {smem_attr_one<false, 8>(), smem_attr_one<true, 8>(), smem_attr_one<false, 16>(),
+                        smem_attr_one<true, 16>(), smem_attr_one<false, 32>(), smem_attr_one<true, 32>()})
+    if (e == cudaSuccess) e = r;
   return e;
 }
 
@@ -659,7 +700,7 @@ int resident_pairs() {
       cfg.gridDim = dim3(2 * (ql::sm_count() / 2));
       cfg.blockDim = dim3(THREADS);
       cfg.dynamicSmemBytes = SMEM_BYTES;
-      if (cudaOccupancyMaxActiveClusters(&n, mdbf_gemm_kernel<false, 1>, &cfg) != cudaSuccess || n <= 0) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, mdbf_gemm_kernel<false, 8>, &cfg) != cudaSuccess || n <= 0) n = 0;
     }
     if (n <= 0) {
       (void)cudaGetLastError();
@@ -718,17 +759,17 @@ Factor make_factor(const mdbf_path *paths, int P, bool f_stage, int n, int m, in
   return f;
 }
 
-template <int LC>
+template <int LK>
 void launch_gemms(const CUtensorMap &mx, const CUtensorMap &mt_, const Factor &fg, const Factor &ff, const GemmWs &L,
                   char *base, void *y, int ydt, bool yvec, int B, int P, int n, int resident, cudaStream_t s) {
   float *part = reinterpret_cast<float *>(base + L.part);
   unsigned *cnt1 = reinterpret_cast<unsigned *>(base + L.cnt);
   unsigned *cnt2 = reinterpret_cast<unsigned *>(base + L.cnt + L.g1.counter_bytes);
   const int items1 = L.g1.full + L.g1.leftover * L.g1.parts, items2 = L.g2.full + L.g2.leftover * L.g2.parts;
-  ql::launch(mdbf_gemm_kernel<false, LC>, 2 * std::min(items1, resident), THREADS, SMEM_BYTES, s, mx, fg,
+  ql::launch(mdbf_gemm_kernel<false, LK>, 2 * std::min(items1, resident), THREADS, SMEM_BYTES, s, mx, fg,
              static_cast<void *>(base + L.ts), P * L.seg, 1, 0, static_cast<const float *>(nullptr), B, P * L.seg,
              L.mp / BK, part, cnt1, L.g1.full, L.g1.parts);
-  ql::launch(mdbf_gemm_kernel<true, LC>, 2 * std::min(items2, resident), THREADS, SMEM_BYTES, s, mt_, ff, y, n,
+  ql::launch(mdbf_gemm_kernel<true, LK>, 2 * std::min(items2, resident), THREADS, SMEM_BYTES, s, mt_, ff, y, n,
              yvec ? 1 : 0, ydt, reinterpret_cast<const float *>(base + L.inv_s), B, n, P * L.seg / BK, part, cnt2,
              L.g2.full, L.g2.parts);
 }
@@ -771,10 +812,12 @@ ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, i
   st = launch_status("mdbf_linear (activation prep)");
   if (st != QL_OK) return st;
   const bool yvec = aligned(y, 16) && (ydt == QL_OUT_F32 ? n % 4 == 0 : n % 8 == 0);
-  if (l <= 16)
-    launch_gemms<1>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+  if (l <= 8)
+    launch_gemms<8>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+  else if (l <= 16)
+    launch_gemms<16>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
   else
-    launch_gemms<2>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+    launch_gemms<32>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
   return launch_status("mdbf_linear (tensor-core GEMMs)");
 }
 
