@@ -33,6 +33,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "pair_gemm.cuh"
 #include "ql_internal.cuh"
@@ -54,7 +55,9 @@ constexpr int A_BYTES = BM * BK * 2;              // 32 KB
 constexpr int B_BYTES = BNH * BK * 2;             // 16 KB
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + SA * A_BYTES;
-constexpr int OFF_BAR = OFF_B + SB * B_BYTES;
+constexpr int CW_BYTES = 512;                     // l <= 4: one warp's fp32 column pairs of a K block
+constexpr int OFF_CW = OFF_B + SB * B_BYTES;      // two of them per decoder warp
+constexpr int OFF_BAR = OFF_CW + 16 * 2 * CW_BYTES;
 constexpr int NBAR = 2 * SA + 3 * SB + 4;
 constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // tensor-memory address, abort flag, last-part flag
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;  // + alignment slack
@@ -83,7 +86,32 @@ struct Factor {
   const uint16_t *Lcol[PMAX];
   int rows, cols, seg, P, l;
   int l_vec2;   // l even and every envelope base 4-byte aligned
+  // l <= 4: the column envelopes once more, as fp32 [P][cpad / 2][4 terms][2 columns] (column pair
+  // q holds columns 2q, 2q + 1), zero past l and past cols; cpad = the padded column count.
+  const float *cpair;
+  int cpad;
 };
+
+// packed fp32 pairs (the f32x2 operands of fma.rn.f32x2)
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2u(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2split(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// a * b + c on both halves, each rounded once (the products of fp16 values are exact in fp32)
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
 
 struct Bars {
   // full_a, peer_b and acc_empty are used in the even CTA only (both CTAs arrive on full_a and
@@ -101,6 +129,15 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
 // {fp16(lo), fp16(hi)} rounded to nearest even, lo in the low half
@@ -141,9 +178,37 @@ __device__ __forceinline__ uint32_t env_pair(const uint16_t *__restrict__ v, int
 // NSL (grid P x 2 x NSL).  Weights are read before the wait on the preceding kernel; the store
 // comes after it.
 constexpr int NSL = 16;
-__global__ void __launch_bounds__(256) mdbf_envmax_kernel(Factor g, float *__restrict__ emax) {
+// Column-pair copy for the l <= 4 decoders: thread q of slice z writes the fp32 pair block of
+// columns 2q, 2q + 1 of path p (grid P x 1 x NSL, one launch per factor).
+__device__ __forceinline__ void write_colpairs(const Factor &f, int p, int z, float *__restrict__ out) {
+  const int npair = f.cpad / 2, per = (npair + NSL - 1) / NSL;
+  const unsigned short *v = reinterpret_cast<const unsigned short *>(f.Lcol[p]);
+  float *o = out + (size_t)p * npair * 8;
+  for (int q = z * per + (int)threadIdx.x; q < min(npair, (z + 1) * per); q += blockDim.x) {
+    float e[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int col = 2 * q + h;
+        e[2 * i + h] = (i < f.l && col < f.cols) ? qld::f16_to_f32(__ldg(v + (size_t)col * f.l + i)) : 0.f;
+      }
+    reinterpret_cast<float4 *>(o + (size_t)q * 8)[0] = make_float4(e[0], e[1], e[2], e[3]);
+    reinterpret_cast<float4 *>(o + (size_t)q * 8)[1] = make_float4(e[4], e[5], e[6], e[7]);
+  }
+}
+
+// blockIdx.y 0, 1: the maxima below; 2: column pairs of g (into g.cpair); 3: of f.
+__global__ void __launch_bounds__(256) mdbf_envmax_kernel(Factor g, Factor f, float *__restrict__ emax,
+                                                          float *__restrict__ gpair, float *__restrict__ fpair) {
   qld::pdl_trigger();
   const int p = blockIdx.x, which = blockIdx.y, z = blockIdx.z;
+  if (which >= 2) {
+    qld::pdl_wait();
+    if (which == 2) write_colpairs(g, p, z, gpair);
+    else write_colpairs(f, p, z, fpair);
+    return;
+  }
   const unsigned short *v = reinterpret_cast<const unsigned short *>(which == 0 ? g.Lrow[p] : g.Lcol[p]);
   const int nrow = which == 0 ? g.rows : g.cols, l = g.l;
   const int per = (nrow + NSL - 1) / NSL, r0 = z * per, r1 = min(nrow, r0 + per);
@@ -307,8 +372,9 @@ __device__ __forceinline__ void put_span(void *out, int ldo, bool ovec, int ydt,
 // ------------------------------------------------------------------ the GEMM
 // C[M][Nout] = A[M][K] D[Nout][K]^T with A an fp16 array read by tensor copies (map_a) and D the
 // factor operand decoded on the fly.  FST false: D = [G_1; ..; G_P] (N = P seg), C = T' in fp16.
-// FST true: D = [F_1 .. F_P] (K = P seg), C = y scaled by row_scale.  LK: envelope terms the
-// warp MMAs cover (8, 16 or 32; l <= LK), in LC chunks of 16.
+// FST true: D = [F_1 .. F_P] (K = P seg), C = y scaled by row_scale.  LK: envelope terms
+// covered (l <= LK).  LK = 4: packed fp32 FMAs, four terms per element pair; LK = 8, 16, 32: warp
+// MMAs in LC chunks of 16 terms.
 template <bool FST, int LK, int LC = (LK + 15) / 16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     mdbf_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ Factor fac,
@@ -472,8 +538,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int ra = (FST ? grow : grow - prow * fac.seg) + g, rb = ra + 8;
       const bool va = pv && ra < fac.rows, vb = pv && rb < fac.rows;
       uint32_t afr[LC][4];
+      uint64_t ra2[4], rb2[4];   // l <= 4: row envelope terms as {v, v} pairs
       auto load_rows = [&](int p) {
         const uint16_t *L = fac.Lrow[p];
+        if constexpr (LK == 4) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float a = (va && i < l) ? qld::f16_to_f32(L[(size_t)ra * l + i]) : 0.f;
+            const float b = (vb && i < l) ? qld::f16_to_f32(L[(size_t)rb * l + i]) : 0.f;
+            ra2[i] = f2(a, a);
+            rb2[i] = f2(b, b);
+          }
+          return;
+        }
 #pragma unroll
         for (int c = 0; c < LC; ++c) {
           const int k0 = 16 * c + 2 * t;
@@ -488,16 +565,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int fkl = FST ? w.kb0 - fp * kbp : w.kb0;
       const uint8_t *sga = nullptr, *sgb = nullptr;   // sign rows ra, rb from the warp's column half
       const uint16_t *lcp = nullptr;                 // column envelope of column 32 hh + g
+      const float *cpp = nullptr;                    // l <= 4: fp32 pair block of columns 32 hh + 2t, +1
       auto set_path = [&](int p) {
         const size_t ld = fac.ld[p];
         sga = fac.S[p] + (size_t)ra * ld + 4 * hh;
         sgb = sga + 8 * ld;
         lcp = fac.Lcol[p] + (size_t)(32 * hh + g) * l;
+        cpp = fac.cpair + ((size_t)p * (fac.cpad / 2) + 16 * hh) * 8;
       };
       if (pv) set_path(fp);
-      struct Pre {
+      struct PreM {
         uint32_t wa, wb, b[4][LC][2];
       };
+      struct PreF {
+        uint32_t wa, wb;
+        uint4 c;   // this lane's 16 bytes of the warp's 512-byte column-pair block
+      };
+      using Pre = std::conditional_t<LK == 4, PreF, PreM>;
       auto fetch = [&](Pre &o) {
         const int kc = fkl * BK + 32 * hh;           // first column of the warp's half in the path
         // The 32 sign bits of the half's columns: rows are 4-byte aligned with strides that are
@@ -508,6 +592,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int lim = win ? cols - kc - g : 0;     // column 8 jj + g of the half is in range iff 8 jj < lim
         o.wa = (va && win) ? __ldg(reinterpret_cast<const unsigned int *>(sga + 8 * fkl)) : 0u;
         o.wb = (vb && win) ? __ldg(reinterpret_cast<const unsigned int *>(sgb + 8 * fkl)) : 0u;
+        if constexpr (LK == 4) {
+          // the warp's 16 column pairs (padded with zeros to cpad columns: no column test), 16
+          // bytes per lane; parked in shared memory before the block is decoded
+          o.c = pv ? __ldg(reinterpret_cast<const uint4 *>(cpp + (size_t)fkl * (BK / 2) * 8) + lane)
+                   : make_uint4(0u, 0u, 0u, 0u);
+        } else {
         const uint16_t *cp = lcp + (size_t)fkl * lblk;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -523,6 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               o.b[jj][c][1] = (LK > 8 && okc) ? env_pair(cp + jj * l8, l, 16 * c + 2 * t + 8, false) : 0u;
             }
           }
+        }
         }
         if (FST && ++fkl == kbp) {
           fkl = 0;
@@ -541,6 +632,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       Pre cur, nxt;
       fetch(cur);
+      const uint32_t cwb = sbase + OFF_CW + dw * 2 * CW_BYTES;   // this warp's two column-pair blocks
+      if constexpr (LK == 4) {
+        sts128(cwb + (it & 1) * CW_BYTES + 16 * lane, cur.c);
+        __syncwarp();
+      }
       for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
         if (kb + 1 < w.kb1) fetch(nxt);
         if (FST && kcl == kbp) {
@@ -558,8 +654,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           float d[4] = {0.f, 0.f, 0.f, 0.f};
+          if constexpr (LK == 4) {
+            // envelope terms in ascending order, one rounding per term, as the oracle sums them
+            const uint32_t cb = cwb + (it & 1) * CW_BYTES + (4 * jj + t) * 32;
+            const uint4 c0 = lds128(cb), c1 = lds128(cb + 16);
+            const uint64_t b[4] = {f2u(c0.x, c0.y), f2u(c0.z, c0.w), f2u(c1.x, c1.y), f2u(c1.z, c1.w)};
+            uint64_t ea = f2(0.f, 0.f), eb = f2(0.f, 0.f);
 #pragma unroll
-          for (int c = 0; c < LC; ++c) mma_f16_16816(d, afr[c], cur.b[jj][c][0], cur.b[jj][c][1]);
+            for (int i = 0; i < 4; ++i) {
+              ea = ffma2(ra2[i], b[i], ea);
+              eb = ffma2(rb2[i], b[i], eb);
+            }
+            f2split(ea, d[0], d[1]);
+            f2split(eb, d[2], d[3]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < LC; ++c) mma_f16_16816(d, afr[c], cur.b[jj][c][0], cur.b[jj][c][1]);
+          }
           const uint32_t sa_ = jj < 2 ? ea : ea2, sb_ = jj < 2 ? eb : eb2;
           const uint32_t fa = (jj & 1) ? sign_flip<1>(sa_) : sign_flip<0>(sa_);
           const uint32_t fb = (jj & 1) ? sign_flip<1>(sb_) : sign_flip<0>(sb_);
@@ -573,7 +684,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(bar.dec_done + 8 * sb);
         if (FST) ++kcl;
-        if (kb + 1 < w.kb1) cur = nxt;
+        if (kb + 1 < w.kb1) {
+          cur = nxt;
+          if constexpr (LK == 4) {
+            // every lane has read block it's pairs (the arrive above follows a __syncwarp)
+            sts128(cwb + ((it + 1) & 1) * CW_BYTES + 16 * lane, cur.c);
+            __syncwarp();
+          }
+        }
       }
       if (!ok) break;
       // epilogue: this warp drains lanes [32q, 32q+32) of both 128-row accumulators
@@ -676,8 +794,9 @@ cudaError_t smem_attr_one() {
 }
 cudaError_t smem_attr() {
   cudaError_t e = cudaSuccess;
-  for (cudaError_t r : {smem_attr_one<false, 8>(), smem_attr_one<true, 8>(), smem_attr_one<false, 16>(),
-                        smem_attr_one<true, 16>(), smem_attr_one<false, 32>(), smem_attr_one<true, 32>()})
+  for (cudaError_t r : {smem_attr_one<false, 4>(), smem_attr_one<true, 4>(), smem_attr_one<false, 8>(),
+                        smem_attr_one<true, 8>(), smem_attr_one<false, 16>(), smem_attr_one<true, 16>(),
+                        smem_attr_one<false, 32>(), smem_attr_one<true, 32>()})
     if (e == cudaSuccess) e = r;
   return e;
 }
@@ -713,13 +832,13 @@ int resident_pairs() {
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Workspace of one call: envelope maxima, inverse row scales, X' [B][mp] fp16, T' [B][P seg]
-// fp16, the split counters of both GEMMs, and one region of fp32 partials that GEMM 1 and then
-// GEMM 2 use in turn.
+// Workspace of one call: envelope maxima, the fp32 column pairs of both factors (l <= 4),
+// inverse row scales, X' [B][mp] fp16, T' [B][P seg] fp16, the split counters of both GEMMs, and
+// one region of fp32 partials that GEMM 1 and then GEMM 2 use in turn.
 struct GemmWs {
   int mp, seg;
   SplitPlan g1, g2;
-  size_t emax, inv_s, xs, ts, cnt, part, total;
+  size_t emax, gpair, fpair, inv_s, xs, ts, cnt, part, total;
 };
 GemmWs gemm_ws(int P, int n, int m, int r, int B, int pairs) {
   GemmWs L;
@@ -730,7 +849,9 @@ GemmWs gemm_ws(int P, int n, int m, int r, int B, int pairs) {
   L.g1 = split_plan(mt * ((P * L.seg + BN - 1) / BN), L.mp / BK, pairs, tile_bytes);
   L.g2 = split_plan(mt * ((n + BN - 1) / BN), P * L.seg / BK, pairs, tile_bytes);
   L.emax = 0;
-  L.inv_s = L.emax + align256((size_t)P * 2 * NSL * LMAX * sizeof(float));
+  L.gpair = L.emax + align256((size_t)P * 2 * NSL * LMAX * sizeof(float));
+  L.fpair = L.gpair + align256((size_t)P * L.mp * 16);
+  L.inv_s = L.fpair + align256((size_t)P * L.seg * 16);
   L.xs = L.inv_s + align256((size_t)B * sizeof(float));
   L.ts = L.xs + align256((size_t)B * L.mp * 2);
   L.cnt = L.ts + align256((size_t)B * P * L.seg * 2);
@@ -739,7 +860,8 @@ GemmWs gemm_ws(int P, int n, int m, int r, int B, int pairs) {
   return L;
 }
 
-Factor make_factor(const mdbf_path *paths, int P, bool f_stage, int n, int m, int r, int l, int seg) {
+Factor make_factor(const mdbf_path *paths, int P, bool f_stage, int n, int m, int r, int l, const GemmWs &L,
+                   const char *base) {
   Factor f = {};
   bool l2 = l % 2 == 0;
   for (int p = 0; p < P; ++p) {
@@ -752,7 +874,9 @@ Factor make_factor(const mdbf_path *paths, int P, bool f_stage, int n, int m, in
   }
   f.rows = f_stage ? n : r;
   f.cols = f_stage ? r : m;
-  f.seg = seg;
+  f.seg = L.seg;
+  f.cpad = f_stage ? L.seg : L.mp;
+  f.cpair = reinterpret_cast<const float *>(base + (f_stage ? L.fpair : L.gpair));
   f.P = P;
   f.l = l;
   f.l_vec2 = l2 ? 1 : 0;
@@ -798,10 +922,11 @@ ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, i
       !encode_rows_sw128(enc, &mtm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + L.ts, B, (uint64_t)P * L.seg,
                          (uint64_t)P * L.seg, BM))
     return fail(QL_ERR_CUDA, "mdbf_linear: cannot encode the activation tensor maps");
-  const Factor fg = make_factor(paths, P, false, n, m, r, l, L.seg);
-  const Factor ff = make_factor(paths, P, true, n, m, r, l, L.seg);
+  const Factor fg = make_factor(paths, P, false, n, m, r, l, L, base);
+  const Factor ff = make_factor(paths, P, true, n, m, r, l, L, base);
   float *emax = reinterpret_cast<float *>(base + L.emax);
-  launch(mdbf_envmax_kernel, dim3(P, 2, NSL), 256, 0, s, fg, emax);
+  launch(mdbf_envmax_kernel, dim3(P, l <= 4 ? 4 : 2, NSL), 256, 0, s, fg, ff, emax,
+         reinterpret_cast<float *>(base + L.gpair), reinterpret_cast<float *>(base + L.fpair));
   ql_status st = launch_status("mdbf_linear (envelope maxima)");
   if (st != QL_OK) return st;
   const bool xvec = m % 8 == 0 && aligned(x, 16);
@@ -812,7 +937,9 @@ ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, i
   st = launch_status("mdbf_linear (activation prep)");
   if (st != QL_OK) return st;
   const bool yvec = aligned(y, 16) && (ydt == QL_OUT_F32 ? n % 4 == 0 : n % 8 == 0);
-  if (l <= 8)
+  if (l <= 4)
+    launch_gemms<4>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+  else if (l <= 8)
     launch_gemms<8>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
   else if (l <= 16)
     launch_gemms<16>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
