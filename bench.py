@@ -1,6 +1,7 @@
 """Benchmark of the weight-only quantized linear layers on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|mdbf|layer]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload decode|prefill|mdbf|mdbf_prefill|layer]
                     [--impl ours|reference]
 
 Prints one JSON line.  Workloads (synthetic, seeded; shapes of a 27B-class
@@ -10,6 +11,7 @@ decoder layer, hidden 5120, intermediate 17408):
            17408->5120 (one step = one pass of each).  Default.
   prefill  BenQ 6-bit prefill GEMM, 2048 tokens, same two shapes, bf16 output.
   mdbf     MDBF P=2, l=4 at 1.5 bits/weight (rank 2886), gate/up and down, batch 1.
+  mdbf_prefill  the same MDBF layers at 2048 tokens (tensor-core path), bf16 output.
   layer    the full decoder-layer linear set at batch 1: BenQ q/k/v/o/gate/up/down
            plus MDBF gate/up/down.
 
@@ -57,6 +59,12 @@ def _peaks():
 def benq_bytes(N, K, B, out_bytes=4):
     """Algorithmic bytes of one BenQ call: packed codes, tables, activations, output."""
     return 0.75 * N * K + 128 * N + 2 * B * K + out_bytes * B * N
+
+
+def mdbf_flops(n, m, r, P, B):
+    """Algorithmic FLOPs of one batched MDBF call: the factored contraction, B x m x (P r) for
+    T = X G^T and B x (P r) x n for Y = T F^T."""
+    return 2.0 * B * P * r * (m + n)
 
 
 def mdbf_bytes(n, m, r, l, P, B, out_bytes=4):
@@ -145,7 +153,7 @@ class Workload:
             return dict(kind="benq", N=N, K=K, B=B, codes=[codes], lut=[lut], x=x, x_h=x_h, y=y, ws=ws,
                         wbytes=codes.numel() + lut.numel() * 2, label=label or f"benq_{K}x{N}_b{B}")
 
-        def mdbf_layer(n, m, B, seed, label=None):
+        def mdbf_layer(n, m, B, seed, label=None, out_dtype=torch.float32):
             paths = synth.mdbf_paths(MLP_P, n, m, MLP_R, MLP_L, seed=seed)
             dps = [dict(S_A=dev(p.S_A), S_B=dev(p.S_B), A_amp=f16(p.A_amp), B_amp=f16(p.B_amp),
                         Q_U=f16(p.Q_U), Q_V=f16(p.Q_V)) for p in paths]
@@ -153,7 +161,8 @@ class Workload:
             ws = torch.empty(ql.mdbf_workspace_bytes(MLP_P, n, m, MLP_R, MLP_L, B), dtype=torch.uint8, device=cuda)
             wbytes = sum(sum(t.numel() * t.element_size() for t in d.values()) for d in dps)
             return dict(kind="mdbf", n=n, m=m, B=B, paths=[dps], x=bf16(x_h), x_h=x_h,
-                        y=torch.empty(B, n, device=cuda), ws=ws, wbytes=wbytes, label=label or f"mdbf_{m}x{n}_b{B}")
+                        y=torch.empty(B, n, dtype=out_dtype, device=cuda), ws=ws, wbytes=wbytes,
+                        label=label or f"mdbf_{m}x{n}_b{B}")
 
         layers = []
         if name == "decode":
@@ -165,6 +174,9 @@ class Workload:
         elif name == "mdbf":
             layers = [mdbf_layer(INTER, HIDDEN, 1, 4001, "mdbf_gate_up_5120x17408_b1"),
                       mdbf_layer(HIDDEN, INTER, 1, 4002, "mdbf_down_17408x5120_b1")]
+        elif name == "mdbf_prefill":
+            layers = [mdbf_layer(INTER, HIDDEN, 2048, 6001, "mdbf_gemm_5120x17408_m2048", torch.bfloat16),
+                      mdbf_layer(HIDDEN, INTER, 2048, 6002, "mdbf_gemm_17408x5120_m2048", torch.bfloat16)]
         elif name == "layer":
             layers = [benq_layer(HIDDEN, HIDDEN, 1, 5001, label="benq_q"),
                       benq_layer(1024, HIDDEN, 1, 5002, label="benq_k"),
@@ -203,7 +215,10 @@ class Workload:
         return tot
 
     def step_flops(self):
-        return sum(2.0 * L["B"] * L["N"] * L["K"] for L in self.layers if L["kind"] == "benq")
+        f = sum(2.0 * L["B"] * L["N"] * L["K"] for L in self.layers if L["kind"] == "benq")
+        if self.name == "mdbf_prefill":
+            f += sum(mdbf_flops(L["n"], L["m"], MLP_R, MLP_P, L["B"]) for L in self.layers if L["kind"] == "mdbf")
+        return f
 
     def run_layer(self, L, c):
         ql = self.ql
@@ -213,7 +228,9 @@ class Workload:
             ql.mdbf_linear(L["paths"][c], L["n"], L["m"], MLP_R, MLP_L, L["x"], L["y"], L["ws"])
 
     def launches_per_step(self):
-        return sum(1 if L["kind"] == "benq" else 3 for L in self.layers)
+        # BenQ: one kernel; MDBF: pack, G stage, F stage, or for batches past the decode kernels
+        # envelope prep, activation prep and the two GEMMs
+        return sum(1 if L["kind"] == "benq" else (4 if MLP_L * L["B"] > 64 else 3) for L in self.layers)
 
 
 # the sources each kernel's DRAM-traffic figure depends on
@@ -221,6 +238,7 @@ _KERNEL_SOURCES = {
     "benq_gemv": ["benq_gemv.cu", "ql_internal.cuh"],
     "benq_gemm": ["benq_gemm_sm100.cu", "sm100_ptx.cuh", "ql_internal.cuh"],
     "mdbf_linear": ["mdbf.cu", "ql_internal.cuh"],
+    "mdbf_gemm": ["mdbf_gemm_sm100.cu", "pair_gemm.cuh", "sm100_ptx.cuh", "ql_internal.cuh"],
 }
 
 
@@ -256,6 +274,7 @@ def oracle_samples(workload, rows=64, seed=0):
     shapes = {"decode": [("benq", INTER, HIDDEN, 1), ("benq", HIDDEN, INTER, 1)],
               "prefill": [("benq", INTER, HIDDEN, 2048), ("benq", HIDDEN, INTER, 2048)],
               "mdbf": [("mdbf", INTER, HIDDEN, 1), ("mdbf", HIDDEN, INTER, 1)],
+              "mdbf_prefill": [("mdbf", INTER, HIDDEN, 2048), ("mdbf", HIDDEN, INTER, 2048)],
               "layer": [("benq", INTER, HIDDEN, 1), ("mdbf", INTER, HIDDEN, 1)]}[workload]
     out = []
     for kind, N, K, B in shapes:
@@ -266,12 +285,13 @@ def oracle_samples(workload, rows=64, seed=0):
             out.append((f"benq {rows} rows x K={K}, B={bb}", lambda w=w, x=x, K=K: ob.linear(w.codes, w.lut, x, K),
                         benq_bytes(rows, K, bb)))
         else:
+            bb = min(B, 16)   # prefill: a 16-row slice of the batch (the oracle's cost is linear in it)
             paths = synth.mdbf_paths(MLP_P, N, K, MLP_R, MLP_L, seed=7)
-            x = synth.activations(B, K, seed=1)
+            x = synth.activations(bb, K, seed=1)
             sel = np.sort(rng.choice(N, rows, replace=False))
-            out.append((f"mdbf {rows} of {N} rows, m={K}, B={B}",
+            out.append((f"mdbf {rows} of {N} rows, m={K}, B={bb}",
                         lambda paths=paths, x=x, N=N, K=K, sel=sel: om.linear_factored(paths, N, K, MLP_R, x, rows=sel),
-                        mdbf_bytes(rows, K, MLP_R, MLP_L, MLP_P, B)))
+                        mdbf_bytes(rows, K, MLP_R, MLP_L, MLP_P, bb)))
     return out
 
 
@@ -351,7 +371,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "mdbf", "layer"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "mdbf", "mdbf_prefill", "layer"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -445,6 +465,15 @@ def main():
                 "frac": achieved / peaks["bf16_tflops"], "traffic": _traffic("benq_gemm"),
                 "kernel": "benq_gemm_tcgen05", "avg_launch_us": 1e3 * dom_ms / dom_launches,
                 "peak_source": peaks["source"] + " (burst)"}
+    elif args.workload == "mdbf_prefill":
+        # the whole call (envelope and activation prep plus both GEMMs) against the fp16 dense
+        # peak, which equals the bf16 one; FLOPs are those of the factored contraction
+        flops = sum(mdbf_flops(L["n"], L["m"], MLP_R, MLP_P, L["B"]) for L in dom) * args.steps
+        achieved = flops / (dom_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": _traffic("mdbf_gemm"),
+                "kernel": "mdbf_gemm_tcgen05 (2 GEMMs + 2 prep kernels per call)",
+                "avg_launch_us": 1e3 * dom_ms / dom_launches, "peak_source": peaks["source"] + " (burst)"}
     else:
         kb = 0.0
         for L in dom:
@@ -486,7 +515,9 @@ def main():
 
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16xu6->f32" if args.workload != "mdbf" else "u1+f16->f32",
+            "vs_baseline": None,
+            "dtype": {"mdbf": "u1+f16->f32", "mdbf_prefill": "u1+f16->f16 (fp32 accumulate)"}.get(args.workload,
+                                                                                            "bf16xu6->f32"),
             "data": "synthetic",
             "config": {"workload": wl.name, "layers": [L["label"] for L in wl.layers],
                        "us_per_step": 1e3 * ms_per_step,

@@ -58,7 +58,7 @@ constexpr int OFF_B = OFF_A + SA * A_BYTES;
 constexpr int CW_BYTES = 512;                     // l <= 4: one warp's fp32 column pairs of a K block
 constexpr int OFF_CW = OFF_B + SB * B_BYTES;      // two of them per decoder warp
 constexpr int OFF_BAR = OFF_CW + 16 * 2 * CW_BYTES;
-constexpr int NBAR = 2 * SA + 3 * SB + 4;
+constexpr int NBAR = 2 * SA + 3 * SB + 6;
 constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // tensor-memory address, abort flag, last-part flag
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;  // + alignment slack
 constexpr int NDEC = 16;                          // decoder / epilogue warps: 8 row groups x 2 column halves
@@ -116,11 +116,12 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 struct Bars {
   // full_a, peer_b and acc_empty are used in the even CTA only (both CTAs arrive on full_a and
   // acc_empty; the odd CTA's forwarder on peer_b).  dec_done collects this CTA's decoder warps.
-  uint32_t full_a, empty_a, dec_done, peer_b, empty_b, acc_full, acc_empty, split_done, split_go;
+  // stg_full / stg_free hand each epilogue round's staging buffer to the tensor stores and back.
+  uint32_t full_a, empty_a, dec_done, peer_b, empty_b, acc_full, acc_empty, split_done, split_go, stg_full, stg_free;
   __device__ Bars(uint32_t base)
       : full_a(base), empty_a(full_a + 8 * SA), dec_done(empty_a + 8 * SA), peer_b(dec_done + 8 * SB),
         empty_b(peer_b + 8 * SB), acc_full(empty_b + 8 * SB), acc_empty(acc_full + 8), split_done(acc_empty + 8),
-        split_go(split_done + 8) {}
+        split_go(split_done + 8), stg_full(split_go + 8), stg_free(stg_full + 8) {}
 };
 
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -378,6 +379,7 @@ __device__ __forceinline__ void put_span(void *out, int ldo, bool ovec, int ydt,
 template <bool FST, int LK, int LC = (LK + 15) / 16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     mdbf_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ Factor fac,
+                     const __grid_constant__ CUtensorMap map_out, int tstore,
                      void *__restrict__ out, int ldo, int ovec, int ydt, const float *__restrict__ row_scale, int M,
                      int Nout, int nkb, float *__restrict__ part_ws, unsigned *__restrict__ part_cnt, int full,
                      int parts) {
@@ -409,9 +411,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     sm100::mbar_init(bar.acc_empty, 2 * NDEC);
     sm100::mbar_init(bar.split_done, NDEC);
     sm100::mbar_init(bar.split_go, 1);
+    sm100::mbar_init(bar.stg_full, NDEC);
+    sm100::mbar_init(bar.stg_free, 1);
     sts32(tmem_slot + 4, 0);
     sm100::fence_barrier_init();
     sm100::prefetch_tensormap(&map_a);
+    if (tstore) sm100::prefetch_tensormap(&map_out);
   }
   if (warp == 1) {
     __syncwarp();
@@ -526,7 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       k0v[c] = 16 * c + 2 * t < l;
       k1v[c] = LK > 8 && 16 * c + 2 * t + 8 < l;
     }
-    int it = 0, tl = 0, ns = 0;
+    int it = 0, tl = 0, ns = 0, ep = 0;
     for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
       const Item w = item_of(wi, full, parts, nkb);
       const int m0 = (w.tile % mt) * PM + (int)rank * BM, n0 = (w.tile / mt) * BN;
@@ -549,15 +554,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             ra2[i] = f2(a, a);
             rb2[i] = f2(b, b);
           }
-          return;
-        }
+        } else {
 #pragma unroll
-        for (int c = 0; c < LC; ++c) {
-          const int k0 = 16 * c + 2 * t;
-          afr[c][0] = va ? env_pair(L + (size_t)ra * l, l, k0, lvec) : 0u;
-          afr[c][1] = vb ? env_pair(L + (size_t)rb * l, l, k0, lvec) : 0u;
-          afr[c][2] = (LK > 8 && va) ? env_pair(L + (size_t)ra * l, l, k0 + 8, lvec) : 0u;
-          afr[c][3] = (LK > 8 && vb) ? env_pair(L + (size_t)rb * l, l, k0 + 8, lvec) : 0u;
+          for (int c = 0; c < LC; ++c) {
+            const int k0 = 16 * c + 2 * t;
+            afr[c][0] = va ? env_pair(L + (size_t)ra * l, l, k0, lvec) : 0u;
+            afr[c][1] = vb ? env_pair(L + (size_t)rb * l, l, k0, lvec) : 0u;
+            afr[c][2] = (LK > 8 && va) ? env_pair(L + (size_t)ra * l, l, k0 + 8, lvec) : 0u;
+            afr[c][3] = (LK > 8 && vb) ? env_pair(L + (size_t)rb * l, l, k0 + 8, lvec) : 0u;
+          }
         }
       };
       // fetch state: path fp and path-local K block fkl of the next block to load
@@ -630,24 +635,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int c = 0; c < LC; ++c) afr[c][0] = afr[c][1] = afr[c][2] = afr[c][3] = 0u;
       }
-      Pre cur, nxt;
-      fetch(cur);
+      // Block buffers in a ring, the loop unrolled by the ring's length so that each buffer keeps
+      // fixed registers.  l <= 4 (three buffers): the loads for block kb + 2 are issued while block
+      // kb is decoded and first needed two blocks later, so the decoders are not paced by the
+      // memory latency.  The larger warp-MMA fragments fit two buffers (one block ahead).
+      constexpr int RING = LK == 4 ? 3 : 2;
+      Pre p0, p1, p2;
+      fetch(p0);
+      if (RING == 3 && w.kb0 + 1 < w.kb1) fetch(p1);
       const uint32_t cwb = sbase + OFF_CW + dw * 2 * CW_BYTES;   // this warp's two column-pair blocks
       if constexpr (LK == 4) {
-        sts128(cwb + (it & 1) * CW_BYTES + 16 * lane, cur.c);
+        sts128(cwb + (it & 1) * CW_BYTES + 16 * lane, p0.c);
         __syncwarp();
       }
-      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
-        if (kb + 1 < w.kb1) fetch(nxt);
+      auto step = [&](int kb, const Pre &cur, const Pre &next, Pre &fill) -> bool {
+        if (kb + RING - 1 < w.kb1) fetch(fill);
         if (FST && kcl == kbp) {
           kcl = 0;
           load_rows(++pc);
         }
         const int sb = it % SB;
-        if (it >= SB && !wt.wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, true)) {
-          ok = false;
-          break;
-        }
+        if (it >= SB && !wt.wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, true)) return false;
         const uint32_t base = sbase + OFF_B + sb * B_BYTES + st_off;
         const uint32_t ea = cur.wa >> (2 * t), eb = cur.wb >> (2 * t);
         const uint32_t ea2 = ea >> 16, eb2 = eb >> 16;
@@ -684,13 +692,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(bar.dec_done + 8 * sb);
         if (FST) ++kcl;
-        if (kb + 1 < w.kb1) {
-          cur = nxt;
-          if constexpr (LK == 4) {
-            // every lane has read block it's pairs (the arrive above follows a __syncwarp)
-            sts128(cwb + ((it + 1) & 1) * CW_BYTES + 16 * lane, cur.c);
+        if constexpr (LK == 4) {
+          if (kb + 1 < w.kb1) {
+            // every lane has read this block's pairs (the arrive above follows a __syncwarp)
+            sts128(cwb + ((it + 1) & 1) * CW_BYTES + 16 * lane, next.c);
             __syncwarp();
           }
+        }
+        ++it;
+        return true;
+      };
+      if constexpr (RING == 3) {
+        for (int kb = w.kb0; kb < w.kb1;) {
+          if (!step(kb, p0, p1, p2)) { ok = false; break; }
+          if (++kb >= w.kb1) break;
+          if (!step(kb, p1, p2, p0)) { ok = false; break; }
+          if (++kb >= w.kb1) break;
+          if (!step(kb, p2, p0, p1)) { ok = false; break; }
+          ++kb;
+        }
+      } else {
+        for (int kb = w.kb0; kb < w.kb1;) {
+          if (!step(kb, p0, p1, p1)) { ok = false; break; }
+          if (++kb >= w.kb1) break;
+          if (!step(kb, p1, p0, p0)) { ok = false; break; }
+          ++kb;
         }
       }
       if (!ok) break;
@@ -699,7 +725,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       qld::pdl_wait();
       sm100::tc_fence_after();
       const bool split = w.part >= 0;
+      if (!split && tstore) {
+        // Whole tile through tensor stores: once acc_full has fired every block of the tile has
+        // been consumed, so the B ring (4 x 16 KB) is free and holds one round of output at a
+        // time, box ch (= this warp's 64 columns) in stage ch, 128 rows x 128 bytes, 128-byte
+        // swizzle.  16-bit output: one round per 128-row half; fp32: two (32 columns per warp).
+        const bool f32o = FST && ydt == QL_OUT_F32;
+        const int cpr = f32o ? 1 : 2, nround = f32o ? 4 : 2;
+        const uint32_t rbase = sbase + OFF_B + (uint32_t)ch * B_BYTES + (uint32_t)(32 * q + lane) * 128u;
+        const uint32_t rsw = (uint32_t)(lane & 7);
+#pragma unroll 1
+        for (int rd = 0; rd < nround && ok; ++rd) {
+          const int h = f32o ? rd >> 1 : rd, cc = f32o ? rd & 1 : 0;
+          const int row = m0 + h * 128 + 32 * q + lane;
+          const float rs = (FST && row < M) ? __ldg(row_scale + row) : 1.f;
+          if (ep > 0 && !wt.wait(bar.stg_free, (ep - 1) & 1, false)) { ok = false; break; }
+#pragma unroll 1
+          for (int k = 0; k < cpr; ++k) {
+            const int c = 2 * ch + (f32o ? cc : k);   // accumulator chunk of 32 columns
+            uint32_t v[32];
+            sm100::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + h * BN + c * 32, v);
+            sm100::tmem_wait_ld();
+            if (f32o) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                sts128(rbase + (((uint32_t)j ^ rsw) << 4),
+                       make_uint4(__float_as_uint(__uint_as_float(v[4 * j]) * rs),
+                                  __float_as_uint(__uint_as_float(v[4 * j + 1]) * rs),
+                                  __float_as_uint(__uint_as_float(v[4 * j + 2]) * rs),
+                                  __float_as_uint(__uint_as_float(v[4 * j + 3]) * rs)));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float a = __uint_as_float(v[8 * j + 2 * e]), b = __uint_as_float(v[8 * j + 2 * e + 1]);
+                  pk[e] = FST ? (uint32_t(qld::f32_to_bf16_rn(a * rs)) | (uint32_t(qld::f32_to_bf16_rn(b * rs)) << 16))
+                              : pack_f16x2(a, b);
+                }
+                sts128(rbase + (((uint32_t)(4 * k + j) ^ rsw) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+              }
+            }
+          }
+          sm100::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(bar.stg_full);
+          if (dw == 0 && lane == 0) {
+            // one thread stores the round's four boxes; parts past the output's edge are clipped
+            if (!wt.wait(bar.stg_full, ep & 1, false)) {
+              ok = false;
+            } else {
+              const int y0 = m0 + h * 128;
+              for (int b = 0; b < 4; ++b) {
+                const int x0 = n0 + 64 * b + 32 * cc;
+                if (x0 < Nout && y0 < M) sm100::tma_store_2d(&map_out, x0, y0, sbase + OFF_B + b * B_BYTES);
+              }
+              sm100::bulk_commit();
+              sm100::bulk_wait_read0();
+              sm100::mbar_arrive(bar.stg_free);
+            }
+          }
+          ++ep;
+        }
+        // the B ring is written again when the next tile is decoded: wait for the last round
+        if (!ok || !wt.wait(bar.stg_free, (ep - 1) & 1, false)) { ok = false; break; }
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive_cluster(lead_acc_empty);
+        continue;
+      }
       // fp32 partials of a split tile: [tile - full][part][rank][BM rows][BN columns]
+
       float *const slot =
           split ? part_ws + ((size_t)((w.tile - full) * parts + w.part) * 2 + rank) * (size_t)(BM * BN) : nullptr;
 #pragma unroll 1
@@ -770,6 +867,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   }
 
+  if (warp == 2 && lane == 0) sm100::bulk_wait0();   // the tensor stores issued by decoder 0
   if (!ok) atomicExch(&g_mgemm_timeout, 1);
   // neither CTA leaves while its peer may still arrive on its barriers, read its shared memory
   // through a pair MMA or write its tensor memory
@@ -883,17 +981,26 @@ Factor make_factor(const mdbf_path *paths, int P, bool f_stage, int n, int m, in
   return f;
 }
 
+// Outputs: T' through tensor stores (mto, always); y through tensor stores when my is valid
+// (ystore), else with direct stores.
+struct OutMaps {
+  CUtensorMap mto, my;
+  bool ystore;
+};
+
 template <int LK>
-void launch_gemms(const CUtensorMap &mx, const CUtensorMap &mt_, const Factor &fg, const Factor &ff, const GemmWs &L,
-                  char *base, void *y, int ydt, bool yvec, int B, int P, int n, int resident, cudaStream_t s) {
+void launch_gemms(const CUtensorMap &mx, const CUtensorMap &mt_, const OutMaps &om, const Factor &fg, const Factor &ff,
+                  const GemmWs &L, char *base, void *y, int ydt, bool yvec, int B, int P, int n, int resident,
+                  cudaStream_t s) {
   float *part = reinterpret_cast<float *>(base + L.part);
   unsigned *cnt1 = reinterpret_cast<unsigned *>(base + L.cnt);
   unsigned *cnt2 = reinterpret_cast<unsigned *>(base + L.cnt + L.g1.counter_bytes);
   const int items1 = L.g1.full + L.g1.leftover * L.g1.parts, items2 = L.g2.full + L.g2.leftover * L.g2.parts;
-  ql::launch(mdbf_gemm_kernel<false, LK>, 2 * std::min(items1, resident), THREADS, SMEM_BYTES, s, mx, fg,
+  ql::launch(mdbf_gemm_kernel<false, LK>, 2 * std::min(items1, resident), THREADS, SMEM_BYTES, s, mx, fg, om.mto, 1,
              static_cast<void *>(base + L.ts), P * L.seg, 1, 0, static_cast<const float *>(nullptr), B, P * L.seg,
              L.mp / BK, part, cnt1, L.g1.full, L.g1.parts);
-  ql::launch(mdbf_gemm_kernel<true, LK>, 2 * std::min(items2, resident), THREADS, SMEM_BYTES, s, mt_, ff, y, n,
+  ql::launch(mdbf_gemm_kernel<true, LK>, 2 * std::min(items2, resident), THREADS, SMEM_BYTES, s, mt_, ff, om.my,
+             om.ystore ? 1 : 0, y, n,
              yvec ? 1 : 0, ydt, reinterpret_cast<const float *>(base + L.inv_s), B, n, P * L.seg / BK, part, cnt2,
              L.g2.full, L.g2.parts);
 }
@@ -922,6 +1029,14 @@ ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, i
       !encode_rows_sw128(enc, &mtm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + L.ts, B, (uint64_t)P * L.seg,
                          (uint64_t)P * L.seg, BM))
     return fail(QL_ERR_CUDA, "mdbf_linear: cannot encode the activation tensor maps");
+  const bool yvec = aligned(y, 16) && (ydt == QL_OUT_F32 ? n % 4 == 0 : n % 8 == 0);
+  OutMaps om = {};
+  if (!encode_rows_sw128(enc, &om.mto, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + L.ts, B, (uint64_t)P * L.seg,
+                         (uint64_t)P * L.seg, 128))
+    return fail(QL_ERR_CUDA, "mdbf_linear: cannot encode the intermediate's tensor map");
+  om.ystore = yvec && encode_rows_sw128(enc, &om.my,
+                                        ydt == QL_OUT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                        y, B, n, n, 128, ydt == QL_OUT_F32 ? 4 : 2);
   const Factor fg = make_factor(paths, P, false, n, m, r, l, L, base);
   const Factor ff = make_factor(paths, P, true, n, m, r, l, L, base);
   float *emax = reinterpret_cast<float *>(base + L.emax);
@@ -936,15 +1051,14 @@ ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, i
          reinterpret_cast<unsigned *>(base + L.cnt), ncnt, xvec ? 1 : 0);
   st = launch_status("mdbf_linear (activation prep)");
   if (st != QL_OK) return st;
-  const bool yvec = aligned(y, 16) && (ydt == QL_OUT_F32 ? n % 4 == 0 : n % 8 == 0);
   if (l <= 4)
-    launch_gemms<4>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+    launch_gemms<4>(mx, mtm, om, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
   else if (l <= 8)
-    launch_gemms<8>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+    launch_gemms<8>(mx, mtm, om, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
   else if (l <= 16)
-    launch_gemms<16>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+    launch_gemms<16>(mx, mtm, om, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
   else
-    launch_gemms<32>(mx, mtm, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
+    launch_gemms<32>(mx, mtm, om, fg, ff, L, base, y, (int)ydt, yvec, B, P, n, resident, s);
   return launch_status("mdbf_linear (tensor-core GEMMs)");
 }
 

@@ -117,13 +117,14 @@ inline EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// Tensor map of a row-major 2-D array [rows][cols] of 2-byte elements (row stride ld elements)
-// read in boxes of box_rows x 64 elements with the 128-byte swizzle the tensor core expects.
+// Tensor map of a row-major 2-D array [rows][cols] of esize-byte elements (row stride ld
+// elements) in boxes of box_rows rows x 128 bytes with the 128-byte swizzle (the tensor core's
+// operand layout, and the staging layout of the tensor-store epilogue).
 inline bool encode_rows_sw128(EncodeTiledFn enc, CUtensorMap *map, CUtensorMapDataType dt, const void *base,
-                              uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+                              uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows, uint32_t esize = 2) {
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * esize};
+  const cuuint32_t box[2] = {128 / esize, box_rows};
   const cuuint32_t es[2] = {1, 1};
   return enc(map, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
