@@ -55,7 +55,7 @@ constexpr int A_BYTES = BM * BK * 2;              // 32 KB
 constexpr int B_BYTES = BNH * BK * 2;             // 16 KB
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + SA * A_BYTES;
-constexpr int CW_BYTES = 512;                     // l <= 4: one warp's fp32 column pairs of a K block
+constexpr int CW_BYTES = 256;                     // l <= 4: one warp's fp32 column pairs of a K block
 constexpr int OFF_CW = OFF_B + SB * B_BYTES;      // two of them per decoder warp
 constexpr int OFF_BAR = OFF_CW + 16 * 2 * CW_BYTES;
 constexpr int NBAR = 2 * SA + 3 * SB + 6;
@@ -136,6 +136,9 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
+}
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
 }
 __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
@@ -535,6 +538,140 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
       const Item w = item_of(wi, full, parts, nkb);
       const int m0 = (w.tile % mt) * PM + (int)rank * BM, n0 = (w.tile / mt) * BN;
+      if constexpr (LK == 4) {
+        // l <= 4, packed fp32 FMAs: warp dw rebuilds rows [32 rq, 32 rq + 32) x columns
+        // [16 cq, 16 cq + 16) of this CTA's 128 x 64 block (rq = dw % 4, cq = dw / 4); lane (g, t)
+        // owns rows g + 8k (k < 4) and the column pairs 8u + 2t, +1 (u < 2).  Four rows per lane
+        // halve the column-envelope reads per element against two; each 32-bit store of a warp
+        // covers 8 rows of one swizzle atom, conflict-free.
+        const int rq = dw & 3, cq = dw >> 2;
+        const int grow = n0 + BNH * (int)rank + 32 * rq;
+        const int prow = FST ? 0 : grow / fac.seg;
+        const bool pv = FST || prow < fac.P;
+        const int r0 = (FST ? grow : grow - prow * fac.seg) + g;   // path-local row of k = 0
+        bool vr[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) vr[k] = pv && r0 + 8 * k < fac.rows;
+        // row envelope terms of row pairs (k = 2j, 2j + 1), [j][term]: each packed FMA computes
+        // one column for two rows
+        uint64_t rr2[2][4];
+        auto load_rows = [&](int p) {
+          const uint16_t *L = fac.Lrow[p];
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int ka = 2 * j, kb2 = 2 * j + 1;
+              const float a = (vr[ka] && i < l) ? qld::f16_to_f32(L[(size_t)(r0 + 8 * ka) * l + i]) : 0.f;
+              const float b = (vr[kb2] && i < l) ? qld::f16_to_f32(L[(size_t)(r0 + 8 * kb2) * l + i]) : 0.f;
+              rr2[j][i] = f2(a, b);
+            }
+        };
+        int fp = FST ? w.kb0 / kbp : prow, fkl = FST ? w.kb0 - fp * kbp : w.kb0;
+        const uint8_t *sg = nullptr;   // sign row r0 of path fp from the warp's 16 columns; row k at + 8k ld
+        size_t sld8 = 0;
+        const float *cpp = nullptr;    // fp32 pair block of the warp's 16 columns
+        auto set_path = [&](int p) {
+          const size_t ld = fac.ld[p];
+          sg = fac.S[p] + (size_t)r0 * ld + 2 * cq;
+          sld8 = 8 * ld;
+          cpp = fac.cpair + ((size_t)p * (fac.cpad / 2) + 8 * cq) * 8;
+        };
+        if (pv) set_path(fp);
+        struct Pre {
+          uint32_t w[4];   // 16 sign bits per row
+          uint2 c;         // this lane's 8 bytes of the warp's 256-byte pair block
+        };
+        auto fetch = [&](Pre &o) {
+          // A 16-bit sign load that starts inside the row's ceil(cols / 8) bytes ends inside its
+          // stride (rows 4-byte aligned, strides multiples of 4, checked by the ABI); bits past
+          // the last column meet a zero column envelope.  Pair blocks are zero-padded to cpad.
+          const int kc = fkl * BK + 16 * cq;
+          const bool win = pv && kc < cols;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            o.w[k] = (vr[k] && win) ? (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sg + k * sld8 + 8 * fkl)) : 0u;
+          o.c = pv ? __ldg(reinterpret_cast<const uint2 *>(cpp + (size_t)fkl * (BK / 2) * 8) + lane) : make_uint2(0u, 0u);
+          if (FST && ++fkl == kbp) {
+            fkl = 0;
+            if (++fp < fac.P) set_path(fp);
+          } else if (!FST) {
+            ++fkl;
+          }
+        };
+        int pc = FST ? w.kb0 / kbp : prow, kcl = FST ? w.kb0 - pc * kbp : 0;
+        if (FST || pv) {
+          load_rows(pc);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rr2[j][i] = f2(0.f, 0.f);
+        }
+        // per-lane store offsets in a B stage: row 32 rq + g + 8k is row g of atom 4 rq + k
+        const uint32_t so0 = (uint32_t)(4 * rq) * 1024u + (uint32_t)g * 128u + 4u * (uint32_t)t;
+        const uint32_t sx0 = ((uint32_t)(2 * cq) ^ (uint32_t)g) << 4, sx1 = ((uint32_t)(2 * cq + 1) ^ (uint32_t)g) << 4;
+        const uint32_t cwb = sbase + OFF_CW + dw * 2 * CW_BYTES;   // this warp's two pair blocks
+        Pre p0, p1;
+        fetch(p0);
+        sts64(cwb + (it & 1) * CW_BYTES + 8 * lane, p0.c.x, p0.c.y);
+        __syncwarp();
+        // two block buffers, the loop unrolled by two so that each keeps fixed registers; the
+        // loads for block kb + 1 are issued before block kb is decoded
+        auto step = [&](int kb, const Pre &cur, Pre &next) -> bool {
+          if (kb + 1 < w.kb1) fetch(next);
+          if (FST && kcl == kbp) {
+            kcl = 0;
+            load_rows(++pc);
+          }
+          const int sb = it % SB;
+          if (it >= SB && !wt.wait(bar.empty_b + 8 * sb, ((it / SB) & 1) ^ 1, true)) return false;
+          const uint32_t base = sbase + OFF_B + sb * B_BYTES + so0;
+          const uint32_t cb = cwb + (it & 1) * CW_BYTES;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            // pair block 4u + t: {C[c][i], C[c + 1][i]} for terms i = 0, 1 then 2, 3
+            const uint4 c0 = lds128(cb + (4 * u + t) * 32), c1 = lds128(cb + (4 * u + t) * 32 + 16);
+            const uint32_t cv[2][4] = {{c0.x, c0.z, c1.x, c1.z}, {c0.y, c0.w, c1.y, c1.w}};   // [column][term]
+            float e[2][4];   // [column][row k]
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                // envelope terms in ascending order, one rounding per term, as the oracle sums them
+                uint64_t acc = f2(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc = ffma2(rr2[j][i], f2u(cv[h][i], cv[h][i]), acc);
+                f2split(acc, e[h][2 * j], e[h][2 * j + 1]);
+              }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t sgn = cur.w[k] >> (2 * t);
+              const uint32_t flip = u ? sign_flip<1>(sgn) : sign_flip<0>(sgn);
+              sts32(base + (uint32_t)k * 1024u + (u ? sx1 : sx0), pack_f16x2(e[0][k], e[1][k]) ^ flip);
+            }
+          }
+          // handed to this CTA's MMA side through a CTA-scope barrier: the even CTA's MMA thread
+          // waits on it directly, the odd CTA's forwarder relays it at cluster scope
+          sm100::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(bar.dec_done + 8 * sb);
+          if (FST) ++kcl;
+          if (kb + 1 < w.kb1) {
+            // every lane has read this block's pairs (the arrive above follows a __syncwarp)
+            sts64(cwb + ((it + 1) & 1) * CW_BYTES + 8 * lane, next.c.x, next.c.y);
+            __syncwarp();
+          }
+          ++it;
+          return true;
+        };
+        for (int kb = w.kb0; kb < w.kb1;) {
+          if (!step(kb, p0, p1)) { ok = false; break; }
+          if (++kb >= w.kb1) break;
+          if (!step(kb, p1, p0)) { ok = false; break; }
+          ++kb;
+        }
+      } else {
       // first operand row of this warp's group (along the GEMM's N); in the G stage it fixes the
       // path, in the F stage the path follows the K block
       const int grow = n0 + BNH * (int)rank + 16 * rg;
@@ -718,6 +855,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           if (!step(kb, p1, p0, p0)) { ok = false; break; }
           ++kb;
         }
+      }
       }
       if (!ok) break;
       // epilogue: this warp drains lanes [32q, 32q+32) of both 128-row accumulators
