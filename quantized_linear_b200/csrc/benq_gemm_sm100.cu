@@ -54,7 +54,7 @@ constexpr int OFF_B = OFF_A + SA * A_BYTES;
 constexpr int OFF_C = OFF_B + SB * B_BYTES;
 constexpr int OFF_LUT = OFF_C + SC * C_BYTES + 128;   // 128 bytes of slack: the last row's second code word
 constexpr int OFF_BAR = OFF_LUT + LUT_BYTES;
-constexpr int NBAR = 2 * (SA + SB + SC) + 6;
+constexpr int NBAR = 2 * (SA + SB + SC) + 8;
 constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;          // tensor-memory address, abort flag, last-part flag
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;      // + alignment slack
 constexpr int NDEC = 16;                              // decoder / epilogue warps (multiple of 8)
@@ -63,6 +63,7 @@ constexpr uint32_t IDESC = sm100::idesc_bf16_f32(2 * 128, BN);   // pair MMA: M 
 constexpr uint16_t PAIR = 0x3;                        // both CTAs of the cluster
 static_assert(OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
 static_assert(OFF_LUT % 128 == 0 && OFF_BAR % 8 == 0, "alignment");
+static_assert(SB * B_BYTES == 4 * 16384, "the decoded-W ring stages one epilogue round: four 16 KB boxes");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 __device__ int g_gemm_timeout = 0;
@@ -71,16 +72,17 @@ struct Bars {
   // full_a, full_b and acc_empty are used in the even CTA only (both CTAs arrive on them);
   // the others are local to each CTA.
   uint32_t full_a, empty_a, full_b, empty_b, full_c, empty_c, lut_full, lut_empty, acc_full, acc_empty, split_done,
-      split_go;
+      split_go, stg_full, stg_free;
   __device__ Bars(uint32_t base)
       : full_a(base), empty_a(full_a + 8 * SA), full_b(empty_a + 8 * SA), empty_b(full_b + 8 * SB),
         full_c(empty_b + 8 * SB), empty_c(full_c + 8 * SC), lut_full(empty_c + 8 * SC), lut_empty(lut_full + 8),
-        acc_full(lut_empty + 8), acc_empty(acc_full + 8), split_done(acc_empty + 8), split_go(split_done + 8) {}
+        acc_full(lut_empty + 8), acc_empty(acc_full + 8), split_done(acc_empty + 8), split_go(split_done + 8),
+        stg_full(split_go + 8), stg_free(stg_full + 8) {}
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     benq_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
-                     const uint16_t *__restrict__ lut, void *__restrict__ y, int ydt, int M, int N, int K,
+                     const __grid_constant__ CUtensorMap map_y, int tstore, const uint16_t *__restrict__ lut, void *__restrict__ y, int ydt, int M, int N, int K,
                      float *__restrict__ part_ws, unsigned *__restrict__ part_cnt, int full, int parts) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
@@ -115,10 +117,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     sm100::mbar_init(bar.acc_empty, 2 * NDEC);
     sm100::mbar_init(bar.split_done, NDEC);
     sm100::mbar_init(bar.split_go, 1);
+    sm100::mbar_init(bar.stg_full, NDEC);
+    sm100::mbar_init(bar.stg_free, 1);
     sts32(tmem_slot + 4, 0);
     sm100::fence_barrier_init();
     sm100::prefetch_tensormap(&map_x);
     sm100::prefetch_tensormap(&map_codes);
+    if (tstore) sm100::prefetch_tensormap(&map_y);
   }
   if (warp == 1) {
     __syncwarp();
@@ -216,7 +221,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int ch = dw >> 2;             // which NDEC/4-th of the 256 accumulator columns it drains
     const uint32_t lead_full_b = sm100::mapa_shared(bar.full_b, 0);
     const uint32_t lead_acc_empty = sm100::mapa_shared(bar.acc_empty, 0);
-    int it = 0, tl = 0, ic = 0, ns = 0;
+    int it = 0, tl = 0, ic = 0, ns = 0, ep = 0;
     // A pass decodes two K blocks: lanes 0-15 the first, 16-31 the second.  Lane l expands the 4
     // codes in bytes [3l, 3l + 3) of the two blocks' 96 code bytes of a row (codes 4(l&15) ..
     // 4(l&15)+3 of its block), so two 32-bit loads serve 4 codes and its output is 8 bytes.
@@ -283,6 +288,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       qld::pdl_wait();
       sm100::tc_fence_after();
       const bool split = w.part >= 0;
+      if (!split && tstore) {
+        // Whole tile through tensor stores: once acc_full has fired every decoded block of the
+        // tile has been consumed, so the decoded-W ring (4 x 16 KB) is free to stage the output.
+        if (!staged_tile_store(tmem, sbase + OFF_B, &map_y, ydt == QL_OUT_F32 ? OUT_F32 : OUT_BF16, nullptr, m0, n0, M,
+                               N, q, ch, dw, lane, wt, bar.stg_full, bar.stg_free, ep)) {
+          ok = false;
+          break;
+        }
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive_cluster(lead_acc_empty);
+        continue;
+      }
       // fp32 partials of a split tile: [tile - full][part][rank][BM rows][BN columns]
       float *const slot =
           split ? part_ws + ((size_t)((w.tile - full) * parts + w.part) * 2 + rank) * (size_t)(BM * BN) : nullptr;
@@ -372,6 +390,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   }
 
+  if (warp == 3 && lane == 0) sm100::bulk_wait0();   // the tensor stores issued by decoder 0
   if (!ok) atomicExch(&g_gemm_timeout, 1);
   // neither CTA leaves while its peer may still arrive on its barriers, read its shared memory
   // through a pair MMA or write its tensor memory
@@ -459,6 +478,11 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return fail(QL_ERR_CUDA, "benq_linear: cannot encode the code tensor map");
   }
+  // y through tensor stores when its rows are 16-byte aligned (N % 256 == 0 here), else direct stores
+  CUtensorMap my = {};
+  const bool tstore = aligned(y, 16) && encode_rows_sw128(enc, &my, ydt == QL_OUT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                                          y, M, N, N, 128, ydt == QL_OUT_F32 ? 4 : 2);
   if (smem_attr() != cudaSuccess) return fail(QL_ERR_CUDA, "benq_linear: cannot reserve GEMM shared memory");
   const int ntiles = ((M + PM - 1) / PM) * (N / BN);
   const int resident = resident_pairs();
@@ -475,7 +499,7 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
   }
   const int nitems = plan.full + plan.leftover * plan.parts;
   const int pairs = std::min(nitems, resident);
-  launch(benq_gemm_kernel, 2 * pairs, THREADS, SMEM_BYTES, s, mx, mc, lut, y, (int)ydt, M, N, K, part_ws, part_cnt,
+  launch(benq_gemm_kernel, 2 * pairs, THREADS, SMEM_BYTES, s, mx, mc, my, tstore ? 1 : 0, lut, y, (int)ydt, M, N, K, part_ws, part_cnt,
          plan.full, plan.parts);
   return launch_status("benq_linear (tensor-core GEMM)");
 }

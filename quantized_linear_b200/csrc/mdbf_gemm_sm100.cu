@@ -70,6 +70,7 @@ constexpr uint16_t PAIR = 0x3;
 constexpr float T_BOUND = 32768.0f;
 static_assert(OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
+static_assert(SB * B_BYTES == 4 * 16384, "the B ring stages one epilogue round: four 16 KB boxes");
 
 __device__ int g_mgemm_timeout = 0;
 
@@ -139,9 +140,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
 }
 __device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
   asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
-}
-__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
 // {fp16(lo), fp16(hi)} rounded to nearest even, lo in the low half
@@ -865,69 +863,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const bool split = w.part >= 0;
       if (!split && tstore) {
         // Whole tile through tensor stores: once acc_full has fired every block of the tile has
-        // been consumed, so the B ring (4 x 16 KB) is free and holds one round of output at a
-        // time, box ch (= this warp's 64 columns) in stage ch, 128 rows x 128 bytes, 128-byte
-        // swizzle.  16-bit output: one round per 128-row half; fp32: two (32 columns per warp).
-        const bool f32o = FST && ydt == QL_OUT_F32;
-        const int cpr = f32o ? 1 : 2, nround = f32o ? 4 : 2;
-        const uint32_t rbase = sbase + OFF_B + (uint32_t)ch * B_BYTES + (uint32_t)(32 * q + lane) * 128u;
-        const uint32_t rsw = (uint32_t)(lane & 7);
-#pragma unroll 1
-        for (int rd = 0; rd < nround && ok; ++rd) {
-          const int h = f32o ? rd >> 1 : rd, cc = f32o ? rd & 1 : 0;
-          const int row = m0 + h * 128 + 32 * q + lane;
-          const float rs = (FST && row < M) ? __ldg(row_scale + row) : 1.f;
-          if (ep > 0 && !wt.wait(bar.stg_free, (ep - 1) & 1, false)) { ok = false; break; }
-#pragma unroll 1
-          for (int k = 0; k < cpr; ++k) {
-            const int c = 2 * ch + (f32o ? cc : k);   // accumulator chunk of 32 columns
-            uint32_t v[32];
-            sm100::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + h * BN + c * 32, v);
-            sm100::tmem_wait_ld();
-            if (f32o) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                sts128(rbase + (((uint32_t)j ^ rsw) << 4),
-                       make_uint4(__float_as_uint(__uint_as_float(v[4 * j]) * rs),
-                                  __float_as_uint(__uint_as_float(v[4 * j + 1]) * rs),
-                                  __float_as_uint(__uint_as_float(v[4 * j + 2]) * rs),
-                                  __float_as_uint(__uint_as_float(v[4 * j + 3]) * rs)));
-            } else {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float a = __uint_as_float(v[8 * j + 2 * e]), b = __uint_as_float(v[8 * j + 2 * e + 1]);
-                  pk[e] = FST ? (uint32_t(qld::f32_to_bf16_rn(a * rs)) | (uint32_t(qld::f32_to_bf16_rn(b * rs)) << 16))
-                              : pack_f16x2(a, b);
-                }
-                sts128(rbase + (((uint32_t)(4 * k + j) ^ rsw) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
-              }
-            }
-          }
-          sm100::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(bar.stg_full);
-          if (dw == 0 && lane == 0) {
-            // one thread stores the round's four boxes; parts past the output's edge are clipped
-            if (!wt.wait(bar.stg_full, ep & 1, false)) {
-              ok = false;
-            } else {
-              const int y0 = m0 + h * 128;
-              for (int b = 0; b < 4; ++b) {
-                const int x0 = n0 + 64 * b + 32 * cc;
-                if (x0 < Nout && y0 < M) sm100::tma_store_2d(&map_out, x0, y0, sbase + OFF_B + b * B_BYTES);
-              }
-              sm100::bulk_commit();
-              sm100::bulk_wait_read0();
-              sm100::mbar_arrive(bar.stg_free);
-            }
-          }
-          ++ep;
+        // been consumed, so the B ring (4 x 16 KB) is free to stage the output.
+        if (!staged_tile_store(tmem, sbase + OFF_B, &map_out, FST ? (ydt == QL_OUT_F32 ? OUT_F32 : OUT_BF16) : OUT_F16,
+                               FST ? row_scale : nullptr, m0, n0, M, Nout, q, ch, dw, lane, wt, bar.stg_full,
+                               bar.stg_free, ep)) {
+          ok = false;
+          break;
         }
-        // the B ring is written again when the next tile is decoded: wait for the last round
-        if (!ok || !wt.wait(bar.stg_free, (ep - 1) & 1, false)) { ok = false; break; }
         sm100::tc_fence_before();
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive_cluster(lead_acc_empty);

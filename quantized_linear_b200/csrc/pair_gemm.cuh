@@ -64,6 +64,89 @@ struct Waiter {
   }
 };
 
+// ----------------------------------------------------------------------------------- epilogue
+enum OutKind { OUT_F16 = 0, OUT_BF16 = 1, OUT_F32 = 2 };
+
+__device__ __forceinline__ void sts128v(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint32_t pack2(float a, float b, int kind) {
+  uint32_t r;
+  if (kind == OUT_F16)
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  else
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// Writes a CTA's 256 x 256 fp32 accumulator tile (rows m0 .. m0 + 255 of the output, two
+// 128-lane halves at tmem and tmem + 256 columns) to columns n0 .. n0 + 255 through tensor
+// stores.  The staging buffer `ring` is four 16 KB boxes of 128 rows x 128 bytes in the 128-byte
+// swizzle of `map`; it holds one round: a 128-row half for 16-bit outputs, a quarter (32 columns
+// per box) for fp32.  Epilogue warp (q, ch) = (its tensor-memory lane quarter, dw / 4) converts
+// rows 32q .. 32q + 31 of box ch.  Each value is multiplied by row_scale[row] when row_scale is
+// not null, then rounded to the output type (nearest even).  All ndec epilogue warps arrive on
+// stg_full per round; warp 0's lane 0 issues the box stores (clipped at the output's edge),
+// waits until the staging has been read and arrives on stg_free, which every warp waits on
+// before reusing the buffer and before returning.  ep counts rounds across calls (phase parity).
+// Returns false when a wait gave up.
+__device__ __forceinline__ bool staged_tile_store(uint32_t tmem, uint32_t ring, const CUtensorMap *map, int kind,
+                                                  const float *__restrict__ row_scale, int m0, int n0, int M,
+                                                  int Nout, int q, int ch, int dw, int lane, const Waiter &wt,
+                                                  uint32_t stg_full, uint32_t stg_free, int &ep) {
+  const bool f32o = kind == OUT_F32;
+  const int cpr = f32o ? 1 : 2, nround = f32o ? 4 : 2;
+  const uint32_t rbase = ring + (uint32_t)ch * 16384u + (uint32_t)(32 * q + lane) * 128u;
+  const uint32_t rsw = (uint32_t)(lane & 7);
+#pragma unroll 1
+  for (int rd = 0; rd < nround; ++rd) {
+    const int h = f32o ? rd >> 1 : rd, cc = f32o ? rd & 1 : 0;
+    const int row = m0 + h * 128 + 32 * q + lane;
+    const float rs = (row_scale != nullptr && row < M) ? __ldg(row_scale + row) : 1.f;
+    if (ep > 0 && !wt.wait(stg_free, (ep - 1) & 1, false)) return false;
+#pragma unroll 1
+    for (int k = 0; k < cpr; ++k) {
+      const int c = 2 * ch + (f32o ? cc : k);   // accumulator chunk of 32 columns
+      uint32_t v[32];
+      sm100::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + h * 256 + c * 32, v);
+      sm100::tmem_wait_ld();
+      if (f32o) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          sts128v(rbase + (((uint32_t)j ^ rsw) << 4), __float_as_uint(__uint_as_float(v[4 * j]) * rs),
+                  __float_as_uint(__uint_as_float(v[4 * j + 1]) * rs), __float_as_uint(__uint_as_float(v[4 * j + 2]) * rs),
+                  __float_as_uint(__uint_as_float(v[4 * j + 3]) * rs));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            pk[e] = pack2(__uint_as_float(v[8 * j + 2 * e]) * rs, __uint_as_float(v[8 * j + 2 * e + 1]) * rs, kind);
+          sts128v(rbase + (((uint32_t)(4 * k + j) ^ rsw) << 4), pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+    sm100::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) sm100::mbar_arrive(stg_full);
+    if (dw == 0 && lane == 0) {
+      if (!wt.wait(stg_full, ep & 1, false)) return false;
+      const int y0 = m0 + h * 128;
+      for (int b = 0; b < 4; ++b) {
+        const int x0 = n0 + 64 * b + 32 * cc;
+        if (x0 < Nout && y0 < M) sm100::tma_store_2d(map, x0, y0, ring + b * 16384u);
+      }
+      sm100::bulk_commit();
+      sm100::bulk_wait_read0();
+      sm100::mbar_arrive(stg_free);
+    }
+    ++ep;
+  }
+  // the staging buffer is written again by the caller: wait for the last round's stores to read it
+  return wt.wait(stg_free, (ep - 1) & 1, false);
+}
+
 // Work items: pair tiles 0 .. full-1 whole, then each of the remaining tiles (the last, partial
 // wave) split into `parts` K ranges so that the otherwise idle pairs share it.  A split item
 // writes an fp32 partial; the last CTA to finish a tile sums the partials in part order.
