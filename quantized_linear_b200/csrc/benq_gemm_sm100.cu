@@ -14,12 +14,16 @@
 //     once per tile) with a bulk copy;
 //   * warps 3..18 (decoders) expand the code tile through the row tables into the bf16 W half
 //     tile, two K blocks per pass, written directly in the K-major 128-byte-swizzled layout the
-//     tensor core reads, fence the writes for the async proxy and arrive on the even CTA's barrier;
-//   * in the even CTA only, warp 1 (one thread) issues the pair MMAs (two M halves share each
-//     decoded W tile) into both CTAs' tensor memory (2 x 128 x 256 fp32 per CTA) and signals
-//     stage release to both CTAs with a multicast commit;
+//     tensor core reads, fence the writes for the async proxy and arrive on a barrier of their
+//     own CTA;
+//   * in the even CTA, warp 1 (one thread) waits for both CTAs' decoded halves and issues the
+//     pair MMAs (two M halves share each decoded W tile) into both CTAs' tensor memory
+//     (2 x 128 x 256 fp32 per CTA), signalling stage release to both CTAs with a multicast
+//     commit; in the odd CTA one thread of warp 1 relays each decoded block to it at cluster
+//     scope (one release per block instead of one per decoder warp);
 //   * after the last K block the decoder warps of each CTA drain their own accumulators
-//     (tcgen05.ld), round to bf16 (or keep fp32) and store Y.
+//     (tcgen05.ld), round to bf16 (or keep fp32) and store Y, through tensor stores staged in the
+//     decoded-W ring when Y's rows are 16-byte aligned.
 // No tensor or bulk load is multicast.  Every wait gives up after a fixed clock budget or as soon
 // as another wait of the pair has given up, sets a device flag read by ql_check(), and the CTA
 // winds down; both CTAs meet at a cluster barrier before tensor memory is freed and they exit.
@@ -54,7 +58,7 @@ constexpr int OFF_B = OFF_A + SA * A_BYTES;
 constexpr int OFF_C = OFF_B + SB * B_BYTES;
 constexpr int OFF_LUT = OFF_C + SC * C_BYTES + 128;   // 128 bytes of slack: the last row's second code word
 constexpr int OFF_BAR = OFF_LUT + LUT_BYTES;
-constexpr int NBAR = 2 * (SA + SB + SC) + 8;
+constexpr int NBAR = 2 * (SA + SB + SC) + SB + 8;
 constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;          // tensor-memory address, abort flag, last-part flag
 constexpr int SMEM_BYTES = OFF_TMEM + 16 + 1024;      // + alignment slack
 constexpr int NDEC = 16;                              // decoder / epilogue warps (multiple of 8)
@@ -69,15 +73,16 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 __device__ int g_gemm_timeout = 0;
 
 struct Bars {
-  // full_a, full_b and acc_empty are used in the even CTA only (both CTAs arrive on them);
+  // full_a, peer_b and acc_empty are used in the even CTA only (both CTAs arrive on full_a and
+  // acc_empty, the odd CTA's forwarder on peer_b); dec_done collects this CTA's decoder warps;
   // the others are local to each CTA.
-  uint32_t full_a, empty_a, full_b, empty_b, full_c, empty_c, lut_full, lut_empty, acc_full, acc_empty, split_done,
-      split_go, stg_full, stg_free;
+  uint32_t full_a, empty_a, dec_done, empty_b, full_c, empty_c, lut_full, lut_empty, acc_full, acc_empty, split_done,
+      split_go, stg_full, stg_free, peer_b;
   __device__ Bars(uint32_t base)
-      : full_a(base), empty_a(full_a + 8 * SA), full_b(empty_a + 8 * SA), empty_b(full_b + 8 * SB),
+      : full_a(base), empty_a(full_a + 8 * SA), dec_done(empty_a + 8 * SA), empty_b(dec_done + 8 * SB),
         full_c(empty_b + 8 * SB), empty_c(full_c + 8 * SC), lut_full(empty_c + 8 * SC), lut_empty(lut_full + 8),
         acc_full(lut_empty + 8), acc_empty(acc_full + 8), split_done(acc_empty + 8), split_go(split_done + 8),
-        stg_full(split_go + 8), stg_free(stg_full + 8) {}
+        stg_full(split_go + 8), stg_free(stg_full + 8), peer_b(stg_free + 8) {}
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
@@ -104,7 +109,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       sm100::mbar_init(bar.empty_a + 8 * s, 1);
     }
     for (int s = 0; s < SB; ++s) {
-      sm100::mbar_init(bar.full_b + 8 * s, 2 * NDEC);
+      sm100::mbar_init(bar.dec_done + 8 * s, NDEC);
+      sm100::mbar_init(bar.peer_b + 8 * s, 1);
       sm100::mbar_init(bar.empty_b + 8 * s, 1);
     }
     for (int s = 0; s < SC; ++s) {
@@ -192,7 +198,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int sa = it % SA, sb = it % SB;
           if (!wt.wait(bar.full_a + 8 * sa, (it / SA) & 1, true) ||
-              !wt.wait(bar.full_b + 8 * sb, (it / SB) & 1, true)) {
+              !wt.wait(bar.dec_done + 8 * sb, (it / SB) & 1, false) ||
+              !wt.wait(bar.peer_b + 8 * sb, (it / SB) & 1, true)) {
             ok = false;
             break;
           }
@@ -213,13 +220,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (!ok) break;
         sm100::mma_commit_pair(bar.acc_full, PAIR);
       }
+    } else if (!lead && lane == 0) {
+      // ---------------------------------------------------------- forwarder (odd CTA)
+      // relays each decoded block of this CTA to the even CTA's MMA thread: one cluster-scope
+      // release per block instead of one per decoder warp
+      const uint32_t lead_peer_b = sm100::mapa_shared(bar.peer_b, 0);
+      int it = 0;
+      for (int wi = pair; wi < nitems && ok; wi += npairs) {
+        const Item w = item_of(wi, full, parts, nkb);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int sb = it % SB;
+          if (!wt.wait(bar.dec_done + 8 * sb, (it / SB) & 1, false)) {
+            ok = false;
+            break;
+          }
+          sm100::mbar_arrive_cluster(lead_peer_b + 8 * sb);
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------ decoders, then epilogue
     const int dw = warp - 3;            // decoder index 0 .. NDEC-1
     const int q = warp & 3;             // tensor-memory lane quarter this warp may read
     const int ch = dw >> 2;             // which NDEC/4-th of the 256 accumulator columns it drains
-    const uint32_t lead_full_b = sm100::mapa_shared(bar.full_b, 0);
     const uint32_t lead_acc_empty = sm100::mapa_shared(bar.acc_empty, 0);
     int it = 0, tl = 0, ic = 0, ns = 0, ep = 0;
     // A pass decodes two K blocks: lanes 0-15 the first, 16-31 the second.  Lane l expands the 4
@@ -272,8 +295,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int step = two ? 2 : 1;
         const bool stage_done = sub + step >= CKB || kb + step == w.kb1;
         if (lane == 0) {
-          sm100::mbar_arrive_cluster(lead_full_b + 8 * sb0);
-          if (two) sm100::mbar_arrive_cluster(lead_full_b + 8 * sb1);
+          // this CTA's MMA side takes the blocks through a CTA-scope barrier: the even CTA's MMA
+          // thread waits on it directly, the odd CTA's forwarder relays it at cluster scope
+          sm100::mbar_arrive(bar.dec_done + 8 * sb0);
+          if (two) sm100::mbar_arrive(bar.dec_done + 8 * sb1);
           if (stage_done) sm100::mbar_arrive(bar.empty_c + 8 * sc);
         }
         if (stage_done) ++ic;
