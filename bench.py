@@ -235,10 +235,10 @@ class Workload:
 
 # the sources each kernel's DRAM-traffic figure depends on
 _KERNEL_SOURCES = {
-    "benq_gemv": ["benq_gemv.cu", "ql_internal.cuh"],
-    "benq_gemm": ["benq_gemm_sm100.cu", "sm100_ptx.cuh", "ql_internal.cuh"],
-    "mdbf_linear": ["mdbf.cu", "ql_internal.cuh"],
-    "mdbf_gemm": ["mdbf_gemm_sm100.cu", "pair_gemm.cuh", "sm100_ptx.cuh", "ql_internal.cuh"],
+    "benq_gemv": ["benq_gemv.cu", "ql_device.cuh"],
+    "benq_gemm": ["benq_gemm_sm100.cu", "pair_gemm.cuh", "sm100_ptx.cuh", "ql_device.cuh"],
+    "mdbf_linear": ["mdbf.cu", "ql_device.cuh"],
+    "mdbf_gemm": ["mdbf_gemm_sm100.cu", "pair_gemm.cuh", "sm100_ptx.cuh", "ql_device.cuh"],
 }
 
 

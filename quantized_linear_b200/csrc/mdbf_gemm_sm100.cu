@@ -93,26 +93,10 @@ struct Factor {
   int cpad;
 };
 
-// packed fp32 pairs (the f32x2 operands of fma.rn.f32x2)
-__device__ __forceinline__ uint64_t f2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2u(uint32_t lo, uint32_t hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2split(uint64_t v, float &lo, float &hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-// a * b + c on both halves, each rounded once (the products of fp16 values are exact in fp32)
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
+using qld::f2;
+using qld::f2split;
+using qld::f2u;
+using qld::ffma2;
 
 struct Bars {
   // full_a, peer_b and acc_empty are used in the even CTA only (both CTAs arrive on full_a and

@@ -76,33 +76,4 @@ ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r
 
 }  // namespace ql
 
-// ---- device helpers ----
-namespace qld {
-
-__device__ __forceinline__ float bf16_to_f32(uint32_t h16) { return __uint_as_float(h16 << 16); }
-
-__device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
-  uint16_t h;
-  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(f));
-  return h;
-}
-
-__device__ __forceinline__ float f16_to_f32(uint16_t h) {
-  float f;
-  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
-  return f;
-}
-
-// Programmatic dependent launch: wait until the preceding grid in the stream has completed and
-// its writes are visible (a no-op when the kernel was launched without overlap), and allow the
-// next grid to be scheduled (it still waits for this one to complete before touching its data).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-// acc + a * b with bf16 a, b and fp32 accumulate; the product is exact in fp32.
-__device__ __forceinline__ float fma_bf16(uint16_t a, uint16_t b, float acc) {
-  asm("fma.rn.f32.bf16 %0, %1, %2, %0;" : "+f"(acc) : "h"(a), "h"(b));
-  return acc;
-}
-
-}  // namespace qld
+#include "ql_device.cuh"
