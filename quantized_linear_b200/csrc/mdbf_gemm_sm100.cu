@@ -412,8 +412,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   sm100::cluster_sync();   // both CTAs' barriers initialised and tensor memory allocated
   sm100::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem_raw + (tmem_slot - raw));
-  // the factor operand is weights: its decoders start at once; A is read and C written only
-  // after the preceding kernel in the stream has completed
+  // the factor operand comes from weights (its decoders may start at once, except that l <= 4
+  // reads column pairs from the workspace); A is read and C written only after the preceding
+  // kernel in the stream has completed
   qld::pdl_trigger();
 
   if (warp == 0) {
@@ -507,6 +508,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int kbp = fac.seg / BK;                      // K blocks per path (F stage)
     const int l = fac.l, cols = fac.cols;
     const bool lvec = fac.l_vec2 != 0;
+    // l <= 4: the fp32 column pairs are workspace written by this call's first kernel, not weights,
+    // so the decoders wait for the preceding kernel (and with it for every earlier one) first
+    if constexpr (LK == 4) qld::pdl_wait();
     const size_t lblk = (size_t)BK * l;                // column-envelope elements per K block
     const int l8 = 8 * l;
     // this lane's envelope terms: 16c + 2t, +1 (k0) and 16c + 2t + 8, +1 (k1) of chunk c

@@ -102,6 +102,14 @@ def test_mixed_chain(ql):
     _compare(ql, chain, bf16(synth.activations(2, 2048, seed=944)))
 
 
+def test_batched_mdbf_chain(ql):
+    # prefill-sized batches: BenQ GEMM -> MDBF on the tensor cores (4 launches per call, l = 4 with its
+    # workspace column pairs; l = 6 on the warp-MMA decoders) -> BenQ GEMM
+    chain = [_benq_fn(ql, 1024, 512, 951, 300), _mdbf_fn(ql, 768, 1024, 300, 4, 2, 300, 952),
+             _mdbf_fn(ql, 512, 768, 256, 6, 2, 300, 953), _benq_fn(ql, 512, 512, 954, 300)]
+    _compare(ql, chain, bf16(synth.activations(300, 512, seed=955)), reps=4)
+
+
 def test_set_pdl_returns_previous(ql):
     prev = ql.ql_set_pdl(False)
     try:
