@@ -60,3 +60,24 @@ def linear(packed: np.ndarray, lut_bits: np.ndarray, x_bits: np.ndarray, K: int,
     W = dequant(packed, lut_bits, K).astype(np.float64)
     x = bf16_to_f32(x_bits).astype(np.float64).reshape(-1, K)
     return x @ W.T
+
+
+# ---------------------------------------------------------------------------- gated MLP (gate, up)
+# The card's model family computes its MLP as down(silu(gate(x)) * up(x)); the pages do not print
+# it, so this is the plain definition of that gate: silu(v) = v * sigmoid(v) = v / (1 + e^-v).
+
+def silu(v: np.ndarray) -> np.ndarray:
+    """v / (1 + exp(-v)) in fp64, written in a form that does not overflow for large |v|."""
+    v = np.asarray(v, dtype=np.float64)
+    e = np.exp(-np.abs(v))                      # in (0, 1]
+    sig = np.where(v >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+    return v * sig
+
+
+def mlp_gate_up(packed_g: np.ndarray, lut_g: np.ndarray, packed_u: np.ndarray, lut_u: np.ndarray,
+                x_bits: np.ndarray, K: int, rows: np.ndarray | None = None) -> np.ndarray:
+    """h = silu(x W_g^T) * (x W_u^T) in fp64, shape [B, N] (or [B, len(rows)]): both projections as
+    ``linear``, the gate and the product taken in fp64."""
+    g = linear(packed_g, lut_g, x_bits, K, rows)
+    u = linear(packed_u, lut_u, x_bits, K, rows)
+    return silu(g) * u

@@ -102,3 +102,51 @@ def test_linear_row_subset_matches_full():
     full = ob.linear(w.codes, w.lut, x, 128)
     rows = np.array([0, 5, 63, 17])
     assert np.array_equal(ob.linear(w.codes, w.lut, x, 128, rows=rows), full[:, rows])
+
+
+# ---------------------------------------------------------------- gated MLP (gate, up) of the oracle
+
+def test_silu_fixed_points_and_identities():
+    # silu(0) = 0; silu(v) - silu(-v) = v (sigmoid(v) + sigmoid(-v) = 1); sigmoid(ln 3) = 3/4
+    v = np.array([-30.0, -4.5, -1.0, -1e-3, 0.0, 1e-3, 0.7, 3.0, 40.0, 700.0])
+    s = ob.silu(v)
+    assert s[4] == 0.0
+    assert np.allclose(s - ob.silu(-v), v, rtol=1e-15, atol=1e-15)
+    assert abs(ob.silu(np.log(3.0)) - 0.75 * np.log(3.0)) < 1e-15
+    # for large v the gate passes v through; for very negative v it vanishes from below
+    assert ob.silu(700.0) == 700.0 and -1e-250 < ob.silu(-700.0) < 0.0
+    # minimum of silu: v* solves 1 + v(1 - sigmoid(v)) = 0, v* ~ -1.2784645, silu(v*) ~ -0.2784645
+    grid = np.linspace(-3, 0, 300001)
+    assert abs(ob.silu(grid).min() - (-0.27846454276)) < 1e-9
+
+
+def test_mlp_gate_up_exact_rational_brute_force():
+    # tiny layer: h[b, n] = silu(sum_k Wg x) * sum_k Wu x with the sums in exact rationals and the
+    # gate from the math library on the exact sum
+    import math
+    K, N = 8, 3
+    wg = synth.benq_weights(N, K, seed=41)
+    wu = synth.benq_weights(N, K, seed=42)
+    x = synth.activations(2, K, seed=43)
+    h = ob.mlp_gate_up(wg.codes, wg.lut, wu.codes, wu.lut, x, K)
+    codes_g = ob.unpack_codes(wg.codes, K)
+    codes_u = ob.unpack_codes(wu.codes, K)
+    for b in range(2):
+        for n in range(N):
+            g = sum(Fraction(float(_f32_of_bf16(wg.lut[n, codes_g[n, k]]))) * Fraction(float(_f32_of_bf16(x[b, k])))
+                    for k in range(K))
+            u = sum(Fraction(float(_f32_of_bf16(wu.lut[n, codes_u[n, k]]))) * Fraction(float(_f32_of_bf16(x[b, k])))
+                    for k in range(K))
+            gf = float(g)
+            ref = gf / (1.0 + math.exp(-gf)) * float(u)
+            assert abs(h[b, n] - ref) <= 1e-15 * max(1.0, abs(ref))
+
+
+def test_mlp_gate_up_row_subset_matches_full():
+    K, N = 64, 40
+    wg = synth.benq_weights(N, K, seed=51)
+    wu = synth.benq_weights(N, K, seed=52)
+    x = synth.activations(3, K, seed=53)
+    full = ob.mlp_gate_up(wg.codes, wg.lut, wu.codes, wu.lut, x, K)
+    rows = np.array([0, 7, 39])
+    assert np.array_equal(ob.mlp_gate_up(wg.codes, wg.lut, wu.codes, wu.lut, x, K, rows=rows), full[:, rows])

@@ -61,6 +61,15 @@ def _factors_swapped_qu_qv(path, n, m, r):
     return F, G
 
 
+def _silu_sign_flipped(v):
+    v = np.asarray(v, dtype=np.float64)
+    return v / (1.0 + np.exp(np.clip(v, -700, 700)))     # v * sigmoid(-v)
+
+
+def _mlp_gate_and_up_swapped(pg, lg, pu, lu, x, K, rows=None):
+    return ob.silu(ob.linear(pu, lu, x, K, rows)) * ob.linear(pg, lg, x, K, rows)
+
+
 def _b_eff_without_2r(n, m, r, P, l, scale_bits=16):
     from fractions import Fraction
     return Fraction(P * (r * (n + m) + scale_bits * l * (n + m)), n * m)
@@ -78,6 +87,7 @@ MDBF_PINS = [
     lambda: tm.test_dequant_exact_rational_dyadic((3, 4, 2, 2, 1)),
     lambda: tm.test_dequant_exact_rational_dyadic((2, 5, 3, 2, 2)),
 ]
+MLP_PINS = [tb.test_silu_fixed_points_and_identities, tb.test_mlp_gate_up_exact_rational_brute_force]
 ACC_PINS = [ta.test_square_layer_rank_2000_is_one_bit, ta.test_mlp_layers_at_one_and_a_half_bits,
             ta.test_b_max_is_b_eff_at_full_rank,
             lambda: ta.test_stored_bits_of_generated_layer_equal_b_eff((64, 96, 40, 2, 1))]
@@ -92,6 +102,8 @@ MUTANTS = [
     ("mdbf: envelope columns misaligned", om, "envelope", _envelope_reversed_columns, MDBF_PINS),
     ("mdbf: Q_U and Q_V swapped", om, "factors", _factors_swapped_qu_qv, MDBF_PINS),
     ("accounting: b_eff without the 2r envelope term", acc, "mdbf_b_eff", _b_eff_without_2r, ACC_PINS),
+    ("mlp: gate uses sigmoid(-v)", ob, "silu", _silu_sign_flipped, MLP_PINS),
+    ("mlp: gate applied to the up projection", ob, "mlp_gate_up", _mlp_gate_and_up_swapped, MLP_PINS),
 ]
 
 
