@@ -108,6 +108,28 @@ QL_API ql_status benq_linear_ws(const uint8_t *codes, const uint16_t *lut, const
                                 ql_out_dtype y_dtype, int B, int N, int K, void *workspace, size_t ws_bytes,
                                 ql_stream_t stream);
 
+/*
+ * benq_mlp_gate_up -- the gated MLP of two BenQ projections of the same input,
+ *     h[b][n] = silu(g[b][n]) * u[b][n],  g = x W_g^T,  u = x W_u^T,  silu(v) = v / (1 + e^-v)
+ *   (the MLP of the card's model family; the gate itself is not printed on the pages).
+ *   W_g and W_u are N x K BenQ layers stored as for benq_linear (codes_g / lut_g, codes_u /
+ *   lut_u); x bf16 [B][K]; h [B][N] of h_dtype (bf16: round to nearest even of the fp32 value).
+ *   g and u are accumulated exactly as benq_linear computes them; the gate is taken in fp32
+ *   (library expf, IEEE division).  B == 1 with K % 1024 == 0 (K <= 20480) and N even runs as one
+ *   fused kernel that needs no workspace; other shapes run both projections (GEMV or tensor-core
+ *   GEMM) into the workspace and a gate kernel.
+ *   workspace  device, 256-byte aligned, ws_bytes >= benq_mlp_workspace_bytes(B, N, K); NULL with 0
+ *              when that is 0.  Owned by the caller, not shared with a concurrent call.
+ *   Errors: as benq_linear (alignment of every pointer 16 bytes, B > 16 needs K % 64 == 0 and
+ *   N % 256 == 0), QL_ERR_INVALID_ARG for a workspace smaller than required.
+ */
+QL_API ql_status benq_mlp_gate_up(const uint8_t *codes_g, const uint16_t *lut_g, const uint8_t *codes_u,
+                                  const uint16_t *lut_u, const uint16_t *x, void *h, ql_out_dtype h_dtype, int B,
+                                  int N, int K, void *workspace, size_t ws_bytes, ql_stream_t stream);
+
+/* Workspace bytes benq_mlp_gate_up needs for these sizes (0 when the fused batch-1 kernel runs). */
+QL_API size_t benq_mlp_workspace_bytes(int B, int N, int K);
+
 /* Workspace bytes benq_linear_ws uses for these sizes on the current device
  * (0 when B <= 16 or when no split applies).  Needs a CUDA device. */
 QL_API size_t benq_linear_workspace_bytes(int B, int N, int K);

@@ -36,6 +36,8 @@ _SIGNATURES = {
     "benq_linear": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "benq_linear_ws": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "benq_linear_workspace_bytes": (_sz, [_i, _i, _i]),
+    "benq_mlp_gate_up": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "benq_mlp_workspace_bytes": (_sz, [_i, _i, _i]),
     "benq_dequant_debug": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
     "benq_bits_per_weight": (_d, [_i]),
     "mdbf_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -69,7 +71,8 @@ def lib() -> ctypes.CDLL:
 def _c(name):
     return getattr(lib(), name)
 
-EXPORTS = ["benq_linear", "benq_linear_ws", "benq_linear_workspace_bytes", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
+EXPORTS = ["benq_linear", "benq_linear_ws", "benq_linear_workspace_bytes", "benq_mlp_gate_up",
+           "benq_mlp_workspace_bytes", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
            "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
            "mdbf_select_rank", "ql_last_error", "ql_check", "ql_set_pdl"]
 
@@ -145,6 +148,32 @@ def benq_linear(codes, lut, x, y, stream=None, workspace=None):
 def benq_linear_workspace_bytes(B: int, N: int, K: int) -> int:
     """Bytes of workspace the GEMM's split last wave uses for these sizes on the current device."""
     return int(_c("benq_linear_workspace_bytes")(B, N, K))
+
+
+def benq_mlp_gate_up(codes_g, lut_g, codes_u, lut_u, x, h, workspace=None, stream=None):
+    """h[B, N] = silu(x @ W_g^T) * (x @ W_u^T) for two BenQ layers of the same shape (codes and
+    tables as for benq_linear); h float32 or bf16 [B, N] (overwritten).  `workspace`: uint8 device
+    tensor of at least benq_mlp_workspace_bytes(B, N, K) bytes when that is non-zero."""
+    N = codes_g.shape[0]
+    B, K = x.shape
+    for c, l, what in ((codes_g, lut_g, "gate"), (codes_u, lut_u, "up")):
+        _want(c, torch.uint8, f"{what} codes")
+        if tuple(c.shape) != (N, 3 * K // 4):
+            raise ValueError(f"{what} codes must be [N, 3K/4]")
+        if l.dtype not in (torch.bfloat16, torch.int16) or tuple(l.shape) != (N, 64) or not l.is_contiguous():
+            raise TypeError(f"{what} lut must be a contiguous bf16 [N, 64] tensor")
+    _want(x, torch.bfloat16, "x")
+    if tuple(h.shape) != (B, N) or not h.is_contiguous():
+        raise ValueError("h must be contiguous [B, N]")
+    ws, nbytes = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() * workspace.element_size())
+    _check(_c("benq_mlp_gate_up")(_ptr(codes_g), _ptr(lut_g), _ptr(codes_u), _ptr(lut_u), _ptr(x), _ptr(h), _ydt(h),
+                                  B, N, K, ws, nbytes, _stream(stream)))
+    return h
+
+
+def benq_mlp_workspace_bytes(B: int, N: int, K: int) -> int:
+    """Bytes of workspace benq_mlp_gate_up needs (0 when the fused batch-1 kernel runs)."""
+    return int(_c("benq_mlp_workspace_bytes")(B, N, K))
 
 
 def benq_dequant_debug(codes, lut, W, stream=None):

@@ -73,6 +73,30 @@ ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t 
   return benq_linear_ws(codes, lut, x, y, y_dtype, B, N, K, nullptr, 0, stream);
 }
 
+size_t benq_mlp_workspace_bytes(int B, int N, int K) { return ql::benq_mlp_workspace_size(B, N, K); }
+
+ql_status benq_mlp_gate_up(const uint8_t *codes_g, const uint16_t *lut_g, const uint8_t *codes_u, const uint16_t *lut_u,
+                           const uint16_t *x, void *h, ql_out_dtype h_dtype, int B, int N, int K, void *workspace,
+                           size_t ws_bytes, ql_stream_t stream) {
+  g_msg[0] = 0;
+  if (!codes_g || !lut_g || !codes_u || !lut_u || !x || !h) return fail(QL_ERR_INVALID_ARG, "benq_mlp_gate_up: null pointer");
+  if ((workspace == nullptr) != (ws_bytes == 0))
+    return fail(QL_ERR_INVALID_ARG, "benq_mlp_gate_up: workspace and ws_bytes must both be set or both be empty");
+  if (workspace && !aligned(workspace, 256)) return fail(QL_ERR_ALIGNMENT, "benq_mlp_gate_up: workspace must be 256-byte aligned");
+  if (B <= 0 || N <= 0 || K <= 0) return fail(QL_ERR_INVALID_ARG, "benq_mlp_gate_up: B, N, K must be positive");
+  if (K % 4) return fail(QL_ERR_INVALID_ARG, "benq_mlp_gate_up: K = %d is not a multiple of 4", K);
+  if (h_dtype != QL_OUT_F32 && h_dtype != QL_OUT_BF16) return fail(QL_ERR_INVALID_ARG, "benq_mlp_gate_up: bad h_dtype");
+  if (!aligned(codes_g, 16) || !aligned(lut_g, 16) || !aligned(codes_u, 16) || !aligned(lut_u, 16) || !aligned(x, 16) ||
+      !aligned(h, 16))
+    return fail(QL_ERR_ALIGNMENT, "benq_mlp_gate_up: codes, tables, x and h must be 16-byte aligned");
+  if (B > 16 && (K % 64 || N % 256))
+    return fail(QL_ERR_UNSUPPORTED, "benq_mlp_gate_up: batch %d > 16 needs K %% 64 == 0 and N %% 256 == 0", B);
+  const size_t need = ql::benq_mlp_workspace_size(B, N, K);
+  if (ws_bytes < need) return fail(QL_ERR_INVALID_ARG, "benq_mlp_gate_up: workspace %zu < %zu bytes", ws_bytes, need);
+  return ql::benq_mlp_launch(codes_g, lut_g, codes_u, lut_u, x, h, h_dtype, B, N, K, workspace, ws_bytes,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
 ql_status benq_linear_ws(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype y_dtype,
                          int B, int N, int K, void *workspace, size_t ws_bytes, ql_stream_t stream) {
   g_msg[0] = 0;

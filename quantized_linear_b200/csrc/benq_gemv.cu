@@ -342,8 +342,13 @@ struct IntC {
   static constexpr int value = V;
 };
 
+// MLP: the gated MLP h = silu(x W_g^T) * (x W_u^T) in the same launch: codes / lut are W_g and
+// codes2 / lut2 W_u; a tile is two output features, its first row group the two gate rows and its
+// second the two up rows, and the tile's sums leave as silu(g) * u.
+template <bool MLP>
 __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
     benq_gemv_b1_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ lut,
+                        const uint8_t *__restrict__ codes2, const uint16_t *__restrict__ lut2,
                         const uint16_t *__restrict__ x, void *__restrict__ y, int ydt, int N, int K) {
   __shared__ __align__(128) B1Tables tb;
   extern __shared__ __align__(16) float b1part[];  // [2][C][B1_T][32]
@@ -352,14 +357,26 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
   const int kc = warp * WARP_CODES + lane * LANE_CODES;
   const uint32_t rowbytes = 3u * K / 4;
   const uint8_t *cbase = codes + 3u * kc / 4;
-  const int ntile = N / B1_T;
+  const uint8_t *cbase2 = MLP ? codes2 + 3u * kc / 4 : nullptr;
+  constexpr int TOUT = MLP ? B1_T / 2 : B1_T;   // output features per tile
+  const int ntile = N / TOUT;
   int tile = blockIdx.x;
   if (tile >= ntile) return;
   // Before waiting on the preceding kernel, pull this CTA's first tile of weights (codes and
   // tables) toward L2; prefetches hold no registers, so the loop below is compiled as if they
   // were absent.  Activations are loaded first after the wait: loading them after the codes
   // made the compiler schedule the decode loop far worse.
-  {
+  if constexpr (MLP) {
+    const uint8_t *p = cbase + (size_t)tile * TOUT * rowbytes, *p2 = cbase2 + (size_t)tile * TOUT * rowbytes;
+#pragma unroll
+    for (int r = 0; r < TOUT; ++r) {
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (size_t)r * rowbytes));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p2 + (size_t)r * rowbytes));
+    }
+    if (threadIdx.x < B1_T)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"((threadIdx.x < TOUT ? lut : lut2) +
+                                                      ((size_t)tile * TOUT + (threadIdx.x % TOUT)) * 64));
+  } else {
     const uint8_t *p = cbase + (size_t)tile * B1_T * rowbytes;
 #pragma unroll
     for (int r = 0; r < B1_T; ++r) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (size_t)r * rowbytes));
@@ -379,8 +396,11 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
       xh[8 * t + 2 * e + 1] = u[e] >> 16;
     }
   }
-  auto load_rows = [&](int n0, uint32_t (&w)[B1_R][6]) {
-    const uint8_t *p = cbase + (size_t)n0 * rowbytes;
+  // rows of tile t's row group grp (grp = 0, 1): B1_R consecutive rows of W, or for MLP the
+  // tile's two gate rows (grp 0) and its two up rows (grp 1)
+  auto load_rows = [&](int t, int grp, uint32_t (&w)[B1_R][6]) {
+    const uint8_t *p = MLP ? (grp == 0 ? cbase : cbase2) + (size_t)t * TOUT * rowbytes
+                           : cbase + (size_t)(t * B1_T + grp * B1_R) * rowbytes;
 #pragma unroll
     for (int r = 0; r < B1_R; ++r) {
       const uint2 a = ldg_u2(p + r * rowbytes), c = ldg_u2(p + r * rowbytes + 8), d = ldg_u2(p + r * rowbytes + 16);
@@ -388,7 +408,12 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
     }
   };
   auto load_lut = [&](int t, uint4 &v) {
-    if (threadIdx.x < 8 * B1_T) v = ldg_u4(lut + ((size_t)t * B1_T + (threadIdx.x >> 3)) * 64 + (threadIdx.x & 7) * 8);
+    if (threadIdx.x < 8 * B1_T) {
+      const int i = threadIdx.x >> 3;   // table row of the tile
+      const uint16_t *src = MLP ? (i < TOUT ? lut : lut2) + ((size_t)t * TOUT + (i % TOUT)) * 64
+                                : lut + ((size_t)t * B1_T + i) * 64;
+      v = ldg_u4(src + (threadIdx.x & 7) * 8);
+    }
   };
   auto store_lut = [&](int buf, const uint4 &v) {
     if (threadIdx.x < 8 * B1_T) reinterpret_cast<uint4 *>(&tb.lut[buf][0][0])[threadIdx.x] = v;
@@ -409,7 +434,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
   load_lut(tile, lv);
   store_lut(0, lv);
   uint32_t ga[B1_R][6], gb[B1_R][6];
-  load_rows(tile * B1_T, ga);
+  load_rows(tile, 0, ga);
   __syncthreads();
   float *mypart = b1part + (warp * B1_T) * 32 + lane;
   constexpr int GP = B1_T / B1_R;  // even
@@ -423,13 +448,13 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
     float *pb = mypart + BUF * C * B1_T * 32;
 #pragma unroll
     for (int g = 0; g < GP; g += 2) {
-      load_rows(tile * B1_T + (g + 1) * B1_R, gb);
+      load_rows(tile, g + 1, gb);
 #pragma unroll
       for (int r = 0; r < B1_R; ++r) pb[(g * B1_R + r) * 32] = dot(ga[r], &tb.lut[BUF][g * B1_R + r][0]);
       if (g + 2 < GP)
-        load_rows(tile * B1_T + (g + 2) * B1_R, ga);
+        load_rows(tile, g + 2, ga);
       else if (has_next)
-        load_rows(nxt * B1_T, ga);
+        load_rows(nxt, 0, ga);
 #pragma unroll
       for (int r = 0; r < B1_R; ++r)
         pb[((g + 1) * B1_R + r) * 32] = dot(gb[r], &tb.lut[BUF][(g + 1) * B1_R + r][0]);
@@ -437,17 +462,40 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
     if (has_next) store_lut(BUF ^ 1, lv);
     __syncthreads();
     const float *pr = b1part + BUF * C * B1_T * 32;
-    for (int o = warp; o < B1_T; o += C) {
-      float s = 0.f;
-      for (int c = 0; c < C; ++c) s += pr[(c * B1_T + o) * 32 + lane];
+    if constexpr (MLP) {
+      for (int o = warp; o < TOUT; o += C) {
+        float g = 0.f, u = 0.f;
+        for (int c = 0; c < C; ++c) {
+          g += pr[(c * B1_T + o) * 32 + lane];
+          u += pr[(c * B1_T + TOUT + o) * 32 + lane];
+        }
 #pragma unroll
-      for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
-      if (lane == 0) {
-        const int n = tile * B1_T + o;
-        if (ydt == QL_OUT_F32)
-          static_cast<float *>(y)[n] = s;
-        else
-          static_cast<uint16_t *>(y)[n] = qld::f32_to_bf16_rn(s);
+        for (int d = 16; d > 0; d >>= 1) {
+          g += __shfl_xor_sync(0xffffffffu, g, d);
+          u += __shfl_xor_sync(0xffffffffu, u, d);
+        }
+        if (lane == 0) {
+          const float h = qld::silu_mul(g, u);
+          const int n = tile * TOUT + o;
+          if (ydt == QL_OUT_F32)
+            static_cast<float *>(y)[n] = h;
+          else
+            static_cast<uint16_t *>(y)[n] = qld::f32_to_bf16_rn(h);
+        }
+      }
+    } else {
+      for (int o = warp; o < B1_T; o += C) {
+        float s = 0.f;
+        for (int c = 0; c < C; ++c) s += pr[(c * B1_T + o) * 32 + lane];
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
+        if (lane == 0) {
+          const int n = tile * B1_T + o;
+          if (ydt == QL_OUT_F32)
+            static_cast<float *>(y)[n] = s;
+          else
+            static_cast<uint16_t *>(y)[n] = qld::f32_to_bf16_rn(s);
+        }
       }
     }
     tile = nxt;
@@ -459,18 +507,19 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
   }
 }
 
-ql_status launch_b1(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y, ql_out_dtype ydt, int N,
-                    int K, cudaStream_t s) {
+template <bool MLP>
+ql_status launch_b1(const uint8_t *codes, const uint16_t *lut, const uint8_t *codes2, const uint16_t *lut2,
+                    const uint16_t *x, void *y, ql_out_dtype ydt, int N, int K, cudaStream_t s) {
   const int C = K / WARP_CODES;
   const int threads = C * 32;
   const size_t smem = (size_t)2 * C * B1_T * 32 * sizeof(float);
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, benq_gemv_b1_kernel, threads, smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, benq_gemv_b1_kernel<MLP>, threads, smem) != cudaSuccess ||
       per_sm < 1)
     return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
-  const int grid = std::min(N / B1_T, per_sm * ql::sm_count());
-  ql::launch(benq_gemv_b1_kernel, grid, threads, smem, s, codes, lut, x, y, (int)ydt, N, K);
-  return ql::launch_status("benq_linear (batch-1 GEMV)");
+  const int grid = std::min(N / (MLP ? B1_T / 2 : B1_T), per_sm * ql::sm_count());
+  ql::launch(benq_gemv_b1_kernel<MLP>, grid, threads, smem, s, codes, lut, codes2, lut2, x, y, (int)ydt, N, K);
+  return ql::launch_status(MLP ? "benq_mlp_gate_up (batch-1 GEMV)" : "benq_linear (batch-1 GEMV)");
 }
 
 template <int R, int BMAX>
@@ -512,7 +561,8 @@ ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint
   const bool fast = (K % LANE_CODES == 0) && K <= MAX_WARPS * WARP_CODES && aligned(codes, 16) &&
                     aligned(x, 16);
   if (fast) {
-    if (B == 1 && K % WARP_CODES == 0 && N % B1_T == 0) return launch_b1(codes, lut, x, y, ydt, N, K, s);
+    if (B == 1 && K % WARP_CODES == 0 && N % B1_T == 0)
+      return launch_b1<false>(codes, lut, nullptr, nullptr, x, y, ydt, N, K, s);
     if (B == 1) return launch_fast<4, 1>(codes, lut, x, y, ydt, B, N, K, s);
     if (B <= 2) return launch_fast<2, 2>(codes, lut, x, y, ydt, B, N, K, s);
     if (B <= 4) return launch_fast<2, 4>(codes, lut, x, y, ydt, B, N, K, s);
@@ -524,6 +574,52 @@ ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint
   const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count() * 8);
   launch(benq_gemv_generic_kernel, grid, threads, 0, s, codes, lut, x, y, (int)ydt, B, N, K);
   return launch_status("benq_linear (generic GEMV)");
+}
+
+// ------------------------------------------------------------------------------- gated MLP
+// h = silu(g) * u elementwise from the two projections' fp32 outputs (batches the fused batch-1
+// kernel does not take).
+__global__ void __launch_bounds__(256) mlp_silu_mul_kernel(const float *__restrict__ g, const float *__restrict__ u,
+                                                           void *__restrict__ h, int ydt, size_t count) {
+  qld::pdl_trigger();
+  qld::pdl_wait();
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x) {
+    const float v = qld::silu_mul(g[i], u[i]);
+    if (ydt == QL_OUT_F32)
+      static_cast<float *>(h)[i] = v;
+    else
+      static_cast<uint16_t *>(h)[i] = qld::f32_to_bf16_rn(v);
+  }
+}
+
+bool mlp_fused_shape(int B, int N, int K) {
+  return B == 1 && K % WARP_CODES == 0 && K <= MAX_WARPS * WARP_CODES && N % (B1_T / 2) == 0;
+}
+
+size_t benq_mlp_workspace_size(int B, int N, int K) {
+  if (B <= 0 || N <= 0 || K <= 0) return 0;
+  if (mlp_fused_shape(B, N, K)) return 0;
+  return ((size_t)2 * B * N * sizeof(float) + 255) / 256 * 256;
+}
+
+ql_status benq_mlp_launch(const uint8_t *codes_g, const uint16_t *lut_g, const uint8_t *codes_u, const uint16_t *lut_u,
+                          const uint16_t *x, void *h, ql_out_dtype ydt, int B, int N, int K, void *ws, size_t ws_bytes,
+                          cudaStream_t s) {
+  // arguments validated by the caller (pointers 16-byte aligned, workspace large enough)
+  if (mlp_fused_shape(B, N, K)) return launch_b1<true>(codes_g, lut_g, codes_u, lut_u, x, h, ydt, N, K, s);
+  (void)ws_bytes;
+  float *g = static_cast<float *>(ws), *u = g + (size_t)B * N;
+  ql_status st = B <= 16 ? benq_gemv_launch(codes_g, lut_g, x, g, QL_OUT_F32, B, N, K, s)
+                         : benq_gemm_launch(codes_g, lut_g, x, g, QL_OUT_F32, B, N, K, nullptr, 0, s);
+  if (st != QL_OK) return st;
+  st = B <= 16 ? benq_gemv_launch(codes_u, lut_u, x, u, QL_OUT_F32, B, N, K, s)
+               : benq_gemm_launch(codes_u, lut_u, x, u, QL_OUT_F32, B, N, K, nullptr, 0, s);
+  if (st != QL_OK) return st;
+  const size_t count = (size_t)B * N;
+  const int grid = (int)std::min<size_t>((count + 255) / 256, (size_t)sm_count() * 8);
+  launch(mlp_silu_mul_kernel, grid, 256, 0, s, static_cast<const float *>(g), static_cast<const float *>(u), h,
+         (int)ydt, count);
+  return launch_status("benq_mlp_gate_up (silu * up)");
 }
 
 }  // namespace ql

@@ -33,6 +33,10 @@ __device__ __forceinline__ float fma_bf16(uint16_t a, uint16_t b, float acc) {
   return acc;
 }
 
+// silu(g) * u = g / (1 + e^-g) * u in fp32: the library expf and IEEE division (for g < -88 the
+// exponential overflows to +inf and the gate is -0, its limit).
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdiv_rn(g, 1.0f + expf(-g)) * u; }
+
 // Packed fp32 pairs, the operands of fma.rn.f32x2 (two fp32 FMAs in one instruction, each
 // rounded as a scalar fma.rn.f32 would be).
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {

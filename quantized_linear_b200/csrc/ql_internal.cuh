@@ -46,6 +46,10 @@ ql_status benq_dequant_launch(const uint8_t *codes, const uint16_t *lut, uint16_
 ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
                            ql_out_dtype ydt, int B, int N, int K, cudaStream_t s);
 size_t benq_gemm_workspace_size(int M, int N, int K);
+size_t benq_mlp_workspace_size(int B, int N, int K);
+ql_status benq_mlp_launch(const uint8_t *codes_g, const uint16_t *lut_g, const uint8_t *codes_u,
+                          const uint16_t *lut_u, const uint16_t *x, void *h, ql_out_dtype ydt, int B, int N,
+                          int K, void *ws, size_t ws_bytes, cudaStream_t s);
 ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
                            ql_out_dtype ydt, int M, int N, int K, void *ws, size_t ws_bytes, cudaStream_t s);
 ql_status benq_gemm_read_timeout(int *flag);  // reads and clears the GEMM's bounded-wait flag

@@ -97,6 +97,22 @@ def test_benq_argument_errors_are_caught_on_the_host(ql):
     assert g(A, A, A, 4, 10, None) == ql.QL_ERR_INVALID_ARG
 
 
+def test_mlp_argument_errors_are_caught_on_the_host(ql):
+    f = _raw(ql, "benq_mlp_gate_up")
+    A = 1 << 20    # never dereferenced: every call below fails validation first
+    assert ql.benq_mlp_workspace_bytes(1, 512, 1024) == 0                         # fused batch-1 kernel
+    need = ql.benq_mlp_workspace_bytes(4, 512, 1024)
+    assert need >= 2 * 4 * 512 * 4
+    assert f(A, A, None, A, A, A, 0, 1, 512, 1024, None, 0, None) == ql.QL_ERR_INVALID_ARG
+    assert f(A, A, A, A, A, A, 0, 1, 512, 1022, None, 0, None) == ql.QL_ERR_INVALID_ARG   # K % 4
+    assert f(A, A, A + 4, A, A, A, 0, 1, 512, 1024, None, 0, None) == ql.QL_ERR_ALIGNMENT
+    assert f(A, A, A, A, A, A, 5, 1, 512, 1024, None, 0, None) == ql.QL_ERR_INVALID_ARG     # h dtype
+    assert f(A, A, A, A, A, A, 0, 4, 512, 1024, A, need - 256, None) == ql.QL_ERR_INVALID_ARG  # workspace
+    assert f(A, A, A, A, A, A, 0, 4, 512, 1024, None, 0, None) == ql.QL_ERR_INVALID_ARG      # none given
+    assert f(A, A, A, A, A, A, 0, 4, 512, 1024, A + 64, need, None) == ql.QL_ERR_ALIGNMENT   # ws 256
+    assert f(A, A, A, A, A, A, 0, 32, 512, 1000, A, 1 << 30, None) == ql.QL_ERR_UNSUPPORTED  # GEMM K % 64
+
+
 def _fake_paths(ql, P, ldSA=16, ldSB=16, base=1 << 20):
     arr = (ql.MDBFPathC * P)()
     for p in range(P):
