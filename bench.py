@@ -12,8 +12,8 @@ decoder layer, hidden 5120, intermediate 17408):
   prefill  BenQ 6-bit prefill GEMM, 2048 tokens, same two shapes, bf16 output.
   mdbf     MDBF P=2, l=4 at 1.5 bits/weight (rank 2886), gate/up and down, batch 1.
   mdbf_prefill  the same MDBF layers at 2048 tokens (tensor-core path), bf16 output.
-  layer    the full decoder-layer linear set at batch 1: BenQ q/k/v/o/gate/up/down
-           plus MDBF gate/up/down.
+  layer    the full decoder-layer linear set at batch 1: BenQ q/k/v/o, gate and up in one
+           call with the SiLU gate (benq_mlp_gate_up), down, plus MDBF gate/up/down.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
 device synchronize on both sides, CUDA events on the launching stream, the max
@@ -153,6 +153,16 @@ class Workload:
             return dict(kind="benq", N=N, K=K, B=B, codes=[codes], lut=[lut], x=x, x_h=x_h, y=y, ws=ws,
                         wbytes=codes.numel() + lut.numel() * 2, label=label or f"benq_{K}x{N}_b{B}")
 
+        def benq_mlp_layer(N, K, seed, label):
+            # gate and up of the same input in one call, h = silu(gate) * up (bf16 out)
+            wg = synth.benq_weights(N, K, seed=seed)
+            wu = synth.benq_weights(N, K, seed=seed + 1)
+            x_h = synth.activations(1, K, seed=seed + 500)
+            cg, lg, cu, lu = dev(wg.codes), bits16(wg.lut), dev(wu.codes), bits16(wu.lut)
+            return dict(kind="benq_mlp", N=N, K=K, B=1, codes=[(cg, lg, cu, lu)], x=bf16(x_h), x_h=x_h,
+                        y=torch.empty(1, N, dtype=torch.bfloat16, device=cuda), ws=None,
+                        wbytes=2 * (cg.numel() + lg.numel() * 2), label=label)
+
         def mdbf_layer(n, m, B, seed, label=None, out_dtype=torch.float32):
             paths = synth.mdbf_paths(MLP_P, n, m, MLP_R, MLP_L, seed=seed)
             dps = [dict(S_A=dev(p.S_A), S_B=dev(p.S_B), A_amp=f16(p.A_amp), B_amp=f16(p.B_amp),
@@ -182,8 +192,7 @@ class Workload:
                       benq_layer(1024, HIDDEN, 1, 5002, label="benq_k"),
                       benq_layer(1024, HIDDEN, 1, 5003, label="benq_v"),
                       benq_layer(HIDDEN, HIDDEN, 1, 5004, label="benq_o"),
-                      benq_layer(INTER, HIDDEN, 1, 5005, label="benq_gate"),
-                      benq_layer(INTER, HIDDEN, 1, 5006, label="benq_up"),
+                      benq_mlp_layer(INTER, HIDDEN, 5005, "benq_gate_up_silu"),
                       benq_layer(HIDDEN, INTER, 1, 5007, label="benq_down"),
                       mdbf_layer(INTER, HIDDEN, 1, 5008, "mdbf_gate"),
                       mdbf_layer(INTER, HIDDEN, 1, 5009, "mdbf_up"),
@@ -199,6 +208,8 @@ class Workload:
                 if L["kind"] == "benq":
                     L["codes"].append(L["codes"][0].clone())
                     L["lut"].append(L["lut"][0].clone())
+                elif L["kind"] == "benq_mlp":
+                    L["codes"].append(tuple(t.clone() for t in L["codes"][0]))
                 else:
                     L["paths"].append([{k: v.clone() for k, v in d.items()} for d in L["paths"][0]])
         self.layers = layers
@@ -210,6 +221,8 @@ class Workload:
             ob = L["y"].element_size()
             if L["kind"] == "benq":
                 tot += benq_bytes(L["N"], L["K"], L["B"], ob)
+            elif L["kind"] == "benq_mlp":
+                tot += 2 * benq_bytes(L["N"], L["K"], L["B"], 0) - 2 * L["B"] * L["K"] + ob * L["B"] * L["N"]
             else:
                 tot += mdbf_bytes(L["n"], L["m"], MLP_R, MLP_L, MLP_P, L["B"], ob)
         return tot
@@ -224,13 +237,15 @@ class Workload:
         ql = self.ql
         if L["kind"] == "benq":
             ql.benq_linear(L["codes"][c], L["lut"][c], L["x"], L["y"], workspace=L["ws"])
+        elif L["kind"] == "benq_mlp":
+            ql.benq_mlp_gate_up(*L["codes"][c], L["x"], L["y"])
         else:
             ql.mdbf_linear(L["paths"][c], L["n"], L["m"], MLP_R, MLP_L, L["x"], L["y"], L["ws"])
 
     def launches_per_step(self):
         # BenQ: one kernel; MDBF: pack, G stage, F stage, or for batches past the decode kernels
         # envelope prep, activation prep and the two GEMMs
-        return sum(1 if L["kind"] == "benq" else (4 if MLP_L * L["B"] > 64 else 3) for L in self.layers)
+        return sum(1 if L["kind"] in ("benq", "benq_mlp") else (4 if MLP_L * L["B"] > 64 else 3) for L in self.layers)
 
 
 # the sources each kernel's DRAM-traffic figure depends on
@@ -317,6 +332,30 @@ def cpu_baseline(workload, budget_s=10.0):
     done, t_used, runs = time_samples(samples, budget_s)
     return {"value": done / t_used / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{runs} runs over {len(samples)} shapes ({samples[0][0]}; ...), {t_used:.1f} s of oracle time"}
+
+
+def cublas_reference(torch, layers, steps, warmup=3):
+    """Dense bf16 GEMMs of the prefill shapes through torch.matmul (cuBLAS) on random dense weights,
+    timed the same way (device events, weights larger than L2): a reference point for the tensor-core
+    rate at these shapes, not part of the measured path."""
+    mats = [(torch.randn(L["B"], L["K"], device="cuda").to(torch.bfloat16),
+             torch.randn(L["N"], L["K"], device="cuda").to(torch.bfloat16)) for L in layers]
+    out = [torch.empty(L["B"], L["N"], device="cuda", dtype=torch.bfloat16) for L in layers]
+    for _ in range(warmup):
+        for (a, w), o in zip(mats, out):
+            torch.matmul(a, w.t(), out=o)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(steps):
+        for (a, w), o in zip(mats, out):
+            torch.matmul(a, w.t(), out=o)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    flops = sum(2.0 * L["B"] * L["N"] * L["K"] for L in layers)
+    del mats, out
+    return {"us_per_step": 1e3 * ms, "tflops": flops / (ms / 1e3) / 1e12, "what": "torch.matmul bf16 (cuBLAS), same shapes, dense random weights"}
 
 
 def max_over_ranks(value, world):
@@ -530,6 +569,8 @@ def main():
                                  "by programmatic dependent launch; e2e uses eager calls"},
             "roofline": roof, "e2e": e2e, "gpu_launches": wl.launches_per_step() * args.steps,
             "clocks": clk.summary()}
+    if rank == 0 and world == 1 and args.workload == "prefill":
+        line["config"]["cublas_bf16_same_shape"] = cublas_reference(torch, wl.layers, min(args.steps, 20))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload)
     if rank == 0:
