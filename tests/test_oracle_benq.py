@@ -150,3 +150,75 @@ def test_mlp_gate_up_row_subset_matches_full():
     full = ob.mlp_gate_up(wg.codes, wg.lut, wu.codes, wu.lut, x, K)
     rows = np.array([0, 7, 39])
     assert np.array_equal(ob.mlp_gate_up(wg.codes, wg.lut, wu.codes, wu.lut, x, K, rows=rows), full[:, rows])
+
+
+# --------------------------------------------------------------------------- encoder of the oracle
+
+def _bits(v):
+    return synth.f32_to_bf16_bits(np.asarray(v, dtype=np.float32))
+
+
+def test_encode_hand_worked_row():
+    # one row, K = 8, dyadic values (exact at every step): max|w| = 3 -> shell width D = 3/32.
+    # |w| / D: 3 -> 32 (tier 31), 0.0625 -> 0.67 (0), 0.25 -> 2.67 (2), 0 (0), 1 -> 10.67 (10),
+    # 0.046875 -> 0.5 (0).  Levels: tier 31 = mean(3, 3) = 3, tier 2 = 0.25, tier 10 = 1, tier 0 =
+    # mean(0.0625, 0, 0.046875) = 0.036458.. rounded to bf16, empty tiers at their shell midpoints
+    # (t + 1/2) D, e.g. tier 5 = 0.515625 (exact in bf16).
+    w = np.array([[3.0, 0.0625, -0.25, 0.0, 1.0, 0.25, -3.0, 0.046875]], dtype=np.float32)
+    packed, lut = ob.encode(_bits(w))
+    L = ob.bf16_to_f32(lut[0, 32:]).astype(np.float64)
+    assert L[31] == 3.0 and L[2] == 0.25 and L[10] == 1.0 and L[5] == 0.515625 and L[1] == 0.140625
+    assert L[0] == float(ob.bf16_to_f32(_bits(np.float32(0.109375 / 3)).reshape(1))[0])
+    assert ob.unpack_codes(packed, 8)[0].tolist() == [63, 32, 29, 32, 42, 34, 0, 32]
+    assert np.array_equal(lut[0, :32], lut[0, 32:][::-1] | np.uint16(0x8000))
+
+
+def test_encode_table_is_sorted_and_codes_are_nearest():
+    rng = np.random.default_rng(3)
+    w = (rng.standard_normal((6, 256)) * rng.uniform(0.01, 0.05, size=(6, 1))).astype(np.float32)
+    wb = _bits(w)
+    for iters in (0, 3):
+        packed, lut = ob.encode(wb, iters)
+        vals = ob.bf16_to_f32(lut).astype(np.float64)
+        assert np.all(np.diff(vals, axis=1) >= 0)                         # ascending value
+        assert np.all(vals[:, :32] <= 0) and np.all(vals[:, 32:] >= 0)
+        W = ob.dequant(packed, lut, 256).astype(np.float64)
+        a = ob.bf16_to_f32(wb).astype(np.float64)
+        # every weight decodes to a level of its own sign at minimum distance among all 64 entries
+        # whose sign matches (zero counts as non-negative)
+        d = np.abs(a[:, :, None] - vals[:, None, :])
+        sign_ok = np.where(a[:, :, None] < 0, vals[:, None, :] <= 0, vals[:, None, :] >= 0)
+        dmin = np.where(sign_ok, d, np.inf).min(axis=2)
+        assert np.array_equal(np.abs(a - W), dmin)
+
+
+def test_lloyd_rounds_do_not_increase_the_error():
+    # each Lloyd round (nearest assignment, then member means) cannot increase the squared error of
+    # the magnitudes beyond what rounding the levels to bf16 adds back
+    rng = np.random.default_rng(4)
+    w = (rng.standard_normal((4, 2048)) * 0.02).astype(np.float32)
+    wb = _bits(w)
+    a = np.abs(ob.bf16_to_f32(wb).astype(np.float64))
+    errs = []
+    for iters in range(4):
+        packed, lut = ob.encode(wb, iters)
+        errs.append(((np.abs(ob.dequant(packed, lut, 2048).astype(np.float64)) - a) ** 2).sum())
+    assert errs[3] <= errs[0] * (1 + 1e-3)
+    assert min(errs[1:]) < errs[0]
+
+
+def test_encode_pack_matches_generator_packing():
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 64, size=(5, 64), dtype=np.uint8)
+    assert np.array_equal(ob.pack(codes), synth.pack_codes(codes))
+    assert np.array_equal(ob.unpack_codes(ob.pack(codes), 64), codes)
+
+
+def test_encode_all_zero_row_and_signed_zero():
+    wb = np.zeros((2, 8), dtype=np.uint16)
+    wb[1, 3] = 0x8000                      # -0.0 counts as non-negative
+    wb[1, 5] = _bits(np.array([0.5], dtype=np.float32))[0]
+    packed, lut = ob.encode(wb)
+    codes = ob.unpack_codes(packed, 8)
+    assert codes[0].tolist() == [32] * 8 and np.all(lut[0, 32:] == 0)
+    assert codes[1, 3] >= 32 and codes[1, 5] == 63

@@ -70,6 +70,22 @@ def _mlp_gate_and_up_swapped(pg, lg, pu, lu, x, K, rows=None):
     return ob.silu(ob.linear(pu, lu, x, K, rows)) * ob.linear(pg, lg, x, K, rows)
 
 
+_orig_shell_levels = ob._shell_levels
+
+
+def _shell_levels_midpoints(a, tier, prev):
+    return _orig_shell_levels(np.zeros_like(a), tier, prev) * 0 + prev      # ignores the members
+
+
+def _encode_width_over_31(w_bits, lloyd_iters=0):
+    w = ob.bf16_to_f32(np.asarray(w_bits, np.uint16)).astype(np.float64)
+    scaled = ob._bf16_rne_of_f32((w * (32.0 / 31.0)).astype(np.float32))     # tiers of max/31 shells
+    return _orig_encode(scaled, lloyd_iters)
+
+
+_orig_encode = ob.encode
+
+
 def _b_eff_without_2r(n, m, r, P, l, scale_bits=16):
     from fractions import Fraction
     return Fraction(P * (r * (n + m) + scale_bits * l * (n + m)), n * m)
@@ -88,6 +104,8 @@ MDBF_PINS = [
     lambda: tm.test_dequant_exact_rational_dyadic((2, 5, 3, 2, 2)),
 ]
 MLP_PINS = [tb.test_silu_fixed_points_and_identities, tb.test_mlp_gate_up_exact_rational_brute_force]
+ENC_PINS = [tb.test_encode_hand_worked_row, tb.test_encode_table_is_sorted_and_codes_are_nearest,
+            tb.test_lloyd_rounds_do_not_increase_the_error]
 ACC_PINS = [ta.test_square_layer_rank_2000_is_one_bit, ta.test_mlp_layers_at_one_and_a_half_bits,
             ta.test_b_max_is_b_eff_at_full_rank,
             lambda: ta.test_stored_bits_of_generated_layer_equal_b_eff((64, 96, 40, 2, 1))]
@@ -103,6 +121,8 @@ MUTANTS = [
     ("mdbf: Q_U and Q_V swapped", om, "factors", _factors_swapped_qu_qv, MDBF_PINS),
     ("accounting: b_eff without the 2r envelope term", acc, "mdbf_b_eff", _b_eff_without_2r, ACC_PINS),
     ("mlp: gate uses sigmoid(-v)", ob, "silu", _silu_sign_flipped, MLP_PINS),
+    ("encoder: levels are shell midpoints, not member means", ob, "_shell_levels", _shell_levels_midpoints, ENC_PINS),
+    ("encoder: shells of max/31", ob, "encode", _encode_width_over_31, ENC_PINS),
     ("mlp: gate applied to the up projection", ob, "mlp_gate_up", _mlp_gate_and_up_swapped, MLP_PINS),
 ]
 
