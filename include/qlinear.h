@@ -135,6 +135,27 @@ QL_API size_t benq_mlp_workspace_bytes(int B, int N, int K);
 QL_API size_t benq_linear_workspace_bytes(int B, int N, int K);
 
 /*
+ * benq_encode -- quantizes a bf16 matrix to BenQ storage ("Why equal-width shells": 32 magnitude
+ *   tiers as equal-width shells of each row's range, member-mean levels refined Lloyd-style,
+ *   nearest-level assignment; the uncalibrated path, no calibration data):
+ *     D = max_k |W[n][k]| / 32, tier t = min(floor(|w| / D), 31) in fp64;
+ *     level t = fp64 mean of the magnitudes in tier t (the shell midpoint (t + 1/2) D when empty),
+ *               rounded fp64 -> fp32 -> bf16 to nearest even;
+ *     lloyd_iters rounds of: assign every magnitude to its nearest level (lower tier on an exact
+ *               tie), level = fp64 mean of its members (unchanged without members), rounded the same;
+ *     code = 32 + t for w >= 0 (zero and -0 included), 31 - t for w < 0 with t the nearest level,
+ *     table [-L31 .. -L0, L0 .. L31]; an all-zero row gets zero levels and codes 32.
+ *   W      device bf16 [N][K] (read);  codes  device uint8 [N][3K/4] (written, the layout
+ *          benq_linear reads);  lut  device bf16 [N][64] (written).  K % 4 == 0, 0 <= lloyd_iters <= 1000.
+ *   W must be finite (NaN or Inf weights give unspecified codes).
+ *   The result is exact and independent of scheduling when every row's nonzero magnitudes span less
+ *   than a factor 2^30 (the tier sums are then exact in fp64); beyond that the tier means are
+ *   rounded in an unspecified order.
+ */
+QL_API ql_status benq_encode(const uint16_t *W, uint8_t *codes, uint16_t *lut, int N, int K, int lloyd_iters,
+                             ql_stream_t stream);
+
+/*
  * benq_dequant_debug -- W[n][k] = lut[n][code(n,k)] as bf16 bits, row-major
  *   [N][K].  Bit-exact by construction; meant for checking, not speed.
  *   Same codes / lut layout as benq_linear; K % 4 == 0.

@@ -38,6 +38,7 @@ _SIGNATURES = {
     "benq_linear_workspace_bytes": (_sz, [_i, _i, _i]),
     "benq_mlp_gate_up": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "benq_mlp_workspace_bytes": (_sz, [_i, _i, _i]),
+    "benq_encode": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "benq_dequant_debug": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
     "benq_bits_per_weight": (_d, [_i]),
     "mdbf_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -72,7 +73,7 @@ def _c(name):
     return getattr(lib(), name)
 
 EXPORTS = ["benq_linear", "benq_linear_ws", "benq_linear_workspace_bytes", "benq_mlp_gate_up",
-           "benq_mlp_workspace_bytes", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
+           "benq_mlp_workspace_bytes", "benq_encode", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
            "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
            "mdbf_select_rank", "ql_last_error", "ql_check", "ql_set_pdl"]
 
@@ -174,6 +175,21 @@ def benq_mlp_gate_up(codes_g, lut_g, codes_u, lut_u, x, h, workspace=None, strea
 def benq_mlp_workspace_bytes(B: int, N: int, K: int) -> int:
     """Bytes of workspace benq_mlp_gate_up needs (0 when the fused batch-1 kernel runs)."""
     return int(_c("benq_mlp_workspace_bytes")(B, N, K))
+
+
+def benq_encode(W, codes, lut, lloyd_iters=0, stream=None):
+    """Quantizes W (bf16 [N, K]) to BenQ storage: codes uint8 [N, 3K/4] and lut bf16 [N, 64], both
+    overwritten (equal-width shells, member-mean levels, lloyd_iters refinement rounds)."""
+    N, K = W.shape
+    if W.dtype not in (torch.bfloat16, torch.int16) or not W.is_contiguous():
+        raise TypeError("W must be a contiguous bf16 [N, K] tensor")
+    _want(codes, torch.uint8, "codes")
+    if tuple(codes.shape) != (N, 3 * K // 4):
+        raise ValueError("codes must be [N, 3K/4]")
+    if lut.dtype not in (torch.bfloat16, torch.int16) or tuple(lut.shape) != (N, 64) or not lut.is_contiguous():
+        raise TypeError("lut must be a contiguous bf16 [N, 64] tensor")
+    _check(_c("benq_encode")(_ptr(W), _ptr(codes), _ptr(lut), N, K, int(lloyd_iters), _stream(stream)))
+    return codes, lut
 
 
 def benq_dequant_debug(codes, lut, W, stream=None):

@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libqlinear.so")
 OBJDIR = os.path.join(HERE, "_build")
-SOURCES = ["abi.cu", "benq_gemv.cu", "benq_gemm_sm100.cu", "mdbf.cu", "mdbf_gemm_sm100.cu"]
+SOURCES = ["abi.cu", "benq_gemv.cu", "benq_gemm_sm100.cu", "mdbf.cu", "mdbf_gemm_sm100.cu", "benq_encode.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

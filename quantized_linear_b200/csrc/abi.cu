@@ -75,6 +75,16 @@ ql_status benq_linear(const uint8_t *codes, const uint16_t *lut, const uint16_t 
 
 size_t benq_mlp_workspace_bytes(int B, int N, int K) { return ql::benq_mlp_workspace_size(B, N, K); }
 
+ql_status benq_encode(const uint16_t *W, uint8_t *codes, uint16_t *lut, int N, int K, int lloyd_iters,
+                      ql_stream_t stream) {
+  g_msg[0] = 0;
+  if (!W || !codes || !lut) return fail(QL_ERR_INVALID_ARG, "benq_encode: null pointer");
+  if (N <= 0 || K <= 0 || K % 4) return fail(QL_ERR_INVALID_ARG, "benq_encode: N, K must be positive and K %% 4 == 0");
+  if (lloyd_iters < 0 || lloyd_iters > 1000) return fail(QL_ERR_INVALID_ARG, "benq_encode: lloyd_iters must be in [0, 1000]");
+  if (!aligned(W, 2) || !aligned(lut, 2)) return fail(QL_ERR_ALIGNMENT, "benq_encode: W and lut must be 2-byte aligned");
+  return ql::benq_encode_launch(W, codes, lut, N, K, lloyd_iters, reinterpret_cast<cudaStream_t>(stream));
+}
+
 ql_status benq_mlp_gate_up(const uint8_t *codes_g, const uint16_t *lut_g, const uint8_t *codes_u, const uint16_t *lut_u,
                            const uint16_t *x, void *h, ql_out_dtype h_dtype, int B, int N, int K, void *workspace,
                            size_t ws_bytes, ql_stream_t stream) {

@@ -47,6 +47,8 @@ ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint
                            ql_out_dtype ydt, int B, int N, int K, cudaStream_t s);
 size_t benq_gemm_workspace_size(int M, int N, int K);
 size_t benq_mlp_workspace_size(int B, int N, int K);
+ql_status benq_encode_launch(const uint16_t *W, uint8_t *codes, uint16_t *lut, int N, int K, int iters,
+                             cudaStream_t s);
 ql_status benq_mlp_launch(const uint8_t *codes_g, const uint16_t *lut_g, const uint8_t *codes_u,
                           const uint16_t *lut_u, const uint16_t *x, void *h, ql_out_dtype ydt, int B, int N,
                           int K, void *ws, size_t ws_bytes, cudaStream_t s);
