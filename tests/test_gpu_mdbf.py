@@ -85,6 +85,18 @@ def test_linear_square_one_bit_layer(ql, B):
     assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
 
 
+@pytest.mark.parametrize("P,B", [(1, 1), (1, 16), (2, 1), (2, 16)])
+def test_linear_rank_one_envelopes(ql, P, B):
+    # l = 1: the envelopes collapse to row and column scalings, W = sum_p diag(a) S_A diag(q_u q_v)
+    # S_B diag(b) ("DBF" at P = 1, "LittleBit" at P = 2): the square one-bit layer at rank 2000
+    n = m = 4096
+    r, l = 2000, 1
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=3200 + P)
+    x = synth.activations(B, m, seed=3300 + B)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+
+
 @pytest.mark.parametrize("n,m", [(17408, 5120), (5120, 17408)])
 def test_linear_mlp_shapes_sampled_rows(ql, n, m):
     # 27B-class gate/up and down at 1.5 bits/weight: P = 2, l = 4, r = 2886

@@ -39,6 +39,8 @@ def _scaled_envelope(bits: np.ndarray, scale: float) -> np.ndarray:
 # tile of tokens, the smallest layer the tensor cores take (n = m = r = 64) and the smallest
 # batch past the decode kernels' limit.
 SHAPES = [
+    (1024, 1024, 512, 1, 1, 300),     # l = 1, P = 1 (DBF) on the tensor cores
+    (512, 768, 256, 1, 2, 129),       # l = 1, P = 2 (LittleBit)
     (256, 512, 200, 4, 2, 40),
     (300, 200, 100, 3, 2, 70),
     (512, 1024, 256, 4, 1, 600),
