@@ -273,6 +273,12 @@ QL_API const char *ql_last_error(void);
  * QL_OK, QL_ERR_TIMEOUT, or QL_ERR_CUDA if the stream itself failed. */
 QL_API ql_status ql_check(ql_stream_t stream);
 
+/* Self-test of the bounded device-side waits (no counterpart in the pages): launches a CTA pair
+ * whose wait on a barrier that nothing arrives on gives up after ~10 ms, propagates the abort to the
+ * other CTA and raises the flag ql_check() reports; the kernel then returns normally, so the next
+ * ql_check(stream) returns QL_ERR_TIMEOUT and the context stays usable. */
+QL_API ql_status ql_selftest_timeout(ql_stream_t stream);
+
 /* Launch overlap (programmatic dependent launch).  No counterpart in the pages:
  * this is launch plumbing.  When enabled (the default; the environment variable
  * QL_PDL=0 at load time disables it), every kernel is launched so that it may

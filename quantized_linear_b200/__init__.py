@@ -51,6 +51,7 @@ _SIGNATURES = {
     "ql_last_error": (ctypes.c_char_p, []),
     "ql_check": (_i, [_vp]),
     "ql_set_pdl": (_i, [_i]),
+    "ql_selftest_timeout": (_i, [_vp]),
 }
 
 
@@ -75,7 +76,7 @@ def _c(name):
 EXPORTS = ["benq_linear", "benq_linear_ws", "benq_linear_workspace_bytes", "benq_mlp_gate_up",
            "benq_mlp_workspace_bytes", "benq_encode", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
            "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
-           "mdbf_select_rank", "ql_last_error", "ql_check", "ql_set_pdl"]
+           "mdbf_select_rank", "ql_last_error", "ql_check", "ql_set_pdl", "ql_selftest_timeout"]
 
 
 class QLinearError(RuntimeError):
@@ -275,6 +276,11 @@ def mdbf_select_rank(n, m, P, l, scale_bits, target_bits):
 def ql_check(stream=None):
     """Waits for the stream and raises QLinearError(QL_ERR_TIMEOUT) if a bounded device wait ran out."""
     _check(_c("ql_check")(_stream(stream)))
+
+
+def ql_selftest_timeout(stream=None):
+    """Launches the bounded-wait self-test: the next ql_check() on the stream raises QL_ERR_TIMEOUT."""
+    _check(_c("ql_selftest_timeout")(_stream(stream)))
 
 
 def ql_set_pdl(enable: bool) -> bool:

@@ -241,6 +241,11 @@ ql_status mdbf_select_rank(int n, int m, int P, int l, int scale_bits, double ta
   return QL_OK;
 }
 
+ql_status ql_selftest_timeout(ql_stream_t stream) {
+  g_msg[0] = 0;
+  return ql::selftest_timeout_launch(reinterpret_cast<cudaStream_t>(stream));
+}
+
 ql_status ql_check(ql_stream_t stream) {
   g_msg[0] = 0;
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

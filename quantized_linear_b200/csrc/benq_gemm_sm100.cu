@@ -428,6 +428,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
 }
 
+// Self-test of the bounded waits: a CTA pair where the even CTA waits on an mbarrier nothing ever
+// arrives on, with a short budget.  Its wait runs out, raises the abort flag in both CTAs (the odd
+// CTA's own wait on an equally idle barrier ends through that flag), and both record the timeout in
+// the flag ql_check() reads; the kernel then returns normally.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(32, 1) selftest_timeout_kernel(long long budget) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+  const uint32_t f = static_cast<uint32_t>(__cvta_generic_to_shared(&abort_flag));
+  const uint32_t rank = sm100::cluster_ctarank();
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(b, 1);
+    sts32(f, 0);
+    sm100::fence_barrier_init();
+  }
+  sm100::cluster_sync();
+  const Waiter wt{f, sm100::mapa_shared(f, rank ^ 1u), rank == 0 ? budget : WAIT_BUDGET};
+  bool ok = true;
+  if (threadIdx.x == 0) ok = wt.wait(b, 0, false);
+  if (!ok) atomicExch(&g_gemm_timeout, 2);
+  sm100::cluster_sync();   // neither CTA leaves while the other may still write its abort flag
+}
+
 // ---------------------------------------------------------------------------- host side
 // Opts the GEMM kernel into its dynamic shared memory (once per process).
 cudaError_t smem_attr() {
@@ -527,6 +550,11 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
   launch(benq_gemm_kernel, 2 * pairs, THREADS, SMEM_BYTES, s, mx, mc, my, tstore ? 1 : 0, lut, y, (int)ydt, M, N, K, part_ws, part_cnt,
          plan.full, plan.parts);
   return launch_status("benq_linear (tensor-core GEMM)");
+}
+
+ql_status selftest_timeout_launch(cudaStream_t s) {
+  launch(selftest_timeout_kernel, 2, 32, 0, s, 20000000LL);   // ~10 ms at 2 GHz
+  return launch_status("ql_selftest_timeout");
 }
 
 ql_status benq_gemm_read_timeout(int *flag) {

@@ -46,6 +46,7 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v
 // flag is set; a thread that runs out sets the flag in both CTAs so that the others stop at once.
 struct Waiter {
   uint32_t abort_local, abort_peer;
+  long long budget = WAIT_BUDGET;
   __device__ bool wait(uint32_t bar, uint32_t parity, bool cluster_scope) const {
     auto probe = [&] {
       return cluster_scope ? sm100::mbar_try_wait_cluster(bar, parity) : sm100::mbar_try_wait(bar, parity);
@@ -54,7 +55,7 @@ struct Waiter {
     const long long t0 = clock64();
     while (!probe()) {
       if (ld_volatile_u32(abort_local) != 0) return false;
-      if (clock64() - t0 > WAIT_BUDGET) {
+      if (clock64() - t0 > budget) {
         sts32(abort_local, 1);
         st_cluster_u32(abort_peer, 1);
         return false;

@@ -54,7 +54,8 @@ ql_status benq_mlp_launch(const uint8_t *codes_g, const uint16_t *lut_g, const u
                           int K, void *ws, size_t ws_bytes, cudaStream_t s);
 ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
                            ql_out_dtype ydt, int M, int N, int K, void *ws, size_t ws_bytes, cudaStream_t s);
-ql_status benq_gemm_read_timeout(int *flag);  // reads and clears the GEMM's bounded-wait flag
+ql_status benq_gemm_read_timeout(int *flag);
+ql_status selftest_timeout_launch(cudaStream_t s);  // reads and clears the GEMM's bounded-wait flag
 
 size_t mdbf_workspace_size(int P, int n, int m, int r, int l, int B);
 ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r, int l,

@@ -117,3 +117,22 @@ def test_set_pdl_returns_previous(ql):
         assert ql.ql_set_pdl(True) is True
     finally:
         ql.ql_set_pdl(prev)
+
+
+def test_bounded_wait_runs_out_and_the_context_survives(ql):
+    # a wait on a barrier that nothing arrives on gives up (~10 ms), the flag reaches ql_check, the
+    # next check is clean, and the library keeps working on the same context
+    ql.ql_check()
+    ql.ql_selftest_timeout()
+    with pytest.raises(ql.QLinearError) as e:
+        ql.ql_check()
+    assert e.value.status == ql.QL_ERR_TIMEOUT
+    ql.ql_check()
+    codes, lut = _benq(256, 1024, 961)
+    x = bf16(synth.activations(1, 1024, seed=962))
+    y = torch.empty(1, 256, device="cuda")
+    ql.benq_linear(codes, lut, x, y)
+    ql.ql_check()
+    from oracle import benq as ob
+    ref = ob.linear(codes.cpu().numpy(), lut.cpu().numpy().view(np.uint16), x.cpu().view(torch.int16).numpy().view(np.uint16), 1024)
+    assert np.max(np.abs(y.cpu().numpy() - ref)) <= 2e-3 * np.max(np.abs(ref))
