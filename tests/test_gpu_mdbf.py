@@ -147,3 +147,16 @@ def test_linear_unaligned_sign_strides(ql, B):
     x = synth.activations(B, m, seed=5500 + B)
     y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
     assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+
+
+@pytest.mark.parametrize("n,m,r,l,P,B", [(1024, 8192, 512, 4, 1, 1), (900, 8000, 333, 2, 2, 1),
+                                         (700, 6000, 300, 3, 2, 2), (640, 6144, 200, 1, 1, 1)])
+def test_linear_long_sign_rows(ql, n, m, r, l, P, B):
+    # few 32-row blocks of S_B with long rows (m up to 8192, ragged in m and r): each G-stage
+    # warp runs many word groups through its shared-memory ring, with a partial last group
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=5600 + m + r)
+    x = synth.activations(B, m, seed=5700 + B)
+    y = _linear(ql, paths, n, m, r, l, x)
+    assert max_rel(y.cpu().numpy(), om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+    for _ in range(2):
+        assert torch.equal(_linear(ql, paths, n, m, r, l, x), y)
