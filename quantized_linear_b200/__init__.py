@@ -91,10 +91,19 @@ def _check(status: int):
 
 
 def _ptr(t):
+    """Device address of a tensor argument (None and plain integers pass through unchanged).
+
+    The library takes device pointers on the current device; a host tensor or one on another GPU
+    is refused here, before any launch could read it as a device address."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must be CUDA tensors (got one on the host)")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor arguments must be on the current device cuda:{torch.cuda.current_device()}, "
+                         f"got one on {t.device}")
     return t.data_ptr()
 
 

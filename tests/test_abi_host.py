@@ -10,6 +10,7 @@ import warnings
 from fractions import Fraction
 
 import numpy as np
+import torch
 import pytest
 
 from oracle import accounting as acc
@@ -147,3 +148,19 @@ def test_binding_fails_loudly_without_the_library(ql, monkeypatch, tmp_path):
     monkeypatch.setattr(ql, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         ql.benq_bits_per_weight(64)
+
+
+def test_binding_refuses_host_tensors(ql):
+    # the Python binding hands the library device addresses only: a host tensor is refused before
+    # any call into the library could launch a kernel on it
+    K, N = 8, 4
+    codes = torch.zeros(N, 3 * K // 4, dtype=torch.uint8)
+    lut = torch.zeros(N, 64, dtype=torch.bfloat16)
+    x = torch.zeros(1, K, dtype=torch.bfloat16)
+    y = torch.zeros(1, N)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        ql.benq_linear(codes, lut, x, y)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        ql.benq_mlp_gate_up(codes, lut, codes, lut, x, y)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        ql.mdbf_paths_c([{"S_A": codes, "S_B": codes, "A_amp": lut, "B_amp": lut, "Q_U": lut, "Q_V": lut}])
