@@ -55,6 +55,19 @@ def test_encode_edge_rows(ql):
         assert np.array_equal(lut, ol) and np.array_equal(codes, oc)
 
 
+def test_encode_exact_tie_row(ql):
+    # 0.75 lies exactly halfway between the levels of tiers 7 (empty, its midpoint 45/64) and 8
+    # (the mean 51/64 of 0.75, 0.8125, 0.828125) of a row with max 3: both sides take the lower
+    # tier; repeated 32 times over a longer row, with the sign flipped on every other copy
+    base = np.array([3.0, 0.75, 0.8125, 0.828125, 0.0, 0.0, 0.0, 0.0], dtype=np.float32)
+    row = np.tile(base, 32) * np.repeat(np.array([1.0, -1.0] * 16, np.float32), 8)
+    wb = synth.f32_to_bf16_bits(row.reshape(1, -1))
+    codes, lut = _encode(ql, wb, 0)
+    oc, ol = ob.encode(wb, 0)
+    assert np.array_equal(lut, ol) and np.array_equal(codes, oc)
+    assert ob.unpack_codes(codes, 256)[0, :8].tolist() == [63, 39, 40, 40, 32, 32, 32, 32]
+
+
 def test_encode_27b_shape_sampled_rows(ql):
     # a 17408 x 5120 matrix in one launch; rows are independent, so sampled rows are checked against
     # the oracle run on those rows alone

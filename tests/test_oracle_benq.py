@@ -173,6 +173,20 @@ def test_encode_hand_worked_row():
     assert np.array_equal(lut[0, :32], lut[0, 32:][::-1] | np.uint16(0x8000))
 
 
+def test_encode_exact_tie_takes_the_lower_level():
+    # max|w| = 3 -> D = 3/32.  Tier 8 = [0.75, 0.84375) holds 0.75, 0.8125 and 0.828125, so its level
+    # is their mean 51/64 = 0.796875; tier 7 is empty and sits at its midpoint 7.5 D = 45/64.  The
+    # magnitude 0.75 is 3/64 from both levels (every value here is exact in bf16 and fp64): an exact
+    # tie, which goes to the lower tier (code 32 + 7), not its own shell (32 + 8).  The other codes
+    # are 63 (tier 31), 40, 40 and 32 for the zeros (tier 0, level 0).
+    w = np.array([[3.0, 0.75, 0.8125, 0.828125, 0.0, 0.0, 0.0, 0.0]], dtype=np.float32)
+    packed, lut = ob.encode(_bits(w))
+    L = ob.bf16_to_f32(lut[0, 32:]).astype(np.float64)
+    assert L[8] == 0.796875 and L[7] == 0.703125 and L[0] == 0.0 and L[31] == 3.0
+    assert abs(0.75 - L[7]) == abs(0.75 - L[8])
+    assert ob.unpack_codes(packed, 8)[0].tolist() == [63, 39, 40, 40, 32, 32, 32, 32]
+
+
 def test_encode_table_is_sorted_and_codes_are_nearest():
     rng = np.random.default_rng(3)
     w = (rng.standard_normal((6, 256)) * rng.uniform(0.01, 0.05, size=(6, 1))).astype(np.float32)

@@ -86,6 +86,17 @@ def _encode_width_over_31(w_bits, lloyd_iters=0):
 _orig_encode = ob.encode
 
 
+def _encode_signs_swapped(w_bits, lloyd_iters=0):
+    packed, lut = _orig_encode(w_bits, lloyd_iters)          # 32 + t for w < 0, 31 - t for w >= 0
+    K = 4 * packed.shape[1] // 3
+    return ob.pack(63 - ob.unpack_codes(packed, K).astype(np.int64)), lut
+
+
+def _nearest_upper_on_tie(a, levels):
+    d = np.abs(a[:, None] - levels[None, :])
+    return levels.shape[0] - 1 - np.argmin(d[:, ::-1], axis=1)   # the last (upper) index of a tie
+
+
 def _b_eff_without_2r(n, m, r, P, l, scale_bits=16):
     from fractions import Fraction
     return Fraction(P * (r * (n + m) + scale_bits * l * (n + m)), n * m)
@@ -105,7 +116,7 @@ MDBF_PINS = [
 ]
 MLP_PINS = [tb.test_silu_fixed_points_and_identities, tb.test_mlp_gate_up_exact_rational_brute_force]
 ENC_PINS = [tb.test_encode_hand_worked_row, tb.test_encode_table_is_sorted_and_codes_are_nearest,
-            tb.test_lloyd_rounds_do_not_increase_the_error]
+            tb.test_lloyd_rounds_do_not_increase_the_error, tb.test_encode_exact_tie_takes_the_lower_level]
 ACC_PINS = [ta.test_square_layer_rank_2000_is_one_bit, ta.test_mlp_layers_at_one_and_a_half_bits,
             ta.test_b_max_is_b_eff_at_full_rank,
             lambda: ta.test_stored_bits_of_generated_layer_equal_b_eff((64, 96, 40, 2, 1))]
@@ -123,6 +134,8 @@ MUTANTS = [
     ("mlp: gate uses sigmoid(-v)", ob, "silu", _silu_sign_flipped, MLP_PINS),
     ("encoder: levels are shell midpoints, not member means", ob, "_shell_levels", _shell_levels_midpoints, ENC_PINS),
     ("encoder: shells of max/31", ob, "encode", _encode_width_over_31, ENC_PINS),
+    ("encoder: code signs swapped", ob, "encode", _encode_signs_swapped, ENC_PINS),
+    ("encoder: exact ties go to the upper level", ob, "_nearest", _nearest_upper_on_tie, ENC_PINS),
     ("mlp: gate applied to the up projection", ob, "mlp_gate_up", _mlp_gate_and_up_swapped, MLP_PINS),
 ]
 
