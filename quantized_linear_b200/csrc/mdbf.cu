@@ -326,6 +326,9 @@ __device__ __forceinline__ uint32_t lds32s(uint32_t a) {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -367,6 +370,22 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
     }
   };
   for (int grp = 0; grp < GR_STAGES - 1 && grp < ngroups; ++grp) issue_signs(grp);
+  // The epilogue's Q_V and Q_U rows (weights) travel to shared memory with the first copy group
+  // when both blocks start on 4-byte boundaries and hold whole 4-byte words; else the epilogue
+  // reads them from global memory.
+  const int rows_b = min(32, r - row0);
+  const uint16_t *const qv0 = ps.QV[p] + (size_t)row0 * l, *const qu0 = ps.QU[p] + (size_t)row0 * l;
+  const bool q_smem = ((reinterpret_cast<uintptr_t>(qv0) | reinterpret_cast<uintptr_t>(qu0)) & 3) == 0 &&
+                      (rows_b * l) % 2 == 0;
+  uint16_t *const qs = reinterpret_cast<uint16_t *>(Ws + 32 * V);   // [2][32 l]: Q_V rows, Q_U rows
+  if (q_smem) {
+    const uint32_t qsa = static_cast<uint32_t>(__cvta_generic_to_shared(qs));
+    const int words = rows_b * l / 2;
+    for (int e = threadIdx.x; e < 2 * words; e += blockDim.x) {
+      const int which = e / words, j = e - which * words;
+      cp_async4(qsa + 4 * (which * 16 * l + j), (which ? qu0 : qv0) + 2 * j);
+    }
+  }
   qld::pdl_trigger();
   qld::pdl_wait();
   for (int grp = 0; grp < GR_STAGES - 1; ++grp) {
@@ -433,7 +452,8 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
       continue;
     }
     const float *Dr = D + rr * (8 * NB);
-    const uint16_t *qv = ps.QV[p] + (int64_t)k * l, *qu = ps.QU[p] + (int64_t)k * l;
+    const uint16_t *qv = q_smem ? qs + rr * l : ps.QV[p] + (int64_t)k * l;
+    const uint16_t *qu = q_smem ? qs + 32 * l + rr * l : ps.QU[p] + (int64_t)k * l;
     float t = 0.f;
     for (int i = 0; i < l; ++i) t = fmaf(qld::f16_to_f32(qv[i]), Dr[b * l + i] + Dr[V + b * l + i], t);
     for (int i = 0; i < l; ++i) wo[i] = qld::f16_to_f32(qu[i]) * t;
@@ -504,9 +524,10 @@ constexpr long long FT_WAIT_BUDGET = 4000000000LL;   // clock cycles (~2 s)
 
 
 struct FTileLayout {
-  uint32_t sign_bytes, frag_bytes, stage_bytes, nstage, off_bars, off_d, off_y, total;
+  uint32_t sign_bytes, frag_bytes, stage_bytes, nstage, off_bars, off_d, off_y, off_a, a_stride, total;
 };
-__host__ __device__ inline FTileLayout ftile_layout(size_t ld_max, int r, int NB, int B, int nstage, int KG,
+constexpr uint32_t FT_A_STAGE_MAX = 16 * 1024;   // shared-memory bytes for the CTA's A_amp rows
+__host__ __device__ inline FTileLayout ftile_layout(size_t ld_max, int r, int NB, int B, int P, int l, int nstage, int KG,
                                                     int tiles) {
   FTileLayout L;
   L.sign_bytes = (uint32_t)((16 * tiles * ld_max + 127) / 128 * 128);
@@ -516,7 +537,10 @@ __host__ __device__ inline FTileLayout ftile_layout(size_t ld_max, int r, int NB
   L.off_bars = L.nstage * L.stage_bytes;
   L.off_d = L.off_bars + 128;                                   // per-warp D scratch [16][8 NB] fp32
   L.off_y = L.off_d + KG * tiles * 16 * 8 * NB * 4;              // per-row-tile y accumulators [16][B] fp32
-  L.total = L.off_y + tiles * 16 * B * 4;
+  L.off_a = L.off_y + tiles * 16 * B * 4;                        // A_amp rows of every path [P][16 tiles][l]
+  const uint32_t a_bytes = (uint32_t)(P * 16 * tiles * l * 2 + 15) / 16 * 16;
+  L.a_stride = a_bytes <= FT_A_STAGE_MAX ? (uint32_t)(16 * tiles * l) : 0u;   // 0: read A_amp from global
+  L.total = L.off_a + (L.a_stride ? a_bytes : 0u);
   return L;
 }
 
@@ -562,6 +586,14 @@ __global__ void __launch_bounds__(NRG * 32 * KG)
     qld::pdl_wait();
     for (int p = 0; p < P && p < (int)L.nstage; ++p) issue(p, p, true);
   }
+  // the epilogue's A_amp rows (weights) to shared memory while the G stage is still running; warp
+  // 0 (whose thread 0 has already waited for the G stage above) takes no share
+  uint16_t *const a_sm = reinterpret_cast<uint16_t *>(fsm + L.off_a);
+  if (L.a_stride && threadIdx.x >= 32)
+    for (int e = threadIdx.x - 32; e < P * rows * l; e += blockDim.x - 32) {
+      const int pp = e / (rows * l), j = e - pp * rows * l;
+      a_sm[pp * L.a_stride + j] = ps.A[pp][(int64_t)row0 * l + j];
+    }
   qld::pdl_wait();
   __syncthreads();
 
@@ -637,7 +669,7 @@ __global__ void __launch_bounds__(NRG * 32 * KG)
           const int rr = e / B, b = e - rr * B, a = row0 + 16 * tile + rr;
           if (a >= n) continue;
           const float *Dr = dsc + rr * 8 * NB;
-          const uint16_t *am = ps.A[p] + (int64_t)a * l;
+          const uint16_t *am = L.a_stride ? a_sm + p * L.a_stride + (16 * tile + rr) * l : ps.A[p] + (int64_t)a * l;
           float sacc = yacc[e];
           for (int i = 0; i < l; ++i) sacc = fmaf(qld::f16_to_f32(am[i]), Dr[b * l + i] + Dr[V + b * l + i], sacc);
           yacc[e] = sacc;
@@ -764,7 +796,7 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
   // G stage through per-warp cp.async rings when sign rows are 16-byte aligned and the vectors
   // are narrow (decode batches); wider ones keep mdbf_g_mma_kernel
   constexpr bool g_ring = VEC16 && NB <= 2;
-  const size_t smg_t = (size_t)SP_WARPS * GR_STAGES * g_ring_stage_bytes<NB>() + smg;
+  const size_t smg_t = (size_t)SP_WARPS * GR_STAGES * g_ring_stage_bytes<NB>() + smg + (size_t)2 * 32 * l * 2;
   if constexpr (g_ring) {
     if (cudaFuncSetAttribute(mdbf_g_tile_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg_t) !=
         cudaSuccess)
@@ -794,8 +826,8 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     // 32-row ones still fit in one round; else 128-row CTAs
     const bool small = RT == 2 && (n + 127) / 128 < ql::sm_count() && (n + 31) / 32 <= 3 * ql::sm_count();
     const int tiles = small ? RT : FT_TILES;
-    FTileLayout L = ftile_layout(ld_max, r, NB, B, small ? 1 : 2, KG, tiles);
-    if (L.total > 227 * 1024) L = ftile_layout(ld_max, r, NB, B, 1, KG, tiles);
+    FTileLayout L = ftile_layout(ld_max, r, NB, B, P, l, small ? 1 : 2, KG, tiles);
+    if (L.total > 227 * 1024) L = ftile_layout(ld_max, r, NB, B, P, l, 1, KG, tiles);
     if (L.total <= 227 * 1024) {
       auto kt = small ? mdbf_f_tile_kernel<NB, KG, RT, 1> : mdbf_f_tile_kernel<NB, KG, RT, FT_TILES / RT>;
       if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total) != cudaSuccess)
