@@ -4,6 +4,7 @@ Every rank must receive the slowest rank's time (the bench's max over ranks), an
 value must count every rank's bytes against that time (weak scaling).  The reference arm prints
 on rank 0 only.
 """
+import json
 import os
 import socket
 
@@ -60,3 +61,21 @@ def test_reference_arm_prints_on_rank_zero_only(capsys):
         workload, steps, warmup, gpus = "decode", 1, 0, 2
     bench.run_reference(A, rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_carries_the_contract_keys(capsys):
+    # rank 0 prints one JSON line: the oracle timed on the host cores, with the keys the bench
+    # contract asks of the reference arm
+    class A:
+        workload, steps, warmup, gpus = "decode", 1, 0, 1
+    bench.run_reference(A, rank=0, world=1)
+    lines = [s for s in capsys.readouterr().out.splitlines() if s.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["vs_baseline"] is None
+    assert (d["n_gpus"], d["steps"], d["warmup"]) == (1, 1, 0) and d["ms_per_step"] > 0
+    assert d["config"]["workload"] == "decode" and d["data"] == "synthetic"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
