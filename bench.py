@@ -1,26 +1,39 @@
 """Benchmark of the weight-only quantized linear layers on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload decode|prefill|mdbf|mdbf_prefill|layer]
-                    [--impl ours|reference]
+                    [--workload all|small|decode|prefill|mdbf_square|layer|mdbf|mdbf_prefill]
+                    [--impl ours|reference] [--no-cpu-baseline]
 
-Prints one JSON line.  Workloads (synthetic, seeded; shapes of a 27B-class
-decoder layer, hidden 5120, intermediate 17408):
+Prints one JSON line.  The default workload, ``all``, times every configuration of the
+benchmark suite in one run; the line's headline (``value``, ``roofline``, ``e2e``) is the
+27B-class BenQ decode GEMV and ``workloads`` holds one record per configuration:
 
-  decode   BenQ 6-bit decode GEMV at batch 1: gate/up 5120->17408 and down
-           17408->5120 (one step = one pass of each).  Default.
-  prefill  BenQ 6-bit prefill GEMM, 2048 tokens, same two shapes, bf16 output.
-  mdbf     MDBF P=2, l=4 at 1.5 bits/weight (rank 2886), gate/up and down, batch 1.
-  mdbf_prefill  the same MDBF layers at 2048 tokens (tensor-core path), bf16 output.
-  layer    the full decoder-layer linear set at batch 1: BenQ q/k/v/o, gate and up in one
-           call with the SiLU gate (benq_mlp_gate_up), down, plus MDBF gate/up/down.
+  cfg0_benq_256x512   BenQ 6-bit 256 out x 512 in at batch 1 and 8 (launch-latency bound).
+  cfg1_decode_27b     BenQ decode GEMV at batch 1: gate/up 5120->17408 and down 17408->5120.
+  cfg2_prefill_m2048  BenQ prefill GEMM, 2048 tokens, the same two shapes, bf16 output.
+  cfg3_mdbf_4096      MDBF n = m = 4096, P = 1, l = 2, rank 2000 (1.0 bit/weight), batch 1 and 16.
+  cfg4_layer_27b      the decoder-layer linear set at batch 1 (q/o 5120->5120, k/v 5120->1024,
+                      gate/up 5120->17408, down 17408->5120): BenQ on all seven; BenQ with gate and
+                      up fused with the SiLU gate; MDBF (P = 2, l = 4, 1.5 bits/weight, rank 2886) on
+                      gate/up/down; and BenQ attention with the MDBF MLP.  Each as a CUDA graph and
+                      as separate launches.
+  next1_mdbf_prefill  the MDBF MLP projections at 2048 tokens (tensor-core path), bf16 output.
 
-Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
-device synchronize on both sides, CUDA events on the launching stream, the max
-over ranks.  Weights rotate over enough device copies that every step reads
-more than the 126 MB L2 before a copy is reused.  With N > 1 each rank runs an
-independent replica of the workload (the layer has no data-path exchange), so
-scaling is weak.
+The other workload names run one of these alone (``mdbf`` is the MDBF MLP of cfg4).
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier and a device synchronize
+on both sides, CUDA events on the launching stream, the max over ranks.  Workloads whose weights
+exceed the L2 rotate over enough device copies that every step reads more than twice the 126 MB
+L2 before a copy is reused; the small ones (cfg0, cfg3) write a 256 MiB buffer between steps and
+time each step alone.  With N > 1 each rank runs an independent replica (the layer has no
+data-path exchange), so scaling is weak.
+
+Inputs: seeded and synthetic.  BenQ weights follow the generator recipe (per-row sigma ~
+U(0.01, 0.03), w ~ N(0, sigma), 32 equal-width shells, member-mean levels, nearest-level codes)
+with the draws made on the device by torch and the shells, levels and codes made by the
+library's own encoder (``benq_encode``, bit-exact to the oracle's); MDBF weights and all
+activations come from ``synth``.  The CPU baselines time the oracle on bounded samples made by
+``synth``.
 """
 from __future__ import annotations
 
@@ -29,7 +42,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -41,8 +53,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "quantized-linear GB/s & TFLOP/s vs B200 roofline; decode us per layer"
 L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 256 * 1024 * 1024
 HIDDEN, INTER = 5120, 17408
-MLP_R, MLP_L, MLP_P = 2886, 4, 2
+MLP_R, MLP_L, MLP_P = 2886, 4, 2         # MDBF at 1.5 bits/weight on the 27B MLP shapes
+SQ_N, SQ_R, SQ_L, SQ_P = 4096, 2000, 2, 1  # MDBF square layer, rank 2000 (1.0 bit/weight)
+DECODE_VLIM = 64                          # the MDBF decode kernels take l * B <= 64
+SM_COUNT, FP32_LANES = 148, 128            # B200: SMs, fp32 lanes per SM
 
 
 def _peaks():
@@ -52,13 +68,26 @@ def _peaks():
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
                 "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
-                "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+                "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
 
+
+def alu_peak_tadds(peaks):
+    """Signed fp32 adds per second of the whole part, in T/s: every SM's 128 fp32 lanes retire one
+    add per clock at the maximum SM clock (148 x 128 x 1965 MHz = 37.2 T/s)."""
+    return SM_COUNT * FP32_LANES * peaks["sm_max_mhz"] * 1e6 / 1e12
+
+
+# ---------------------------------------------------------------------------------- algorithmic work
 
 def benq_bytes(N, K, B, out_bytes=4):
     """Algorithmic bytes of one BenQ call: packed codes, tables, activations, output."""
     return 0.75 * N * K + 128 * N + 2 * B * K + out_bytes * B * N
+
+
+def benq_weight_bytes(N, K):
+    return 0.75 * N * K + 128 * N
 
 
 def mdbf_flops(n, m, r, P, B):
@@ -67,11 +96,177 @@ def mdbf_flops(n, m, r, P, B):
     return 2.0 * B * P * r * (m + n)
 
 
+def mdbf_adds(n, m, r, l, P, B):
+    """Signed adds of one MDBF call evaluated through the factors: the G stage sums l * B vectors
+    over every sign of S_B (r x m), the F stage over every sign of S_A (n x r), per path."""
+    return float(P) * l * B * r * (n + m)
+
+
+def mdbf_weight_bytes(n, m, r, l, P):
+    """Both packed sign matrices and the four fp16 envelopes of every path."""
+    return P * (n * ((r + 7) // 8) + r * ((m + 7) // 8)) + P * 2 * l * (n + m + 2 * r)
+
+
 def mdbf_bytes(n, m, r, l, P, B, out_bytes=4):
     """Algorithmic bytes of one MDBF call: both sign matrices, four fp16 envelopes, x and y."""
-    signs = P * (n * ((r + 7) // 8) + r * ((m + 7) // 8))
-    env = P * 2 * l * (n + m + 2 * r)
-    return signs + env + 2 * B * m + out_bytes * B * n
+    return mdbf_weight_bytes(n, m, r, l, P) + 2 * B * m + out_bytes * B * n
+
+
+# ---------------------------------------------------------------------------------- layer specs
+
+def L_benq(N, K, B, seed, label, out="f32"):
+    return dict(kind="benq", N=N, K=K, B=B, seed=seed, label=label, out=out)
+
+
+def L_mlp(N, K, seed_g, seed_u, label):
+    """Gate and up projections of the same x in one call, h = silu(gate) * up (bf16 out)."""
+    return dict(kind="benq_mlp", N=N, K=K, B=1, seed=seed_g, seed_u=seed_u, label=label, out="bf16")
+
+
+def L_mdbf(P, n, m, r, l, B, seed, label, out="f32"):
+    return dict(kind="mdbf", P=P, n=n, m=m, r=r, l=l, B=B, seed=seed, label=label, out=out)
+
+
+# BenQ weight seeds: one matrix per shape and role, shared between the records that use it
+SEED_GATE, SEED_DOWN, SEED_UP = 1001, 1002, 1003
+
+
+def layer_set(attention, mlp):
+    """One decoder layer's linears at batch 1: the BenQ attention projections (q, k, v, o) when
+    `attention`, then the MLP: "benq" (gate, up, down), "benq_fused" (gate and up in one call
+    with the SiLU gate, then down) or "mdbf" (gate, up, down in MDBF)."""
+    out = []
+    if attention:
+        out += [L_benq(HIDDEN, HIDDEN, 1, 5001, "benq_q"), L_benq(1024, HIDDEN, 1, 5002, "benq_k"),
+                L_benq(1024, HIDDEN, 1, 5003, "benq_v"), L_benq(HIDDEN, HIDDEN, 1, 5004, "benq_o")]
+    if mlp == "benq":
+        out += [L_benq(INTER, HIDDEN, 1, SEED_GATE, "benq_gate"), L_benq(INTER, HIDDEN, 1, SEED_UP, "benq_up")]
+    elif mlp == "benq_fused":
+        out += [L_mlp(INTER, HIDDEN, SEED_GATE, SEED_UP, "benq_gate_up_silu")]
+    if mlp in ("benq", "benq_fused"):
+        out += [L_benq(HIDDEN, INTER, 1, SEED_DOWN, "benq_down")]
+    if mlp == "mdbf":
+        out += [L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 1, 5008, "mdbf_gate"),
+                L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 1, 5009, "mdbf_up"),
+                L_mdbf(MLP_P, HIDDEN, INTER, MLP_R, MLP_L, 1, 5010, "mdbf_down")]
+    return out
+
+
+DECODE = [L_benq(INTER, HIDDEN, 1, SEED_GATE, "benq_gate_up_5120x17408_b1"),
+          L_benq(HIDDEN, INTER, 1, SEED_DOWN, "benq_down_17408x5120_b1")]
+
+# workload -> [(record key, [(variant, layers, timing)])]; timing "rotate" (weights larger than
+# L2, rotating copies) or "flush" (an L2 flush before each timed step)
+RECORDS = {
+    "small": [("cfg0_benq_256x512", [
+        ("b1", [L_benq(256, 512, 1, 1, "benq_256x512_b1")], "flush"),
+        ("b8", [L_benq(256, 512, 8, 2, "benq_256x512_b8")], "flush")])],
+    "decode": [("cfg1_decode_27b", [("b1", DECODE, "rotate")])],
+    "prefill": [("cfg2_prefill_m2048", [
+        ("m2048", [L_benq(INTER, HIDDEN, 2048, SEED_GATE, "benq_gemm_5120x17408_m2048", "bf16"),
+                   L_benq(HIDDEN, INTER, 2048, SEED_DOWN, "benq_gemm_17408x5120_m2048", "bf16")], "rotate")])],
+    "mdbf_square": [("cfg3_mdbf_4096", [
+        ("b1", [L_mdbf(SQ_P, SQ_N, SQ_N, SQ_R, SQ_L, 1, 3001, "mdbf_4096_r2000_b1")], "flush"),
+        ("b16", [L_mdbf(SQ_P, SQ_N, SQ_N, SQ_R, SQ_L, 16, 3002, "mdbf_4096_r2000_b16")], "flush")])],
+    "layer": [("cfg4_layer_27b", [
+        ("benq_7_linears", layer_set(True, "benq"), "rotate"),
+        ("benq_fused_mlp", layer_set(True, "benq_fused"), "rotate"),
+        ("mdbf_mlp", layer_set(False, "mdbf"), "rotate"),
+        ("mixed_benq_attention_mdbf_mlp", layer_set(True, "mdbf"), "rotate")])],
+    "mdbf": [("cfg4_mdbf_mlp_27b", [("b1", layer_set(False, "mdbf"), "rotate")])],
+    "mdbf_prefill": [("next1_mdbf_prefill_m2048", [
+        ("m2048", [L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 2048, 6001, "mdbf_gemm_5120x17408_m2048", "bf16"),
+                   L_mdbf(MLP_P, HIDDEN, INTER, MLP_R, MLP_L, 2048, 6002, "mdbf_gemm_17408x5120_m2048", "bf16")],
+         "rotate")])],
+}
+ALL_ORDER = ["decode", "small", "prefill", "mdbf_square", "layer", "mdbf_prefill"]
+WORKLOADS = ["all"] + list(RECORDS)
+
+
+def headline_workload(workload):
+    return "decode" if workload == "all" else workload
+
+
+def out_bytes(L):
+    return 4 if L["out"] == "f32" else 2
+
+
+def layer_bytes(L):
+    if L["kind"] == "benq":
+        return benq_bytes(L["N"], L["K"], L["B"], out_bytes(L))
+    if L["kind"] == "benq_mlp":
+        return 2 * benq_weight_bytes(L["N"], L["K"]) + 2 * L["K"] + out_bytes(L) * L["N"]
+    return mdbf_bytes(L["n"], L["m"], L["r"], L["l"], L["P"], L["B"], out_bytes(L))
+
+
+def layer_weight_bytes(L):
+    if L["kind"] == "benq":
+        return benq_weight_bytes(L["N"], L["K"])
+    if L["kind"] == "benq_mlp":
+        return 2 * benq_weight_bytes(L["N"], L["K"])
+    return mdbf_weight_bytes(L["n"], L["m"], L["r"], L["l"], L["P"])
+
+
+def layer_flops(L):
+    if L["kind"] == "benq":
+        return 2.0 * L["B"] * L["N"] * L["K"]
+    if L["kind"] == "benq_mlp":
+        return 4.0 * L["N"] * L["K"]
+    return mdbf_flops(L["n"], L["m"], L["r"], L["P"], L["B"])
+
+
+def is_gemm(L):
+    if L["kind"] == "benq":
+        return L["B"] > 16
+    if L["kind"] == "mdbf":
+        return L["l"] * L["B"] > DECODE_VLIM
+    return False
+
+
+def layer_launches(L):
+    """Kernels of this library one call launches: BenQ one; MDBF decode pack z, G stage, F stage;
+    MDBF batched envelope prep, activation prep and the two GEMMs."""
+    if L["kind"] in ("benq", "benq_mlp"):
+        return 1
+    return 4 if is_gemm(L) else 3
+
+
+def layer_ideal_us(L, peaks):
+    """The layer's roofline time: HBM time of its algorithmic bytes, tensor time of its FLOPs for the
+    GEMMs, and for the MDBF decode the larger of its HBM and signed-add (ALU) times."""
+    t_hbm = layer_bytes(L) / (peaks["hbm_gbs"] * 1e3)
+    if is_gemm(L):
+        return max(t_hbm, layer_flops(L) / (peaks["bf16_tflops"] * 1e6))
+    if L["kind"] == "mdbf":
+        return max(t_hbm, mdbf_adds(L["n"], L["m"], L["r"], L["l"], L["P"], L["B"]) / (alu_peak_tadds(peaks) * 1e6))
+    return t_hbm
+
+
+def copies_for(layers, timing):
+    if timing == "flush":
+        return 1
+    per_step = sum(layer_weight_bytes(L) for L in layers)
+    return max(1, int(np.ceil(2 * L2_BYTES / per_step)) + 1)
+
+
+def l2_note(layers, timing):
+    if timing == "flush":
+        return f"L2 flushed: a {FLUSH_BYTES >> 20} MiB buffer is written before each timed step"
+    c = copies_for(layers, timing)
+    ws = c * sum(layer_weight_bytes(L) for L in layers)
+    return f"inputs larger than L2: {c} rotating weight copies, {ws / 2**20:.0f} MiB working set vs 126 MiB L2"
+
+
+def line_config(workload, world):
+    """The line's `config` (the same for both arms: it depends on the workload only)."""
+    wl = headline_workload(workload)
+    key, variants = RECORDS[wl][0]
+    name, layers, timing = variants[0]
+    cfg = {"workload": workload, "headline": f"{key}/{name}", "layers": [L["label"] for L in layers],
+           "l2": l2_note(layers, timing), "parallelism": f"replicas x{world}"}
+    if workload == "all":
+        cfg["records"] = [f"{k}/{v[0]}" for w in ALL_ORDER for k, vs in RECORDS[w] for v in vs]
+    return cfg
 
 
 # ---------------------------------------------------------------------------------------------- clocks
@@ -127,126 +322,208 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-# ---------------------------------------------------------------------------------------------- workloads
+# ---------------------------------------------------------------------------------------------- device inputs
 
-class Workload:
-    """Device-resident inputs for one workload plus the calls of one step."""
+class Inputs:
+    """Device-resident weights, activations and outputs of a list of layers, with rotating copies of
+    the weights.  BenQ weights of one (N, K, seed) are made once and shared between records."""
 
-    def __init__(self, name, ql, torch, copies_hint=None):
+    _benq_cache = {}
+
+    def __init__(self, layers, copies, ql, torch):
         import synth
-        from tests.qlhelpers import bf16, bits16, dev, f16
-        self.name, self.ql, self.torch = name, ql, torch
-        self.calls = []          # (label, fn(copy_index), algorithmic bytes, flops)
-        self.inputs_h = []       # host copies of step inputs (for the end-to-end number)
-        self.outputs = []
-        self.desc = {}
+        from tests.qlhelpers import bf16, dev, f16
+        self.layers, self.copies = [], copies
         cuda = torch.device("cuda")
-
-        def benq_layer(N, K, B, seed, out_dtype=torch.float32, label=None):
-            w = synth.benq_weights(N, K, seed=seed)
-            codes, lut = dev(w.codes), bits16(w.lut)
-            x_h = synth.activations(B, K, seed=seed + 500)
-            x = bf16(x_h)
-            y = torch.empty(B, N, dtype=out_dtype, device=cuda)
-            nws = ql.benq_linear_workspace_bytes(B, N, K)
-            ws = torch.empty(nws, dtype=torch.uint8, device=cuda) if nws else None
-            return dict(kind="benq", N=N, K=K, B=B, codes=[codes], lut=[lut], x=x, x_h=x_h, y=y, ws=ws,
-                        wbytes=codes.numel() + lut.numel() * 2, label=label or f"benq_{K}x{N}_b{B}")
-
-        def benq_mlp_layer(N, K, seed, label):
-            # gate and up of the same input in one call, h = silu(gate) * up (bf16 out)
-            wg = synth.benq_weights(N, K, seed=seed)
-            wu = synth.benq_weights(N, K, seed=seed + 1)
-            x_h = synth.activations(1, K, seed=seed + 500)
-            cg, lg, cu, lu = dev(wg.codes), bits16(wg.lut), dev(wu.codes), bits16(wu.lut)
-            return dict(kind="benq_mlp", N=N, K=K, B=1, codes=[(cg, lg, cu, lu)], x=bf16(x_h), x_h=x_h,
-                        y=torch.empty(1, N, dtype=torch.bfloat16, device=cuda), ws=None,
-                        wbytes=2 * (cg.numel() + lg.numel() * 2), label=label)
-
-        def mdbf_layer(n, m, B, seed, label=None, out_dtype=torch.float32):
-            paths = synth.mdbf_paths(MLP_P, n, m, MLP_R, MLP_L, seed=seed)
-            dps = [dict(S_A=dev(p.S_A), S_B=dev(p.S_B), A_amp=f16(p.A_amp), B_amp=f16(p.B_amp),
-                        Q_U=f16(p.Q_U), Q_V=f16(p.Q_V)) for p in paths]
-            x_h = synth.activations(B, m, seed=seed + 500)
-            ws = torch.empty(ql.mdbf_workspace_bytes(MLP_P, n, m, MLP_R, MLP_L, B), dtype=torch.uint8, device=cuda)
-            wbytes = sum(sum(t.numel() * t.element_size() for t in d.values()) for d in dps)
-            return dict(kind="mdbf", n=n, m=m, B=B, paths=[dps], x=bf16(x_h), x_h=x_h,
-                        y=torch.empty(B, n, dtype=out_dtype, device=cuda), ws=ws, wbytes=wbytes,
-                        label=label or f"mdbf_{m}x{n}_b{B}")
-
-        layers = []
-        if name == "decode":
-            layers = [benq_layer(INTER, HIDDEN, 1, 1001, label="benq_gate_up_5120x17408_b1"),
-                      benq_layer(HIDDEN, INTER, 1, 1002, label="benq_down_17408x5120_b1")]
-        elif name == "prefill":
-            layers = [benq_layer(INTER, HIDDEN, 2048, 2001, torch.bfloat16, "benq_gemm_5120x17408_m2048"),
-                      benq_layer(HIDDEN, INTER, 2048, 2002, torch.bfloat16, "benq_gemm_17408x5120_m2048")]
-        elif name == "mdbf":
-            layers = [mdbf_layer(INTER, HIDDEN, 1, 4001, "mdbf_gate_up_5120x17408_b1"),
-                      mdbf_layer(HIDDEN, INTER, 1, 4002, "mdbf_down_17408x5120_b1")]
-        elif name == "mdbf_prefill":
-            layers = [mdbf_layer(INTER, HIDDEN, 2048, 6001, "mdbf_gemm_5120x17408_m2048", torch.bfloat16),
-                      mdbf_layer(HIDDEN, INTER, 2048, 6002, "mdbf_gemm_17408x5120_m2048", torch.bfloat16)]
-        elif name == "layer":
-            layers = [benq_layer(HIDDEN, HIDDEN, 1, 5001, label="benq_q"),
-                      benq_layer(1024, HIDDEN, 1, 5002, label="benq_k"),
-                      benq_layer(1024, HIDDEN, 1, 5003, label="benq_v"),
-                      benq_layer(HIDDEN, HIDDEN, 1, 5004, label="benq_o"),
-                      benq_mlp_layer(INTER, HIDDEN, 5005, "benq_gate_up_silu"),
-                      benq_layer(HIDDEN, INTER, 1, 5007, label="benq_down"),
-                      mdbf_layer(INTER, HIDDEN, 1, 5008, "mdbf_gate"),
-                      mdbf_layer(INTER, HIDDEN, 1, 5009, "mdbf_up"),
-                      mdbf_layer(HIDDEN, INTER, 1, 5010, "mdbf_down")]
-        else:
-            raise SystemExit(f"unknown workload {name}")
-
-        # rotate weight copies so that a copy is reused only after > 2 x L2 of other reads
-        per_step = sum(L["wbytes"] for L in layers)
-        self.copies = copies_hint or max(1, int(np.ceil(2 * L2_BYTES / per_step)) + 1)
         for L in layers:
-            for _ in range(self.copies - 1):
-                if L["kind"] == "benq":
-                    L["codes"].append(L["codes"][0].clone())
-                    L["lut"].append(L["lut"][0].clone())
-                elif L["kind"] == "benq_mlp":
-                    L["codes"].append(tuple(t.clone() for t in L["codes"][0]))
-                else:
-                    L["paths"].append([{k: v.clone() for k, v in d.items()} for d in L["paths"][0]])
-        self.layers = layers
-        self.working_set = per_step * self.copies
-
-    def step_bytes(self):
-        tot = 0.0
-        for L in self.layers:
-            ob = L["y"].element_size()
+            L = dict(L)
+            x_h = synth.activations(L["B"], L["K"] if "K" in L else L["m"], seed=L["seed"] + 500)
+            L["x_h"], L["x"] = x_h, bf16(x_h)
+            odt = torch.float32 if L["out"] == "f32" else torch.bfloat16
+            nout = L["N"] if "N" in L else L["n"]
+            L["y"] = torch.empty(L["B"], nout, dtype=odt, device=cuda)
+            L["ws"] = None
             if L["kind"] == "benq":
-                tot += benq_bytes(L["N"], L["K"], L["B"], ob)
+                w0 = self.benq_device_weights(L["N"], L["K"], L["seed"], ql, torch)
+                nws = ql.benq_linear_workspace_bytes(L["B"], L["N"], L["K"])
+                L["ws"] = torch.empty(nws, dtype=torch.uint8, device=cuda) if nws else None
             elif L["kind"] == "benq_mlp":
-                tot += 2 * benq_bytes(L["N"], L["K"], L["B"], 0) - 2 * L["B"] * L["K"] + ob * L["B"] * L["N"]
+                w0 = (self.benq_device_weights(L["N"], L["K"], L["seed"], ql, torch)
+                      + self.benq_device_weights(L["N"], L["K"], L["seed_u"], ql, torch))
             else:
-                tot += mdbf_bytes(L["n"], L["m"], MLP_R, MLP_L, MLP_P, L["B"], ob)
-        return tot
+                paths = synth.mdbf_paths(L["P"], L["n"], L["m"], L["r"], L["l"], seed=L["seed"])
+                w0 = [dict(S_A=dev(p.S_A), S_B=dev(p.S_B), A_amp=f16(p.A_amp), B_amp=f16(p.B_amp),
+                           Q_U=f16(p.Q_U), Q_V=f16(p.Q_V)) for p in paths]
+                L["ws"] = torch.empty(ql.mdbf_workspace_bytes(L["P"], L["n"], L["m"], L["r"], L["l"], L["B"]),
+                                      dtype=torch.uint8, device=cuda)
+            L["w"] = [w0] + [self.clone(w0) for _ in range(copies - 1)]
+            self.layers.append(L)
 
-    def step_flops(self):
-        f = sum(2.0 * L["B"] * L["N"] * L["K"] for L in self.layers if L["kind"] == "benq")
-        if self.name == "mdbf_prefill":
-            f += sum(mdbf_flops(L["n"], L["m"], MLP_R, MLP_P, L["B"]) for L in self.layers if L["kind"] == "mdbf")
-        return f
+    @classmethod
+    def benq_device_weights(cls, N, K, seed, ql, torch):
+        key = (N, K, seed)
+        if key not in cls._benq_cache:
+            g = torch.Generator(device="cuda")
+            g.manual_seed(seed)
+            sigma = torch.rand(N, 1, generator=g, device="cuda") * 0.02 + 0.01
+            w = (torch.randn(N, K, generator=g, device="cuda") * sigma).to(torch.bfloat16)
+            codes = torch.empty(N, 3 * K // 4, dtype=torch.uint8, device="cuda")
+            lut = torch.empty(N, 64, dtype=torch.int16, device="cuda")
+            ql.benq_encode(w, codes, lut, lloyd_iters=0)
+            del w, sigma
+            cls._benq_cache[key] = (codes, lut)
+        return cls._benq_cache[key]
 
-    def run_layer(self, L, c):
-        ql = self.ql
+    @staticmethod
+    def clone(w):
+        if isinstance(w, tuple):
+            return tuple(t.clone() for t in w)
+        return [{k: v.clone() for k, v in d.items()} for d in w]
+
+    def run(self, ql, L, c):
+        w = L["w"][c]
         if L["kind"] == "benq":
-            ql.benq_linear(L["codes"][c], L["lut"][c], L["x"], L["y"], workspace=L["ws"])
+            ql.benq_linear(w[0], w[1], L["x"], L["y"], workspace=L["ws"])
         elif L["kind"] == "benq_mlp":
-            ql.benq_mlp_gate_up(*L["codes"][c], L["x"], L["y"])
+            ql.benq_mlp_gate_up(*w, L["x"], L["y"])
         else:
-            ql.mdbf_linear(L["paths"][c], L["n"], L["m"], MLP_R, MLP_L, L["x"], L["y"], L["ws"])
+            ql.mdbf_linear(w, L["n"], L["m"], L["r"], L["l"], L["x"], L["y"], L["ws"])
 
-    def launches_per_step(self):
-        # BenQ: one kernel; MDBF: pack, G stage, F stage, or for batches past the decode kernels
-        # envelope prep, activation prep and the two GEMMs
-        return sum(1 if L["kind"] in ("benq", "benq_mlp") else (4 if MLP_L * L["B"] > 64 else 3) for L in self.layers)
 
+# ---------------------------------------------------------------------------------------------- timing
+
+def max_over_ranks(value, world):
+    """The largest of the ranks' `value` (a device time in ms), every rank getting the result.
+    One rank returns its own value; otherwise an all-reduce on the process group (NCCL: a CUDA
+    tensor, gloo: a CPU one)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step, steps, ms, world):
+    """Whole-job GB/s: every rank processes bytes_per_step per step (weak scaling), timed by the
+    slowest rank's `ms` for `steps` steps."""
+    return world * bytes_per_step * steps / (ms / 1e3) / 1e9
+
+
+class Timer:
+    """Runs a record's steps (graph replays or eager calls) and times them on the launching stream."""
+
+    def __init__(self, ql, torch, world, warmup):
+        self.ql, self.torch, self.world, self.warmup = ql, torch, world, warmup
+        self.stream = torch.cuda.current_stream()
+        self._flush = None
+
+    def sync_all(self):
+        import torch.distributed as dist
+        if self.world > 1:
+            dist.barrier()
+        self.torch.cuda.synchronize()
+
+    def capture(self, inp, layers, copies):
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for c in copies:
+                for L in layers:
+                    inp.run(self.ql, L, c)
+        return g
+
+    def graphs(self, inp, layers):
+        n = inp.copies
+        return {"cycle": self.capture(inp, layers, range(n)), "one": [self.capture(inp, layers, [c]) for c in range(n)]}
+
+    def replay(self, gs, steps, n):
+        for _ in range(steps // n):
+            gs["cycle"].replay()
+        for c in range(steps % n):
+            gs["one"][c].replay()
+
+    def flush(self):
+        if self._flush is None:
+            self._flush = self.torch.empty(FLUSH_BYTES, dtype=self.torch.uint8, device="cuda")
+        self._flush.fill_(1)
+
+    def time_graph(self, inp, gs, steps, timing):
+        """Milliseconds for `steps` graph-replayed steps (max over ranks)."""
+        torch, n = self.torch, inp.copies
+        self.replay(gs, max(self.warmup, n), n)
+        if timing == "rotate":
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            self.sync_all()
+            a.record(self.stream)
+            self.replay(gs, steps, n)
+            b.record(self.stream)
+            self.sync_all()
+            return max_over_ranks(a.elapsed_time(b), self.world)
+        ev = []
+        self.sync_all()
+        for _ in range(steps):
+            self.flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+            gs["one"][0].replay()
+            b.record(self.stream)
+            ev.append((a, b))
+        self.sync_all()
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), self.world)
+
+    def time_eager(self, inp, layers, steps, timing):
+        """Milliseconds for `steps` steps of separate launches (no graph)."""
+        torch, n = self.torch, inp.copies
+        for i in range(self.warmup):
+            for L in layers:
+                inp.run(self.ql, L, i % n)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        self.sync_all()
+        if timing == "flush":
+            tot = 0.0
+            for i in range(steps):
+                self.flush()
+                a.record(self.stream)
+                for L in layers:
+                    inp.run(self.ql, L, 0)
+                b.record(self.stream)
+                b.synchronize()
+                tot += a.elapsed_time(b)
+            self.sync_all()
+            return max_over_ranks(tot, self.world)
+        a.record(self.stream)
+        for i in range(steps):
+            for L in layers:
+                inp.run(self.ql, L, i % n)
+        b.record(self.stream)
+        self.sync_all()
+        return max_over_ranks(a.elapsed_time(b), self.world)
+
+    def time_e2e(self, inp, layers, steps):
+        """The same steps through the public API with the inputs copied in from pinned host memory and
+        the results copied back each step (eager calls); returns (ms, h2d bytes, d2h bytes) per run."""
+        torch, n = self.torch, inp.copies
+        xs_h = [torch.from_numpy(np.ascontiguousarray(L["x_h"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+                for L in layers]
+        ys_h = [torch.empty(L["y"].shape, dtype=L["y"].dtype).pin_memory() for L in layers]
+        h2d = sum(t.numel() * t.element_size() for t in xs_h)
+        d2h = sum(t.numel() * t.element_size() for t in ys_h)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        self.sync_all()
+        a.record(self.stream)
+        for i in range(steps):
+            for L, xh, yh in zip(layers, xs_h, ys_h):
+                L["x"].copy_(xh, non_blocking=True)
+                inp.run(self.ql, L, i % n)
+                yh.copy_(L["y"], non_blocking=True)
+        b.record(self.stream)
+        self.sync_all()
+        return max_over_ranks(a.elapsed_time(b), self.world), h2d, d2h
+
+
+# ---------------------------------------------------------------------------------------------- records
 
 # the sources each kernel's DRAM-traffic figure depends on
 _KERNEL_SOURCES = {
@@ -279,141 +556,215 @@ def _traffic(kernel_key):
     return e.get("dram_bytes_per_launch")
 
 
-def oracle_samples(workload, rows=64, seed=0):
-    """A bounded sample of the workload for the oracle: per shape, `rows` output rows with their
-    inputs (generated once, outside any timing).  Returns [(label, run, algorithmic bytes)]."""
+def kernel_name(L):
+    if L["kind"] in ("benq", "benq_mlp"):
+        return "benq_gemm" if is_gemm(L) else "benq_gemv"
+    return "mdbf_gemm" if is_gemm(L) else "mdbf_linear"
+
+
+def roofline(layers, us, peaks):
+    """Roofline of one step of `layers` taking `us` microseconds.
+
+    Homogeneous steps report their own bound: GB/s against the measured copy bandwidth (BenQ
+    GEMV), TFLOP/s against the measured bf16 peak (the GEMMs), and for the MDBF decode kernels the
+    larger of the HBM and ALU (signed-add) times, with both fractions.  A step that mixes bounds
+    reports the sum of its layers' roofline times against the measured time."""
+    ideal = sum(layer_ideal_us(L, peaks) for L in layers)
+    byts = sum(layer_bytes(L) for L in layers)
+    kinds = {kernel_name(L) for L in layers}
+    kname = kinds.pop() if len(kinds) == 1 else "mixed"
+    hbm = {"bound": "hbm", "achieved": byts / us / 1e3, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+           "peak_source": peaks["source"] + " (STREAM copy)"}
+    if kname in ("benq_gemm", "mdbf_gemm"):
+        fl = sum(layer_flops(L) for L in layers)
+        r = {"bound": "tensor", "achieved": fl / us / 1e6, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+             "peak_source": peaks["source"] + " (burst)"}
+    elif kname == "mdbf_linear":
+        adds = sum(mdbf_adds(L["n"], L["m"], L["r"], L["l"], L["P"], L["B"]) for L in layers)
+        t_hbm = byts / (peaks["hbm_gbs"] * 1e3)
+        t_alu = adds / (alu_peak_tadds(peaks) * 1e6)
+        r = dict(hbm) if t_hbm >= t_alu else {
+            "bound": "alu", "achieved": adds / us / 1e6, "peak": alu_peak_tadds(peaks), "unit": "T add/s",
+            "peak_source": "derived: 148 SMs x 128 fp32 lanes x max SM clock, one add per lane per clock"}
+        r.update(hbm_us=t_hbm, alu_us=t_alu, hbm_frac=t_hbm / us, alu_frac=t_alu / us,
+                 hbm_achieved_gbs=byts / us / 1e3)
+    elif kname == "mixed":
+        r = {"bound": "mixed", "achieved": byts / us / 1e3, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "peak_source": peaks["source"] + " (STREAM copy); frac = sum of the layers' roofline times / time"}
+    else:
+        r = hbm
+    r.update(frac=(ideal / us) if kname in ("mixed", "mdbf_linear") else r["achieved"] / r["peak"],
+             ideal_us=ideal, kernel=kname, traffic=None if kname == "mixed" else _traffic(kname))
+    return r
+
+
+def measure_variant(timer, layers, timing, steps, peaks, eager=False):
+    inp = Inputs(layers, copies_for(layers, timing), timer.ql, timer.torch)
+    for L in inp.layers:   # first calls outside any capture (kernel attributes, tensor maps)
+        inp.run(timer.ql, L, 0)
+    timer.torch.cuda.synchronize()
+    gs = timer.graphs(inp, inp.layers)
+    ms = timer.time_graph(inp, gs, steps, timing)
+    us = 1e3 * ms / steps
+    byts = sum(layer_bytes(L) for L in layers)
+    rec = {"us": us, "layers": [L["label"] for L in layers], "algorithmic_bytes": byts,
+           "gbs": byts / us / 1e3, "launches_per_step": sum(layer_launches(L) for L in layers),
+           "roofline": roofline(layers, us, peaks), "l2": l2_note(layers, timing),
+           "launch": "CUDA graph, kernels chained by programmatic dependent launch"}
+    fl = sum(layer_flops(L) for L in layers)
+    if any(is_gemm(L) for L in layers):
+        rec["tflops"] = fl / us / 1e6
+    if eager:
+        ems = timer.time_eager(inp, inp.layers, steps, timing)
+        rec["us_separate_launches"] = 1e3 * ems / steps
+    ems, h2d, d2h = timer.time_e2e(inp, inp.layers, steps)
+    rec["e2e"] = {"value": byts * steps / (ems / 1e3) / 1e9, "unit": "GB/s", "us": 1e3 * ems / steps,
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del gs
+    return rec, inp
+
+
+# ---------------------------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(layers, rows=64, seed=0):
+    """A bounded sample of a step for the oracle: per layer, `rows` output rows (all of them when the
+    layer has fewer) with their inputs, and at most 16 token rows of a batch; generated once,
+    outside any timing.  Returns [(label, run, algorithmic bytes, flops)]."""
     import synth
     from oracle import benq as ob
     from oracle import mdbf as om
     rng = np.random.default_rng(seed)
-    shapes = {"decode": [("benq", INTER, HIDDEN, 1), ("benq", HIDDEN, INTER, 1)],
-              "prefill": [("benq", INTER, HIDDEN, 2048), ("benq", HIDDEN, INTER, 2048)],
-              "mdbf": [("mdbf", INTER, HIDDEN, 1), ("mdbf", HIDDEN, INTER, 1)],
-              "mdbf_prefill": [("mdbf", INTER, HIDDEN, 2048), ("mdbf", HIDDEN, INTER, 2048)],
-              "layer": [("benq", INTER, HIDDEN, 1), ("mdbf", INTER, HIDDEN, 1)]}[workload]
     out = []
-    for kind, N, K, B in shapes:
-        if kind == "benq":
-            bb = min(B, 16)   # prefill: a 16-row slice of the batch (the oracle's cost is linear in it)
-            w = synth.benq_weights(rows, K, seed=int(rng.integers(1 << 30)))
+    for L in layers:
+        bb = min(L["B"], 16)
+        if L["kind"] in ("benq", "benq_mlp"):
+            N, K = L["N"], L["K"]
+            rr = min(rows, N)
+            w = synth.benq_weights(rr, K, seed=int(rng.integers(1 << 30)))
             x = synth.activations(bb, K, seed=1)
-            out.append((f"benq {rows} rows x K={K}, B={bb}", lambda w=w, x=x, K=K: ob.linear(w.codes, w.lut, x, K),
-                        benq_bytes(rows, K, bb)))
+            if L["kind"] == "benq":
+                run = (lambda w=w, x=x, K=K: ob.linear(w.codes, w.lut, x, K))
+                out.append((f"benq {rr} of {N} rows x K={K}, B={bb}", run, benq_bytes(rr, K, bb), 2.0 * bb * rr * K))
+            else:
+                wu = synth.benq_weights(rr, K, seed=int(rng.integers(1 << 30)))
+                run = (lambda w=w, wu=wu, x=x, K=K: ob.mlp_gate_up(w.codes, w.lut, wu.codes, wu.lut, x, K))
+                out.append((f"benq gate/up {rr} of {N} rows x K={K}", run,
+                            2 * benq_weight_bytes(rr, K) + 2 * K + 4 * rr, 4.0 * rr * K))
         else:
-            bb = min(B, 16)   # prefill: a 16-row slice of the batch (the oracle's cost is linear in it)
-            paths = synth.mdbf_paths(MLP_P, N, K, MLP_R, MLP_L, seed=7)
-            x = synth.activations(bb, K, seed=1)
-            sel = np.sort(rng.choice(N, rows, replace=False))
-            out.append((f"mdbf {rows} of {N} rows, m={K}, B={bb}",
-                        lambda paths=paths, x=x, N=N, K=K, sel=sel: om.linear_factored(paths, N, K, MLP_R, x, rows=sel),
-                        mdbf_bytes(rows, K, MLP_R, MLP_L, MLP_P, bb)))
+            n, m, r, l, P = L["n"], L["m"], L["r"], L["l"], L["P"]
+            rr = min(rows, n)
+            paths = synth.mdbf_paths(P, n, m, r, l, seed=7)
+            x = synth.activations(bb, m, seed=1)
+            sel = np.sort(rng.choice(n, rr, replace=False))
+            run = (lambda paths=paths, x=x, n=n, m=m, r=r, sel=sel: om.linear_factored(paths, n, m, r, x, rows=sel))
+            out.append((f"mdbf {rr} of {n} rows, m={m}, r={r}, l={l}, P={P}, B={bb}", run,
+                        mdbf_bytes(rr, m, r, l, P, bb), mdbf_flops(rr, m, r, P, bb)))
     return out
 
 
-def time_samples(samples, budget_s):
-    """Runs the samples round-robin (single-threaded BLAS) until `budget_s` of oracle time; returns
-    (bytes, seconds, runs)."""
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_sample(sample, budget_s, threads):
+    """Runs the sample (every entry once per pass) until `budget_s` seconds of oracle time have been
+    spent, with BLAS limited to `threads` threads (None: the library's default, all cores).  Returns
+    (bytes, flops, seconds, passes, threads used)."""
     from threadpoolctl import threadpool_limits
-    done, t_used, runs = 0.0, 0.0, 0
-    with threadpool_limits(limits=1):
-        while t_used < budget_s or runs == 0:
-            for _, run, nbytes in samples:
+    done_b, done_f, t_used, passes = 0.0, 0.0, 0.0, 0
+    with threadpool_limits(limits=threads):
+        used = _blas_threads()
+        while t_used < budget_s or passes == 0:
+            for _, run, nb, nf in sample:
                 t0 = time.perf_counter()
                 run()
                 t_used += time.perf_counter() - t0
-                done += nbytes
-                runs += 1
-    return done, t_used, runs
+                done_b += nb
+                done_f += nf
+            passes += 1
+    return done_b, done_f, t_used, passes, used
 
 
-def cpu_baseline(workload, budget_s=10.0):
-    """The oracle as it stands, on a bounded sample of the workload's rows, single-threaded BLAS."""
-    samples = oracle_samples(workload)
-    done, t_used, runs = time_samples(samples, budget_s)
-    return {"value": done / t_used / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{runs} runs over {len(samples)} shapes ({samples[0][0]}; ...), {t_used:.1f} s of oracle time"}
+def cpu_baseline(layers, budget_s, unit):
+    """The oracle as it stands on a bounded sample of the step: one thread, and all cores."""
+    sample = oracle_sample(layers)
+    res = {"kind": "oracle", "unit": unit, "os_cpu_count": os.cpu_count(),
+           "affinity_cores": len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else None}
+    for tag, threads in (("", 1), ("all_cores_", None)):
+        b, f, t, passes, used = time_sample(sample, budget_s, threads)
+        v = b / t / 1e9 if unit == "GB/s" else f / t / 1e12
+        res[tag + "value"] = v
+        res[tag + "cores"] = used
+        res[tag + "sample"] = (f"{passes} passes over {len(sample)} layers ({sample[0][0]}; ...), "
+                               f"{t:.1f} s of oracle time")
+    return res
 
 
-def cublas_reference(torch, layers, steps, warmup=3):
-    """Dense bf16 GEMMs of the prefill shapes through torch.matmul (cuBLAS) on random dense weights,
-    timed the same way (device events, weights larger than L2): a reference point for the tensor-core
-    rate at these shapes, not part of the measured path."""
-    mats = [(torch.randn(L["B"], L["K"], device="cuda").to(torch.bfloat16),
-             torch.randn(L["N"], L["K"], device="cuda").to(torch.bfloat16)) for L in layers]
-    out = [torch.empty(L["B"], L["N"], device="cuda", dtype=torch.bfloat16) for L in layers]
-    for _ in range(warmup):
-        for (a, w), o in zip(mats, out):
-            torch.matmul(a, w.t(), out=o)
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    s.record()
-    for _ in range(steps):
-        for (a, w), o in zip(mats, out):
-            torch.matmul(a, w.t(), out=o)
-    e.record()
-    torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / steps
-    flops = sum(2.0 * L["B"] * L["N"] * L["K"] for L in layers)
-    del mats, out
-    return {"us_per_step": 1e3 * ms, "tflops": flops / (ms / 1e3) / 1e12, "what": "torch.matmul bf16 (cuBLAS), same shapes, dense random weights"}
-
-
-def max_over_ranks(value, world):
-    """The largest of the ranks' `value` (a device time in ms), every rank getting the result.
-    One rank returns its own value; otherwise an all-reduce on the process group (NCCL: a CUDA
-    tensor, gloo: a CPU one)."""
-    if world <= 1:
-        return value
-    import torch
-    import torch.distributed as dist
-    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
-    t = torch.tensor([value], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def job_throughput(bytes_per_step, steps, ms, world):
-    """Whole-job GB/s: every rank processes bytes_per_step per step (weak scaling), timed by the
-    slowest rank's `ms` for `steps` steps."""
-    return world * bytes_per_step * steps / (ms / 1e3) / 1e9
-
+# ---------------------------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
-    """The oracle as the reference arm: each step is one pass of the oracle over the sample
-    (generated once), so the run's length is bounded by the sample, not by the weights' size."""
+    """The oracle as the reference arm: each step is one pass of the oracle over the headline's sample
+    (generated once), so the run's length is bounded by the sample, not by the weights' size; the
+    other records of the workload get a bounded single-threaded timing each."""
     if rank != 0:
         return
-    samples = oracle_samples(args.workload)
+    from threadpoolctl import threadpool_limits
+    wl = headline_workload(args.workload)
+    key, variants = RECORDS[wl][0]
+    sample = oracle_sample(variants[0][1])
+    unit = "TFLOP/s" if any(is_gemm(L) for L in variants[0][1]) else "GB/s"
     for _ in range(args.warmup):
-        time_samples(samples, 0.0)
-    done, t_used = 0.0, 0.0
+        time_sample(sample, 0.0, 1)
+    done_b, done_f, t_used = 0.0, 0.0, 0.0
     t0 = time.perf_counter()   # the timed steps only
-    for _ in range(args.steps):
-        d, t, _ = time_samples(samples, 0.0)
-        done += d
-        t_used += t
+    with threadpool_limits(limits=1):
+        for _ in range(args.steps):
+            b, f, t, _, _ = time_sample(sample, 0.0, 1)
+            done_b += b
+            done_f += f
+            t_used += t
     t_steps = time.perf_counter() - t0
-    v = done / t_used / 1e9
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+    v = done_b / t_used / 1e9 if unit == "GB/s" else done_f / t_used / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * t_steps / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "oracle": "CPU numpy, fp32 W materialised, fp64 contraction"},
-            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"one pass per step over {len(samples)} shapes: "
-                                       + "; ".join(lbl for lbl, _, _ in samples)},
-            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "config": line_config(args.workload, world),
+            "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle",
+                             "os_cpu_count": os.cpu_count(),
+                             "sample": f"one pass per step over {len(sample)} layers: "
+                                       + "; ".join(s[0] for s in sample)},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if args.workload == "all":
+        recs = {}
+        for w in ALL_ORDER:
+            for k, vs in RECORDS[w]:
+                for name, layers, _ in vs:
+                    u = "TFLOP/s" if any(is_gemm(L) for L in layers) else "GB/s"
+                    s = oracle_sample(layers)
+                    b, f, t, passes, _ = time_sample(s, getattr(args, "ref_budget", 1.0), 1)
+                    recs[f"{k}/{name}"] = {"value": b / t / 1e9 if u == "GB/s" else f / t / 1e12, "unit": u,
+                                           "cores": 1, "sample": f"{passes} passes over {len(s)} layers"}
+        line["workloads"] = recs
     print(json.dumps(line), flush=True)
 
+
+# ---------------------------------------------------------------------------------------------- main
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "mdbf", "mdbf_prefill", "layer"])
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="all", choices=WORKLOADS)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=1.5, help="seconds of oracle time per record and thread setting")
+    ap.add_argument("--ref-budget", type=float, default=1.0, help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -433,150 +784,68 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
-    wl = Workload(args.workload, ql, torch)
-    stream = torch.cuda.current_stream()
-    ncopy = wl.copies
-
-    def step(i):
-        c = i % ncopy
-        for L in wl.layers:
-            wl.run_layer(L, c)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-
-    # A decode step is launch-bound at this size, so it is replayed as a CUDA graph: one graph
-    # per rotating weight copy, kernels chained by programmatic dependent launch.
-    dom = [L for L in wl.layers if L["kind"] == ("benq" if args.workload in ("decode", "prefill", "layer") else "mdbf")]
-
-    def capture(layers, copies):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, capture_error_mode="thread_local"):
-            for c in copies:
-                for L in layers:
-                    wl.run_layer(L, c)
-        return g
-
-    # one graph per rotation cycle (steps on copies 0 .. ncopy-1), as a model graph holds many
-    # layers; single-step graphs cover a remainder so that exactly `steps` steps run
-    def graph_set(layers):
-        return {"cycle": capture(layers, range(ncopy)), "one": [capture(layers, [c]) for c in range(ncopy)]}
-
-    graphs = graph_set(wl.layers)
-    dom_graphs = graphs if len(dom) == len(wl.layers) else graph_set(dom)
-
-    def replay(gs, steps):
-        for _ in range(steps // ncopy):
-            gs["cycle"].replay()
-        for c in range(steps % ncopy):
-            gs["one"][c].replay()
-
-    def timed(gs, steps):
-        """Replays `steps` steps between two events on the launching stream; returns
-        milliseconds, the max over ranks."""
-        replay(gs, max(args.warmup, ncopy))
-        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        start.record(stream)
-        replay(gs, steps)
-        stop.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        return max_over_ranks(start.elapsed_time(stop), world)
-
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        ms = timed(graphs, args.steps)
-        # the dominant kernel's average duration: its own launches back to back, in the same
-        # graphs when the step holds nothing else
-        dom_ms = ms if dom_graphs is graphs else timed(dom_graphs, args.steps)
-    ms_per_step = ms / args.steps
-    step_bytes = wl.step_bytes()
-    value = job_throughput(step_bytes, args.steps, ms, world)
-    dom_launches = len(dom) * args.steps
     peaks = _peaks()
-    if args.workload == "prefill":
-        flops = sum(2.0 * L["B"] * L["N"] * L["K"] for L in dom) * args.steps
-        achieved = flops / (dom_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": _traffic("benq_gemm"),
-                "kernel": "benq_gemm_tcgen05", "avg_launch_us": 1e3 * dom_ms / dom_launches,
-                "peak_source": peaks["source"] + " (burst)"}
-    elif args.workload == "mdbf_prefill":
-        # the whole call (envelope and activation prep plus both GEMMs) against the fp16 dense
-        # peak, which equals the bf16 one; FLOPs are those of the factored contraction
-        flops = sum(mdbf_flops(L["n"], L["m"], MLP_R, MLP_P, L["B"]) for L in dom) * args.steps
-        achieved = flops / (dom_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": _traffic("mdbf_gemm"),
-                "kernel": "mdbf_gemm_tcgen05 (2 GEMMs + 2 prep kernels per call)",
-                "avg_launch_us": 1e3 * dom_ms / dom_launches, "peak_source": peaks["source"] + " (burst)"}
-    else:
-        kb = 0.0
-        for L in dom:
-            ob = L["y"].element_size()
-            kb += (benq_bytes(L["N"], L["K"], L["B"], ob) if L["kind"] == "benq"
-                   else mdbf_bytes(L["n"], L["m"], MLP_R, MLP_L, MLP_P, L["B"], ob))
-        achieved = kb * args.steps / (dom_ms / 1e3) / 1e9
-        kname = "benq_gemv" if dom[0]["kind"] == "benq" else "mdbf_linear"
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": _traffic(kname), "kernel": kname,
-                "avg_launch_us": 1e3 * dom_ms / dom_launches, "peak_source": peaks["source"] + " (STREAM copy)"}
+    timer = Timer(ql, torch, world, args.warmup)
+    order = ALL_ORDER if args.workload == "all" else [args.workload]
+    records, head = {}, None
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for w in order:
+            for key, variants in RECORDS[w]:
+                rec = {}
+                for name, layers, timing in variants:
+                    r, inp = measure_variant(timer, layers, timing, args.steps, peaks, eager=(w == "layer"))
+                    rec[name] = r
+                    if head is None:
+                        head = (key, name, layers, r)
+                    del inp
+                records[key] = rec
+                torch.cuda.empty_cache()
 
-    # end to end through the public API: pinned host inputs in, results back to pinned host memory
-    e2e = None
-    try:
-        xs_h = [torch.from_numpy(np.ascontiguousarray(L["x_h"]).view(np.int16)).view(torch.bfloat16).pin_memory()
-                for L in wl.layers]
-        ys_h = [torch.empty(L["y"].shape, dtype=L["y"].dtype).pin_memory() for L in wl.layers]
-        h2d = sum(t.numel() * t.element_size() for t in xs_h)
-        d2h = sum(t.numel() * t.element_size() for t in ys_h)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for i in range(args.steps):
-            c = i % ncopy
-            for L, xh, yh in zip(wl.layers, xs_h, ys_h):
-                L["x"].copy_(xh, non_blocking=True)
-                wl.run_layer(L, c)
-                yh.copy_(L["y"], non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1), world)
-        e2e = {"value": job_throughput(step_bytes, args.steps, ems, world), "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems / args.steps}
-    except Exception as exc:  # pragma: no cover - reported, not hidden
-        e2e = {"error": repr(exc)}
+    key, name, layers, hr = head
+    ms = hr["us"] * args.steps / 1e3
+    step_bytes = hr["algorithmic_bytes"]
+    value = job_throughput(step_bytes, args.steps, ms, world)
+    roof = dict(hr["roofline"])
+    roof["avg_launch_us"] = hr["us"] / len(layers)
+    headline_gemm = any(is_gemm(L) for L in layers)
 
-    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": {"mdbf": "u1+f16->f32", "mdbf_prefill": "u1+f16->f16 (fp32 accumulate)"}.get(args.workload,
-                                                                                            "bf16xu6->f32"),
-            "data": "synthetic",
-            "config": {"workload": wl.name, "layers": [L["label"] for L in wl.layers],
-                       "us_per_step": 1e3 * ms_per_step,
-                       "algorithmic_bytes_per_step": step_bytes,
-                       "tflops": (wl.step_flops() * args.steps / (ms / 1e3) / 1e12) if wl.step_flops() else None,
-                       "l2": f"inputs larger than L2: {ncopy} rotating weight copies, "
-                             f"{wl.working_set / 2**20:.0f} MiB working set vs 126 MiB L2",
-                       "parallelism": f"replicas x{world}",
-                       "launch": f"CUDA graphs of {ncopy} steps (one weight-copy rotation), kernels chained "
-                                 "by programmatic dependent launch; e2e uses eager calls"},
-            "roofline": roof, "e2e": e2e, "gpu_launches": wl.launches_per_step() * args.steps,
-            "clocks": clk.summary()}
-    if rank == 0 and world == 1 and args.workload == "prefill":
-        line["config"]["cublas_bf16_same_shape"] = cublas_reference(torch, wl.layers, min(args.steps, 20))
+    # CPU baselines (rank 0, one GPU only): the oracle on bounded samples, after all GPU timing
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.workload)
+        for w in order:
+            for k, variants in RECORDS[w]:
+                for vname, vlayers, _ in variants:
+                    unit = "TFLOP/s" if any(is_gemm(L) for L in vlayers) else "GB/s"
+                    budget = 3 * args.cpu_budget if (k, vname) == (key, name) else args.cpu_budget
+                    records[k][vname]["cpu_baseline"] = cpu_baseline(vlayers, budget, unit)
+
+    e2e = hr["e2e"]
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "u1+f16->f32" if layers[0]["kind"] == "mdbf" else "bf16xu6->f32",
+            "data": "synthetic (seeded; BenQ codes made on the device by benq_encode, see the docstring)",
+            "config": line_config(args.workload, world),
+            "roofline": roof,
+            "e2e": {"value": job_throughput(step_bytes, args.steps, e2e["us"] * args.steps / 1e3, world),
+                    "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                    "d2h_bytes_per_step": e2e["d2h_bytes_per_step"], "ms_per_step": e2e["us"] / 1e3},
+            "gpu_launches": hr["launches_per_step"] * args.steps,
+            "clocks": clk.summary()}
+    if headline_gemm:
+        line["unit_note"] = "value is GB/s of algorithmic bytes; roofline is TFLOP/s"
+    if "cpu_baseline" in hr:
+        cb = hr["cpu_baseline"]
+        line["cpu_baseline"] = {"value": cb["value"], "unit": cb["unit"], "cores": cb["cores"], "kind": "oracle",
+                                "sample": cb["sample"], "all_cores_value": cb["all_cores_value"],
+                                "all_cores": cb["all_cores_cores"], "os_cpu_count": cb["os_cpu_count"],
+                                "affinity_cores": cb["affinity_cores"]}
+    if args.workload in ("all", "layer"):
+        lay = records.get("cfg4_layer_27b")
+        if lay:
+            line["decode_us_per_layer"] = {k: v["us"] for k, v in lay.items()}
+    line["workloads"] = records
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs, dom_graphs
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
