@@ -1,7 +1,7 @@
 """Benchmark of the weight-only quantized linear layers on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload all|small|decode|prefill|mdbf_square|layer|mdbf|mdbf_prefill]
+                    [--workload all|small|decode|prefill|mdbf_square|mdbf_l1|layer|mdbf|mdbf_prefill]
                     [--impl ours|reference] [--no-cpu-baseline]
 
 Prints one JSON line.  The default workload, ``all``, times every configuration of the
@@ -18,6 +18,7 @@ benchmark suite in one run; the line's headline (``value``, ``roofline``, ``e2e`
                       gate/up/down; and BenQ attention with the MDBF MLP.  Each as a CUDA graph and
                       as separate launches.
   next1_mdbf_prefill  the MDBF MLP projections at 2048 tokens (tensor-core path), bf16 output.
+  next4_mdbf_l1_4096  the square layer of cfg3 at l = 1: DBF (P = 1) and LittleBit (P = 2), batch 1 and 16.
 
 The other workload names run one of these alone (``mdbf`` is the MDBF MLP of cfg4).
 
@@ -174,12 +175,18 @@ RECORDS = {
         ("mdbf_mlp", layer_set(False, "mdbf"), "rotate"),
         ("mixed_benq_attention_mdbf_mlp", layer_set(True, "mdbf"), "rotate")])],
     "mdbf": [("cfg4_mdbf_mlp_27b", [("b1", layer_set(False, "mdbf"), "rotate")])],
+    # the l = 1 cases (DBF at P = 1, LittleBit at P = 2) on the square layer, next to cfg3's l = 2
+    "mdbf_l1": [("next4_mdbf_l1_4096", [
+        ("dbf_b1", [L_mdbf(1, SQ_N, SQ_N, SQ_R, 1, 1, 3101, "mdbf_4096_r2000_l1_p1_b1")], "flush"),
+        ("dbf_b16", [L_mdbf(1, SQ_N, SQ_N, SQ_R, 1, 16, 3102, "mdbf_4096_r2000_l1_p1_b16")], "flush"),
+        ("littlebit_b1", [L_mdbf(2, SQ_N, SQ_N, SQ_R, 1, 1, 3103, "mdbf_4096_r2000_l1_p2_b1")], "flush"),
+        ("littlebit_b16", [L_mdbf(2, SQ_N, SQ_N, SQ_R, 1, 16, 3104, "mdbf_4096_r2000_l1_p2_b16")], "flush")])],
     "mdbf_prefill": [("next1_mdbf_prefill_m2048", [
         ("m2048", [L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 2048, 6001, "mdbf_gemm_5120x17408_m2048", "bf16"),
                    L_mdbf(MLP_P, HIDDEN, INTER, MLP_R, MLP_L, 2048, 6002, "mdbf_gemm_17408x5120_m2048", "bf16")],
          "rotate")])],
 }
-ALL_ORDER = ["decode", "small", "prefill", "mdbf_square", "layer", "mdbf_prefill"]
+ALL_ORDER = ["decode", "small", "prefill", "mdbf_square", "mdbf_l1", "layer", "mdbf_prefill"]
 WORKLOADS = ["all"] + list(RECORDS)
 
 

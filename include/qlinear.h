@@ -203,10 +203,11 @@ QL_API size_t mdbf_workspace_bytes(int P, int n, int m, int r, int l, int B);
  *   Execution: l * B <= 64 runs the decode kernels once (sign products on the warp MMA with
  *   the dense operand split into bf16 high and low parts).  Larger batches with l <= 32 and
  *   n, m, r >= 64 run as two tensor-core GEMMs, T = X G^T and y = T F^T, each factor element
- *   rebuilt in fp16 inside the GEMM (fp32 accumulation); each token row of x is first scaled by
- *   a power of two so that x and T fit fp16, and y is scaled back exactly.  This assumes every
- *   factor element |F[a][k]|, |G[k][j]| is below 65504.  All other batches run through the
- *   decode kernels floor(64 / l) rows at a time.
+ *   rebuilt in fp16 inside the GEMM (fp32 accumulation).  Powers of two keep every fp16 value
+ *   in range: each factor is rebuilt times 2^-e (e >= 0 from the envelope column maxima, so that
+ *   no element's bound sum_i max|L_i| max|R_i| exceeds 2^15), each token row of x is scaled so
+ *   that x and T fit fp16, and y is scaled back exactly; any envelope magnitudes are accepted.
+ *   All other batches run through the decode kernels floor(64 / l) rows at a time.
  *   Limits: l <= 64 (else QL_ERR_UNSUPPORTED), P <= 8.
  */
 QL_API ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r, int l,
@@ -227,7 +228,8 @@ QL_API ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r,
  *   threads with no ordering between their streams) race and must be serialised by the caller.
  *   Every scratch byte that is read is first written by the same call, so nothing needs
  *   clearing between calls.  The first call on each device looks up the array's device address
- *   with that device current; make that first call before any stream capture.
+ *   with that device current (and so does the first call after the device's context has been
+ *   destroyed and created again); make that first call before any stream capture.
  */
 QL_API ql_status mdbf_linear_noalloc(const mdbf_path *paths, int P, int n, int m, int r, int l,
                                      const uint16_t *x, void *y, ql_out_dtype y_dtype, int B,

@@ -809,7 +809,7 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
-  if (g_ring)
+  if constexpr (g_ring)
     ql::launch(mdbf_g_tile_kernel<NB>, dim3((r + 31) / 32, P), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
                m, r, l, B);
   else
@@ -962,7 +962,33 @@ static __device__ __align__(256) unsigned char g_mdbf_scratch[NOALLOC_SCRATCH_BY
 
 namespace {
 std::mutex g_scratch_mu;
-void *g_scratch_ptr[64] = {nullptr};
+// The array's device address, per device, with the unique id of the context it was looked up in.
+struct ScratchAddr {
+  bool valid;
+  unsigned long long ctx_id;
+  void *ptr;
+};
+ScratchAddr g_scratch_addr[64] = {};
+
+using CtxGetCurrentFn = int (*)(void **);                     // cuCtxGetCurrent
+using CtxGetIdFn = int (*)(void *, unsigned long long *);     // cuCtxGetId
+template <typename F>
+F driver_fn(const char *name) {
+  void *p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<F>(p);
+  return nullptr;
+}
+// Id of the calling thread's current context.  The driver never hands the same id to two
+// contexts of one process, so a context torn down and created again (cudaDeviceReset, a host
+// that resets its device) gets a new id even where its handle is reused.
+bool current_ctx_id(unsigned long long *id) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  void *ctx = nullptr;
+  return get_current && get_id && get_current(&ctx) == 0 && ctx && get_id(ctx, id) == 0;
+}
 }  // namespace
 
 namespace ql {
@@ -970,20 +996,29 @@ namespace ql {
 size_t mdbf_noalloc_scratch_limit() { return NOALLOC_SCRATCH_BYTES; }
 
 // Device address of the scratch array on the current device.  The host-side symbol is only a
-// stand-in, so the address is looked up once per device (with that device current) and cached.
+// stand-in, so the address is looked up with the device current and cached with the context it
+// belongs to; a new context on the device (the module then loads at another address) is looked
+// up again, and where the context cannot be identified the lookup runs on every call.
 ql_status mdbf_noalloc_scratch(void **ptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return fail(QL_ERR_CUDA, "mdbf_linear_noalloc: no current CUDA device");
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_mdbf_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(QL_ERR_CUDA, "mdbf_linear_noalloc: cannot resolve the scratch array: %s", cudaGetErrorString(e));
-    g_scratch_ptr[dev] = p;
+  ScratchAddr &e = g_scratch_addr[dev];
+  unsigned long long id = 0;
+  if (e.valid && current_ctx_id(&id) && id == e.ctx_id) {
+    *ptr = e.ptr;
+    return QL_OK;
   }
-  *ptr = g_scratch_ptr[dev];
+  void *p = nullptr;
+  const cudaError_t err = cudaGetSymbolAddress(&p, g_mdbf_scratch);
+  if (err != cudaSuccess || !p)
+    return fail(QL_ERR_CUDA, "mdbf_linear_noalloc: cannot resolve the scratch array: %s", cudaGetErrorString(err));
+  // the lookup made the device's primary context current if the thread had none
+  e.valid = current_ctx_id(&id);
+  e.ctx_id = id;
+  e.ptr = p;
+  *ptr = p;
   return QL_OK;
 }
 

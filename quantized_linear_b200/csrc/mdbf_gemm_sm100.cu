@@ -18,8 +18,15 @@
 // the smallest exponent for which the envelope bound
 //   |T'[b][k]| <= m * max|X'| * beta,   beta = max_p sum_i max_k|Q_V[k][i]| * max_j|B_amp[j][i]|,
 // stays below half the fp16 maximum, so the intermediate T' = X' G^T is stored in fp16 without
-// overflow.  The last epilogue multiplies each row by the inverse power of two.  Decoded factor
-// elements are assumed to lie within fp16 range (|F|, |G| < 65504).
+// overflow.  The factors get the same treatment: every element of G obeys
+// |G[k][j]| <= sum_i |Q_V[k][i]| |B_amp[j][i]| <= beta, and every element of F likewise
+// |F[a][k]| <= alpha = max_p sum_i max_a|A_amp[a][i]| * max_k|Q_U[k][i]|, so G is rebuilt as
+// G 2^-eg and F as F 2^-ef with eg, ef >= 0 the smallest exponents that put the bounds at or below
+// 2^15 (beta in the bound above is then beta 2^-eg).  A power of two commutes with every fp32
+// rounding of the envelope sum, so each rebuilt element is the oracle's envelope times 2^-e
+// exactly before its rounding to fp16, and no factor element can leave fp16's range whatever the
+// envelopes' magnitudes.  The last epilogue multiplies each row by 2^(eg + ef - s_b), the inverse
+// of all three powers of two.
 //
 // Launches per call: envelope column maxima, activation prep (scale, convert, pad), GEMM 1
 // (decodes G), GEMM 2 (decodes F).  The GEMMs share the CTA-pair structure of the BenQ GEMM: CTA
@@ -68,6 +75,8 @@ constexpr uint16_t PAIR = 0x3;
 // Bound the intermediate T' is kept under: half the fp16 maximum, which leaves room for the fp16
 // rounding of the decoded G and for the fp32 accumulation order.
 constexpr float T_BOUND = 32768.0f;
+// Bound each rebuilt factor element is kept under (the same margin below the fp16 maximum).
+constexpr float F_BOUND = 32768.0f;
 static_assert(OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 static_assert(SB * B_BYTES == 4 * 16384, "the B ring stages one epilogue round: four 16 KB boxes");
@@ -91,6 +100,8 @@ struct Factor {
   // q holds columns 2q, 2q + 1), zero past l and past cols; cpad = the padded column count.
   const float *cpair;
   int cpad;
+  // the power of two 2^-e the rebuilt elements are scaled by (written by the activation prep)
+  const float *scale;
 };
 
 using qld::f2;
@@ -160,9 +171,9 @@ __device__ __forceinline__ uint32_t env_pair(const uint16_t *__restrict__ v, int
 }
 
 // ------------------------------------------------------------------ envelope column maxima
-// emax[p][0][z][i] = max |Q_V[k][i]| and emax[p][1][z][i] = max |B_amp[j][i]| over row slice z of
-// NSL (grid P x 2 x NSL).  Weights are read before the wait on the preceding kernel; the store
-// comes after it.
+// emax[p][w][z][i] = max |E_w[.][i]| over row slice z of NSL for the four envelopes E_0 = Q_V,
+// E_1 = B_amp (G), E_2 = A_amp, E_3 = Q_U (F) (grid P x 4 x NSL, plus the column pairs).
+// Weights are read before the wait on the preceding kernel; the store comes after it.
 constexpr int NSL = 16;
 // Column-pair copy for the l <= 4 decoders: thread q of slice z writes the fp32 pair block of
 // columns 2q, 2q + 1 of path p (grid P x 1 x NSL, one launch per factor).
@@ -184,19 +195,20 @@ __device__ __forceinline__ void write_colpairs(const Factor &f, int p, int z, fl
   }
 }
 
-// blockIdx.y 0, 1: the maxima below; 2: column pairs of g (into g.cpair); 3: of f.
+// blockIdx.y 0 .. 3: the maxima below; 4: column pairs of g (into g.cpair); 5: of f.
 __global__ void __launch_bounds__(256) mdbf_envmax_kernel(Factor g, Factor f, float *__restrict__ emax,
                                                           float *__restrict__ gpair, float *__restrict__ fpair) {
   qld::pdl_trigger();
   const int p = blockIdx.x, which = blockIdx.y, z = blockIdx.z;
-  if (which >= 2) {
+  if (which >= 4) {
     qld::pdl_wait();
-    if (which == 2) write_colpairs(g, p, z, gpair);
+    if (which == 4) write_colpairs(g, p, z, gpair);
     else write_colpairs(f, p, z, fpair);
     return;
   }
-  const unsigned short *v = reinterpret_cast<const unsigned short *>(which == 0 ? g.Lrow[p] : g.Lcol[p]);
-  const int nrow = which == 0 ? g.rows : g.cols, l = g.l;
+  const Factor &fc = which < 2 ? g : f;
+  const unsigned short *v = reinterpret_cast<const unsigned short *>((which & 1) == 0 ? fc.Lrow[p] : fc.Lcol[p]);
+  const int nrow = (which & 1) == 0 ? fc.rows : fc.cols, l = g.l;
   const int per = (nrow + NSL - 1) / NSL, r0 = z * per, r1 = min(nrow, r0 + per);
   __shared__ float red[8][LMAX];
   float mx[LMAX];
@@ -218,17 +230,44 @@ __global__ void __launch_bounds__(256) mdbf_envmax_kernel(Factor g, Factor f, fl
   if ((int)threadIdx.x < l) {
     float a = 0.f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) a = fmaxf(a, red[w][threadIdx.x]);
-    emax[((p * 2 + which) * NSL + z) * LMAX + threadIdx.x] = a;
+    emax[((p * 4 + which) * NSL + z) * LMAX + threadIdx.x] = a;
   }
 }
 
 // ------------------------------------------------------------------ activation prep
+// The bound (max over paths) of sum_i max|E_w0[.][i]| * max|E_w1[.][i]| from the slice maxima.
+__device__ float envelope_bound(const float *__restrict__ emax, int P, int l, int w0) {
+  float bound = 0.f;
+  for (int p = 0; p < P; ++p) {
+    float sp = 0.f;
+    for (int i = 0; i < l; ++i) {
+      float a = 0.f, b = 0.f;
+      for (int z = 0; z < NSL; ++z) {
+        a = fmaxf(a, emax[((p * 4 + w0) * NSL + z) * LMAX + i]);
+        b = fmaxf(b, emax[((p * 4 + w0 + 1) * NSL + z) * LMAX + i]);
+      }
+      sp += a * b;
+    }
+    bound = fmaxf(bound, sp);
+  }
+  return bound;
+}
+// Smallest e >= 0 with v 2^-e <= lim (v finite and >= 0).
+__device__ int down_exponent(float v, float lim) {
+  const float need = v / lim;
+  if (!(need > 1.0f)) return 0;
+  int ex;
+  const float f = frexpf(need, &ex);   // need = f 2^ex, f in [0.5, 1)
+  return f == 0.5f ? ex - 1 : ex;
+}
 // One CTA per token row b: X'[b][j] = fp16(x[b][j] * 2^s_b) for j < m, 0 for m <= j < mp, and
-// inv_s[b] = 2^-s_b, with s_b chosen as described at the top of this file.  CTA 0 also clears the
-// split-tile counters of both GEMMs.
+// inv_s[b] = 2^(eg + ef - s_b), with s_b, eg and ef chosen as described at the top of this file.
+// CTA 0 also writes the factor scales fsc = {2^-eg, 2^-ef} and clears the split-tile counters of
+// both GEMMs.
 __global__ void __launch_bounds__(256) mdbf_xprep_kernel(const uint16_t *__restrict__ x, int m, int mp,
                                                          const float *__restrict__ emax, int P, int l,
                                                          uint16_t *__restrict__ xs, float *__restrict__ inv_s,
+                                                         float *__restrict__ fsc,
                                                          unsigned *__restrict__ counters, int ncounters, int vec8) {
   qld::pdl_trigger();
   qld::pdl_wait();
@@ -256,27 +295,16 @@ __global__ void __launch_bounds__(256) mdbf_xprep_kernel(const uint16_t *__restr
   if (tid == 0) {
     float rmax = 0.f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) rmax = fmaxf(rmax, red[w]);
-    float beta = 0.f;
-    for (int p = 0; p < P; ++p) {
-      float sp = 0.f;
-      for (int i = 0; i < l; ++i) {
-        float mq = 0.f, mb = 0.f;
-        for (int z = 0; z < NSL; ++z) {
-          mq = fmaxf(mq, emax[((p * 2) * NSL + z) * LMAX + i]);
-          mb = fmaxf(mb, emax[((p * 2 + 1) * NSL + z) * LMAX + i]);
-        }
-        sp += mq * mb;
-      }
-      beta = fmaxf(beta, sp);
+    // factor scales: |G| <= beta 2^-eg and |F| <= alpha 2^-ef stay at or below F_BOUND
+    const float beta0 = envelope_bound(emax, P, l, 0), alpha = envelope_bound(emax, P, l, 2);
+    const int eg = down_exponent(beta0, F_BOUND), ef = down_exponent(alpha, F_BOUND);
+    const float beta = ldexpf(beta0, -eg);
+    if (b == 0) {
+      fsc[0] = ldexpf(1.0f, -eg);
+      fsc[1] = ldexpf(1.0f, -ef);
     }
     // e: smallest e >= 0 with m * 2^(1-e) * beta <= T_BOUND
-    int e = 0;
-    const float need = 2.0f * (float)m * beta / T_BOUND;
-    if (need > 1.0f) {
-      int ex;
-      const float f = frexpf(need, &ex);   // need = f 2^ex, f in [0.5, 1)
-      e = f == 0.5f ? ex - 1 : ex;
-    }
+    const int e = down_exponent(2.0f * (float)m * beta, T_BOUND);
     int se = 0;   // scale exponent: max|x'| = rmax 2^se in [2^-e, 2^(1-e))
     if (rmax > 0.f) {
       int ex;
@@ -285,7 +313,7 @@ __global__ void __launch_bounds__(256) mdbf_xprep_kernel(const uint16_t *__restr
     }
     se = max(-126, min(127, se));
     s_exp = se;
-    inv_s[b] = ldexpf(1.0f, -se);
+    inv_s[b] = ldexpf(1.0f, eg + ef - se);
   }
   __syncthreads();
   const float s = ldexpf(1.0f, s_exp);
@@ -508,9 +536,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int kbp = fac.seg / BK;                      // K blocks per path (F stage)
     const int l = fac.l, cols = fac.cols;
     const bool lvec = fac.l_vec2 != 0;
-    // l <= 4: the fp32 column pairs are workspace written by this call's first kernel, not weights,
-    // so the decoders wait for the preceding kernel (and with it for every earlier one) first
-    if constexpr (LK == 4) qld::pdl_wait();
+    // The factor scale (and for l <= 4 the fp32 column pairs) is workspace written by this call's
+    // first kernels, not weights, so the decoders wait for the preceding kernel (and with it for
+    // every earlier one) first.
+    qld::pdl_wait();
+    const float fsc = __ldcg(fac.scale);
     const size_t lblk = (size_t)BK * l;                // column-envelope elements per K block
     const int l8 = 8 * l;
     // this lane's envelope terms: 16c + 2t, +1 (k0) and 16c + 2t + 8, +1 (k1) of chunk c
@@ -548,8 +578,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int ka = 2 * j, kb2 = 2 * j + 1;
-              const float a = (vr[ka] && i < l) ? qld::f16_to_f32(L[(size_t)(r0 + 8 * ka) * l + i]) : 0.f;
-              const float b = (vr[kb2] && i < l) ? qld::f16_to_f32(L[(size_t)(r0 + 8 * kb2) * l + i]) : 0.f;
+              // times the factor's power-of-two scale: exact, and exact through every FMA below
+              const float a = (vr[ka] && i < l) ? qld::f16_to_f32(L[(size_t)(r0 + 8 * ka) * l + i]) * fsc : 0.f;
+              const float b = (vr[kb2] && i < l) ? qld::f16_to_f32(L[(size_t)(r0 + 8 * kb2) * l + i]) * fsc : 0.f;
               rr2[j][i] = f2(a, b);
             }
         };
@@ -801,6 +832,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           } else {
 #pragma unroll
             for (int c = 0; c < LC; ++c) mma_f16_16816(d, afr[c], cur.b[jj][c][0], cur.b[jj][c][1]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) d[c] *= fsc;
           }
           const uint32_t sa_ = jj < 2 ? ea : ea2, sb_ = jj < 2 ? eb : eb2;
           const uint32_t fa = (jj & 1) ? sign_flip<1>(sa_) : sign_flip<0>(sa_);
@@ -999,12 +1032,12 @@ int resident_pairs() {
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace of one call: envelope maxima, the fp32 column pairs of both factors (l <= 4),
-// inverse row scales, X' [B][mp] fp16, T' [B][P seg] fp16, the split counters of both GEMMs, and
-// one region of fp32 partials that GEMM 1 and then GEMM 2 use in turn.
+// inverse row scales, the two factor scales, X' [B][mp] fp16, T' [B][P seg] fp16, the split
+// counters of both GEMMs, and one region of fp32 partials that GEMM 1 and then GEMM 2 use in turn.
 struct GemmWs {
   int mp, seg;
   SplitPlan g1, g2;
-  size_t emax, gpair, fpair, inv_s, xs, ts, cnt, part, total;
+  size_t emax, gpair, fpair, inv_s, fsc, xs, ts, cnt, part, total;
 };
 GemmWs gemm_ws(int P, int n, int m, int r, int B, int pairs) {
   GemmWs L;
@@ -1015,10 +1048,11 @@ GemmWs gemm_ws(int P, int n, int m, int r, int B, int pairs) {
   L.g1 = split_plan(mt * ((P * L.seg + BN - 1) / BN), L.mp / BK, pairs, tile_bytes);
   L.g2 = split_plan(mt * ((n + BN - 1) / BN), P * L.seg / BK, pairs, tile_bytes);
   L.emax = 0;
-  L.gpair = L.emax + align256((size_t)P * 2 * NSL * LMAX * sizeof(float));
+  L.gpair = L.emax + align256((size_t)P * 4 * NSL * LMAX * sizeof(float));
   L.fpair = L.gpair + align256((size_t)P * L.mp * 16);
   L.inv_s = L.fpair + align256((size_t)P * L.seg * 16);
-  L.xs = L.inv_s + align256((size_t)B * sizeof(float));
+  L.fsc = L.inv_s + align256((size_t)B * sizeof(float));
+  L.xs = L.fsc + 256;
   L.ts = L.xs + align256((size_t)B * L.mp * 2);
   L.cnt = L.ts + align256((size_t)B * P * L.seg * 2);
   L.part = L.cnt + L.g1.counter_bytes + L.g2.counter_bytes;
@@ -1043,6 +1077,7 @@ Factor make_factor(const mdbf_path *paths, int P, bool f_stage, int n, int m, in
   f.seg = L.seg;
   f.cpad = f_stage ? L.seg : L.mp;
   f.cpair = reinterpret_cast<const float *>(base + (f_stage ? L.fpair : L.gpair));
+  f.scale = reinterpret_cast<const float *>(base + L.fsc) + (f_stage ? 1 : 0);
   f.P = P;
   f.l = l;
   f.l_vec2 = l2 ? 1 : 0;
@@ -1108,7 +1143,7 @@ ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, i
   const Factor fg = make_factor(paths, P, false, n, m, r, l, L, base);
   const Factor ff = make_factor(paths, P, true, n, m, r, l, L, base);
   float *emax = reinterpret_cast<float *>(base + L.emax);
-  launch(mdbf_envmax_kernel, dim3(P, l <= 4 ? 4 : 2, NSL), 256, 0, s, fg, ff, emax,
+  launch(mdbf_envmax_kernel, dim3(P, l <= 4 ? 6 : 4, NSL), 256, 0, s, fg, ff, emax,
          reinterpret_cast<float *>(base + L.gpair), reinterpret_cast<float *>(base + L.fpair));
   ql_status st = launch_status("mdbf_linear (envelope maxima)");
   if (st != QL_OK) return st;
@@ -1116,7 +1151,7 @@ ql_status mdbf_gemm_launch(const mdbf_path *paths, int P, int n, int m, int r, i
   const int ncnt = (int)((L.g1.counter_bytes + L.g2.counter_bytes) / sizeof(unsigned));
   launch(mdbf_xprep_kernel, B, 256, 0, s, x, m, L.mp, static_cast<const float *>(emax), P, l,
          reinterpret_cast<uint16_t *>(base + L.xs), reinterpret_cast<float *>(base + L.inv_s),
-         reinterpret_cast<unsigned *>(base + L.cnt), ncnt, xvec ? 1 : 0);
+         reinterpret_cast<float *>(base + L.fsc), reinterpret_cast<unsigned *>(base + L.cnt), ncnt, xvec ? 1 : 0);
   st = launch_status("mdbf_linear (activation prep)");
   if (st != QL_OK) return st;
   if (l <= 4)

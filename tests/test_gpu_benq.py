@@ -77,6 +77,20 @@ def test_linear_fast_path_shapes(ql, N, K, B):
     assert max_rel(y, ob.linear(w.codes, w.lut, x, K)) <= BENQ_TOL
 
 
+@pytest.mark.parametrize("N,K", [(2, 1024), (6, 1024), (10, 2048), (4098, 1024), (1026, 17408), (2050, 20480),
+                                 (10242, 12288)])
+def test_linear_batch1_row_counts(ql, N, K):
+    # batch 1 with few rows (fewer row tiles than SMs), N % 4 == 2, one warp per CTA (K = 1024), 20
+    # warps (K = 20480) and CTAs that walk many row tiles (K = 12288, one CTA per SM)
+    w = synth.benq_weights(N, K, seed=N * 3 + K)
+    x = synth.activations(1, K, seed=K + 1)
+    y = _linear(ql, w, x).cpu().numpy()
+    rows = np.arange(N) if N <= 4098 else np.r_[np.arange(0, N, 37), N - 2, N - 1]
+    assert max_rel(y[:, rows], ob.linear(w.codes, w.lut, x, K, rows=rows)) <= BENQ_TOL
+    yb = _linear(ql, w, x, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(yb, f32_to_bf16_rne(y))
+
+
 @pytest.mark.parametrize("N,K,B", [(1, 4, 1), (10, 100, 1), (9, 36, 4), (17, 20484, 2), (5, 1000, 16)])
 def test_linear_generic_path_shapes(ql, N, K, B):
     w = synth.benq_weights(N, K, seed=N * K + B)

@@ -116,6 +116,32 @@ def test_batched_large_envelopes(ql):
     assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
 
 
+@pytest.mark.parametrize("which", ["G", "F", "both"])
+def test_batched_factors_past_fp16_range(ql, which):
+    # Envelopes 2^11 times larger put factor elements well past fp16's maximum (65504): G's when
+    # Q_V and B_amp are scaled, F's when A_amp and Q_U are.  The tensor-core path rebuilds each
+    # factor times a power of two chosen from the envelope maxima and scales the output back, so
+    # the result still meets the tolerance (and the decode kernels, which have no such limit, are
+    # not needed for it).
+    n, m, r, l, P, B = 512, 1024, 384, 4, 2, 40      # l * B = 160: the tensor-core path
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=51)
+    for p in paths:
+        if which in ("G", "both"):
+            p.Q_V = _scaled_envelope(p.Q_V, 2048.0)
+            p.B_amp = _scaled_envelope(p.B_amp, 2048.0)
+        if which in ("F", "both"):
+            p.A_amp = _scaled_envelope(p.A_amp, 2048.0)
+            p.Q_U = _scaled_envelope(p.Q_U, 2048.0)
+    big = max(max(np.abs(F).max(), np.abs(G).max()) for F, G in (om.factors(p, n, m, r) for p in paths))
+    assert big > 65504.0
+    x = synth.activations(B, m, seed=52)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    assert np.all(np.isfinite(y))
+    assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+    yb = _linear(ql, paths, n, m, r, l, x, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(yb, f32_to_bf16_rne(y))
+
+
 @pytest.mark.parametrize("ldSA,ldSB", [(40, 128), (44, 132)])
 def test_batched_narrow_sign_strides(ql, ldSA, ldSB):
     # strides that are multiples of 4 bytes but not of 16, the last 32-bit word of a row reaching

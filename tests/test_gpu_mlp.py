@@ -53,7 +53,8 @@ def _check_against_oracle(h, wg, wu, x, K, rows=None):
     assert np.all(err <= bound), float((err / np.maximum(bound, 1e-300)).max())
 
 
-@pytest.mark.parametrize("N,K", [(256, 1024), (1000, 2048), (34, 5120), (1024, 20480)])
+@pytest.mark.parametrize("N,K", [(256, 1024), (1000, 2048), (34, 5120), (1024, 20480), (2, 1024), (6, 3072),
+                                 (2050, 17408)])
 def test_fused_decode_matches_oracle(ql, N, K):
     wg, wu = _layers(N, K, seed=N + K)
     x = synth.activations(1, K, seed=K)

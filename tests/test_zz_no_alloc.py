@@ -3,20 +3,27 @@
 Some callers may not call cudaMalloc (allocator-internal code, real-time threads that must not
 block in the driver, hosts with a memory budget fixed at start-up).  mdbf_linear_noalloc serves
 them from a fixed scratch array compiled into the library.  This test calls it through the C ABI
-and checks each result against mdbf_linear (the workspace entry point) on two calls in a row with
-different problems, so stale scratch from the first call cannot leak into the second.  It lives in
-a file of its own that pytest collects last, and passes alone or after the other tests.
+on each of the paths its scratch feeds -- the batch decode kernels, the envelope chunks of l > 32,
+and the tensor-core GEMMs whose split counters live in the scratch -- twice in a row on different
+inputs, so stale scratch from one call cannot leak into the next.  Each result is checked against
+the oracle (within the MDBF tolerance) and against mdbf_linear, the workspace entry point (bit for
+bit).  The file is collected last and passes alone or after the other tests.
 """
-import ctypes
-
 import numpy as np
 import pytest
 import torch
 
 import synth
+from oracle import mdbf as om
 from tests.qlhelpers import MDBF_TOL, bf16, max_rel, mdbf_dev_paths
 
 pytestmark = pytest.mark.gpu
+
+# (n, m, r, l, P, B, seed): decode kernels (l*B <= 64), envelope chunks (l > 32), and the tensor
+# cores (l*B > 64 with n, m, r >= 64) on a layer small enough for the array whose two K blocks per
+# GEMM make both GEMMs split their last wave, so the split counters in the scratch are used
+PROBLEMS = [(1024, 768, 300, 4, 2, 3, 71), (640, 1280, 257, 2, 1, 16, 72),
+            (256, 256, 128, 40, 1, 2, 74), (300, 128, 64, 4, 2, 20, 73)]
 
 
 def _reference(ql, paths_c, n, m, r, l, x):
@@ -33,19 +40,22 @@ def _noalloc_raw(ql, paths_c, n, m, r, l, x, y):
              torch.cuda.current_stream().cuda_stream)
 
 
-def test_noalloc_matches_workspace_entry_on_two_calls(ql):
-    problems = [(1024, 768, 300, 4, 2, 3, 71), (640, 1280, 257, 2, 1, 16, 72)]
-    for n, m, r, l, P, B, seed in problems:
-        paths = synth.mdbf_paths(P, n, m, r, l, seed=seed)
-        dp = mdbf_dev_paths(paths)
-        pc = ql.mdbf_paths_c(dp)
-        x = bf16(synth.activations(B, m, seed=seed + 1))
-        assert ql.mdbf_workspace_bytes(P, n, m, r, l, B) <= ql.mdbf_noalloc_scratch_bytes()
+@pytest.mark.parametrize("n,m,r,l,P,B,seed", PROBLEMS)
+def test_noalloc_matches_oracle_and_workspace_entry_on_two_calls(ql, n, m, r, l, P, B, seed):
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=seed)
+    dp = mdbf_dev_paths(paths)
+    pc = ql.mdbf_paths_c(dp)
+    assert ql.mdbf_workspace_bytes(P, n, m, r, l, B) <= ql.mdbf_noalloc_scratch_bytes()
+    for call in range(2):
+        x_h = synth.activations(B, m, seed=seed + 1 + call)
+        x = bf16(x_h)
         y = torch.full((B, n), float("nan"), device="cuda")
         assert _noalloc_raw(ql, pc, n, m, r, l, x, y) == ql.QL_OK
         y_ref = _reference(ql, pc, n, m, r, l, x)
         torch.cuda.synchronize()
-        assert max_rel(y.cpu().numpy(), y_ref.cpu().numpy()) <= MDBF_TOL
+        got = y.cpu().numpy()
+        assert np.isfinite(got).all()
+        assert max_rel(got, om.linear_factored(paths, n, m, r, x_h)) <= MDBF_TOL
         assert torch.equal(y, y_ref)
 
 
