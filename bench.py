@@ -605,6 +605,31 @@ def roofline(layers, us, peaks):
     return r
 
 
+def cublas_reference(torch, layers, steps, warmup=3):
+    """Dense bf16 GEMMs of the same shapes through torch.matmul (cuBLAS) on random dense weights,
+    timed the same way (device events, weights larger than L2): a reference point for the
+    tensor-core rate at these shapes, not part of the measured path."""
+    mats = [(torch.randn(L["B"], L["K"], device="cuda").to(torch.bfloat16),
+             torch.randn(L["N"], L["K"], device="cuda").to(torch.bfloat16)) for L in layers]
+    out = [torch.empty(L["B"], L["N"], device="cuda", dtype=torch.bfloat16) for L in layers]
+    for _ in range(warmup):
+        for (a, w), o in zip(mats, out):
+            torch.matmul(a, w.t(), out=o)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(steps):
+        for (a, w), o in zip(mats, out):
+            torch.matmul(a, w.t(), out=o)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    flops = sum(2.0 * L["B"] * L["N"] * L["K"] for L in layers)
+    del mats, out
+    return {"us_per_step": 1e3 * ms, "tflops": flops / (ms / 1e3) / 1e12,
+            "what": "torch.matmul bf16 (cuBLAS), same shapes, dense random weights"}
+
+
 def measure_variant(timer, layers, timing, steps, peaks, eager=False):
     inp = Inputs(layers, copies_for(layers, timing), timer.ql, timer.torch)
     for L in inp.layers:   # first calls outside any capture (kernel attributes, tensor maps)
@@ -624,6 +649,8 @@ def measure_variant(timer, layers, timing, steps, peaks, eager=False):
     if eager:
         ems = timer.time_eager(inp, inp.layers, steps, timing)
         rec["us_separate_launches"] = 1e3 * ems / steps
+    if all(L["kind"] == "benq" and is_gemm(L) for L in layers) and timer.world == 1:
+        rec["cublas_bf16_same_shape"] = cublas_reference(timer.torch, layers, min(steps, 20))
     ems, h2d, d2h = timer.time_e2e(inp, inp.layers, steps)
     rec["e2e"] = {"value": byts * steps / (ems / 1e3) / 1e9, "unit": "GB/s", "us": 1e3 * ems / steps,
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
