@@ -707,6 +707,174 @@ __global__ void __launch_bounds__(NRG * 32 * KG)
   }
 }
 
+// ------------------------------------------------ F stage, one fragment block per word ----------
+// For NB == 1 (l * B <= 4, the decode batches) and at most two paths.  One CTA per 16 * RT * NRG
+// rows holds both paths in shared memory: each path's sign block arrives by bulk copy before the
+// wait on the G stage (weights) and its w fragments by a bulk copy right after it, both counted on
+// the path's mbarrier.  Every warp then runs both paths in one pass over its K-word group, one
+// accumulator set per path, with no barrier between the paths.  The A_amp epilogue runs in
+// registers: lane (g, q) holds columns 2q, 2q + 1 of rows g and g + 8 of each 16-row tile, i.e. the
+// high or low part of vector (b, i), so it adds A_amp[row][i] times its values into the row's sum
+// for b and the four lanes of a row combine them by shuffles; the K-word groups' sums are then
+// added in group order.  Paths are summed inside each lane in p order.  One barrier per CTA,
+// before the group sums.
+constexpr int F1_PMAX = 2;
+
+template <int RT, int NRG>
+__global__ void __launch_bounds__(NRG * 32 * 8)
+    mdbf_f_nb1_kernel(Paths ps, int P, const uint4 *__restrict__ wpk, void *__restrict__ y, int ydt, int n, int r,
+                      int l, int B, uint32_t sign_stride, uint32_t frag_bytes) {
+  constexpr int KG = 8, TILES = RT * NRG, ROWS = 16 * TILES;
+  extern __shared__ __align__(128) unsigned char fsm[];
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(fsm));
+  const int QW = (r + 31) / 32, V = l * B;
+  const int row0 = blockIdx.x * ROWS, rows = min(ROWS, n - row0);
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int rg = wid % NRG, kg = wid / NRG;
+  const int qw0 = kg * QW / KG, qw1 = (kg + 1) * QW / KG;
+  const int rbase = 16 * RT * rg;
+  const uint32_t frag_base = base + F1_PMAX * sign_stride;                  // [P][frag_bytes]
+  const uint32_t bars = frag_base + F1_PMAX * frag_bytes;                   // one mbarrier per path
+  const uint32_t abort_a = bars + 64;                                        // set when a wait ran out
+  uint16_t *const a_sm = reinterpret_cast<uint16_t *>(fsm + F1_PMAX * (sign_stride + frag_bytes) + 128);   // [P][ROWS][l]
+  float *const ypart = reinterpret_cast<float *>(fsm + F1_PMAX * (sign_stride + frag_bytes) + 128 +
+                                                 ((F1_PMAX * ROWS * l * 2 + 15) / 16) * 16);   // [KG][ROWS][B]
+  if (threadIdx.x == 0) {
+    for (int p = 0; p < P; ++p) sm100::mbar_init(bars + 8 * p, 1);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(abort_a), "r"(0u) : "memory");
+    sm100::fence_barrier_init();
+    for (int p = 0; p < P; ++p) {
+      const uint32_t sbytes = (uint32_t)(rows * ps.ldSA[p]);
+      sm100::mbar_arrive_expect_tx(bars + 8 * p, sbytes + frag_bytes);
+      sm100::bulk_g2s(base + p * sign_stride, ps.SA[p] + (size_t)row0 * ps.ldSA[p], sbytes, bars + 8 * p);
+    }
+  }
+  for (int e = threadIdx.x; e < P * rows * l; e += blockDim.x) {
+    const int pp = e / (rows * l), j = e - pp * (rows * l);
+    a_sm[pp * ROWS * l + j] = ps.A[pp][(int64_t)row0 * l + j];
+  }
+  qld::pdl_trigger();
+  qld::pdl_wait();
+  // the w fragments are made by the G stage: copied after the wait
+  if (threadIdx.x == 0)
+    for (int p = 0; p < P; ++p) sm100::bulk_g2s(frag_base + p * frag_bytes, wpk + (size_t)p * QW * 32, frag_bytes, bars + 8 * p);
+  __syncthreads();
+
+  bool ok = true;
+  const bool live = rbase < rows;   // rows past `rows` read stale bytes and are never stored
+  float acc[F1_PMAX][RT][4];
+#pragma unroll
+  for (int p = 0; p < F1_PMAX; ++p)
+#pragma unroll
+    for (int t = 0; t < RT; ++t) acc[p][t][0] = acc[p][t][1] = acc[p][t][2] = acc[p][t][3] = 0.f;
+#pragma unroll
+  for (int p = 0; p < F1_PMAX; ++p) {
+    if (p >= P) break;
+    if (!sm100::mbar_wait(bars + 8 * p, 0, FT_WAIT_BUDGET)) ok = false;
+    if (!ok || !live || qw0 >= qw1) continue;
+    const uint32_t sb = base + p * sign_stride;
+    const uint32_t ldp = (uint32_t)ps.ldSA[p];
+    uint32_t r0[RT];
+#pragma unroll
+    for (int t = 0; t < RT; ++t) r0[t] = sb + (rbase + 16 * t + g) * ldp;
+    const uint32_t fb = frag_base + p * frag_bytes + lane * 16;
+#pragma unroll 2
+    for (int qw = qw0; qw < qw1; ++qw) {
+      const uint4 bf = lds128(fb + qw * 512);
+      uint32_t s0[RT], s1[RT];
+#pragma unroll
+      for (int t = 0; t < RT; ++t) {
+        s0[t] = lds32s(r0[t] + 4 * qw);
+        s1[t] = lds32s(r0[t] + 8 * ldp + 4 * qw);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t ma = 1u << (15 - 8 * h - q), mb = 1u << (11 - 8 * h - q);
+#pragma unroll
+        for (int t = 0; t < RT; ++t) {
+          const uint32_t a0 = sign_pair_mul(s0[t], ma), a1 = sign_pair_mul(s1[t], ma),
+                         a2 = sign_pair_mul(s0[t], mb), a3 = sign_pair_mul(s1[t], mb);
+          mma16816(acc[p][t], a0, a1, a2, a3, h ? bf.z : bf.x, h ? bf.w : bf.y);
+        }
+      }
+    }
+  }
+  // register epilogue: this lane's columns c = 2q + j (j = 0, 1) are the high (c < V) or low
+  // (V <= c < 2V) part of vector v = b * l + i; add A_amp[row][i] times them into the row's sum for b
+  float yb[2 * RT][4];   // [tile t, half hh][b]
+#pragma unroll
+  for (int k = 0; k < 2 * RT; ++k) yb[k][0] = yb[k][1] = yb[k][2] = yb[k][3] = 0.f;
+  if (live) {
+#pragma unroll
+    for (int p = 0; p < F1_PMAX; ++p) {
+      if (p >= P) break;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int c = 2 * q + j;
+        if (c >= 2 * V) continue;
+        const int v = c < V ? c : c - V, b = v / l, i = v - b * l;
+#pragma unroll
+        for (int t = 0; t < RT; ++t)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int rl = rbase + 16 * t + g + 8 * hh;   // block-local row
+            const float a = qld::f16_to_f32(a_sm[(p * ROWS + rl) * l + i]);
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb)
+              if (bb == b) yb[2 * t + hh][bb] = fmaf(a, acc[p][t][2 * hh + j], yb[2 * t + hh][bb]);
+          }
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 2 * RT; ++k)
+#pragma unroll
+    for (int bb = 0; bb < 4; ++bb) {
+      float v = yb[k][bb];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      yb[k][bb] = v;
+    }
+  if (live && q == 0) {
+#pragma unroll
+    for (int t = 0; t < RT; ++t)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int rl = rbase + 16 * t + g + 8 * hh;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb)
+          if (bb < B) ypart[((size_t)kg * ROWS + rl) * B + bb] = yb[2 * t + hh][bb];
+      }
+  }
+  if (!ok) asm volatile("st.shared.u32 [%0], %1;" ::"r"(abort_a), "r"(1u) : "memory");
+  __syncthreads();   // every thread arrives here exactly once, whether its waits ran out or not
+  uint32_t aborted;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(aborted) : "r"(abort_a) : "memory");
+  if (aborted) {
+    if (threadIdx.x == 0) {
+      atomicExch(&g_mdbf_timeout, 1);
+      // leave no copy in flight: wait (bounded) for every path's sign block
+      for (int p = 0; p < P; ++p) (void)sm100::mbar_wait(bars + 8 * p, 0, FT_WAIT_BUDGET);
+    }
+    return;
+  }
+  for (int e = threadIdx.x; e < rows * B; e += blockDim.x) {
+    const int rl = e / B, b = e - rl * B, a = row0 + rl;
+    float sacc = 0.f;
+#pragma unroll
+    for (int k = 0; k < KG; ++k) sacc += ypart[((size_t)k * ROWS + rl) * B + b];
+    if (ydt == QL_OUT_F32)
+      static_cast<float *>(y)[(int64_t)b * n + a] = sacc;
+    else
+      static_cast<uint16_t *>(y)[(int64_t)b * n + a] = qld::f32_to_bf16_rn(sacc);
+  }
+}
+
+inline size_t f_nb1_smem(uint32_t sign_stride, uint32_t frag_bytes, int rows, int l, int B) {
+  return (size_t)F1_PMAX * (sign_stride + frag_bytes) + 128 + ((F1_PMAX * rows * l * 2 + 15) / 16) * 16 +
+         (size_t)8 * rows * B * 4;
+}
+
 // ---------------------------------------------------------------- debug dequantizer ----------
 __device__ __forceinline__ float envelope(const uint16_t *L, const uint16_t *R, int l) {
   float e = qld::f16_to_f32(L[0]) * qld::f16_to_f32(R[0]);
@@ -816,6 +984,26 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     ql::launch(kg, dim3((r + 31) / 32, P), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
   ql_status st = ql::launch_status("mdbf_linear (G stage)");
   if (st != QL_OK) return st;
+  if constexpr (VEC16 && NB == 1) {
+    if (P <= F1_PMAX) {
+      // both paths in one pass: 128-row CTAs when they fill the SMs, else 32-row ones
+      size_t ld_max = 0;
+      for (int p = 0; p < P; ++p) ld_max = std::max(ld_max, ps.ldSA[p]);
+      const bool big = (n + 127) / 128 >= ql::sm_count() * 3 / 4;
+      const int rows = big ? 128 : 32;
+      const uint32_t sign_stride = (uint32_t)((rows * ld_max + 127) / 128 * 128);
+      const uint32_t frag_bytes = (uint32_t)((r + 31) / 32) * 32 * 16;
+      const size_t sm = f_nb1_smem(sign_stride, frag_bytes, rows, l, B);
+      if (sm <= 227 * 1024) {
+        auto kt = big ? mdbf_f_nb1_kernel<2, 4> : mdbf_f_nb1_kernel<2, 1>;
+        if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+          return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
+        ql::launch(kt, (n + rows - 1) / rows, (big ? 4 : 1) * 32 * 8, sm, s, ps, P, (const uint4 *)wpk, y, (int)ydt, n,
+                   r, l, B, sign_stride, frag_bytes);
+        return ql::launch_status("mdbf_linear (F stage)");
+      }
+    }
+  }
   if constexpr (VEC16) {
     // staged-tile F stage when two (else one) path stages fit in shared memory
     size_t ld_max = 0;

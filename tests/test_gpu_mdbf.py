@@ -62,7 +62,10 @@ def test_dequant_hand_worked_example(ql, golden):
 
 @pytest.mark.parametrize("n,m,r,l,P,B", [(5, 7, 3, 1, 1, 1), (33, 65, 31, 2, 2, 3), (100, 40, 40, 4, 2, 16),
                                          (64, 64, 64, 8, 1, 8), (70, 90, 50, 3, 3, 5), (300, 200, 100, 1, 2, 1),
-                                         (96, 1000, 95, 2, 1, 32), (1, 1, 1, 1, 1, 1)])
+                                         (96, 1000, 95, 2, 1, 32), (1, 1, 1, 1, 1, 1),
+                                         # l * B <= 4 with several token rows (the F stage's per-row
+                                         # sums for each b), one and two paths, ragged n, m and r
+                                         (130, 200, 64, 2, 2, 2), (77, 50, 40, 1, 2, 4), (4000, 300, 128, 1, 1, 3)])
 def test_linear_shapes(ql, n, m, r, l, P, B):
     paths = synth.mdbf_paths(P, n, m, r, l, seed=3 * n + m)
     x = synth.activations(B, m, seed=B)
@@ -106,6 +109,16 @@ def test_linear_mlp_shapes_sampled_rows(ql, n, m):
     y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
     rows = np.r_[np.random.default_rng(2).choice(n, 256, replace=False), 0, n - 1]
     assert max_rel(y[:, rows], om.linear_factored(paths, n, m, r, x, rows=rows)) <= MDBF_TOL
+
+
+@pytest.mark.parametrize("P", [1, 2])
+def test_linear_more_g_blocks_than_sms(ql, P):
+    # more 32-row blocks of S_B than SMs (the G stage then runs 16 warps per block), ragged r
+    n, m, r, l, B = 5200, 4800, 4790 // P, 4, 1
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=4400 + P)
+    x = synth.activations(B, m, seed=4500 + P)
+    y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
+    assert max_rel(y, om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
 
 
 def test_linear_is_deterministic(ql):
