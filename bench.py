@@ -124,6 +124,13 @@ def L_mlp(N, K, seed_g, seed_u, label):
     return dict(kind="benq_mlp", N=N, K=K, B=1, seed=seed_g, seed_u=seed_u, label=label, out="bf16")
 
 
+def L_multi(parts, K, label):
+    """BenQ layers of the same K that read the same x, in one call (benq_linear_multi, batch 1);
+    parts: [(N, seed, label)]."""
+    return dict(kind="benq_multi", parts=parts, N=sum(p[0] for p in parts), K=K, B=1, seed=parts[0][1], label=label,
+                out="f32")
+
+
 def L_mdbf(P, n, m, r, l, B, seed, label, out="f32"):
     return dict(kind="mdbf", P=P, n=n, m=m, r=r, l=l, B=B, seed=seed, label=label, out=out)
 
@@ -134,10 +141,14 @@ SEED_GATE, SEED_DOWN, SEED_UP = 1001, 1002, 1003
 
 def layer_set(attention, mlp):
     """One decoder layer's linears at batch 1: the BenQ attention projections (q, k, v, o) when
-    `attention`, then the MLP: "benq" (gate, up, down), "benq_fused" (gate and up in one call
-    with the SiLU gate, then down) or "mdbf" (gate, up, down in MDBF)."""
+    `attention` ("fused": q, k and v in one call), then the MLP: "benq" (gate, up, down),
+    "benq_fused" (gate and up in one call with the SiLU gate, then down) or "mdbf" (gate, up, down
+    in MDBF)."""
     out = []
-    if attention:
+    if attention == "fused":
+        out += [L_multi([(HIDDEN, 5001, "q"), (1024, 5002, "k"), (1024, 5003, "v")], HIDDEN, "benq_qkv"),
+                L_benq(HIDDEN, HIDDEN, 1, 5004, "benq_o")]
+    elif attention:
         out += [L_benq(HIDDEN, HIDDEN, 1, 5001, "benq_q"), L_benq(1024, HIDDEN, 1, 5002, "benq_k"),
                 L_benq(1024, HIDDEN, 1, 5003, "benq_v"), L_benq(HIDDEN, HIDDEN, 1, 5004, "benq_o")]
     if mlp == "benq":
@@ -172,6 +183,7 @@ RECORDS = {
     "layer": [("cfg4_layer_27b", [
         ("benq_7_linears", layer_set(True, "benq"), "rotate"),
         ("benq_fused_mlp", layer_set(True, "benq_fused"), "rotate"),
+        ("benq_4_launches", layer_set("fused", "benq_fused"), "rotate"),
         ("mdbf_mlp", layer_set(False, "mdbf"), "rotate"),
         ("mixed_benq_attention_mdbf_mlp", layer_set(True, "mdbf"), "rotate")])],
     "mdbf": [("cfg4_mdbf_mlp_27b", [("b1", layer_set(False, "mdbf"), "rotate")])],
@@ -201,13 +213,15 @@ def out_bytes(L):
 def layer_bytes(L):
     if L["kind"] == "benq":
         return benq_bytes(L["N"], L["K"], L["B"], out_bytes(L))
+    if L["kind"] == "benq_multi":   # x read once for all parts
+        return benq_bytes(L["N"], L["K"], L["B"], out_bytes(L))
     if L["kind"] == "benq_mlp":
         return 2 * benq_weight_bytes(L["N"], L["K"]) + 2 * L["K"] + out_bytes(L) * L["N"]
     return mdbf_bytes(L["n"], L["m"], L["r"], L["l"], L["P"], L["B"], out_bytes(L))
 
 
 def layer_weight_bytes(L):
-    if L["kind"] == "benq":
+    if L["kind"] in ("benq", "benq_multi"):
         return benq_weight_bytes(L["N"], L["K"])
     if L["kind"] == "benq_mlp":
         return 2 * benq_weight_bytes(L["N"], L["K"])
@@ -215,7 +229,7 @@ def layer_weight_bytes(L):
 
 
 def layer_flops(L):
-    if L["kind"] == "benq":
+    if L["kind"] in ("benq", "benq_multi"):
         return 2.0 * L["B"] * L["N"] * L["K"]
     if L["kind"] == "benq_mlp":
         return 4.0 * L["N"] * L["K"]
@@ -223,7 +237,7 @@ def layer_flops(L):
 
 
 def is_gemm(L):
-    if L["kind"] == "benq":
+    if L["kind"] in ("benq", "benq_multi"):
         return L["B"] > 16
     if L["kind"] == "mdbf":
         return L["l"] * L["B"] > DECODE_VLIM
@@ -233,7 +247,7 @@ def is_gemm(L):
 def layer_launches(L):
     """Kernels of this library one call launches: BenQ one; MDBF decode pack z, G stage, F stage;
     MDBF batched envelope prep, activation prep and the two GEMMs."""
-    if L["kind"] in ("benq", "benq_mlp"):
+    if L["kind"] in ("benq", "benq_mlp", "benq_multi"):
         return 1
     return 4 if is_gemm(L) else 3
 
@@ -357,6 +371,11 @@ class Inputs:
             elif L["kind"] == "benq_mlp":
                 w0 = (self.benq_device_weights(L["N"], L["K"], L["seed"], ql, torch)
                       + self.benq_device_weights(L["N"], L["K"], L["seed_u"], ql, torch))
+            elif L["kind"] == "benq_multi":
+                # one output buffer, a contiguous view per part (batch 1, parts of 4k rows: 16-byte aligned)
+                w0 = tuple(self.benq_device_weights(N, L["K"], sd, ql, torch) for N, sd, _ in L["parts"])
+                offs = np.cumsum([0] + [N for N, _, _ in L["parts"]])
+                L["ys"] = [L["y"][:, offs[i]:offs[i + 1]] for i in range(len(L["parts"]))]
             else:
                 paths = synth.mdbf_paths(L["P"], L["n"], L["m"], L["r"], L["l"], seed=L["seed"])
                 w0 = [dict(S_A=dev(p.S_A), S_B=dev(p.S_B), A_amp=f16(p.A_amp), B_amp=f16(p.B_amp),
@@ -384,7 +403,7 @@ class Inputs:
     @staticmethod
     def clone(w):
         if isinstance(w, tuple):
-            return tuple(t.clone() for t in w)
+            return tuple(tuple(u.clone() for u in t) if isinstance(t, tuple) else t.clone() for t in w)
         return [{k: v.clone() for k, v in d.items()} for d in w]
 
     def run(self, ql, L, c):
@@ -393,6 +412,8 @@ class Inputs:
             ql.benq_linear(w[0], w[1], L["x"], L["y"], workspace=L["ws"])
         elif L["kind"] == "benq_mlp":
             ql.benq_mlp_gate_up(*w, L["x"], L["y"])
+        elif L["kind"] == "benq_multi":
+            ql.benq_linear_multi([(c, t, y) for (c, t), y in zip(w, L["ys"])], L["x"])
         else:
             ql.mdbf_linear(w, L["n"], L["m"], L["r"], L["l"], L["x"], L["y"], L["ws"])
 
@@ -564,7 +585,7 @@ def _traffic(kernel_key):
 
 
 def kernel_name(L):
-    if L["kind"] in ("benq", "benq_mlp"):
+    if L["kind"] in ("benq", "benq_mlp", "benq_multi"):
         return "benq_gemm" if is_gemm(L) else "benq_gemv"
     return "mdbf_gemm" if is_gemm(L) else "mdbf_linear"
 
@@ -671,12 +692,12 @@ def oracle_sample(layers, rows=64, seed=0):
     out = []
     for L in layers:
         bb = min(L["B"], 16)
-        if L["kind"] in ("benq", "benq_mlp"):
+        if L["kind"] in ("benq", "benq_mlp", "benq_multi"):
             N, K = L["N"], L["K"]
             rr = min(rows, N)
             w = synth.benq_weights(rr, K, seed=int(rng.integers(1 << 30)))
             x = synth.activations(bb, K, seed=1)
-            if L["kind"] == "benq":
+            if L["kind"] != "benq_mlp":
                 run = (lambda w=w, x=x, K=K: ob.linear(w.codes, w.lut, x, K))
                 out.append((f"benq {rr} of {N} rows x K={K}, B={bb}", run, benq_bytes(rr, K, bb), 2.0 * bb * rr * K))
             else:

@@ -130,6 +130,29 @@ QL_API ql_status benq_mlp_gate_up(const uint8_t *codes_g, const uint16_t *lut_g,
 /* Workspace bytes benq_mlp_gate_up needs for these sizes (0 when the fused batch-1 kernel runs). */
 QL_API size_t benq_mlp_workspace_bytes(int B, int N, int K);
 
+/*
+ * benq_linear_multi -- several BenQ layers that read the same input, y_s = x W_s^T for
+ *   s < S ("What BenQ stores": each layer stored as for benq_linear), as the attention
+ *   projections q, k and v of a decoder layer are.  At B == 1, with K % 1024 == 0 (K <= 20480)
+ *   and every N % 4 == 0, all layers run in one launch of the batch-1 GEMV, which walks the row
+ *   tiles of every layer as one range (a small layer then shares the SMs with the others instead
+ *   of leaving them idle); each y_s equals benq_linear's result for that layer bit for bit.
+ *   Other shapes run the layers one after another through benq_linear.
+ *   layers  host array of S entries {codes, lut, y, N}: device pointers and the layer's output
+ *           features, each as for benq_linear (16-byte aligned).
+ *   S       1 <= S <= 4.
+ *   x       device, bf16 bits [B][K], shared by all layers; y_s [B][N_s] of y_dtype.
+ *   Errors: as benq_linear for every layer; QL_ERR_INVALID_ARG for S outside [1, 4].
+ */
+typedef struct {
+  const uint8_t *codes;   /* [N][3K/4] packed codes */
+  const uint16_t *lut;    /* [N][64] bf16 tables */
+  void *y;                /* [B][N] output */
+  int N;                  /* output features */
+} benq_layer;
+QL_API ql_status benq_linear_multi(const benq_layer *layers, int S, const uint16_t *x, ql_out_dtype y_dtype,
+                                   int B, int K, ql_stream_t stream);
+
 /* Workspace bytes benq_linear_ws uses for these sizes on the current device
  * (0 when B <= 16 or when no split applies).  Needs a CUDA device. */
 QL_API size_t benq_linear_workspace_bytes(int B, int N, int K);

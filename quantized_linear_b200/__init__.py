@@ -27,6 +27,10 @@ STATUS_NAMES = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED", 3:
 _vp, _i, _sz, _d = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_double
 
 
+class BenQLayerC(ctypes.Structure):
+    _fields_ = [("codes", _vp), ("lut", _vp), ("y", _vp), ("N", _i)]
+
+
 class MDBFPathC(ctypes.Structure):
     _fields_ = [("S_A", _vp), ("S_B", _vp), ("ldSA", _sz), ("ldSB", _sz),
                 ("A_amp", _vp), ("B_amp", _vp), ("Q_U", _vp), ("Q_V", _vp)]
@@ -36,6 +40,7 @@ _SIGNATURES = {
     "benq_linear": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "benq_linear_ws": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "benq_linear_workspace_bytes": (_sz, [_i, _i, _i]),
+    "benq_linear_multi": (_i, [ctypes.POINTER(BenQLayerC), _i, _vp, _i, _i, _i, _vp]),
     "benq_mlp_gate_up": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "benq_mlp_workspace_bytes": (_sz, [_i, _i, _i]),
     "benq_encode": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
@@ -73,7 +78,7 @@ def lib() -> ctypes.CDLL:
 def _c(name):
     return getattr(lib(), name)
 
-EXPORTS = ["benq_linear", "benq_linear_ws", "benq_linear_workspace_bytes", "benq_mlp_gate_up",
+EXPORTS = ["benq_linear", "benq_linear_ws", "benq_linear_workspace_bytes", "benq_linear_multi", "benq_mlp_gate_up",
            "benq_mlp_workspace_bytes", "benq_encode", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
            "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
            "mdbf_select_rank", "ql_last_error", "ql_check", "ql_set_pdl", "ql_selftest_timeout"]
@@ -154,6 +159,30 @@ def benq_linear(codes, lut, x, y, stream=None, workspace=None):
         _check(_c("benq_linear_ws")(_ptr(codes), _ptr(lut), _ptr(x), _ptr(y), _ydt(y), B, N, K, _ptr(workspace),
                                     nbytes, _stream(stream)))
     return y
+
+
+def benq_linear_multi(layers, x, stream=None):
+    """y_s = x @ W_s^T for several BenQ layers of the same K that read the same x (at batch 1 in one
+    launch).  layers: list of (codes, lut, y) with codes uint8 [N_s, 3K/4], lut bf16 [N_s, 64] and y
+    float32 or bf16 [B, N_s] (all the same dtype, overwritten)."""
+    B, K = x.shape
+    _want(x, torch.bfloat16, "x")
+    if not 1 <= len(layers) <= 4:
+        raise ValueError("benq_linear_multi takes 1 to 4 layers")
+    ydt = _ydt(layers[0][2])
+    arr = (BenQLayerC * len(layers))()
+    for i, (codes, lut, y) in enumerate(layers):
+        N = codes.shape[0]
+        _want(codes, torch.uint8, "codes")
+        if codes.shape[1] != 3 * K // 4:
+            raise ValueError("codes must be [N, 3K/4]")
+        if lut.dtype not in (torch.bfloat16, torch.int16) or tuple(lut.shape) != (N, 64) or not lut.is_contiguous():
+            raise TypeError("lut must be a contiguous bf16 [N, 64] tensor")
+        if tuple(y.shape) != (B, N) or not y.is_contiguous() or _ydt(y) != ydt:
+            raise ValueError("each y must be contiguous [B, N] of the first y's dtype")
+        arr[i] = BenQLayerC(_ptr(codes), _ptr(lut), _ptr(y), N)
+    _check(_c("benq_linear_multi")(arr, len(layers), _ptr(x), ydt, B, K, _stream(stream)))
+    return [y for _, _, y in layers]
 
 
 def benq_linear_workspace_bytes(B: int, N: int, K: int) -> int:

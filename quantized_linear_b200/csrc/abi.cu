@@ -126,6 +126,27 @@ ql_status benq_linear_ws(const uint8_t *codes, const uint16_t *lut, const uint16
   return ql::benq_gemm_launch(codes, lut, x, y, y_dtype, B, N, K, workspace, ws_bytes, s);
 }
 
+ql_status benq_linear_multi(const benq_layer *layers, int S, const uint16_t *x, ql_out_dtype y_dtype, int B, int K,
+                            ql_stream_t stream) {
+  g_msg[0] = 0;
+  if (!layers || !x) return fail(QL_ERR_INVALID_ARG, "benq_linear_multi: null pointer");
+  if (S < 1 || S > 4) return fail(QL_ERR_INVALID_ARG, "benq_linear_multi: S = %d must be in [1, 4]", S);
+  if (B <= 0 || K <= 0) return fail(QL_ERR_INVALID_ARG, "benq_linear_multi: B, K must be positive");
+  if (K % 4) return fail(QL_ERR_INVALID_ARG, "benq_linear_multi: K = %d is not a multiple of 4", K);
+  if (y_dtype != QL_OUT_F32 && y_dtype != QL_OUT_BF16) return fail(QL_ERR_INVALID_ARG, "benq_linear_multi: bad y_dtype");
+  if (!aligned(x, 16)) return fail(QL_ERR_ALIGNMENT, "benq_linear_multi: x must be 16-byte aligned");
+  for (int i = 0; i < S; ++i) {
+    const benq_layer &L = layers[i];
+    if (!L.codes || !L.lut || !L.y) return fail(QL_ERR_INVALID_ARG, "benq_linear_multi: null pointer in layer %d", i);
+    if (L.N <= 0) return fail(QL_ERR_INVALID_ARG, "benq_linear_multi: layer %d has N = %d", i, L.N);
+    if (!aligned(L.codes, 16) || !aligned(L.lut, 16) || !aligned(L.y, 16))
+      return fail(QL_ERR_ALIGNMENT, "benq_linear_multi: codes, lut and y of layer %d must be 16-byte aligned", i);
+    if (B > 16 && (K % 64 || L.N % 256))
+      return fail(QL_ERR_UNSUPPORTED, "benq_linear_multi: batch %d > 16 needs K %% 64 == 0 and N %% 256 == 0", B);
+  }
+  return ql::benq_gemv_multi_launch(layers, S, x, y_dtype, B, K, reinterpret_cast<cudaStream_t>(stream));
+}
+
 ql_status benq_dequant_debug(const uint8_t *codes, const uint16_t *lut, uint16_t *W, int N, int K,
                              ql_stream_t stream) {
   g_msg[0] = 0;

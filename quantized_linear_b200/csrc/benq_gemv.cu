@@ -21,6 +21,7 @@
 //    the C x 32 partials of each output are summed in a fixed order
 //    (deterministic), and the next block's codes and tables are already in flight.
 #include <algorithm>
+#include <climits>
 
 #include "ql_internal.cuh"
 
@@ -342,26 +343,59 @@ struct IntC {
   static constexpr int value = V;
 };
 
-// MLP: the gated MLP h = silu(x W_g^T) * (x W_u^T) in the same launch: codes / lut are W_g and
-// codes2 / lut2 W_u; a tile is two output features, its first row group the two gate rows and its
-// second the two up rows, and the tile's sums leave as silu(g) * u.
-template <bool MLP>
+// Up to B1_MAXSEG layers of the same K read in one launch (MODE B1_MULTI): layer s owns the row
+// tiles [tend[s - 1], tend[s]) of the launch (tend of unused entries is INT_MAX).
+constexpr int B1_MAXSEG = 4;
+struct B1Multi {
+  const uint8_t *codes[B1_MAXSEG];
+  const uint16_t *lut[B1_MAXSEG];
+  void *y[B1_MAXSEG];
+  int tend[B1_MAXSEG];
+};
+enum { B1_PLAIN = 0, B1_MLP = 1, B1_MULTI = 2 };
+
+// MODE B1_MLP: the gated MLP h = silu(x W_g^T) * (x W_u^T) in the same launch: codes / lut are W_g
+// and codes2 / lut2 W_u; a tile is two output features, its first row group the two gate rows and
+// its second the two up rows, and the tile's sums leave as silu(g) * u.  MODE B1_MULTI: the layers
+// of `ms` one after another, each tile taking its codes, tables and output from its own layer.
+template <int MODE>
 __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
     benq_gemv_b1_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ lut,
                         const uint8_t *__restrict__ codes2, const uint16_t *__restrict__ lut2,
-                        const uint16_t *__restrict__ x, void *__restrict__ y, int ydt, int N, int K) {
+                        const uint16_t *__restrict__ x, void *__restrict__ y, int ydt, int N, int K,
+                        const __grid_constant__ B1Multi ms) {
+  constexpr bool MLP = MODE == B1_MLP;
   __shared__ __align__(128) B1Tables tb;
   extern __shared__ __align__(16) float b1part[];  // [2][C][B1_T][32]
   const int C = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kc = warp * WARP_CODES + lane * LANE_CODES;
   const uint32_t rowbytes = 3u * K / 4;
-  const uint8_t *cbase = codes + 3u * kc / 4;
+  const uint8_t *cbase = MODE == B1_MULTI ? nullptr : codes + 3u * kc / 4;
   const uint8_t *cbase2 = MLP ? codes2 + 3u * kc / 4 : nullptr;
   constexpr int TOUT = MLP ? B1_T / 2 : B1_T;   // output features per tile
   const int ntile = N / TOUT;
   int tile = blockIdx.x;
   if (tile >= ntile) return;
+  // where tile t's rows live: this lane's code slice, the tables and the output, and the tile's index
+  // within its layer
+  struct Src {
+    const uint8_t *c;
+    const uint16_t *l;
+    void *yy;
+    int lt;
+  };
+  auto src_of = [&](int t) -> Src {
+    if constexpr (MODE == B1_MULTI) {
+      int sg = 0;
+#pragma unroll
+      for (int i = 1; i < B1_MAXSEG; ++i)
+        if (t >= ms.tend[i - 1]) sg = i;
+      return {ms.codes[sg] + 3u * kc / 4, ms.lut[sg], ms.y[sg], t - (sg ? ms.tend[sg - 1] : 0)};
+    } else {
+      return {cbase, lut, y, t};
+    }
+  };
   // Before waiting on the preceding kernel, pull this CTA's first tile of weights (codes and
   // tables) toward L2; prefetches hold no registers, so the loop below is compiled as if they
   // were absent.  Activations are loaded first after the wait: loading them after the codes
@@ -377,11 +411,12 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
       asm volatile("prefetch.global.L2 [%0];" ::"l"((threadIdx.x < TOUT ? lut : lut2) +
                                                       ((size_t)tile * TOUT + (threadIdx.x % TOUT)) * 64));
   } else {
-    const uint8_t *p = cbase + (size_t)tile * B1_T * rowbytes;
+    const Src sr = src_of(tile);
+    const uint8_t *p = sr.c + (size_t)sr.lt * B1_T * rowbytes;
 #pragma unroll
     for (int r = 0; r < B1_T; ++r) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (size_t)r * rowbytes));
     if (threadIdx.x < B1_T)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(lut + ((size_t)tile * B1_T + threadIdx.x) * 64));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(sr.l + ((size_t)sr.lt * B1_T + threadIdx.x) * 64));
   }
   qld::pdl_trigger();
   qld::pdl_wait();
@@ -399,8 +434,9 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
   // rows of tile t's row group grp (grp = 0, 1): B1_R consecutive rows of W, or for MLP the
   // tile's two gate rows (grp 0) and its two up rows (grp 1)
   auto load_rows = [&](int t, int grp, uint32_t (&w)[B1_R][6]) {
+    const Src sr = src_of(t);
     const uint8_t *p = MLP ? (grp == 0 ? cbase : cbase2) + (size_t)t * TOUT * rowbytes
-                           : cbase + (size_t)(t * B1_T + grp * B1_R) * rowbytes;
+                           : sr.c + (size_t)(sr.lt * B1_T + grp * B1_R) * rowbytes;
 #pragma unroll
     for (int r = 0; r < B1_R; ++r) {
       const uint2 a = ldg_u2(p + r * rowbytes), c = ldg_u2(p + r * rowbytes + 8), d = ldg_u2(p + r * rowbytes + 16);
@@ -410,8 +446,9 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
   auto load_lut = [&](int t, uint4 &v) {
     if (threadIdx.x < 8 * B1_T) {
       const int i = threadIdx.x >> 3;   // table row of the tile
+      const Src sr = src_of(t);
       const uint16_t *src = MLP ? (i < TOUT ? lut : lut2) + ((size_t)t * TOUT + (i % TOUT)) * 64
-                                : lut + ((size_t)t * B1_T + i) * 64;
+                                : sr.l + ((size_t)sr.lt * B1_T + i) * 64;
       v = ldg_u4(src + (threadIdx.x & 7) * 8);
     }
   };
@@ -484,17 +521,18 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
         }
       }
     } else {
+      const Src sr = src_of(tile);
       for (int o = warp; o < B1_T; o += C) {
         float s = 0.f;
         for (int c = 0; c < C; ++c) s += pr[(c * B1_T + o) * 32 + lane];
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
         if (lane == 0) {
-          const int n = tile * B1_T + o;
+          const int n = sr.lt * B1_T + o;
           if (ydt == QL_OUT_F32)
-            static_cast<float *>(y)[n] = s;
+            static_cast<float *>(sr.yy)[n] = s;
           else
-            static_cast<uint16_t *>(y)[n] = qld::f32_to_bf16_rn(s);
+            static_cast<uint16_t *>(sr.yy)[n] = qld::f32_to_bf16_rn(s);
         }
       }
     }
@@ -507,19 +545,23 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
   }
 }
 
-template <bool MLP>
+template <int MODE>
 ql_status launch_b1(const uint8_t *codes, const uint16_t *lut, const uint8_t *codes2, const uint16_t *lut2,
-                    const uint16_t *x, void *y, ql_out_dtype ydt, int N, int K, cudaStream_t s) {
+                    const uint16_t *x, void *y, ql_out_dtype ydt, int N, int K, cudaStream_t s,
+                    const B1Multi &ms = B1Multi{}) {
+  constexpr bool MLP = MODE == B1_MLP;
   const int C = K / WARP_CODES;
   const int threads = C * 32;
   const size_t smem = (size_t)2 * C * B1_T * 32 * sizeof(float);
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, benq_gemv_b1_kernel<MLP>, threads, smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, benq_gemv_b1_kernel<MODE>, threads, smem) != cudaSuccess ||
       per_sm < 1)
     return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
   const int grid = std::min(N / (MLP ? B1_T / 2 : B1_T), per_sm * ql::sm_count());
-  ql::launch(benq_gemv_b1_kernel<MLP>, grid, threads, smem, s, codes, lut, codes2, lut2, x, y, (int)ydt, N, K);
-  return ql::launch_status(MLP ? "benq_mlp_gate_up (batch-1 GEMV)" : "benq_linear (batch-1 GEMV)");
+  ql::launch(benq_gemv_b1_kernel<MODE>, grid, threads, smem, s, codes, lut, codes2, lut2, x, y, (int)ydt, N, K, ms);
+  return ql::launch_status(MODE == B1_MLP     ? "benq_mlp_gate_up (batch-1 GEMV)"
+                           : MODE == B1_MULTI ? "benq_linear_multi (batch-1 GEMV)"
+                                              : "benq_linear (batch-1 GEMV)");
 }
 
 template <int R, int BMAX>
@@ -562,7 +604,7 @@ ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint
                     aligned(x, 16);
   if (fast) {
     if (B == 1 && K % WARP_CODES == 0 && N % B1_T == 0)
-      return launch_b1<false>(codes, lut, nullptr, nullptr, x, y, ydt, N, K, s);
+      return launch_b1<B1_PLAIN>(codes, lut, nullptr, nullptr, x, y, ydt, N, K, s);
     if (B == 1) return launch_fast<4, 1>(codes, lut, x, y, ydt, B, N, K, s);
     if (B <= 2) return launch_fast<2, 2>(codes, lut, x, y, ydt, B, N, K, s);
     if (B <= 4) return launch_fast<2, 4>(codes, lut, x, y, ydt, B, N, K, s);
@@ -574,6 +616,37 @@ ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint
   const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count() * 8);
   launch(benq_gemv_generic_kernel, grid, threads, 0, s, codes, lut, x, y, (int)ydt, B, N, K);
   return launch_status("benq_linear (generic GEMV)");
+}
+
+// Several layers of the same K that read the same x: one batch-1 launch over all their row tiles
+// when every layer takes the batch-1 kernel, else one call per layer.
+ql_status benq_gemv_multi_launch(const benq_layer *layers, int S, const uint16_t *x, ql_out_dtype ydt, int B, int K,
+                                 cudaStream_t s) {
+  bool one = B == 1 && S <= B1_MAXSEG && K % WARP_CODES == 0 && K <= MAX_WARPS * WARP_CODES && aligned(x, 16);
+  for (int i = 0; i < S && one; ++i) one = layers[i].N % B1_T == 0 && aligned(layers[i].codes, 16);
+  if (!one) {
+    for (int i = 0; i < S; ++i) {
+      const ql_status st = B <= 16 ? benq_gemv_launch(layers[i].codes, layers[i].lut, x, layers[i].y, ydt, B, layers[i].N, K, s)
+                                   : benq_gemm_launch(layers[i].codes, layers[i].lut, x, layers[i].y, ydt, B, layers[i].N, K,
+                                                      nullptr, 0, s);
+      if (st != QL_OK) return st;
+    }
+    return QL_OK;
+  }
+  B1Multi ms{};
+  int rows = 0;
+  for (int i = 0; i < B1_MAXSEG; ++i) {
+    if (i < S) {
+      ms.codes[i] = layers[i].codes;
+      ms.lut[i] = layers[i].lut;
+      ms.y[i] = layers[i].y;
+      rows += layers[i].N;
+      ms.tend[i] = rows / B1_T;
+    } else {
+      ms.tend[i] = INT_MAX;
+    }
+  }
+  return launch_b1<B1_MULTI>(nullptr, nullptr, nullptr, nullptr, x, nullptr, ydt, rows, K, s, ms);
 }
 
 // ------------------------------------------------------------------------------- gated MLP
@@ -606,7 +679,7 @@ ql_status benq_mlp_launch(const uint8_t *codes_g, const uint16_t *lut_g, const u
                           const uint16_t *x, void *h, ql_out_dtype ydt, int B, int N, int K, void *ws, size_t ws_bytes,
                           cudaStream_t s) {
   // arguments validated by the caller (pointers 16-byte aligned, workspace large enough)
-  if (mlp_fused_shape(B, N, K)) return launch_b1<true>(codes_g, lut_g, codes_u, lut_u, x, h, ydt, N, K, s);
+  if (mlp_fused_shape(B, N, K)) return launch_b1<B1_MLP>(codes_g, lut_g, codes_u, lut_u, x, h, ydt, N, K, s);
   (void)ws_bytes;
   float *g = static_cast<float *>(ws), *u = g + (size_t)B * N;
   ql_status st = B <= 16 ? benq_gemv_launch(codes_g, lut_g, x, g, QL_OUT_F32, B, N, K, s)

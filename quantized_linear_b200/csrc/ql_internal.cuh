@@ -45,6 +45,8 @@ ql_status benq_dequant_launch(const uint8_t *codes, const uint16_t *lut, uint16_
                               cudaStream_t s);
 ql_status benq_gemv_launch(const uint8_t *codes, const uint16_t *lut, const uint16_t *x, void *y,
                            ql_out_dtype ydt, int B, int N, int K, cudaStream_t s);
+ql_status benq_gemv_multi_launch(const benq_layer *layers, int S, const uint16_t *x, ql_out_dtype ydt, int B,
+                                 int K, cudaStream_t s);
 size_t benq_gemm_workspace_size(int M, int N, int K);
 size_t benq_mlp_workspace_size(int B, int N, int K);
 ql_status benq_encode_launch(const uint16_t *W, uint8_t *codes, uint16_t *lut, int N, int K, int iters,

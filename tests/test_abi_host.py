@@ -98,6 +98,27 @@ def test_benq_argument_errors_are_caught_on_the_host(ql):
     assert g(A, A, A, 4, 10, None) == ql.QL_ERR_INVALID_ARG
 
 
+def test_multi_argument_errors_are_caught_on_the_host(ql):
+    f = _raw(ql, "benq_linear_multi")
+    A = 1 << 20    # never dereferenced: every call below fails validation first
+    arr = (ql.BenQLayerC * 5)()
+    for i in range(5):
+        arr[i] = ql.BenQLayerC(A, A, A, 8)
+    assert f(None, 1, A, 0, 1, 8, None) == ql.QL_ERR_INVALID_ARG              # no layers
+    assert f(arr, 0, A, 0, 1, 8, None) == ql.QL_ERR_INVALID_ARG               # S < 1
+    assert f(arr, 5, A, 0, 1, 8, None) == ql.QL_ERR_INVALID_ARG               # S > 4
+    assert f(arr, 2, A, 0, 1, 6, None) == ql.QL_ERR_INVALID_ARG               # K % 4
+    assert f(arr, 2, A + 2, 0, 1, 8, None) == ql.QL_ERR_ALIGNMENT             # x
+    arr[1] = ql.BenQLayerC(A, A, A + 4, 8)
+    assert f(arr, 2, A, 0, 1, 8, None) == ql.QL_ERR_ALIGNMENT                 # y of layer 1
+    arr[1] = ql.BenQLayerC(A, None, A, 8)
+    assert f(arr, 2, A, 0, 1, 8, None) == ql.QL_ERR_INVALID_ARG               # null table
+    arr[1] = ql.BenQLayerC(A, A, A, 0)
+    assert f(arr, 2, A, 0, 1, 8, None) == ql.QL_ERR_INVALID_ARG               # N
+    arr[1] = ql.BenQLayerC(A, A, A, 8)
+    assert f(arr, 2, A, 0, 32, 40, None) == ql.QL_ERR_UNSUPPORTED             # GEMM needs K % 64
+
+
 def test_mlp_argument_errors_are_caught_on_the_host(ql):
     f = _raw(ql, "benq_mlp_gate_up")
     A = 1 << 20    # never dereferenced: every call below fails validation first

@@ -221,3 +221,39 @@ def test_workspace_arguments(ql):
     assert raw(*args, ws.data_ptr() + 16, 1024, s) == ql.QL_ERR_ALIGNMENT
     assert raw(*args, ws.data_ptr(), 4096, s) == ql.QL_OK     # too small for a split: whole tiles
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("B,K,Ns", [(1, 5120, (5120, 1024, 1024)), (1, 2048, (8, 4, 100, 36)), (1, 1024, (4,)),
+                                    (3, 2048, (64, 32)), (1, 1000, (16, 8)), (20, 512, (256, 512))])
+def test_linear_multi_matches_each_layer(ql, B, K, Ns):
+    # several layers that read the same x (the attention projections q, k, v of the 27B-class layer
+    # first): every output equals benq_linear's result for that layer bit for bit, and the oracle's
+    # within the bar; batch 1 with K % 1024 == 0 runs one launch, the other shapes one call per layer
+    ws = [synth.benq_weights(N, K, seed=17 * N + K + i) for i, N in enumerate(Ns)]
+    x = synth.activations(B, K, seed=K + B)
+    xd = bf16(x)
+    for dt in (torch.float32, torch.bfloat16):
+        ys = [torch.full((B, w.N), float("nan"), dtype=dt, device="cuda") for w in ws]
+        ql.benq_linear_multi([(dev(w.codes), bits16(w.lut), y) for w, y in zip(ws, ys)], xd)
+        for w, y in zip(ws, ys):
+            ref = torch.empty(B, w.N, dtype=dt, device="cuda")
+            ql.benq_linear(dev(w.codes), bits16(w.lut), xd, ref)
+            torch.cuda.synchronize()
+            assert torch.equal(y, ref)
+            if dt == torch.float32:
+                assert max_rel(y.cpu().numpy(), ob.linear(w.codes, w.lut, x, K)) <= BENQ_TOL
+
+
+def test_linear_multi_argument_errors(ql):
+    w = synth.benq_weights(8, 1024, seed=3)
+    x = bf16(synth.activations(1, 1024, seed=4))
+    y = torch.empty(1, 8, device="cuda")
+    with pytest.raises(ValueError):
+        ql.benq_linear_multi([], x)
+    with pytest.raises(ValueError):
+        ql.benq_linear_multi([(dev(w.codes), bits16(w.lut), y)] * 5, x)
+    arr = (ql.BenQLayerC * 1)()
+    arr[0] = ql.BenQLayerC(dev(w.codes).data_ptr(), bits16(w.lut).data_ptr(), y.data_ptr() + 4, 8)
+    s = torch.cuda.current_stream().cuda_stream
+    assert ql.lib().benq_linear_multi(arr, 1, x.data_ptr(), ql.QL_OUT_F32, 1, 1024, s) == ql.QL_ERR_ALIGNMENT
+    assert ql.lib().benq_linear_multi(arr, 0, x.data_ptr(), ql.QL_OUT_F32, 1, 1024, s) == ql.QL_ERR_INVALID_ARG
