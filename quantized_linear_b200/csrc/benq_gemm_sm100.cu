@@ -88,7 +88,7 @@ struct Bars {
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     benq_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
                      const __grid_constant__ CUtensorMap map_y, int tstore, const uint16_t *__restrict__ lut, void *__restrict__ y, int ydt, int M, int N, int K,
-                     float *__restrict__ part_ws, unsigned *__restrict__ part_cnt, int full, int parts) {
+                     float *__restrict__ part_ws, unsigned *__restrict__ part_cnt, int full, int parts, int nfast) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -152,7 +152,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int it = 0;
       for (int wi = pair; wi < nitems && ok; wi += npairs) {
         const Item w = item_of(wi, full, parts, nkb);
-        const int m0 = (w.tile % mt) * PM + (int)rank * BM;
+        int mi, ni;
+        tile_mn(w.tile, mt, nt, nfast, mi, ni);
+        const int m0 = mi * PM + (int)rank * BM;
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % SA;
           if (it >= SA && !wt.wait(bar.empty_a + 8 * s, ((it / SA) & 1) ^ 1, true)) {
@@ -170,7 +172,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int ic = 0, tl = 0;
       for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
         const Item w = item_of(wi, full, parts, nkb);
-        const int n0 = (w.tile / mt) * BN + (int)rank * BNH;
+        int mi, ni;
+        tile_mn(w.tile, mt, nt, nfast, mi, ni);
+        const int n0 = ni * BN + (int)rank * BNH;
         const int ncs = (w.kb1 - w.kb0 + CKB - 1) / CKB;   // code stages; a ragged last one reads zeros
         if (tl > 0 && !wt.wait(bar.lut_empty, (tl - 1) & 1, false)) { ok = false; break; }
         sm100::mbar_arrive_expect_tx(bar.lut_full, LUT_BYTES);
@@ -255,7 +259,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         (dw >> 3) * 1024 + (dw & 7) * 128 + ((((lane & 15) >> 1) ^ (dw & 7)) << 4) + (lane & 1) * 8;
     for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
       const Item w = item_of(wi, full, parts, nkb);
-      const int m0 = (w.tile % mt) * PM + (int)rank * BM, n0 = (w.tile / mt) * BN;
+      int mi, ni;
+      tile_mn(w.tile, mt, nt, nfast, mi, ni);
+      const int m0 = mi * PM + (int)rank * BM, n0 = ni * BN;
       if (!wt.wait(bar.lut_full, tl & 1, false)) { ok = false; break; }
       for (int kb = w.kb0; kb < w.kb1;) {
         const bool two = kb + 1 < w.kb1;
@@ -547,8 +553,10 @@ ql_status benq_gemm_launch(const uint8_t *codes, const uint16_t *lut, const uint
   }
   const int nitems = plan.full + plan.leftover * plan.parts;
   const int pairs = std::min(nitems, resident);
+  // N-fastest tiles when the activations (2 bytes per element) outweigh the packed codes (0.75)
+  const int nfast = 2.0 * M > 0.75 * N ? 1 : 0;
   launch(benq_gemm_kernel, 2 * pairs, THREADS, SMEM_BYTES, s, mx, mc, my, tstore ? 1 : 0, lut, y, (int)ydt, M, N, K, part_ws, part_cnt,
-         plan.full, plan.parts);
+         plan.full, plan.parts, nfast);
   return launch_status("benq_linear (tensor-core GEMM)");
 }
 

@@ -395,7 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                      const __grid_constant__ CUtensorMap map_out, int tstore,
                      void *__restrict__ out, int ldo, int ovec, int ydt, const float *__restrict__ row_scale, int M,
                      int Nout, int nkb, float *__restrict__ part_ws, unsigned *__restrict__ part_cnt, int full,
-                     int parts) {
+                     int parts, int nfast) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -453,7 +453,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int it = 0;
       for (int wi = pair; wi < nitems && ok; wi += npairs) {
         const Item w = item_of(wi, full, parts, nkb);
-        const int m0 = (w.tile % mt) * PM + (int)rank * BM;
+        int mi, ni;
+        tile_mn(w.tile, mt, nt, nfast, mi, ni);
+        const int m0 = mi * PM + (int)rank * BM;
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % SA;
           if (it >= SA && !wt.wait(bar.empty_a + 8 * s, ((it / SA) & 1) ^ 1, true)) {
@@ -553,7 +555,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     int it = 0, tl = 0, ns = 0, ep = 0;
     for (int wi = pair; wi < nitems && ok; wi += npairs, ++tl) {
       const Item w = item_of(wi, full, parts, nkb);
-      const int m0 = (w.tile % mt) * PM + (int)rank * BM, n0 = (w.tile / mt) * BN;
+      int mi, ni;
+      tile_mn(w.tile, mt, nt, nfast, mi, ni);
+      const int m0 = mi * PM + (int)rank * BM, n0 = ni * BN;
       if constexpr (LK == 4) {
         // l <= 4, packed fp32 FMAs: warp dw rebuilds rows [32 rq, 32 rq + 32) x columns
         // [16 cq, 16 cq + 16) of this CTA's 128 x 64 block (rq = dw % 4, cq = dw / 4); lane (g, t)
@@ -1099,13 +1103,15 @@ void launch_gemms(const CUtensorMap &mx, const CUtensorMap &mt_, const OutMaps &
   unsigned *cnt1 = reinterpret_cast<unsigned *>(base + L.cnt);
   unsigned *cnt2 = reinterpret_cast<unsigned *>(base + L.cnt + L.g1.counter_bytes);
   const int items1 = L.g1.full + L.g1.leftover * L.g1.parts, items2 = L.g2.full + L.g2.leftover * L.g2.parts;
+  // N-fastest tiles when the activations (2 bytes per element) outweigh the sign bits (1/8 byte)
+  const int nfast1 = 16.0 * B > (double)P * L.seg ? 1 : 0, nfast2 = 16.0 * B > (double)n ? 1 : 0;
   ql::launch(mdbf_gemm_kernel<false, LK>, 2 * std::min(items1, resident), THREADS, SMEM_BYTES, s, mx, fg, om.mto, 1,
              static_cast<void *>(base + L.ts), P * L.seg, 1, 0, static_cast<const float *>(nullptr), B, P * L.seg,
-             L.mp / BK, part, cnt1, L.g1.full, L.g1.parts);
+             L.mp / BK, part, cnt1, L.g1.full, L.g1.parts, nfast1);
   ql::launch(mdbf_gemm_kernel<true, LK>, 2 * std::min(items2, resident), THREADS, SMEM_BYTES, s, mt_, ff, om.my,
              om.ystore ? 1 : 0, y, n,
              yvec ? 1 : 0, ydt, reinterpret_cast<const float *>(base + L.inv_s), B, n, P * L.seg / BK, part, cnt2,
-             L.g2.full, L.g2.parts);
+             L.g2.full, L.g2.parts, nfast2);
 }
 
 }  // namespace

@@ -148,6 +148,20 @@ __device__ __forceinline__ bool staged_tile_store(uint32_t tmem, uint32_t ring, 
   return wt.wait(stg_free, (ep - 1) & 1, false);
 }
 
+// M panel and N tile of pair tile t.  N-fastest (consecutive tiles, which run in the same wave, share
+// an activation panel) when the activations outweigh the weight stream the decoders read, else
+// M-fastest (they share a weight tile): the larger operand is then read from DRAM about once, and
+// the split last wave re-reads what the previous wave has just brought into L2.
+__device__ __forceinline__ void tile_mn(int t, int mt, int nt, int nfast, int &m, int &n) {
+  if (nfast) {
+    m = t / nt;
+    n = t - m * nt;
+  } else {
+    n = t / mt;
+    m = t - n * mt;
+  }
+}
+
 // Work items: pair tiles 0 .. full-1 whole, then each of the remaining tiles (the last, partial
 // wave) split into `parts` K ranges so that the otherwise idle pairs share it.  A split item
 // writes an fp32 partial; the last CTA to finish a tile sums the partials in part order.
