@@ -104,7 +104,7 @@ __device__ __forceinline__ uint4 pack_fragment(Get get, int qw, int nb, int lane
 // loaded before any is used, and the weights (B_amp) are pulled toward L2 before the wait on
 // the preceding kernel.
 __global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uint4 *__restrict__ out, int m, int l,
-                                   int B, int NB) {
+                                   int B, int NB, unsigned *__restrict__ cnt, int ncnt) {
   const int p = blockIdx.y;
   const int QW = (m + 31) / 32, V = l * B;
   const int64_t total = (int64_t)QW * NB * 32;
@@ -116,6 +116,9 @@ __global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uin
     }
   qld::pdl_trigger();
   qld::pdl_wait();
+  // the arrival counts of the split G stage that follows (the launch before this one has completed)
+  if (p == 0)
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < ncnt; e += gridDim.x * blockDim.x) cnt[e] = 0u;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
     const int lane = int(e & 31), g = lane >> 2, q = lane & 3;
     const int64_t f = e >> 5;
@@ -875,6 +878,219 @@ inline size_t f_nb1_smem(uint32_t sign_stride, uint32_t frag_bytes, int rows, in
          (size_t)8 * rows * B * 4;
 }
 
+// ------------------------------------------------------ G stage in split-K units (NB == 1) ----------
+// A unit is GS_ROWS = 128 rows of S_B of one path over one K slice, a run of 4-word groups.  Its
+// sign segments (one bulk copy per row, requested before the wait on pack z: signs are weights) and
+// the slice's z fragments (one bulk copy after the wait) sit in shared memory, where 16 warps (4 row
+// groups of 32 rows x 4 K-word groups) multiply them as the F stage does.  The K groups' sums are
+// added in group order.  With several slices per row block every unit writes its 128 x 8 partial
+// sums to the workspace and counts itself in; the last unit of the row block to arrive adds the
+// slices' partials in slice order (so the result does not depend on which unit that is) and runs
+// the epilogue
+//   t[k][b] = sum_i Q_V[k][i] u[k][b*l+i],  w[k][b*l+i] = Q_U[k][i] t[k][b],
+// writing the block's w as the F stage's packed fragments (4 words).  It also clears the count
+// for the next call; pack z clears the counts as well, so a fresh workspace needs no preparation.
+// Slices are sized so that the units fill the SMs: a row block of S_B per SM is too little work
+// for the 27B-class layers (r = 2886: 23 row blocks per path).  Used for long sign rows, where
+// each unit's shared-memory staging replaces many small ring copies per warp.
+constexpr int GS_RT = 2, GS_NRG = 4, GS_KG = 4, GS_ROWS = 16 * GS_RT * GS_NRG;
+constexpr int GS_SMAX = 16;   // slices per row block at most (sizes the workspace)
+
+struct GsLayout {
+  int S;              // K slices per row block
+  uint32_t sstride;   // bytes per sign row in shared memory (word count = 4 mod 8: conflict-free rows)
+  uint32_t frag_off;  // z fragments, then (after the products) the K groups' partial sums
+  uint32_t bar_off, total;
+};
+
+inline GsLayout gs_layout(int S, int m, int l, int B) {
+  const int QWm = (m + 31) / 32, G4 = (QWm + 3) / 4;
+  const int gps = (G4 + S - 1) / S;   // 4-word groups of the largest slice
+  int words = 4 * gps;
+  while (words % 8 != 4) words += 4;
+  GsLayout L;
+  L.S = S;
+  L.sstride = 4u * (uint32_t)words;
+  const uint32_t sign_bytes = (uint32_t)GS_ROWS * L.sstride;
+  // after the products the sign region holds the row sums D [128][8] and the w rows [128][V]
+  const uint32_t sign_region = std::max(sign_bytes, (uint32_t)(GS_ROWS * 8 + GS_ROWS * l * B) * 4);
+  L.frag_off = (sign_region + 127) / 128 * 128;
+  const uint32_t frag_region = std::max((uint32_t)(4 * gps) * 512, (uint32_t)(GS_KG * GS_ROWS * 8) * 4);
+  L.bar_off = L.frag_off + frag_region;
+  L.total = L.bar_off + 32;
+  return L;
+}
+
+__global__ void __launch_bounds__(GS_KG * GS_NRG * 32, 1)
+    mdbf_g_split_kernel(Paths ps, const uint4 *__restrict__ zpk, uint4 *__restrict__ wpk, float *__restrict__ part,
+                        unsigned *__restrict__ cnt, int m, int r, int l, int B, GsLayout L) {
+  constexpr int RT = GS_RT, NRG = GS_NRG, KG = GS_KG, ROWS = GS_ROWS;
+  extern __shared__ __align__(128) unsigned char gsm[];
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(gsm));
+  const int QWm = (m + 31) / 32, QWr = (r + 31) / 32, G4 = (QWm + 3) / 4, V = l * B;
+  const int nrb = (r + ROWS - 1) / ROWS, S = L.S;
+  const int unit = blockIdx.x, ks = unit % S, pr = unit / S, rb = pr % nrb, p = pr / nrb;
+  const int g0 = ks * G4 / S, g1 = (ks + 1) * G4 / S;
+  const int w0 = 4 * g0, wn = min(4 * g1, QWm) - w0;   // the slice's words of z
+  const int k0 = rb * ROWS, rows = min(ROWS, r - k0);
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const uint32_t sign_bar = base + L.bar_off, frag_bar = sign_bar + 8, flag_a = sign_bar + 16;
+  const size_t ld = ps.ldSB[p];
+  const uint32_t seg = 16u * (uint32_t)(g1 - g0);   // sign bytes of one row in the slice
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(sign_bar, 1);
+    sm100::mbar_init(frag_bar, 1);
+    sm100::fence_barrier_init();
+    sm100::mbar_arrive_expect_tx(sign_bar, (uint32_t)rows * seg);
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < rows)
+    sm100::bulk_g2s(base + threadIdx.x * L.sstride, ps.SB[p] + (size_t)(k0 + threadIdx.x) * ld + 16 * g0, seg,
+                    sign_bar);
+  {
+    // the epilogue's Q_V and Q_U rows (weights) toward L2
+    const int lines = (rows * l * 2 + 127) / 128;
+    if ((int)threadIdx.x < 2 * lines) {
+      const int which = threadIdx.x / lines, c = threadIdx.x - which * lines;
+      const char *src = reinterpret_cast<const char *>((which ? ps.QU[p] : ps.QV[p]) + (size_t)k0 * l);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(src + std::min(128 * c, rows * l * 2 - 1)));
+    }
+  }
+  qld::pdl_trigger();
+  qld::pdl_wait();
+  if (threadIdx.x == 0) {
+    sm100::mbar_arrive_expect_tx(frag_bar, (uint32_t)wn * 512);
+    sm100::bulk_g2s(base + L.frag_off, zpk + ((size_t)p * QWm + w0) * 32, (uint32_t)wn * 512, frag_bar);
+  }
+
+  bool ok = true;
+  const int rg = wid % NRG, kg = wid / NRG;
+  const int q0 = kg * wn / KG, q1 = (kg + 1) * wn / KG;
+  const int rbase = 16 * RT * rg;
+  float acc[RT][4];
+#pragma unroll
+  for (int t = 0; t < RT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  if (!sm100::mbar_wait(sign_bar, 0, FT_WAIT_BUDGET) || !sm100::mbar_wait(frag_bar, 0, FT_WAIT_BUDGET)) ok = false;
+  // rows past `rows` hold stale bytes: +-1 signs all the same, whose sums are never used
+  if (ok && rbase < rows) {
+    uint32_t r0[RT];
+#pragma unroll
+    for (int t = 0; t < RT; ++t) r0[t] = base + (rbase + 16 * t + g) * L.sstride;
+    const uint32_t fb = base + L.frag_off + lane * 16;
+    const uint32_t l8 = 8 * L.sstride;
+#pragma unroll 2
+    for (int qw = q0; qw < q1; ++qw) {
+      const uint4 bf = lds128(fb + qw * 512);
+      uint32_t s0[RT], s1[RT];
+#pragma unroll
+      for (int t = 0; t < RT; ++t) {
+        s0[t] = lds32s(r0[t] + 4 * qw);
+        s1[t] = lds32s(r0[t] + l8 + 4 * qw);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t ma = 1u << (15 - 8 * h - q), mb = 1u << (11 - 8 * h - q);
+#pragma unroll
+        for (int t = 0; t < RT; ++t) {
+          const uint32_t a0 = sign_pair_mul(s0[t], ma), a1 = sign_pair_mul(s1[t], ma),
+                         a2 = sign_pair_mul(s0[t], mb), a3 = sign_pair_mul(s1[t], mb);
+          mma16816(acc[t], a0, a1, a2, a3, h ? bf.z : bf.x, h ? bf.w : bf.y);
+        }
+      }
+    }
+  }
+  if (!ok) atomicExch(&g_mdbf_timeout, 1);
+  // A wait that ran out leaves its copy in flight: wait again (bounded) before the region is reused.
+  if (!ok && threadIdx.x == 0) {
+    (void)sm100::mbar_wait(sign_bar, 0, FT_WAIT_BUDGET);
+    (void)sm100::mbar_wait(frag_bar, 0, FT_WAIT_BUDGET);
+  }
+  __syncthreads();   // every warp is done with the fragments: their region takes the partial sums
+  float *const red = reinterpret_cast<float *>(gsm + L.frag_off);   // [KG][ROWS][8]
+#pragma unroll
+  for (int t = 0; t < RT; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      red[(kg * ROWS + rbase + 16 * t + g + 8 * (i >> 1)) * 8 + 2 * q + (i & 1)] = acc[t][i];
+  __syncthreads();
+  float *const D = reinterpret_cast<float *>(gsm);   // [ROWS][8], over the sign rows
+  float *const Ws = D + ROWS * 8;                     // [ROWS][V]
+  for (int e = threadIdx.x; e < ROWS * 8; e += blockDim.x) {
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < KG; ++k) sum += red[k * ROWS * 8 + e];
+    if (S == 1)
+      D[e] = sum;
+    else
+      part[(size_t)unit * ROWS * 8 + e] = sum;
+  }
+  if (S > 1) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const bool last = atomicAdd(cnt + pr, 1u) == (unsigned)S - 1;
+      if (last) atomicExch(cnt + pr, 0u);
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(flag_a), "r"(last ? 1u : 0u) : "memory");
+    }
+    __syncthreads();
+    uint32_t last;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(last) : "r"(flag_a) : "memory");
+    if (!last) return;
+    __threadfence();
+    const float *pb = part + (size_t)pr * S * ROWS * 8;
+    for (int e = threadIdx.x; e < ROWS * 8; e += blockDim.x) {
+      float sum = 0.f;
+      for (int s2 = 0; s2 < S; ++s2) sum += __ldcg(pb + (size_t)s2 * ROWS * 8 + e);
+      D[e] = sum;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < ROWS * B; e += blockDim.x) {
+    const int rr = e / B, b = e - rr * B, k = k0 + rr;
+    float *wo = Ws + rr * V + b * l;
+    if (k >= r) {
+      for (int i = 0; i < l; ++i) wo[i] = 0.f;
+      continue;
+    }
+    const float *Dr = D + rr * 8;
+    const uint16_t *qv = ps.QV[p] + (int64_t)k * l, *qu = ps.QU[p] + (int64_t)k * l;
+    float t = 0.f;
+    for (int i = 0; i < l; ++i) t = fmaf(qld::f16_to_f32(qv[i]), Dr[b * l + i] + Dr[V + b * l + i], t);
+    for (int i = 0; i < l; ++i) wo[i] = qld::f16_to_f32(qu[i]) * t;
+  }
+  __syncthreads();
+  if (threadIdx.x < ROWS) {
+    const int qw = k0 / 32 + (threadIdx.x >> 5);
+    if (qw < QWr) {
+      auto get = [&](int c, int v) { return Ws[(c - k0) * V + v]; };
+      wpk[((size_t)p * QWr + qw) * 32 + lane] = pack_fragment(get, qw, 0, lane, r, V);
+    }
+  }
+}
+
+// The split G stage for a layer, if its shared memory fits: slices enough to fill the SMs, more
+// if a slice would not fit.
+struct GsPlan {
+  bool ok;
+  int units;
+  GsLayout L;
+};
+inline GsPlan gs_plan(int P, int m, int r, int l, int B) {
+  GsPlan gp{};
+  const int nrb = (r + GS_ROWS - 1) / GS_ROWS, G4 = ((m + 31) / 32 + 3) / 4;
+  const int smax = std::min(GS_SMAX, G4);
+  for (int S = std::max(1, std::min(smax, ql::sm_count() / (P * nrb))); S <= smax; ++S) {
+    const GsLayout L = gs_layout(S, m, l, B);
+    if (L.total <= 227 * 1024) {
+      gp.ok = true;
+      gp.units = P * nrb * S;
+      gp.L = L;
+      return gp;
+    }
+  }
+  return gp;
+}
+
 // ---------------------------------------------------------------- debug dequantizer ----------
 __device__ __forceinline__ float envelope(const uint16_t *L, const uint16_t *R, int l) {
   float e = qld::f16_to_f32(L[0]) * qld::f16_to_f32(R[0]);
@@ -951,9 +1167,27 @@ int nb_for(int V) {
   return nb;
 }
 
+// workspace: packed z fragments, packed w fragments, and for NB == 1 the split G stage's partial
+// sums and arrival counts
+struct WsLayout {
+  size_t zpk, wpk, part, cnt, total;
+};
+WsLayout ws_layout(int P, int m, int r, int l, int B) {
+  const int NB = nb_for(l * B), nrb = (r + GS_ROWS - 1) / GS_ROWS;
+  WsLayout L;
+  L.zpk = 0;
+  L.wpk = align256((size_t)P * ((m + 31) / 32) * NB * 32 * sizeof(uint4));
+  L.part = L.wpk + align256((size_t)P * ((r + 31) / 32) * NB * 32 * sizeof(uint4));
+  const int smax = std::min(GS_SMAX, ((m + 31) / 32 + 3) / 4);   // as gs_plan: at most one slice per 4-word group
+  const size_t part_bytes = NB == 1 && smax > 1 ? (size_t)P * nrb * smax * GS_ROWS * 8 * sizeof(float) : 0;
+  L.cnt = L.part + align256(part_bytes);
+  L.total = L.cnt + (NB == 1 ? align256((size_t)P * nrb * sizeof(unsigned)) : 0);
+  return L;
+}
+
 template <int NB, int RTF, bool VEC16>
 ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk,
-                         uint4 *wpk, void *y, ql_out_dtype ydt, cudaStream_t s) {
+                         uint4 *wpk, float *part, unsigned *cnt, void *y, ql_out_dtype ydt, cudaStream_t s) {
   const size_t smg = (size_t)(SP_WARPS * 2 * NB * 128 + 32 * 8 * NB + 32 * l * B) * sizeof(float);
   const size_t smf = (size_t)(SP_WARPS * RTF * NB * 128 + RTF * 16 * 8 * NB + RTF * 16 * B) * sizeof(float);
   auto kg = mdbf_g_mma_kernel<NB, VEC16>;
@@ -970,14 +1204,27 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
         cudaSuccess)
       return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
   }
+  // the split G stage for NB == 1 on long sign rows (m >= 8192: 256 words or more), when its shared
+  // memory fits; shorter rows keep the ring kernel, which is faster there (27B-class gate/up,
+  // m = 5120: 26.5 against 28.1 us per call; down, m = 17408: 33.4 against 35.4 us)
+  GsPlan gsp{};
+  if constexpr (VEC16 && NB == 1)
+    if (m >= 8192) gsp = gs_plan(P, m, r, l, B);
   {
     const int64_t total = (int64_t)((m + 31) / 32) * NB * 32;
     const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)ql::sm_count() * 4);
-    ql::launch(mdbf_pack_z_kernel, dim3(grid, P), 256, 0, s, ps, x, zpk, m, l, B, NB);
+    ql::launch(mdbf_pack_z_kernel, dim3(grid, P), 256, 0, s, ps, x, zpk, m, l, B, NB, cnt,
+               gsp.ok && gsp.L.S > 1 ? P * ((r + GS_ROWS - 1) / GS_ROWS) : 0);
     ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
-  if constexpr (g_ring)
+  if (gsp.ok) {
+    if (cudaFuncSetAttribute(mdbf_g_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsp.L.total) !=
+        cudaSuccess)
+      return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
+    ql::launch(mdbf_g_split_kernel, gsp.units, GS_KG * GS_NRG * 32, gsp.L.total, s, ps, (const uint4 *)zpk, wpk, part,
+               cnt, m, r, l, B, gsp.L);
+  } else if constexpr (g_ring)
     ql::launch(mdbf_g_tile_kernel<NB>, dim3((r + 31) / 32, P), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
                m, r, l, B);
   else
@@ -1033,35 +1280,23 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
 
 template <int NB, bool VEC16>
 ql_status run_nb(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk, uint4 *wpk,
-                 void *y, ql_out_dtype ydt, cudaStream_t s) {
+                 float *part, unsigned *cnt, void *y, ql_out_dtype ydt, cudaStream_t s) {
   // two 16-row tiles per F block once there are enough rows to fill the machine twice over
   if (NB == 1 && n >= 16 * 2 * 4 * ql::sm_count())
-    return run_mma_stages<NB, 2, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
-  return run_mma_stages<NB, 1, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+    return run_mma_stages<NB, 2, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+  return run_mma_stages<NB, 1, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
 }
 
 template <bool VEC16>
 ql_status run_vec(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk,
-                  uint4 *wpk, void *y, ql_out_dtype ydt, cudaStream_t s) {
+                  uint4 *wpk, float *part, unsigned *cnt, void *y, ql_out_dtype ydt, cudaStream_t s) {
   switch (nb_for(l * B)) {
-    case 1: return run_nb<1, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
-    case 2: return run_nb<2, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
-    case 4: return run_nb<4, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
-    case 8: return run_nb<8, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
-    default: return run_nb<16, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+    case 1: return run_nb<1, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+    case 2: return run_nb<2, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+    case 4: return run_nb<4, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+    case 8: return run_nb<8, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+    default: return run_nb<16, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
   }
-}
-
-struct WsLayout {
-  size_t zpk, wpk, total;
-};
-WsLayout ws_layout(int P, int m, int r, int l, int B) {
-  const int NB = nb_for(l * B);
-  WsLayout L;
-  L.zpk = 0;
-  L.wpk = align256((size_t)P * ((m + 31) / 32) * NB * 32 * sizeof(uint4));
-  L.total = L.wpk + align256((size_t)P * ((r + 31) / 32) * NB * 32 * sizeof(uint4));
-  return L;
 }
 
 }  // namespace
@@ -1112,12 +1347,14 @@ ql_status mdbf_decode_launch(const mdbf_path *paths, int P, int n, int m, int r,
   char *base = static_cast<char *>(ws);
   uint4 *zpk = reinterpret_cast<uint4 *>(base + L.zpk);
   uint4 *wpk = reinterpret_cast<uint4 *>(base + L.wpk);
+  float *part = reinterpret_cast<float *>(base + L.part);
+  unsigned *cnt = reinterpret_cast<unsigned *>(base + L.cnt);
   bool vec16 = true;
   for (int p = 0; p < P; ++p)
     vec16 = vec16 && paths[p].ldSA % 16 == 0 && paths[p].ldSB % 16 == 0 && aligned(paths[p].S_A, 16) &&
             aligned(paths[p].S_B, 16);
-  if (vec16) return run_vec<true>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
-  return run_vec<false>(ps, P, n, m, r, l, B, x, zpk, wpk, y, ydt, s);
+  if (vec16) return run_vec<true>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+  return run_vec<false>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
 }
 
 ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W, float *F,

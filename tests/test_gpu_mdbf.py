@@ -173,3 +173,22 @@ def test_linear_long_sign_rows(ql, n, m, r, l, P, B):
     assert max_rel(y.cpu().numpy(), om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
     for _ in range(2):
         assert torch.equal(_linear(ql, paths, n, m, r, l, x), y)
+
+
+@pytest.mark.parametrize("n,m,r,l,P,B", [(700, 9000, 333, 2, 2, 2), (1100, 8192, 1000, 4, 1, 1), (200, 16400, 130, 1, 2, 4)])
+def test_linear_split_g_stage(ql, n, m, r, l, P, B):
+    # sign rows of 8192 columns or more run the G stage in split-K units (128 rows x a K slice, the
+    # slices' partial sums added by the last unit of each row block): ragged m and r, one and two
+    # paths; a workspace full of stale bytes (arrival counts included) gives the same result, and
+    # repeated calls are bit-identical whichever unit of a row block arrives last
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=5800 + m + r)
+    xbits = synth.activations(B, m, seed=5900 + B)
+    y = _linear(ql, paths, n, m, r, l, xbits)
+    assert max_rel(y.cpu().numpy(), om.linear_factored(paths, n, m, r, xbits)) <= MDBF_TOL
+    dp = mdbf_dev_paths(paths)
+    ws = torch.full((ql.mdbf_workspace_bytes(P, n, m, r, l, B),), 0xA5, dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        y2 = torch.empty(B, n, device="cuda")
+        ql.mdbf_linear(dp, n, m, r, l, bf16(xbits), y2, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y2, y)
