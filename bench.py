@@ -131,8 +131,11 @@ def L_multi(parts, K, label):
                 out="f32")
 
 
-def L_mdbf(P, n, m, r, l, B, seed, label, out="f32"):
-    return dict(kind="mdbf", P=P, n=n, m=m, r=r, l=l, B=B, seed=seed, label=label, out=out)
+def L_mdbf(P, n, m, r, l, B, seed, label, out="f32", group=None, group_skip=False):
+    """An MDBF layer.  Layers with the same `group` read one x and run as one mdbf_linear_multi call,
+    issued by the first of them (the others have `group_skip`)."""
+    return dict(kind="mdbf", P=P, n=n, m=m, r=r, l=l, B=B, seed=seed, label=label, out=out, group=group,
+                group_skip=group_skip)
 
 
 # BenQ weight seeds: one matrix per shape and role, shared between the records that use it
@@ -142,8 +145,8 @@ SEED_GATE, SEED_DOWN, SEED_UP = 1001, 1002, 1003
 def layer_set(attention, mlp):
     """One decoder layer's linears at batch 1: the BenQ attention projections (q, k, v, o) when
     `attention` ("fused": q, k and v in one call), then the MLP: "benq" (gate, up, down),
-    "benq_fused" (gate and up in one call with the SiLU gate, then down) or "mdbf" (gate, up, down
-    in MDBF)."""
+    "benq_fused" (gate and up in one call with the SiLU gate, then down), "mdbf" (gate, up, down
+    in MDBF) or "mdbf_multi" (the MDBF gate and up in one mdbf_linear_multi call, then down)."""
     out = []
     if attention == "fused":
         out += [L_multi([(HIDDEN, 5001, "q"), (1024, 5002, "k"), (1024, 5003, "v")], HIDDEN, "benq_qkv"),
@@ -159,8 +162,12 @@ def layer_set(attention, mlp):
         out += [L_benq(HIDDEN, INTER, 1, SEED_DOWN, "benq_down")]
     if mlp == "mdbf":
         out += [L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 1, 5008, "mdbf_gate"),
-                L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 1, 5009, "mdbf_up"),
-                L_mdbf(MLP_P, HIDDEN, INTER, MLP_R, MLP_L, 1, 5010, "mdbf_down")]
+                L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 1, 5009, "mdbf_up")]
+    if mlp == "mdbf_multi":
+        out += [L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 1, 5008, "mdbf_gate", group="gate_up"),
+                L_mdbf(MLP_P, INTER, HIDDEN, MLP_R, MLP_L, 1, 5009, "mdbf_up", group="gate_up", group_skip=True)]
+    if mlp in ("mdbf", "mdbf_multi"):
+        out += [L_mdbf(MLP_P, HIDDEN, INTER, MLP_R, MLP_L, 1, 5010, "mdbf_down")]
     return out
 
 
@@ -185,7 +192,9 @@ RECORDS = {
         ("benq_fused_mlp", layer_set(True, "benq_fused"), "rotate"),
         ("benq_4_launches", layer_set("fused", "benq_fused"), "rotate"),
         ("mdbf_mlp", layer_set(False, "mdbf"), "rotate"),
-        ("mixed_benq_attention_mdbf_mlp", layer_set(True, "mdbf"), "rotate")])],
+        ("mdbf_mlp_2_calls", layer_set(False, "mdbf_multi"), "rotate"),
+        ("mixed_benq_attention_mdbf_mlp", layer_set(True, "mdbf"), "rotate"),
+        ("mixed_5_calls", layer_set("fused", "mdbf_multi"), "rotate")])],
     "mdbf": [("cfg4_mdbf_mlp_27b", [("b1", layer_set(False, "mdbf"), "rotate")])],
     # the l = 1 cases (DBF at P = 1, LittleBit at P = 2) on the square layer, next to cfg3's l = 2
     "mdbf_l1": [("next4_mdbf_l1_4096", [
@@ -249,6 +258,8 @@ def layer_launches(L):
     MDBF batched envelope prep, activation prep and the two GEMMs."""
     if L["kind"] in ("benq", "benq_mlp", "benq_multi"):
         return 1
+    if L.get("group_skip"):   # run by its group's first layer
+        return 0
     return 4 if is_gemm(L) else 3
 
 
@@ -384,6 +395,15 @@ class Inputs:
                                       dtype=torch.uint8, device=cuda)
             L["w"] = [w0] + [self.clone(w0) for _ in range(copies - 1)]
             self.layers.append(L)
+        # layers of one group read the first one's x; its workspace serves all of their paths
+        for L in self.layers:
+            if L.get("group") and not L.get("group_skip"):
+                members = [M for M in self.layers if M.get("group") == L["group"]]
+                for M in members[1:]:
+                    M["x_h"], M["x"] = L["x_h"], L["x"]
+                L["group_members"] = members
+                L["ws"] = torch.empty(ql.mdbf_workspace_bytes(len(members) * L["P"], L["n"], L["m"], L["r"], L["l"],
+                                                              L["B"]), dtype=torch.uint8, device=cuda)
 
     @classmethod
     def benq_device_weights(cls, N, K, seed, ql, torch):
@@ -414,6 +434,12 @@ class Inputs:
             ql.benq_mlp_gate_up(*w, L["x"], L["y"])
         elif L["kind"] == "benq_multi":
             ql.benq_linear_multi([(c, t, y) for (c, t), y in zip(w, L["ys"])], L["x"])
+        elif L.get("group_skip"):
+            return
+        elif "group_members" in L:
+            ms = L["group_members"]
+            ql.mdbf_linear_multi([M["w"][c] for M in ms], L["n"], L["m"], L["r"], L["l"], L["x"], [M["y"] for M in ms],
+                                 L["ws"])
         else:
             ql.mdbf_linear(w, L["n"], L["m"], L["r"], L["l"], L["x"], L["y"], L["ws"])
 
@@ -533,17 +559,20 @@ class Timer:
         """The same steps through the public API with the inputs copied in from pinned host memory and
         the results copied back each step (eager calls); returns (ms, h2d bytes, d2h bytes) per run."""
         torch, n = self.torch, inp.copies
-        xs_h = [torch.from_numpy(np.ascontiguousarray(L["x_h"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        # a layer run by its group's first layer reads that layer's x: no copy of its own
+        xs_h = [None if L.get("group_skip") else
+                torch.from_numpy(np.ascontiguousarray(L["x_h"]).view(np.int16)).view(torch.bfloat16).pin_memory()
                 for L in layers]
         ys_h = [torch.empty(L["y"].shape, dtype=L["y"].dtype).pin_memory() for L in layers]
-        h2d = sum(t.numel() * t.element_size() for t in xs_h)
+        h2d = sum(t.numel() * t.element_size() for t in xs_h if t is not None)
         d2h = sum(t.numel() * t.element_size() for t in ys_h)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         self.sync_all()
         a.record(self.stream)
         for i in range(steps):
             for L, xh, yh in zip(layers, xs_h, ys_h):
-                L["x"].copy_(xh, non_blocking=True)
+                if xh is not None:
+                    L["x"].copy_(xh, non_blocking=True)
                 inp.run(self.ql, L, i % n)
                 yh.copy_(L["y"], non_blocking=True)
         b.record(self.stream)

@@ -238,6 +238,25 @@ QL_API ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r,
                       size_t ws_bytes, ql_stream_t stream);
 
 /*
+ * mdbf_linear_multi -- S MDBF layers of the same sizes that read the same x (the gate and up
+ *   projections of a gated MLP): y_s = W_s x for s < S, each exactly as mdbf_linear computes it
+ *   (the same kernels and arithmetic, bit for bit).
+ *   paths      host array of S * P paths, layer s's paths at [s * P, s * P + P).
+ *   S, P       layers and paths per layer: 1 <= S <= 4, S * P <= 8.
+ *   ys         host array of S device outputs, each [B][n] of y_dtype (4-byte aligned), fully
+ *              overwritten.
+ *   workspace  device scratch of ws_bytes >= mdbf_workspace_bytes(S * P, n, m, r, l, B), 256-byte
+ *              aligned; contents on entry are ignored and on return undefined.
+ *   Execution: where the layers run the decode kernels with the one-pass F stage (l * B <= 4, at
+ *   most two paths per layer, 16-byte aligned sign rows), each of the three launches covers all
+ *   layers, so S layers take three launches instead of 3 S.  Otherwise the layers run one after
+ *   another as mdbf_linear calls on the same workspace.  Other sizes and limits as mdbf_linear.
+ */
+QL_API ql_status mdbf_linear_multi(const mdbf_path *paths, int S, int P, int n, int m, int r, int l,
+                                   const uint16_t *x, void *const *ys, ql_out_dtype y_dtype, int B,
+                                   void *workspace, size_t ws_bytes, ql_stream_t stream);
+
+/*
  * mdbf_linear_noalloc -- mdbf_linear for callers that cannot allocate device memory.
  *   The paper has no counterpart: this is a deployment convenience.  Some callers can't call
  *   cudaMalloc (or must not: allocator-internal code, real-time threads that may not block in

@@ -48,6 +48,8 @@ _SIGNATURES = {
     "benq_bits_per_weight": (_d, [_i]),
     "mdbf_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "mdbf_linear": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _sz, _vp]),
+    "mdbf_linear_multi": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _i, _vp, ctypes.POINTER(_vp), _i, _i,
+                               _vp, _sz, _vp]),
     "mdbf_dequant_debug": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "mdbf_linear_noalloc": (_i, [ctypes.POINTER(MDBFPathC), _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp]),
     "mdbf_noalloc_scratch_bytes": (_sz, []),
@@ -80,7 +82,7 @@ def _c(name):
 
 EXPORTS = ["benq_linear", "benq_linear_ws", "benq_linear_workspace_bytes", "benq_linear_multi", "benq_mlp_gate_up",
            "benq_mlp_workspace_bytes", "benq_encode", "benq_dequant_debug", "benq_bits_per_weight", "mdbf_workspace_bytes", "mdbf_linear",
-           "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
+           "mdbf_linear_multi", "mdbf_linear_noalloc", "mdbf_noalloc_scratch_bytes", "mdbf_dequant_debug", "mdbf_effective_bits",
            "mdbf_select_rank", "ql_last_error", "ql_check", "ql_set_pdl", "ql_selftest_timeout"]
 
 
@@ -272,6 +274,31 @@ def mdbf_linear(paths, n, m, r, l, x, y, workspace, stream=None):
     _check(_c("mdbf_linear")(arr, len(arr), n, m, r, l, _ptr(x), _ptr(y), _ydt(y), B, _ptr(workspace),
                         workspace.numel() * workspace.element_size(), _stream(stream)))
     return y
+
+
+def mdbf_linear_multi(layers, n, m, r, l, x, ys, workspace, stream=None):
+    """y_s[B, n] = x[B, m] @ W_s^T for S MDBF layers of the same sizes that read the same x (the gate and
+    up projections of an MLP), bit for bit as mdbf_linear gives each; at decode batches the three
+    launches cover all layers.  layers: S lists of P paths each (dicts / objects as for mdbf_linear);
+    ys: S outputs [B, n] of one dtype; workspace: at least mdbf_workspace_bytes(S * P, n, m, r, l, B)
+    bytes."""
+    _want(x, torch.bfloat16, "x")
+    B = x.shape[0]
+    S = len(layers)
+    if S != len(ys) or not 1 <= S <= 4:
+        raise ValueError("mdbf_linear_multi takes 1 to 4 layers and one output per layer")
+    P = len(layers[0])
+    if any(len(lp) != P for lp in layers):
+        raise ValueError("every layer must have the same number of paths")
+    if x.shape[1] != m or any(tuple(y.shape) != (B, n) or not y.is_contiguous() for y in ys):
+        raise ValueError("x must be [B, m] and every y [B, n]")
+    if any(y.dtype != ys[0].dtype for y in ys):
+        raise TypeError("all outputs must have one dtype")
+    arr = mdbf_paths_c([p for lp in layers for p in lp])
+    yp = (_vp * S)(*[_ptr(y) for y in ys])
+    _check(_c("mdbf_linear_multi")(arr, S, P, n, m, r, l, _ptr(x), yp, _ydt(ys[0]), B, _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+    return ys
 
 
 def mdbf_linear_noalloc(paths, n, m, r, l, x, y, stream=None):

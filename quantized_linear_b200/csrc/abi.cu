@@ -199,6 +199,31 @@ ql_status mdbf_linear(const mdbf_path *paths, int P, int n, int m, int r, int l,
                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
+ql_status mdbf_linear_multi(const mdbf_path *paths, int S, int P, int n, int m, int r, int l, const uint16_t *x,
+                            void *const *ys, ql_out_dtype y_dtype, int B, void *workspace, size_t ws_bytes,
+                            ql_stream_t stream) {
+  g_msg[0] = 0;
+  if (S < 1 || S > 4) return fail(QL_ERR_INVALID_ARG, "mdbf_linear_multi: S = %d must be in [1, 4]", S);
+  if (P < 1 || S * P > 8) return fail(QL_ERR_INVALID_ARG, "mdbf_linear_multi: S * P = %d must be in [1, 8]", S * P);
+  ql_status st = check_paths("mdbf_linear_multi", paths, S * P, n, m, r, l);
+  if (st != QL_OK) return st;
+  if (!x || !ys || !workspace) return fail(QL_ERR_INVALID_ARG, "mdbf_linear_multi: null x, ys or workspace");
+  if (B <= 0) return fail(QL_ERR_INVALID_ARG, "mdbf_linear_multi: B must be positive");
+  if (y_dtype != QL_OUT_F32 && y_dtype != QL_OUT_BF16)
+    return fail(QL_ERR_INVALID_ARG, "mdbf_linear_multi: bad y_dtype");
+  if (!aligned(x, 2) || !aligned(workspace, 256))
+    return fail(QL_ERR_ALIGNMENT, "mdbf_linear_multi: x 2- and workspace 256-byte alignment required");
+  for (int s = 0; s < S; ++s) {
+    if (!ys[s]) return fail(QL_ERR_INVALID_ARG, "mdbf_linear_multi: null output %d", s);
+    if (!aligned(ys[s], 4)) return fail(QL_ERR_ALIGNMENT, "mdbf_linear_multi: output %d must be 4-byte aligned", s);
+  }
+  const size_t need = ql::mdbf_workspace_size(S * P, n, m, r, l, B);
+  if (ws_bytes < need)
+    return fail(QL_ERR_INVALID_ARG, "mdbf_linear_multi: workspace %zu < %zu bytes", ws_bytes, need);
+  return ql::mdbf_linear_multi_launch(paths, S, P, n, m, r, l, x, ys, y_dtype, B, workspace,
+                                      reinterpret_cast<cudaStream_t>(stream));
+}
+
 ql_status mdbf_linear_noalloc(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x, void *y,
                               ql_out_dtype y_dtype, int B, ql_stream_t stream) {
   g_msg[0] = 0;

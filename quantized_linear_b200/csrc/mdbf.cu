@@ -722,16 +722,24 @@ __global__ void __launch_bounds__(NRG * 32 * KG)
 // added in group order.  Paths are summed inside each lane in p order.  One barrier per CTA,
 // before the group sums.
 constexpr int F1_PMAX = 2;
+constexpr int LAYERS_MAX = 4;
+// outputs of the layers of one launch (mdbf_linear_multi); one entry for a single layer
+struct LayerOuts {
+  void *y[LAYERS_MAX];
+};
 
 template <int RT, int NRG>
 __global__ void __launch_bounds__(NRG * 32 * 8)
-    mdbf_f_nb1_kernel(Paths ps, int P, const uint4 *__restrict__ wpk, void *__restrict__ y, int ydt, int n, int r,
-                      int l, int B, uint32_t sign_stride, uint32_t frag_bytes) {
+    mdbf_f_nb1_kernel(Paths ps, int P, const uint4 *__restrict__ wpk, const __grid_constant__ LayerOuts outs, int ydt,
+                      int n, int r, int l, int B, uint32_t sign_stride, uint32_t frag_bytes) {
   constexpr int KG = 8, TILES = RT * NRG, ROWS = 16 * TILES;
   extern __shared__ __align__(128) unsigned char fsm[];
   const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(fsm));
   const int QW = (r + 31) / 32, V = l * B;
-  const int row0 = blockIdx.x * ROWS, rows = min(ROWS, n - row0);
+  // layer of this CTA (several layers of one x in one launch): its paths are [p0, p0 + P)
+  const int nfb = (n + ROWS - 1) / ROWS, layer = blockIdx.x / nfb, p0 = layer * P;
+  void *const y = outs.y[layer];
+  const int row0 = (blockIdx.x - layer * nfb) * ROWS, rows = min(ROWS, n - row0);
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
   const int rg = wid % NRG, kg = wid / NRG;
   const int qw0 = kg * QW / KG, qw1 = (kg + 1) * QW / KG;
@@ -747,20 +755,20 @@ __global__ void __launch_bounds__(NRG * 32 * 8)
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(abort_a), "r"(0u) : "memory");
     sm100::fence_barrier_init();
     for (int p = 0; p < P; ++p) {
-      const uint32_t sbytes = (uint32_t)(rows * ps.ldSA[p]);
+      const uint32_t sbytes = (uint32_t)(rows * ps.ldSA[p0 + p]);
       sm100::mbar_arrive_expect_tx(bars + 8 * p, sbytes + frag_bytes);
-      sm100::bulk_g2s(base + p * sign_stride, ps.SA[p] + (size_t)row0 * ps.ldSA[p], sbytes, bars + 8 * p);
+      sm100::bulk_g2s(base + p * sign_stride, ps.SA[p0 + p] + (size_t)row0 * ps.ldSA[p0 + p], sbytes, bars + 8 * p);
     }
   }
   for (int e = threadIdx.x; e < P * rows * l; e += blockDim.x) {
     const int pp = e / (rows * l), j = e - pp * (rows * l);
-    a_sm[pp * ROWS * l + j] = ps.A[pp][(int64_t)row0 * l + j];
+    a_sm[pp * ROWS * l + j] = ps.A[p0 + pp][(int64_t)row0 * l + j];
   }
   qld::pdl_trigger();
   qld::pdl_wait();
   // the w fragments are made by the G stage: copied after the wait
   if (threadIdx.x == 0)
-    for (int p = 0; p < P; ++p) sm100::bulk_g2s(frag_base + p * frag_bytes, wpk + (size_t)p * QW * 32, frag_bytes, bars + 8 * p);
+    for (int p = 0; p < P; ++p) sm100::bulk_g2s(frag_base + p * frag_bytes, wpk + (size_t)(p0 + p) * QW * 32, frag_bytes, bars + 8 * p);
   __syncthreads();
 
   bool ok = true;
@@ -776,7 +784,7 @@ __global__ void __launch_bounds__(NRG * 32 * 8)
     if (!sm100::mbar_wait(bars + 8 * p, 0, FT_WAIT_BUDGET)) ok = false;
     if (!ok || !live || qw0 >= qw1) continue;
     const uint32_t sb = base + p * sign_stride;
-    const uint32_t ldp = (uint32_t)ps.ldSA[p];
+    const uint32_t ldp = (uint32_t)ps.ldSA[p0 + p];
     uint32_t r0[RT];
 #pragma unroll
     for (int t = 0; t < RT; ++t) r0[t] = sb + (rbase + 16 * t + g) * ldp;
@@ -1185,9 +1193,15 @@ WsLayout ws_layout(int P, int m, int r, int l, int B) {
   return L;
 }
 
+// The three launches of a decode call.  S layers of P paths each (S > 1 only where the F stage is
+// mdbf_f_nb1_kernel, see nb1_fits): pack z and the G stage run over all S * P paths, whose
+// workspace entries are laid out path by path; the F stage sums each layer's paths into its output.
 template <int NB, int RTF, bool VEC16>
-ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk,
-                         uint4 *wpk, float *part, unsigned *cnt, void *y, ql_out_dtype ydt, cudaStream_t s) {
+ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int l, int B, const uint16_t *x,
+                         uint4 *zpk, uint4 *wpk, float *part, unsigned *cnt, const LayerOuts &outs, ql_out_dtype ydt,
+                         cudaStream_t s) {
+  const int PT = S * P;
+  void *const y = outs.y[0];
   const size_t smg = (size_t)(SP_WARPS * 2 * NB * 128 + 32 * 8 * NB + 32 * l * B) * sizeof(float);
   const size_t smf = (size_t)(SP_WARPS * RTF * NB * 128 + RTF * 16 * 8 * NB + RTF * 16 * B) * sizeof(float);
   auto kg = mdbf_g_mma_kernel<NB, VEC16>;
@@ -1213,8 +1227,8 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
   {
     const int64_t total = (int64_t)((m + 31) / 32) * NB * 32;
     const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)ql::sm_count() * 4);
-    ql::launch(mdbf_pack_z_kernel, dim3(grid, P), 256, 0, s, ps, x, zpk, m, l, B, NB, cnt,
-               gsp.ok && gsp.L.S > 1 ? P * ((r + GS_ROWS - 1) / GS_ROWS) : 0);
+    ql::launch(mdbf_pack_z_kernel, dim3(grid, PT), 256, 0, s, ps, x, zpk, m, l, B, NB, cnt,
+               gsp.ok && gsp.L.S > 1 ? PT * ((r + GS_ROWS - 1) / GS_ROWS) : 0);
     ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
@@ -1222,20 +1236,20 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
     if (cudaFuncSetAttribute(mdbf_g_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsp.L.total) !=
         cudaSuccess)
       return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-    ql::launch(mdbf_g_split_kernel, gsp.units, GS_KG * GS_NRG * 32, gsp.L.total, s, ps, (const uint4 *)zpk, wpk, part,
+    ql::launch(mdbf_g_split_kernel, S * gsp.units, GS_KG * GS_NRG * 32, gsp.L.total, s, ps, (const uint4 *)zpk, wpk, part,
                cnt, m, r, l, B, gsp.L);
   } else if constexpr (g_ring)
-    ql::launch(mdbf_g_tile_kernel<NB>, dim3((r + 31) / 32, P), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
+    ql::launch(mdbf_g_tile_kernel<NB>, dim3((r + 31) / 32, PT), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
                m, r, l, B);
   else
-    ql::launch(kg, dim3((r + 31) / 32, P), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
+    ql::launch(kg, dim3((r + 31) / 32, PT), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
   ql_status st = ql::launch_status("mdbf_linear (G stage)");
   if (st != QL_OK) return st;
   if constexpr (VEC16 && NB == 1) {
     if (P <= F1_PMAX) {
       // both paths in one pass: 128-row CTAs when they fill the SMs, else 32-row ones
       size_t ld_max = 0;
-      for (int p = 0; p < P; ++p) ld_max = std::max(ld_max, ps.ldSA[p]);
+      for (int p = 0; p < PT; ++p) ld_max = std::max(ld_max, ps.ldSA[p]);
       const bool big = (n + 127) / 128 >= ql::sm_count() * 3 / 4;
       const int rows = big ? 128 : 32;
       const uint32_t sign_stride = (uint32_t)((rows * ld_max + 127) / 128 * 128);
@@ -1245,12 +1259,13 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
         auto kt = big ? mdbf_f_nb1_kernel<2, 4> : mdbf_f_nb1_kernel<2, 1>;
         if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
           return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-        ql::launch(kt, (n + rows - 1) / rows, (big ? 4 : 1) * 32 * 8, sm, s, ps, P, (const uint4 *)wpk, y, (int)ydt, n,
-                   r, l, B, sign_stride, frag_bytes);
+        ql::launch(kt, S * ((n + rows - 1) / rows), (big ? 4 : 1) * 32 * 8, sm, s, ps, P, (const uint4 *)wpk, outs,
+                   (int)ydt, n, r, l, B, sign_stride, frag_bytes);
         return ql::launch_status("mdbf_linear (F stage)");
       }
     }
   }
+  if (S > 1) return ql::fail(QL_ERR_UNSUPPORTED, "mdbf_linear_multi: layers in one launch need the one-pass F stage");
   if constexpr (VEC16) {
     // staged-tile F stage when two (else one) path stages fit in shared memory
     size_t ld_max = 0;
@@ -1279,24 +1294,42 @@ ql_status run_mma_stages(const Paths &ps, int P, int n, int m, int r, int l, int
 }
 
 template <int NB, bool VEC16>
-ql_status run_nb(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk, uint4 *wpk,
-                 float *part, unsigned *cnt, void *y, ql_out_dtype ydt, cudaStream_t s) {
+ql_status run_nb(const Paths &ps, int S, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk,
+                 uint4 *wpk, float *part, unsigned *cnt, const LayerOuts &outs, ql_out_dtype ydt, cudaStream_t s) {
   // two 16-row tiles per F block once there are enough rows to fill the machine twice over
   if (NB == 1 && n >= 16 * 2 * 4 * ql::sm_count())
-    return run_mma_stages<NB, 2, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
-  return run_mma_stages<NB, 1, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+    return run_mma_stages<NB, 2, VEC16>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
+  return run_mma_stages<NB, 1, VEC16>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
 }
 
 template <bool VEC16>
-ql_status run_vec(const Paths &ps, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk,
-                  uint4 *wpk, float *part, unsigned *cnt, void *y, ql_out_dtype ydt, cudaStream_t s) {
+ql_status run_vec(const Paths &ps, int S, int P, int n, int m, int r, int l, int B, const uint16_t *x, uint4 *zpk,
+                  uint4 *wpk, float *part, unsigned *cnt, const LayerOuts &outs, ql_out_dtype ydt, cudaStream_t s) {
   switch (nb_for(l * B)) {
-    case 1: return run_nb<1, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
-    case 2: return run_nb<2, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
-    case 4: return run_nb<4, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
-    case 8: return run_nb<8, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
-    default: return run_nb<16, VEC16>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+    case 1: return run_nb<1, VEC16>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
+    case 2: return run_nb<2, VEC16>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
+    case 4: return run_nb<4, VEC16>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
+    case 8: return run_nb<8, VEC16>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
+    default: return run_nb<16, VEC16>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
   }
+}
+
+// Whether S > 1 layers can share the decode launches: their F stage must be the one-pass kernel
+// (NB == 1, at most two paths per layer, 16-byte aligned sign rows, its shared memory within the
+// limit); the same test run_mma_stages makes before it picks that kernel.
+bool nb1_fits(const mdbf_path *paths, int PT, int P, int n, int r, int l, int B) {
+  if (l * B > 4 || P > F1_PMAX) return false;
+  size_t ld_max = 0;
+  for (int p = 0; p < PT; ++p) {
+    if (paths[p].ldSA % 16 || paths[p].ldSB % 16 || !ql::aligned(paths[p].S_A, 16) || !ql::aligned(paths[p].S_B, 16))
+      return false;
+    ld_max = std::max(ld_max, paths[p].ldSA);
+  }
+  const bool big = (n + 127) / 128 >= ql::sm_count() * 3 / 4;
+  const int rows = big ? 128 : 32;
+  const uint32_t sign_stride = (uint32_t)((rows * ld_max + 127) / 128 * 128);
+  const uint32_t frag_bytes = (uint32_t)((r + 31) / 32) * 32 * 16;
+  return f_nb1_smem(sign_stride, frag_bytes, rows, l, B) <= 227 * 1024;
 }
 
 }  // namespace
@@ -1319,42 +1352,64 @@ size_t mdbf_workspace_size(int P, int n, int m, int r, int l, int B) {
   return ws_layout(P, m, r, l, B).total;
 }
 
-ql_status mdbf_decode_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x, void *y,
-                             ql_out_dtype ydt, int B, void *ws, cudaStream_t s);
+ql_status mdbf_decode_launch(const mdbf_path *paths, int S, int P, int n, int m, int r, int l, const uint16_t *x,
+                             const LayerOuts &outs, ql_out_dtype ydt, int B, void *ws, cudaStream_t s);
 
 ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x,
                              void *y, ql_out_dtype ydt, int B, void *ws, cudaStream_t s) {
   if (P > PMAX) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: P = %d exceeds %d paths", P, PMAX);
-  if (l * B <= VLIM) return mdbf_decode_launch(paths, P, n, m, r, l, x, y, ydt, B, ws, s);
+  LayerOuts outs{};
+  outs.y[0] = y;
+  if (l * B <= VLIM) return mdbf_decode_launch(paths, 1, P, n, m, r, l, x, outs, ydt, B, ws, s);
   if (mdbf_use_gemm(n, m, r, l, B, VLIM)) return mdbf_gemm_launch(paths, P, n, m, r, l, x, y, ydt, B, ws, s);
   if (l > VLIM) return fail(QL_ERR_UNSUPPORTED, "mdbf_linear: l = %d exceeds %d", l, VLIM);
   const int bc = VLIM / l;
   const size_t ysz = ydt == QL_OUT_F32 ? 4 : 2;
   for (int b0 = 0; b0 < B; b0 += bc) {
-    const ql_status st = mdbf_decode_launch(paths, P, n, m, r, l, x + (size_t)b0 * m,
-                                            static_cast<char *>(y) + (size_t)b0 * n * ysz, ydt, std::min(bc, B - b0),
-                                            ws, s);
+    outs.y[0] = static_cast<char *>(y) + (size_t)b0 * n * ysz;
+    const ql_status st = mdbf_decode_launch(paths, 1, P, n, m, r, l, x + (size_t)b0 * m, outs, ydt,
+                                            std::min(bc, B - b0), ws, s);
     if (st != QL_OK) return st;
   }
   return QL_OK;
 }
 
-// The decode kernels: one pass for l * B <= VLIM token rows.
-ql_status mdbf_decode_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, const uint16_t *x, void *y,
-                             ql_out_dtype ydt, int B, void *ws, cudaStream_t s) {
-  const Paths ps = pack_paths(paths, P);
-  const WsLayout L = ws_layout(P, m, r, l, B);
+// S layers of one x: one set of decode launches for all of them where their F stage is the one-pass
+// kernel, else the layers one after another (the workspace, sized for S * P paths, serves each).
+ql_status mdbf_linear_multi_launch(const mdbf_path *paths, int S, int P, int n, int m, int r, int l, const uint16_t *x,
+                                   void *const *ys, ql_out_dtype ydt, int B, void *ws, cudaStream_t s) {
+  if (S < 1 || S > LAYERS_MAX || S * P > PMAX)
+    return fail(QL_ERR_UNSUPPORTED, "mdbf_linear_multi: %d layers of %d paths (at most %d layers and %d paths)", S, P,
+                LAYERS_MAX, PMAX);
+  if (S > 1 && l * B <= VLIM && nb1_fits(paths, S * P, P, n, r, l, B)) {
+    LayerOuts outs{};
+    for (int i = 0; i < S; ++i) outs.y[i] = ys[i];
+    return mdbf_decode_launch(paths, S, P, n, m, r, l, x, outs, ydt, B, ws, s);
+  }
+  for (int i = 0; i < S; ++i) {
+    const ql_status st = mdbf_linear_launch(paths + (size_t)i * P, P, n, m, r, l, x, ys[i], ydt, B, ws, s);
+    if (st != QL_OK) return st;
+  }
+  return QL_OK;
+}
+
+// The decode kernels: one pass for l * B <= VLIM token rows, S layers of P paths.
+ql_status mdbf_decode_launch(const mdbf_path *paths, int S, int P, int n, int m, int r, int l, const uint16_t *x,
+                             const LayerOuts &outs, ql_out_dtype ydt, int B, void *ws, cudaStream_t s) {
+  const int PT = S * P;
+  const Paths ps = pack_paths(paths, PT);
+  const WsLayout L = ws_layout(PT, m, r, l, B);
   char *base = static_cast<char *>(ws);
   uint4 *zpk = reinterpret_cast<uint4 *>(base + L.zpk);
   uint4 *wpk = reinterpret_cast<uint4 *>(base + L.wpk);
   float *part = reinterpret_cast<float *>(base + L.part);
   unsigned *cnt = reinterpret_cast<unsigned *>(base + L.cnt);
   bool vec16 = true;
-  for (int p = 0; p < P; ++p)
+  for (int p = 0; p < PT; ++p)
     vec16 = vec16 && paths[p].ldSA % 16 == 0 && paths[p].ldSB % 16 == 0 && aligned(paths[p].S_A, 16) &&
             aligned(paths[p].S_B, 16);
-  if (vec16) return run_vec<true>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
-  return run_vec<false>(ps, P, n, m, r, l, B, x, zpk, wpk, part, cnt, y, ydt, s);
+  if (vec16) return run_vec<true>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
+  return run_vec<false>(ps, S, P, n, m, r, l, B, x, zpk, wpk, part, cnt, outs, ydt, s);
 }
 
 ql_status mdbf_dequant_launch(const mdbf_path *paths, int P, int n, int m, int r, int l, float *W, float *F,

@@ -63,6 +63,9 @@ size_t mdbf_workspace_size(int P, int n, int m, int r, int l, int B);
 ql_status mdbf_linear_launch(const mdbf_path *paths, int P, int n, int m, int r, int l,
                              const uint16_t *x, void *y, ql_out_dtype ydt, int B, void *ws,
                              cudaStream_t s);
+ql_status mdbf_linear_multi_launch(const mdbf_path *paths, int S, int P, int n, int m, int r, int l,
+                                   const uint16_t *x, void *const *ys, ql_out_dtype ydt, int B, void *ws,
+                                   cudaStream_t s);
 ql_status mdbf_read_timeout(int *flag);   // reads and clears the MDBF kernels' bounded-wait flag
 // batched MDBF (l * B above the decode kernels' limit) on the tensor cores, mdbf_gemm_sm100.cu:
 // envelope ranks up to MDBF_GEMM_LMAX and layers whose n, m and r are all at least

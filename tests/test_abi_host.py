@@ -164,6 +164,28 @@ def test_mdbf_argument_errors_are_caught_on_the_host(ql):
     assert g(ok, 1, 64, 64, 32, 2, None, None, None, None) == ql.QL_ERR_INVALID_ARG
 
 
+def test_mdbf_multi_argument_errors_are_caught_on_the_host(ql):
+    f = _raw(ql, "mdbf_linear_multi")
+    A = 1 << 20    # never dereferenced: every call below fails validation first
+    ok = _fake_paths(ql, 8)
+    ws = ql.mdbf_workspace_bytes(4, 64, 64, 32, 2, 1)
+    ys = (ctypes.c_void_p * 4)(A, A, A, A)
+    assert f(ok, 0, 2, 64, 64, 32, 2, A, ys, 0, 1, A, ws, None) == ql.QL_ERR_INVALID_ARG    # S < 1
+    assert f(ok, 5, 1, 64, 64, 32, 2, A, ys, 0, 1, A, ws, None) == ql.QL_ERR_INVALID_ARG    # S > 4
+    assert f(ok, 3, 3, 64, 64, 32, 2, A, ys, 0, 1, A, ws, None) == ql.QL_ERR_INVALID_ARG    # S * P > 8
+    assert f(None, 2, 2, 64, 64, 32, 2, A, ys, 0, 1, A, ws, None) == ql.QL_ERR_INVALID_ARG  # no paths
+    assert f(ok, 2, 2, 64, 64, 32, 2, A, None, 0, 1, A, ws, None) == ql.QL_ERR_INVALID_ARG  # no outputs
+    assert f(ok, 2, 2, 64, 64, 32, 2, A, ys, 0, 1, A, ws - 1, None) == ql.QL_ERR_INVALID_ARG   # workspace
+    assert f(ok, 2, 2, 64, 64, 32, 2, A + 1, ys, 0, 1, A, ws, None) == ql.QL_ERR_ALIGNMENT     # x
+    bad = (ctypes.c_void_p * 2)(A, A + 2)
+    assert f(ok, 2, 2, 64, 64, 32, 2, A, bad, 0, 1, A, ws, None) == ql.QL_ERR_ALIGNMENT        # y of layer 1
+    none = (ctypes.c_void_p * 2)(A, None)
+    assert f(ok, 2, 2, 64, 64, 32, 2, A, none, 0, 1, A, ws, None) == ql.QL_ERR_INVALID_ARG     # null y
+    paths = _fake_paths(ql, 4)
+    paths[3] = ql.MDBFPathC(A, A, 2, 16, A, A, A, A)
+    assert f(paths, 2, 2, 64, 64, 32, 2, A, ys, 0, 1, A, ws, None) == ql.QL_ERR_INVALID_ARG    # stride of path 3
+
+
 def test_binding_fails_loudly_without_the_library(ql, monkeypatch, tmp_path):
     monkeypatch.setattr(ql, "_lib", None)
     monkeypatch.setattr(ql, "LIB_PATH", str(tmp_path / "missing.so"))

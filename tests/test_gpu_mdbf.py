@@ -192,3 +192,44 @@ def test_linear_split_g_stage(ql, n, m, r, l, P, B):
         ql.mdbf_linear(dp, n, m, r, l, bf16(xbits), y2, ws)
         torch.cuda.synchronize()
         assert torch.equal(y2, y)
+
+
+@pytest.mark.parametrize("S,P,n,m,r,l,B,aligned16,ydtype", [
+    (2, 2, 2048, 1536, 700, 4, 1, True, torch.float32),     # one launch per stage, ring G stage
+    (2, 2, 2048, 1536, 700, 4, 1, True, torch.bfloat16),
+    (3, 1, 500, 300, 200, 2, 2, True, torch.float32),       # three layers, l * B = 4
+    (2, 2, 600, 9000, 300, 4, 1, True, torch.float32),      # long sign rows: split G stage
+    (2, 2, 300, 200, 100, 4, 2, True, torch.float32),       # l * B = 8: the layers one after another
+    (2, 1, 300, 200, 100, 2, 1, False, torch.float32),      # 4-byte sign strides: one after another
+])
+def test_linear_multi_matches_each_layer(ql, S, P, n, m, r, l, B, aligned16, ydtype):
+    # mdbf_linear_multi gives each layer exactly what mdbf_linear gives it (same kernels, same
+    # arithmetic), whether the stages run once for all layers or the layers run in turn
+    kw = {} if aligned16 else {"ldSA": 20, "ldSB": 28}
+    layers = [synth.mdbf_paths(P, n, m, r, l, seed=6000 + 17 * s + m, **kw) for s in range(S)]
+    xbits = synth.activations(B, m, seed=6100 + B)
+    single = [_linear(ql, paths, n, m, r, l, xbits, ydtype) for paths in layers]
+    dls = [mdbf_dev_paths(paths) for paths in layers]
+    ws = torch.empty(ql.mdbf_workspace_bytes(S * P, n, m, r, l, B), dtype=torch.uint8, device="cuda")
+    ys = [torch.empty(B, n, dtype=ydtype, device="cuda") for _ in range(S)]
+    ql.mdbf_linear_multi(dls, n, m, r, l, bf16(xbits), ys, ws)
+    torch.cuda.synchronize()
+    for s in range(S):
+        assert torch.equal(ys[s], single[s]), s
+    if ydtype == torch.float32:
+        assert max_rel(ys[-1].cpu().numpy(), om.linear_factored(layers[-1], n, m, r, xbits)) <= MDBF_TOL
+
+
+def test_linear_multi_argument_errors(ql):
+    paths = synth.mdbf_paths(1, 64, 64, 32, 2, seed=6200)
+    dp = mdbf_dev_paths(paths)
+    x = bf16(synth.activations(1, 64, seed=6201))
+    ws = torch.empty(ql.mdbf_workspace_bytes(2, 64, 64, 32, 2, 1), dtype=torch.uint8, device="cuda")
+    y = torch.empty(1, 64, device="cuda")
+    with pytest.raises(ValueError):
+        ql.mdbf_linear_multi([dp] * 5, 64, 64, 32, 2, x, [y] * 5, ws)                # more than 4 layers
+    with pytest.raises(TypeError):
+        ql.mdbf_linear_multi([dp, dp], 64, 64, 32, 2, x, [y, y.to(torch.bfloat16)], ws)   # mixed dtypes
+    small = torch.empty(ql.mdbf_workspace_bytes(1, 64, 64, 32, 2, 1) - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ql.QLinearError):
+        ql.mdbf_linear_multi([dp, dp], 64, 64, 32, 2, x, [y, y.clone()], small)      # workspace for one layer
