@@ -175,12 +175,14 @@ def test_linear_long_sign_rows(ql, n, m, r, l, P, B):
         assert torch.equal(_linear(ql, paths, n, m, r, l, x), y)
 
 
-@pytest.mark.parametrize("n,m,r,l,P,B", [(700, 9000, 333, 2, 2, 2), (1100, 8192, 1000, 4, 1, 1), (200, 16400, 130, 1, 2, 4)])
+@pytest.mark.parametrize("n,m,r,l,P,B", [(700, 9000, 333, 2, 2, 2), (1100, 8192, 1000, 4, 1, 1), (200, 16400, 130, 1, 2, 4),
+                                         # one, two and three vectors (l * B = 1, 2, 3)
+                                         (600, 8200, 300, 1, 1, 1), (600, 8300, 300, 2, 2, 1), (600, 8192, 300, 3, 1, 1)])
 def test_linear_split_g_stage(ql, n, m, r, l, P, B):
     # sign rows of 8192 columns or more run the G stage in split-K units (128 rows x a K slice, the
     # slices' partial sums added by the last unit of each row block): ragged m and r, one and two
-    # paths; a workspace full of stale bytes (arrival counts included) gives the same result, and
-    # repeated calls are bit-identical whichever unit of a row block arrives last
+    # paths, one to four vectors; a workspace full of stale bytes (arrival counts included) gives the
+    # same result, and repeated calls are bit-identical whichever unit of a row block arrives last
     paths = synth.mdbf_paths(P, n, m, r, l, seed=5800 + m + r)
     xbits = synth.activations(B, m, seed=5900 + B)
     y = _linear(ql, paths, n, m, r, l, xbits)
