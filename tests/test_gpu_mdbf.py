@@ -203,6 +203,7 @@ def test_linear_split_g_stage(ql, n, m, r, l, P, B):
     (2, 2, 600, 9000, 300, 4, 1, True, torch.float32),      # long sign rows: split G stage
     (2, 2, 300, 200, 100, 4, 2, True, torch.float32),       # l * B = 8: the layers one after another
     (2, 1, 300, 200, 100, 2, 1, False, torch.float32),      # 4-byte sign strides: one after another
+    (2, 1, 256, 256, 128, 4, 20, True, torch.float32),      # l * B = 80: tensor-core GEMMs, in turn
 ])
 def test_linear_multi_matches_each_layer(ql, S, P, n, m, r, l, B, aligned16, ydtype):
     # mdbf_linear_multi gives each layer exactly what mdbf_linear gives it (same kernels, same
