@@ -42,6 +42,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -591,12 +592,19 @@ _KERNEL_SOURCES = {
 }
 
 
+_COMMENT = re.compile(r"/\*.*?\*/|//[^\n]*", re.S)
+
+
 def _kernel_source_sha(kernel_key):
+    """Hash of the code (comments and trailing blanks removed) of the sources a kernel's traffic
+    figure depends on: a comment edit leaves the figure valid, any code change voids it."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "quantized_linear_b200", "csrc")
     for f in _KERNEL_SOURCES[kernel_key]:
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            code = _COMMENT.sub("", fh.read())
+        code = "\n".join(line.rstrip() for line in code.splitlines() if line.strip())
+        h.update(f.encode() + code.encode())
     return h.hexdigest()[:16]
 
 

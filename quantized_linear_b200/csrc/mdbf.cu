@@ -720,7 +720,9 @@ __global__ void __launch_bounds__(NRG * 32 * KG)
 // high or low part of vector (b, i), so it adds A_amp[row][i] times its values into the row's sum
 // for b and the four lanes of a row combine them by shuffles; the K-word groups' sums are then
 // added in group order.  Paths are summed inside each lane in p order.  One barrier per CTA,
-// before the group sums.
+// before the group sums.  Several layers of one x (mdbf_linear_multi) share a launch: CTA i works on
+// layer i / (row blocks per layer), whose paths are P consecutive entries of the path list and
+// whose w fragments are those paths' entries of the workspace.
 constexpr int F1_PMAX = 2;
 constexpr int LAYERS_MAX = 4;
 // outputs of the layers of one launch (mdbf_linear_multi); one entry for a single layer
