@@ -177,7 +177,9 @@ def test_linear_long_sign_rows(ql, n, m, r, l, P, B):
 
 @pytest.mark.parametrize("n,m,r,l,P,B", [(700, 9000, 333, 2, 2, 2), (1100, 8192, 1000, 4, 1, 1), (200, 16400, 130, 1, 2, 4),
                                          # one, two and three vectors (l * B = 1, 2, 3)
-                                         (600, 8200, 300, 1, 1, 1), (600, 8300, 300, 2, 2, 1), (600, 8192, 300, 3, 1, 1)])
+                                         (600, 8200, 300, 1, 1, 1), (600, 8300, 300, 2, 2, 1), (600, 8192, 300, 3, 1, 1),
+                                         # a rank below one 32-row word
+                                         (100, 8500, 20, 4, 2, 1)])
 def test_linear_split_g_stage(ql, n, m, r, l, P, B):
     # sign rows of 8192 columns or more run the G stage in split-K units (128 rows x a K slice, the
     # slices' partial sums added by the last unit of each row block): ragged m and r, one and two
@@ -200,6 +202,7 @@ def test_linear_split_g_stage(ql, n, m, r, l, P, B):
     (2, 2, 2048, 1536, 700, 4, 1, True, torch.float32),     # one launch per stage, ring G stage
     (2, 2, 2048, 1536, 700, 4, 1, True, torch.bfloat16),
     (3, 1, 500, 300, 200, 2, 2, True, torch.float32),       # three layers, l * B = 4
+    (4, 2, 400, 9000, 120, 1, 1, True, torch.float32),      # four layers, eight paths (the limits), split G
     (2, 2, 600, 9000, 300, 4, 1, True, torch.float32),      # long sign rows: split G stage
     (2, 2, 300, 200, 100, 4, 2, True, torch.float32),       # l * B = 8: the layers one after another
     (2, 1, 300, 200, 100, 2, 1, False, torch.float32),      # 4-byte sign strides: one after another
