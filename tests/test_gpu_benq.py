@@ -78,10 +78,11 @@ def test_linear_fast_path_shapes(ql, N, K, B):
 
 
 @pytest.mark.parametrize("N,K", [(2, 1024), (6, 1024), (10, 2048), (4098, 1024), (1026, 17408), (2050, 20480),
-                                 (10242, 12288)])
+                                 (10242, 12288), (4096, 12288), (1032, 7168), (2052, 19456), (40, 8192)])
 def test_linear_batch1_row_counts(ql, N, K):
     # batch 1 with few rows (fewer row tiles than SMs), N % 4 == 2, one warp per CTA (K = 1024), 20
-    # warps (K = 20480) and CTAs that walk many row tiles (K = 12288, one CTA per SM)
+    # warps (K = 20480) and CTAs that walk many row tiles (K = 12288, one CTA per SM); 7, 8, 12 and 19
+    # warps per CTA with whole row tiles, and fewer row tiles than SMs
     w = synth.benq_weights(N, K, seed=N * 3 + K)
     x = synth.activations(1, K, seed=K + 1)
     y = _linear(ql, w, x).cpu().numpy()
@@ -257,3 +258,12 @@ def test_linear_multi_argument_errors(ql):
     s = torch.cuda.current_stream().cuda_stream
     assert ql.lib().benq_linear_multi(arr, 1, x.data_ptr(), ql.QL_OUT_F32, 1, 1024, s) == ql.QL_ERR_ALIGNMENT
     assert ql.lib().benq_linear_multi(arr, 0, x.data_ptr(), ql.QL_OUT_F32, 1, 1024, s) == ql.QL_ERR_INVALID_ARG
+
+
+def test_linear_batch1_long_rows_are_deterministic(ql):
+    # the warps' partial row sums are added in a fixed order
+    w = synth.benq_weights(4096, 17408, seed=77)
+    x = synth.activations(1, 17408, seed=78)
+    a = _linear(ql, w, x)
+    for _ in range(3):
+        assert torch.equal(_linear(ql, w, x), a)
