@@ -489,9 +489,12 @@ class Timer:
                     inp.run(self.ql, L, c)
         return g
 
-    def graphs(self, inp, layers):
+    def graphs(self, inp, layers, steps):
+        """Graphs of one rotation of the weight copies, of each single copy, and of the `steps` timed
+        steps in one piece (copies in turn), so that the timed region holds no graph boundary."""
         n = inp.copies
-        return {"cycle": self.capture(inp, layers, range(n)), "one": [self.capture(inp, layers, [c]) for c in range(n)]}
+        return {"cycle": self.capture(inp, layers, range(n)), "one": [self.capture(inp, layers, [c]) for c in range(n)],
+                "all": self.capture(inp, layers, [i % n for i in range(steps)]) if steps else None}
 
     def replay(self, gs, steps, n):
         for _ in range(steps // n):
@@ -509,13 +512,15 @@ class Timer:
         torch, n = self.torch, inp.copies
         self.replay(gs, max(self.warmup, n), n)
         if timing == "rotate":
+            gs["all"].replay()   # the first replay of a graph also uploads it
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             self.sync_all()
             a.record(self.stream)
-            self.replay(gs, steps, n)
+            gs["all"].replay()
             b.record(self.stream)
             self.sync_all()
             return max_over_ranks(a.elapsed_time(b), self.world)
+        gs["one"][0].replay()
         ev = []
         self.sync_all()
         for _ in range(steps):
@@ -693,7 +698,7 @@ def measure_variant(timer, layers, timing, steps, peaks, eager=False):
     for L in inp.layers:   # first calls outside any capture (kernel attributes, tensor maps)
         inp.run(timer.ql, L, 0)
     timer.torch.cuda.synchronize()
-    gs = timer.graphs(inp, inp.layers)
+    gs = timer.graphs(inp, inp.layers, steps if timing == "rotate" else 0)
     ms = timer.time_graph(inp, gs, steps, timing)
     us = 1e3 * ms / steps
     byts = sum(layer_bytes(L) for L in layers)

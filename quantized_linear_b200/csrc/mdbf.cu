@@ -888,6 +888,16 @@ inline size_t f_nb1_smem(uint32_t sign_stride, uint32_t frag_bytes, int rows, in
          (size_t)8 * rows * B * 4;
 }
 
+// Rows per CTA of mdbf_f_nb1_kernel for S layers of n rows: 32 or 64 when the CTAs then run in one
+// round on the SMs (each holds both paths' w fragments, so one CTA per SM is the norm), else 128.
+// The 27B-class down shape (n = 5120) takes 64: 80 CTAs, where 32-row ones ran 160 CTAs in two rounds.
+inline int nb1_rows(int S, int n) {
+  const int sms = ql::sm_count();
+  if (S * ((n + 31) / 32) <= sms) return 32;
+  if (S * ((n + 63) / 64) <= sms) return 64;
+  return 128;
+}
+
 // ------------------------------------------------------ G stage in split-K units (NB == 1) ----------
 // A unit is GS_ROWS = 128 rows of S_B of one path over one K slice, a run of 4-word groups.  Its
 // sign segments (one bulk copy per row, requested before the wait on pack z: signs are weights) and
@@ -1249,19 +1259,18 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
   if (st != QL_OK) return st;
   if constexpr (VEC16 && NB == 1) {
     if (P <= F1_PMAX) {
-      // both paths in one pass: 128-row CTAs when they fill the SMs, else 32-row ones
+      // both paths in one pass
       size_t ld_max = 0;
       for (int p = 0; p < PT; ++p) ld_max = std::max(ld_max, ps.ldSA[p]);
-      const bool big = (n + 127) / 128 >= ql::sm_count() * 3 / 4;
-      const int rows = big ? 128 : 32;
+      const int rows = nb1_rows(S, n);
       const uint32_t sign_stride = (uint32_t)((rows * ld_max + 127) / 128 * 128);
       const uint32_t frag_bytes = (uint32_t)((r + 31) / 32) * 32 * 16;
       const size_t sm = f_nb1_smem(sign_stride, frag_bytes, rows, l, B);
       if (sm <= 227 * 1024) {
-        auto kt = big ? mdbf_f_nb1_kernel<2, 4> : mdbf_f_nb1_kernel<2, 1>;
+        auto kt = rows == 128 ? mdbf_f_nb1_kernel<2, 4> : rows == 64 ? mdbf_f_nb1_kernel<2, 2> : mdbf_f_nb1_kernel<2, 1>;
         if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
           return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-        ql::launch(kt, S * ((n + rows - 1) / rows), (big ? 4 : 1) * 32 * 8, sm, s, ps, P, (const uint4 *)wpk, outs,
+        ql::launch(kt, S * ((n + rows - 1) / rows), rows / 32 * 32 * 8, sm, s, ps, P, (const uint4 *)wpk, outs,
                    (int)ydt, n, r, l, B, sign_stride, frag_bytes);
         return ql::launch_status("mdbf_linear (F stage)");
       }
@@ -1327,8 +1336,7 @@ bool nb1_fits(const mdbf_path *paths, int PT, int P, int n, int r, int l, int B)
       return false;
     ld_max = std::max(ld_max, paths[p].ldSA);
   }
-  const bool big = (n + 127) / 128 >= ql::sm_count() * 3 / 4;
-  const int rows = big ? 128 : 32;
+  const int rows = nb1_rows(PT / P, n);
   const uint32_t sign_stride = (uint32_t)((rows * ld_max + 127) / 128 * 128);
   const uint32_t frag_bytes = (uint32_t)((r + 31) / 32) * 32 * 16;
   return f_nb1_smem(sign_stride, frag_bytes, rows, l, B) <= 227 * 1024;

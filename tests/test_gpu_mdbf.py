@@ -131,13 +131,32 @@ def test_linear_is_deterministic(ql):
 
 @pytest.mark.parametrize("B", [1, 2])
 def test_linear_tall_layer_full_size_blocks(ql, B):
-    # n >= 128 x 148 rows: the F stage runs 128-row blocks (smaller n runs 32-row blocks)
+    # n >= 128 x 148 rows: the F stage runs 128-row blocks
     n, m, r, l, P = 20480, 1024, 256, 4, 2
     paths = synth.mdbf_paths(P, n, m, r, l, seed=5000 + B)
     x = synth.activations(B, m, seed=5100 + B)
     y = _linear(ql, paths, n, m, r, l, x).cpu().numpy()
     rows = np.r_[np.random.default_rng(4).choice(n, 256, replace=False), 0, 127, 128, n - 129, n - 1]
     assert max_rel(y[:, rows], om.linear_factored(paths, n, m, r, x, rows=rows)) <= MDBF_TOL
+
+
+@pytest.mark.parametrize("n,P,l,B", [(4700, 2, 4, 1), (6000, 2, 2, 2), (9400, 1, 4, 1), (9500, 2, 1, 4)])
+def test_linear_f_stage_row_blocks(ql, n, P, l, B):
+    # the one-pass F stage takes 32-row CTAs while they fit in one round on 148 SMs (n = 4700), then
+    # 64-row ones (n = 6000, a 48-row tail; n = 9400), then 128-row ones (n = 9500, a 28-row tail);
+    # the results match the oracle and do not depend on the row count per CTA (bit-identical to a
+    # two-layer call of the same layer, which halves the row count that fits)
+    m, r = 640, 300
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=5250 + n + P)
+    x = synth.activations(B, m, seed=5350 + B)
+    y = _linear(ql, paths, n, m, r, l, x)
+    assert max_rel(y.cpu().numpy(), om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+    dp = mdbf_dev_paths(paths)
+    ws = torch.empty(ql.mdbf_workspace_bytes(2 * P, n, m, r, l, B), dtype=torch.uint8, device="cuda")
+    ys = [torch.empty(B, n, device="cuda") for _ in range(2)]
+    ql.mdbf_linear_multi([dp, dp], n, m, r, l, bf16(x), ys, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], y) and torch.equal(ys[1], y)
 
 
 @pytest.mark.parametrize("l,B", [(4, 4), (4, 8), (2, 16)])
@@ -204,6 +223,7 @@ def test_linear_split_g_stage(ql, n, m, r, l, P, B):
     (3, 1, 500, 300, 200, 2, 2, True, torch.float32),       # three layers, l * B = 4
     (4, 2, 400, 9000, 120, 1, 1, True, torch.float32),      # four layers, eight paths (the limits), split G
     (2, 2, 600, 9000, 300, 4, 1, True, torch.float32),      # long sign rows: split G stage
+    (2, 2, 3000, 2000, 500, 2, 2, True, torch.float32),     # 64-row F blocks here, 32-row ones alone
     (2, 2, 300, 200, 100, 4, 2, True, torch.float32),       # l * B = 8: the layers one after another
     (2, 1, 300, 200, 100, 2, 1, False, torch.float32),      # 4-byte sign strides: one after another
     (2, 1, 256, 256, 128, 4, 20, True, torch.float32),      # l * B = 80: tensor-core GEMMs, in turn
