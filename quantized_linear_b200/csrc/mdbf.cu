@@ -305,11 +305,12 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_mma_kernel(Paths ps, con
     wpk[((size_t)p * QWr + qw) * NB * 32 + e] = pack_fragment(get, qw, e >> 5, e & 31, r, V);
 }
 
-// G stage as above, with each warp streaming its word groups through a private 4-stage ring in
+// G stage as above, with each warp streaming its word groups through a private STG-stage ring in
 // shared memory filled by cp.async: per group of SP_U words, lane (g, q) copies 16 bytes of sign
-// row g + 8q (the 32 rows of the block) and its own 16-byte fragment register sets, three groups
+// row g + 8q (the 32 rows of the block) and its own 16-byte fragment register sets, STG - 1 groups
 // ahead of the one being multiplied.  The first groups' signs are requested before the wait on
-// the preceding kernel.  Needs 16-byte aligned sign rows.
+// the preceding kernel.  Needs 16-byte aligned sign rows.  Four stages fit two CTAs per SM, three
+// stages three (NB = 1); the host takes three when the blocks would otherwise need a second round.
 constexpr int GR_STAGES = 4;
 
 // set when a bounded wait of an MDBF kernel runs out; read and cleared by ql_check()
@@ -339,20 +340,20 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 template <int NB>
 __host__ __device__ constexpr int g_ring_stage_bytes() { return 32 * 16 + SP_U * NB * 32 * 16; }
 
-template <int NB>
+template <int NB, int STG>
 __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, const uint4 *__restrict__ zpk,
                                                                       uint4 *__restrict__ wpk, int m, int r, int l,
                                                                       int B) {
   constexpr int STAGE = g_ring_stage_bytes<NB>();
   extern __shared__ __align__(128) unsigned char gsm[];
   const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(gsm));
-  float *red = reinterpret_cast<float *>(gsm + SP_WARPS * GR_STAGES * STAGE), *D = red + SP_WARPS * 2 * NB * 128,
+  float *red = reinterpret_cast<float *>(gsm + SP_WARPS * STG * STAGE), *D = red + SP_WARPS * 2 * NB * 128,
         *Ws = D + 32 * 8 * NB;
   const int p = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
   const int QW = (m + 31) / 32, V = l * B;
   const int row0 = blockIdx.x * 32;
   const size_t ld = ps.ldSB[p];
-  const uint32_t ring = sbase + warp * GR_STAGES * STAGE;
+  const uint32_t ring = sbase + warp * STG * STAGE;
   const uint4 *vb = zpk + (size_t)p * QW * NB * 32;
   // this lane's sign row (rows past r repeat the last row; their results are dropped)
   const uint8_t *srow = ps.SB[p] + (size_t)min(row0 + g + 8 * q, r - 1) * ld;
@@ -360,11 +361,11 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
   warp_words(QW, warp, w0, w1);
   const int ngroups = (w1 - w0 + SP_U - 1) / SP_U;
   auto issue_signs = [&](int grp) {
-    const uint32_t st = ring + (grp % GR_STAGES) * STAGE;
+    const uint32_t st = ring + (grp % STG) * STAGE;
     cp_async16(st + (g + 8 * q) * 16, srow + 4 * (w0 + SP_U * grp));   // 16 bytes: SP_U sign words
   };
   auto issue_frags = [&](int grp) {
-    const uint32_t st = ring + (grp % GR_STAGES) * STAGE + 32 * 16;
+    const uint32_t st = ring + (grp % STG) * STAGE + 32 * 16;
 #pragma unroll
     for (int u = 0; u < SP_U; ++u) {
       const int qw = min(w0 + SP_U * grp + u, QW - 1);   // words past the range are loaded but multiply zero-padding... see below
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
       for (int nb = 0; nb < NB; ++nb) cp_async16(st + ((u * NB + nb) * 32 + lane) * 16, vb + ((size_t)qw * NB + nb) * 32 + lane);
     }
   };
-  for (int grp = 0; grp < GR_STAGES - 1 && grp < ngroups; ++grp) issue_signs(grp);
+  for (int grp = 0; grp < STG - 1 && grp < ngroups; ++grp) issue_signs(grp);
   // The epilogue's Q_V and Q_U rows (weights) travel to shared memory with the first copy group
   // when both blocks start on 4-byte boundaries and hold whole 4-byte words; else the epilogue
   // reads them from global memory.
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
   }
   qld::pdl_trigger();
   qld::pdl_wait();
-  for (int grp = 0; grp < GR_STAGES - 1; ++grp) {
+  for (int grp = 0; grp < STG - 1; ++grp) {
     if (grp < ngroups) issue_frags(grp);
     cp_async_commit();
   }
@@ -404,9 +405,9 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
   for (int grp = 0; grp < ngroups; ++grp) {
-    cp_async_wait<GR_STAGES - 2>();
+    cp_async_wait<STG - 2>();
     __syncwarp();   // sign rows were copied by other lanes of the warp
-    const uint32_t st = ring + (grp % GR_STAGES) * STAGE;
+    const uint32_t st = ring + (grp % STG) * STAGE;
     uint32_t sw[SP_U][2][2];
 #pragma unroll
     for (int rt = 0; rt < 2; ++rt)
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) bf[u][nb] = lds128(st + 32 * 16 + ((u * NB + nb) * 32 + lane) * 16);
     __syncwarp();   // every lane has read this stage before it is refilled
-    const int nxt = grp + GR_STAGES - 1;
+    const int nxt = grp + STG - 1;
     if (nxt < ngroups) {
       issue_signs(nxt);
       issue_frags(nxt);
@@ -920,7 +921,9 @@ struct GsLayout {
   int S;              // K slices per row block
   uint32_t sstride;   // bytes per sign row in shared memory (word count = 4 mod 8: conflict-free rows)
   uint32_t frag_off;  // z fragments, then (after the products) the K groups' partial sums
-  uint32_t bar_off, total;
+  uint32_t bar_off;   // mbarriers and the last-unit flag (32 bytes)
+  uint32_t q_off;     // the block's Q_V rows, then its Q_U rows: [2][GS_ROWS][l] fp16
+  uint32_t total;
 };
 
 inline GsLayout gs_layout(int S, int m, int l, int B) {
@@ -937,7 +940,8 @@ inline GsLayout gs_layout(int S, int m, int l, int B) {
   L.frag_off = (sign_region + 127) / 128 * 128;
   const uint32_t frag_region = std::max((uint32_t)(4 * gps) * 512, (uint32_t)(GS_KG * GS_ROWS * 8) * 4);
   L.bar_off = L.frag_off + frag_region;
-  L.total = L.bar_off + 32;
+  L.q_off = L.bar_off + 32;
+  L.total = L.q_off + 2u * GS_ROWS * (uint32_t)l * 2u;
   return L;
 }
 
@@ -967,14 +971,13 @@ __global__ void __launch_bounds__(GS_KG * GS_NRG * 32, 1)
   if ((int)threadIdx.x < rows)
     sm100::bulk_g2s(base + threadIdx.x * L.sstride, ps.SB[p] + (size_t)(k0 + threadIdx.x) * ld + 16 * g0, seg,
                     sign_bar);
-  {
-    // the epilogue's Q_V and Q_U rows (weights) toward L2
-    const int lines = (rows * l * 2 + 127) / 128;
-    if ((int)threadIdx.x < 2 * lines) {
-      const int which = threadIdx.x / lines, c = threadIdx.x - which * lines;
-      const char *src = reinterpret_cast<const char *>((which ? ps.QU[p] : ps.QV[p]) + (size_t)k0 * l);
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(src + std::min(128 * c, rows * l * 2 - 1)));
-    }
+  // the epilogue's Q_V and Q_U rows (weights) into shared memory, before the wait: only the last
+  // unit of the row block uses them, and reading them there from global memory put a chain of
+  // dependent loads on the block's critical path
+  uint16_t *const qs = reinterpret_cast<uint16_t *>(gsm + L.q_off);
+  for (int e = threadIdx.x; e < 2 * rows * l; e += blockDim.x) {
+    const int which = e / (rows * l), j = e - which * (rows * l);
+    qs[which * ROWS * l + j] = (which ? ps.QU[p] : ps.QV[p])[(size_t)k0 * l + j];
   }
   qld::pdl_trigger();
   qld::pdl_wait();
@@ -1059,8 +1062,13 @@ __global__ void __launch_bounds__(GS_KG * GS_NRG * 32, 1)
     __threadfence();
     const float *pb = part + (size_t)pr * S * ROWS * 8;
     for (int e = threadIdx.x; e < ROWS * 8; e += blockDim.x) {
+      float v[GS_SMAX];   // every slice's load issued before the first add
+#pragma unroll
+      for (int s2 = 0; s2 < GS_SMAX; ++s2) v[s2] = s2 < S ? __ldcg(pb + (size_t)s2 * ROWS * 8 + e) : 0.f;
       float sum = 0.f;
-      for (int s2 = 0; s2 < S; ++s2) sum += __ldcg(pb + (size_t)s2 * ROWS * 8 + e);
+#pragma unroll
+      for (int s2 = 0; s2 < GS_SMAX; ++s2)
+        if (s2 < S) sum += v[s2];
       D[e] = sum;
     }
   }
@@ -1073,7 +1081,7 @@ __global__ void __launch_bounds__(GS_KG * GS_NRG * 32, 1)
       continue;
     }
     const float *Dr = D + rr * 8;
-    const uint16_t *qv = ps.QV[p] + (int64_t)k * l, *qu = ps.QU[p] + (int64_t)k * l;
+    const uint16_t *qv = qs + rr * l, *qu = qs + ROWS * l + rr * l;
     float t = 0.f;
     for (int i = 0; i < l; ++i) t = fmaf(qld::f16_to_f32(qv[i]), Dr[b * l + i] + Dr[V + b * l + i], t);
     for (int i = 0; i < l; ++i) wo[i] = qld::f16_to_f32(qu[i]) * t;
@@ -1208,6 +1216,15 @@ WsLayout ws_layout(int P, int m, int r, int l, int B) {
 // The three launches of a decode call.  S layers of P paths each (S > 1 only where the F stage is
 // mdbf_f_nb1_kernel, see nb1_fits): pack z and the G stage run over all S * P paths, whose
 // workspace entries are laid out path by path; the F stage sums each layer's paths into its output.
+// the ring G kernel with three stages (NB = 1 only, where that fits three CTAs per SM) or four
+template <int NB>
+auto ring_g_kernel(bool three) {
+  if constexpr (NB == 1)
+    return three ? mdbf_g_tile_kernel<1, 3> : mdbf_g_tile_kernel<1, GR_STAGES>;
+  else
+    return mdbf_g_tile_kernel<NB, GR_STAGES>;
+}
+
 template <int NB, int RTF, bool VEC16>
 ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int l, int B, const uint16_t *x,
                          uint4 *zpk, uint4 *wpk, float *part, unsigned *cnt, const LayerOuts &outs, ql_out_dtype ydt,
@@ -1224,10 +1241,11 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
   // G stage through per-warp cp.async rings when sign rows are 16-byte aligned and the vectors
   // are narrow (decode batches); wider ones keep mdbf_g_mma_kernel
   constexpr bool g_ring = VEC16 && NB <= 2;
-  const size_t smg_t = (size_t)SP_WARPS * GR_STAGES * g_ring_stage_bytes<NB>() + smg + (size_t)2 * 32 * l * 2;
+  const bool g_ring3 = NB == 1 && (int64_t)((r + 31) / 32) * PT > 2LL * ql::sm_count();   // three CTAs per SM
+  const size_t smg_t = (size_t)SP_WARPS * (g_ring3 ? 3 : GR_STAGES) * g_ring_stage_bytes<NB>() + smg + (size_t)2 * 32 * l * 2;
   if constexpr (g_ring) {
-    if (cudaFuncSetAttribute(mdbf_g_tile_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg_t) !=
-        cudaSuccess)
+    auto kg_ring = ring_g_kernel<NB>(g_ring3);
+    if (cudaFuncSetAttribute(kg_ring, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg_t) != cudaSuccess)
       return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
   }
   // the split G stage for NB == 1 on long sign rows (m >= 8192: 256 words or more), when its shared
@@ -1250,10 +1268,11 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
       return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
     ql::launch(mdbf_g_split_kernel, S * gsp.units, GS_KG * GS_NRG * 32, gsp.L.total, s, ps, (const uint4 *)zpk, wpk, part,
                cnt, m, r, l, B, gsp.L);
-  } else if constexpr (g_ring)
-    ql::launch(mdbf_g_tile_kernel<NB>, dim3((r + 31) / 32, PT), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
+  } else if constexpr (g_ring) {
+    auto kg_ring = ring_g_kernel<NB>(g_ring3);
+    ql::launch(kg_ring, dim3((r + 31) / 32, PT), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
                m, r, l, B);
-  else
+  } else
     ql::launch(kg, dim3((r + 31) / 32, PT), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
   ql_status st = ql::launch_status("mdbf_linear (G stage)");
   if (st != QL_OK) return st;

@@ -159,6 +159,28 @@ def test_linear_f_stage_row_blocks(ql, n, P, l, B):
     assert torch.equal(ys[0], y) and torch.equal(ys[1], y)
 
 
+def test_linear_ring_g_three_stages(ql):
+    # more than two 32-row G blocks per SM (4790 / 32 -> 150 per path, two paths) take the ring G
+    # kernel with three stages (three CTAs per SM); its sums equal the four-stage kernel's
+    n, m, r, l, P, B = 4800, 4800, 4790, 4, 2, 1
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=5270)
+    x = synth.activations(B, m, seed=5370)
+    y = _linear(ql, paths, n, m, r, l, x)
+    assert max_rel(y.cpu().numpy(), om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+    # the 27B-class gate and up projections in one call: 2 x 2 x 91 blocks, three stages; each
+    # alone (182 blocks) keeps four
+    n, m, r = 2900, 5120, 2886
+    layers = [synth.mdbf_paths(P, n, m, r, l, seed=5280 + s) for s in range(2)]
+    x = synth.activations(B, m, seed=5380)
+    single = [_linear(ql, paths, n, m, r, l, x) for paths in layers]
+    ws = torch.empty(ql.mdbf_workspace_bytes(2 * P, n, m, r, l, B), dtype=torch.uint8, device="cuda")
+    ys = [torch.empty(B, n, device="cuda") for _ in range(2)]
+    ql.mdbf_linear_multi([mdbf_dev_paths(p) for p in layers], n, m, r, l, bf16(x), ys, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], single[0]) and torch.equal(ys[1], single[1])
+    assert max_rel(ys[1].cpu().numpy(), om.linear_factored(layers[1], n, m, r, x)) <= MDBF_TOL
+
+
 @pytest.mark.parametrize("l,B", [(4, 4), (4, 8), (2, 16)])
 def test_linear_wider_vector_blocks(ql, l, B):
     # l * B = 16, 32, 32: four and eight 8-column MMA blocks per word
