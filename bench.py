@@ -357,6 +357,15 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------------------------- device inputs
 
+def packed_offsets(sizes, align=256):
+    """Byte offsets of consecutive segments of the given sizes, each start aligned, and the total."""
+    offs, o = [], 0
+    for nb in sizes:
+        offs.append(o)
+        o += (nb + align - 1) // align * align
+    return offs, max(o, align)
+
+
 class Inputs:
     """Device-resident weights, activations and outputs of a list of layers, with rotating copies of
     the weights.  BenQ weights of one (N, K, seed) are made once and shared between records."""
@@ -368,13 +377,30 @@ class Inputs:
         from tests.qlhelpers import bf16, dev, f16
         self.layers, self.copies = [], copies
         cuda = torch.device("cuda")
+        layers = [dict(L) for L in layers]
         for L in layers:
-            L = dict(L)
-            x_h = synth.activations(L["B"], L["K"] if "K" in L else L["m"], seed=L["seed"] + 500)
-            L["x_h"], L["x"] = x_h, bf16(x_h)
-            odt = torch.float32 if L["out"] == "f32" else torch.bfloat16
-            nout = L["N"] if "N" in L else L["n"]
-            L["y"] = torch.empty(L["B"], nout, dtype=odt, device=cuda)
+            L["x_h"] = synth.activations(L["B"], L["K"] if "K" in L else L["m"], seed=L["seed"] + 500)
+        # The step's activations sit in one device buffer and its outputs in another (a 256-byte aligned
+        # view per layer), so that the end-to-end step copies its inputs in and its results out with
+        # one copy each.  Layers after the first of a group read the first one's x.
+        own_x = [L for L in layers if not L.get("group_skip")]
+        xoff, xbytes = packed_offsets([L["x_h"].size * 2 for L in own_x])
+        self.xbuf = torch.empty(xbytes, dtype=torch.uint8, device=cuda)
+        xh = np.zeros(xbytes, dtype=np.uint8)
+        for L, o in zip(own_x, xoff):
+            nb = L["x_h"].size * 2
+            xh[o:o + nb] = np.ascontiguousarray(L["x_h"]).view(np.uint8).reshape(-1)
+            L["x"] = self.xbuf[o:o + nb].view(torch.bfloat16).view(L["x_h"].shape)
+        self.xbuf.copy_(torch.from_numpy(xh))
+        self.x_host = xh
+        odts = [torch.float32 if L["out"] == "f32" else torch.bfloat16 for L in layers]
+        nouts = [L["N"] if "N" in L else L["n"] for L in layers]
+        yoff, ybytes = packed_offsets([L["B"] * n * (4 if d == torch.float32 else 2) for L, n, d in zip(layers, nouts, odts)])
+        self.ybuf = torch.empty(ybytes, dtype=torch.uint8, device=cuda)
+        for L, o, n, d in zip(layers, yoff, nouts, odts):
+            nb = L["B"] * n * (4 if d == torch.float32 else 2)
+            L["y"] = self.ybuf[o:o + nb].view(d).view(L["B"], n)
+        for L in layers:
             L["ws"] = None
             if L["kind"] == "benq":
                 w0 = self.benq_device_weights(L["N"], L["K"], L["seed"], ql, torch)
@@ -395,13 +421,15 @@ class Inputs:
                 L["ws"] = torch.empty(ql.mdbf_workspace_bytes(L["P"], L["n"], L["m"], L["r"], L["l"], L["B"]),
                                       dtype=torch.uint8, device=cuda)
             L["w"] = [w0] + [self.clone(w0) for _ in range(copies - 1)]
+            if L["kind"] not in ("benq", "benq_mlp", "benq_multi"):
+                L["wc"] = [ql.mdbf_paths_c(w) for w in L["w"]]   # path arrays made once, not per call
             self.layers.append(L)
         # layers of one group read the first one's x; its workspace serves all of their paths
         for L in self.layers:
             if L.get("group") and not L.get("group_skip"):
                 members = [M for M in self.layers if M.get("group") == L["group"]]
                 for M in members[1:]:
-                    M["x_h"], M["x"] = L["x_h"], L["x"]
+                    M["x"] = L["x"]
                 L["group_members"] = members
                 L["ws"] = torch.empty(ql.mdbf_workspace_bytes(len(members) * L["P"], L["n"], L["m"], L["r"], L["l"],
                                                               L["B"]), dtype=torch.uint8, device=cuda)
@@ -439,10 +467,10 @@ class Inputs:
             return
         elif "group_members" in L:
             ms = L["group_members"]
-            ql.mdbf_linear_multi([M["w"][c] for M in ms], L["n"], L["m"], L["r"], L["l"], L["x"], [M["y"] for M in ms],
-                                 L["ws"])
+            ql.mdbf_linear_multi([M["wc"][c] for M in ms], L["n"], L["m"], L["r"], L["l"], L["x"],
+                                 [M["y"] for M in ms], L["ws"])
         else:
-            ql.mdbf_linear(w, L["n"], L["m"], L["r"], L["l"], L["x"], L["y"], L["ws"])
+            ql.mdbf_linear(L["wc"][c], L["n"], L["m"], L["r"], L["l"], L["x"], L["y"], L["ws"])
 
 
 # ---------------------------------------------------------------------------------------------- timing
@@ -562,28 +590,23 @@ class Timer:
         return max_over_ranks(a.elapsed_time(b), self.world)
 
     def time_e2e(self, inp, layers, steps):
-        """The same steps through the public API with the inputs copied in from pinned host memory and
-        the results copied back each step (eager calls); returns (ms, h2d bytes, d2h bytes) per run."""
+        """The same steps through the public API with the step's inputs copied in from pinned host
+        memory and its results copied back every step (eager calls, one copy each way: the layers'
+        activations and outputs are views of one buffer each); returns (ms, h2d bytes, d2h bytes)."""
         torch, n = self.torch, inp.copies
-        # a layer run by its group's first layer reads that layer's x: no copy of its own
-        xs_h = [None if L.get("group_skip") else
-                torch.from_numpy(np.ascontiguousarray(L["x_h"]).view(np.int16)).view(torch.bfloat16).pin_memory()
-                for L in layers]
-        ys_h = [torch.empty(L["y"].shape, dtype=L["y"].dtype).pin_memory() for L in layers]
-        h2d = sum(t.numel() * t.element_size() for t in xs_h if t is not None)
-        d2h = sum(t.numel() * t.element_size() for t in ys_h)
+        x_h = torch.from_numpy(inp.x_host).pin_memory()
+        y_h = torch.empty(inp.ybuf.numel(), dtype=torch.uint8).pin_memory()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         self.sync_all()
         a.record(self.stream)
         for i in range(steps):
-            for L, xh, yh in zip(layers, xs_h, ys_h):
-                if xh is not None:
-                    L["x"].copy_(xh, non_blocking=True)
+            inp.xbuf.copy_(x_h, non_blocking=True)
+            for L in layers:
                 inp.run(self.ql, L, i % n)
-                yh.copy_(L["y"], non_blocking=True)
+            y_h.copy_(inp.ybuf, non_blocking=True)
         b.record(self.stream)
         self.sync_all()
-        return max_over_ranks(a.elapsed_time(b), self.world), h2d, d2h
+        return max_over_ranks(a.elapsed_time(b), self.world), x_h.numel(), y_h.numel()
 
 
 # ---------------------------------------------------------------------------------------------- records

@@ -106,16 +106,23 @@ def _ptr(t):
         return None
     if isinstance(t, int):
         return t
-    if not t.is_cuda:
+    d = t.get_device()
+    if d < 0:
         raise ValueError("tensor arguments must be CUDA tensors (got one on the host)")
-    if t.device.index != torch.cuda.current_device():
+    if d != torch.cuda.current_device():
         raise ValueError(f"tensor arguments must be on the current device cuda:{torch.cuda.current_device()}, "
                          f"got one on {t.device}")
     return t.data_ptr()
 
 
+# the current stream's handle without building a torch.cuda.Stream object (a few microseconds per call)
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream=None):
     if stream is None:
+        if _raw_stream is not None:
+            return _raw_stream(torch.cuda.current_device())
         stream = torch.cuda.current_stream()
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
 
@@ -250,9 +257,14 @@ def benq_bits_per_weight(K: int) -> float:
 
 def mdbf_paths_c(paths):
     """ctypes array of mdbf_path from a list of dicts / objects with S_A, S_B, A_amp, B_amp, Q_U, Q_V tensors
-    (S_A, S_B uint8 [rows, ld]; envelopes fp16 [*, l])."""
+    (S_A, S_B uint8 [rows, ld]; envelopes fp16 [*, l]), or of entries of such arrays.  The array holds
+    device addresses only: the tensors must outlive every call it is passed to.  mdbf_linear and
+    mdbf_linear_multi take such arrays in place of the lists, which saves building them per call."""
     arr = (MDBFPathC * len(paths))()
     for i, p in enumerate(paths):
+        if isinstance(p, MDBFPathC):   # an entry of an array made by an earlier call
+            arr[i] = p
+            continue
         g = (lambda k: p[k]) if isinstance(p, dict) else (lambda k: getattr(p, k))
         arr[i] = MDBFPathC(_ptr(g("S_A")), _ptr(g("S_B")), g("S_A").shape[1], g("S_B").shape[1],
                            _ptr(g("A_amp")), _ptr(g("B_amp")), _ptr(g("Q_U")), _ptr(g("Q_V")))

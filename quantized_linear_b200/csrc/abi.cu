@@ -6,7 +6,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "ql_internal.cuh"
 
@@ -37,6 +39,47 @@ ql_status launch_status(const char *what) {
 }
 
 bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
+
+// Per-launch host work that depends only on the device, the kernel and its launch shape is done
+// once: each of these runtime calls costs about a microsecond of host time per launch otherwise.
+// (A cudaDeviceReset() on a device clears the function attributes but not these caches.)
+cudaError_t set_max_smem(const void *k, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, int> done;   // (kernel, device) -> bytes already allowed
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  const auto key = std::make_pair(k, dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = done.find(key);
+    if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  }
+  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(mu);
+    int &v = done[key];
+    v = std::max(v, bytes);
+  }
+  return e;
+}
+
+int blocks_per_sm(const void *k, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void *, int, int, size_t>, int> cache;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const auto key = std::make_tuple(k, dev, threads, smem);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess || n < 0) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = n;
+  return n;
+}
 
 int sm_count() {
   static std::mutex mu;

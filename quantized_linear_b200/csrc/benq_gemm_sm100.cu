@@ -458,15 +458,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(32, 1) selftest_time
 }
 
 // ---------------------------------------------------------------------------- host side
-// Opts the GEMM kernel into its dynamic shared memory (once per process).
-cudaError_t smem_attr() {
-  static std::once_flag once;
-  static cudaError_t err = cudaSuccess;
-  std::call_once(once, [] {
-    err = cudaFuncSetAttribute(benq_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
-  return err;
-}
+// Opts the GEMM kernel into its dynamic shared memory (once per device).
+cudaError_t smem_attr() { return ql::set_max_smem(benq_gemm_kernel, SMEM_BYTES); }
 
 // CTA pairs that can be resident at once on the current device (cached per device).
 int resident_pairs() {

@@ -553,10 +553,8 @@ ql_status launch_b1(const uint8_t *codes, const uint16_t *lut, const uint8_t *co
   const int C = K / WARP_CODES;
   const int threads = C * 32;
   const size_t smem = (size_t)2 * C * B1_T * 32 * sizeof(float);
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, benq_gemv_b1_kernel<MODE>, threads, smem) != cudaSuccess ||
-      per_sm < 1)
-    return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
+  const int per_sm = ql::blocks_per_sm(benq_gemv_b1_kernel<MODE>, threads, smem);
+  if (per_sm < 1) return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
   const int grid = std::min(N / (MLP ? B1_T / 2 : B1_T), per_sm * ql::sm_count());
   ql::launch(benq_gemv_b1_kernel<MODE>, grid, threads, smem, s, codes, lut, codes2, lut2, x, y, (int)ydt, N, K, ms);
   return ql::launch_status(MODE == B1_MLP     ? "benq_mlp_gate_up (batch-1 GEMV)"
@@ -572,12 +570,11 @@ ql_status launch_fast(const uint8_t *codes, const uint16_t *lut, const uint16_t 
   const size_t smem = 2 * R * 128 + (size_t)2 * C * R * BMAX * 32 * sizeof(float);
   auto kern = benq_gemv_kernel<R, BMAX>;
   if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (ql::set_max_smem(kern, (int)smem) != cudaSuccess)
       return ql::fail(QL_ERR_CUDA, "benq_linear: cannot reserve %zu bytes of shared memory", smem);
   }
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1)
-    return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
+  const int per_sm = ql::blocks_per_sm(kern, threads, smem);
+  if (per_sm < 1) return ql::fail(QL_ERR_CUDA, "benq_linear: occupancy query failed");
   const int nblk = (N + R - 1) / R;
   const int grid = std::min(nblk, per_sm * ql::sm_count());
   ql::launch(kern, grid, threads, smem, s, codes, lut, x, y, (int)ydt, B, N, K);

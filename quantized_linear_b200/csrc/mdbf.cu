@@ -1235,8 +1235,8 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
   const size_t smf = (size_t)(SP_WARPS * RTF * NB * 128 + RTF * 16 * 8 * NB + RTF * 16 * B) * sizeof(float);
   auto kg = mdbf_g_mma_kernel<NB, VEC16>;
   auto kf = mdbf_f_mma_kernel<NB, RTF, VEC16>;
-  if (cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg) != cudaSuccess ||
-      cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smf) != cudaSuccess)
+  if (ql::set_max_smem(kg, (int)smg) != cudaSuccess ||
+      ql::set_max_smem(kf, (int)smf) != cudaSuccess)
     return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
   // G stage through per-warp cp.async rings when sign rows are 16-byte aligned and the vectors
   // are narrow (decode batches); wider ones keep mdbf_g_mma_kernel
@@ -1245,7 +1245,7 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
   const size_t smg_t = (size_t)SP_WARPS * (g_ring3 ? 3 : GR_STAGES) * g_ring_stage_bytes<NB>() + smg + (size_t)2 * 32 * l * 2;
   if constexpr (g_ring) {
     auto kg_ring = ring_g_kernel<NB>(g_ring3);
-    if (cudaFuncSetAttribute(kg_ring, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg_t) != cudaSuccess)
+    if (ql::set_max_smem(kg_ring, (int)smg_t) != cudaSuccess)
       return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
   }
   // the split G stage for NB == 1 on long sign rows (m >= 8192: 256 words or more), when its shared
@@ -1263,7 +1263,7 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
     if (st != QL_OK) return st;
   }
   if (gsp.ok) {
-    if (cudaFuncSetAttribute(mdbf_g_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsp.L.total) !=
+    if (ql::set_max_smem(mdbf_g_split_kernel, (int)gsp.L.total) !=
         cudaSuccess)
       return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
     ql::launch(mdbf_g_split_kernel, S * gsp.units, GS_KG * GS_NRG * 32, gsp.L.total, s, ps, (const uint4 *)zpk, wpk, part,
@@ -1287,7 +1287,7 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
       const size_t sm = f_nb1_smem(sign_stride, frag_bytes, rows, l, B);
       if (sm <= 227 * 1024) {
         auto kt = rows == 128 ? mdbf_f_nb1_kernel<2, 4> : rows == 64 ? mdbf_f_nb1_kernel<2, 2> : mdbf_f_nb1_kernel<2, 1>;
-        if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+        if (ql::set_max_smem(kt, (int)sm) != cudaSuccess)
           return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
         ql::launch(kt, S * ((n + rows - 1) / rows), rows / 32 * 32 * 8, sm, s, ps, P, (const uint4 *)wpk, outs,
                    (int)ydt, n, r, l, B, sign_stride, frag_bytes);
@@ -1310,7 +1310,7 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
     if (L.total > 227 * 1024) L = ftile_layout(ld_max, r, NB, B, P, l, 1, KG, tiles);
     if (L.total <= 227 * 1024) {
       auto kt = small ? mdbf_f_tile_kernel<NB, KG, RT, 1> : mdbf_f_tile_kernel<NB, KG, RT, FT_TILES / RT>;
-      if (cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total) != cudaSuccess)
+      if (ql::set_max_smem(kt, (int)L.total) != cudaSuccess)
         return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
       const int threads = (small ? 1 : FT_TILES / RT) * 32 * KG;
       ql::launch(kt, (n + 16 * tiles - 1) / (16 * tiles), threads, L.total, s, ps, P, (const uint4 *)wpk, y,

@@ -986,14 +986,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------- host side
+// Opts each GEMM instance into its dynamic shared memory (once per device).
 template <bool FST, int LK>
 cudaError_t smem_attr_one() {
-  static std::once_flag once;
-  static cudaError_t err = cudaSuccess;
-  std::call_once(once, [] {
-    err = cudaFuncSetAttribute(mdbf_gemm_kernel<FST, LK>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
-  return err;
+  return ql::set_max_smem(mdbf_gemm_kernel<FST, LK>, SMEM_BYTES);
 }
 cudaError_t smem_attr() {
   cudaError_t e = cudaSuccess;

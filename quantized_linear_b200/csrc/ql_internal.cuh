@@ -16,6 +16,20 @@ ql_status fail(ql_status s, const char *fmt, ...);
 ql_status launch_status(const char *what);
 // Multiprocessor count of the current device (cached per device).
 int sm_count();
+// cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes), skipped when the
+// current device has already allowed `k` at least `bytes`.
+cudaError_t set_max_smem(const void *k, int bytes);
+template <typename... KArgs>
+cudaError_t set_max_smem(void (*k)(KArgs...), int bytes) {
+  return set_max_smem(reinterpret_cast<const void *>(k), bytes);
+}
+// Resident blocks of `k` per SM at this block size and dynamic shared memory on the current device
+// (cudaOccupancyMaxActiveBlocksPerMultiprocessor, cached); 0 if the query fails.
+int blocks_per_sm(const void *k, int threads, size_t smem);
+template <typename... KArgs>
+int blocks_per_sm(void (*k)(KArgs...), int threads, size_t smem) {
+  return blocks_per_sm(reinterpret_cast<const void *>(k), threads, smem);
+}
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

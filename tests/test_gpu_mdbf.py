@@ -264,6 +264,12 @@ def test_linear_multi_matches_each_layer(ql, S, P, n, m, r, l, B, aligned16, ydt
     torch.cuda.synchronize()
     for s in range(S):
         assert torch.equal(ys[s], single[s]), s
+    # the same call with path arrays made once beforehand
+    ys2 = [torch.empty(B, n, dtype=ydtype, device="cuda") for _ in range(S)]
+    ql.mdbf_linear_multi([ql.mdbf_paths_c(d) for d in dls], n, m, r, l, bf16(xbits), ys2, ws)
+    torch.cuda.synchronize()
+    for s in range(S):
+        assert torch.equal(ys2[s], single[s]), s
     if ydtype == torch.float32:
         assert max_rel(ys[-1].cpu().numpy(), om.linear_factored(layers[-1], n, m, r, xbits)) <= MDBF_TOL
 
