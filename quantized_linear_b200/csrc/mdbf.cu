@@ -152,6 +152,133 @@ __global__ void mdbf_pack_z_kernel(Paths ps, const uint16_t *__restrict__ x, uin
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// Sign products on the s8 warp MMA (the split G stage, NB = 1: l * B <= 4 vectors).
+//
+// z is quantised once, by the pack kernel below, per group of 4 words (128 columns) and vector v:
+//   q[j][v] = rint(z[j][v] / s[v]),  s[v] the smallest power of two >= max_j |z[j][v]| / Z8_QMAX
+// over the group's columns (so z / s and s q are exact scalings),
+// and q = 256 h + lo is split into two signed bytes (lo in [-128, 127]; |q| <= Z8_QMAX keeps h in
+// [-128, 127]).  The sign operand enters as 0/1 bytes b = (sign + 1) / 2, so with the group's byte
+// sums H = sum_j h_j and L = sum_j lo_j,
+//   sum_j sign_j q_j = 256 (2 sum_j b_j h_j - H) + (2 sum_j b_j lo_j - L),
+// exact integers; each group's two int32 sums are scaled into fp32 once.  One quantised z is
+// within 2^-16 of its group's largest |z|, i.e. a relative error of ~1e-4 at most on u = S_B z
+// where the bf16 high + low split of the other G kernels gives ~1e-6; both are far inside the
+// forward pass's tolerance.  mma.m16n8k32 (s8 in, s32 accumulate) takes one 32-column word per
+// instruction, with the K order inside a word permuted so that an A register is one shift and one
+// mask of a sign word: byte e of register a0 (a2) of lane q holds physical column q + 8e
+// (q + 4 + 8e), i.e. logical k = 4q + e (16 + 4q + e) is physical column q + 8e (q + 4 + 8e).  B
+// column n (n < V: the high bytes of vector n; V <= n < 2V: the low bytes of vector n - V; else
+// zero) is packed with the same map: register b0 (b1) of lane (n, q) holds the bytes of columns
+// q + 8e (q + 4 + 8e), e = 0 .. 3, of the word.  Columns past m pack as zero.
+// ------------------------------------------------------------------------------------------
+constexpr int Z8_QMAX = 32639;   // 32767 - 128
+// per path and 4-word group: the scales and byte sums of its vectors (zero past V)
+struct __align__(16) Z8Meta {
+  float s[4];
+  int hs[4];
+  int ls[4];
+};
+__device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One CTA per (path, group), warp u on word u of the group: z of the group's 128 columns, its
+// scales and byte sums (meta) and its 4 words of B fragments (out[p][qw][lane] = {b0, b1}).  The
+// B_amp values (weights) are loaded before the wait on the preceding kernel.  A group holding a
+// non-finite z gets a NaN scale, so the outputs it reaches are NaN.  Also clears the split G
+// stage's arrival counts.
+__global__ void __launch_bounds__(128)
+    mdbf_pack_z8_kernel(Paths ps, const uint16_t *__restrict__ x, uint2 *__restrict__ out, Z8Meta *__restrict__ meta,
+                        int m, int l, int B, unsigned *__restrict__ cnt, int ncnt) {
+  __shared__ int8_t qs[8][128];     // [B column n][column of the group]
+  __shared__ float wmax[4][4];      // [warp][vector]
+  __shared__ int wsum[4][2][4];     // [warp][high, low][vector]
+  __shared__ int nonfinite;
+  const int p = blockIdx.y, grp = blockIdx.x, u = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int QW = (m + 31) / 32, G4 = (QW + 3) / 4, V = l * B;
+  const int j = 128 * grp + 32 * u + lane;
+  const bool in = j < m;
+  const uint16_t *bm = ps.Bm[p];
+  float bv[4];
+#pragma unroll
+  for (int v = 0; v < 4; ++v) bv[v] = (v < V && in) ? qld::f16_to_f32(bm[(int64_t)j * l + (v % l)]) : 0.f;
+  if (threadIdx.x == 0) nonfinite = 0;
+  qld::pdl_trigger();
+  qld::pdl_wait();
+  if (p == 0)
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < ncnt; e += gridDim.x * blockDim.x) cnt[e] = 0u;
+  float z[4];
+  bool finite = true;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    z[v] = (v < V && in) ? bv[v] * qld::bf16_to_f32(x[(int64_t)(v / l) * m + j]) : 0.f;
+    finite = finite && isfinite(z[v]);
+  }
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {   // |z| as bits: non-negative floats order as unsigned integers
+    const unsigned mx = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(z[v])));
+    if (lane == 0) wmax[u][v] = __uint_as_float(mx);
+  }
+  __syncthreads();   // also orders nonfinite = 0 before the flags below
+  if (!finite) nonfinite = 1;
+  int hq[4], lq[4];
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const float mx = fmaxf(fmaxf(wmax[0][v], wmax[1][v]), fmaxf(wmax[2][v], wmax[3][v]));
+    // s = 2^e, the smallest power of two with max|z| / s <= Z8_QMAX: z / s is exact, and so is s q
+    int ex;
+    const float fr = frexpf(mx, &ex);   // mx = fr 2^ex, fr in [0.5, 1) (0 for mx = 0)
+    const int e = ex - 15 + (fr * 32768.f > (float)Z8_QMAX ? 1 : 0);
+    const int qv = isfinite(mx) ? min(Z8_QMAX, max(-Z8_QMAX, __float2int_rn(ldexpf(z[v], -e)))) : 0;
+    lq[v] = ((qv + 128) & 255) - 128;
+    hq[v] = (qv - lq[v]) >> 8;
+    const int hs = __reduce_add_sync(0xffffffffu, hq[v]), ls = __reduce_add_sync(0xffffffffu, lq[v]);
+    if (lane == 0) {
+      wsum[u][0][v] = hs;
+      wsum[u][1][v] = ls;
+    }
+    if (threadIdx.x == 0) meta[(size_t)p * G4 + grp].s[v] = ldexpf(1.f, e);   // NaN scales below if not finite
+  }
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    int val = 0;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      if (v < V && n == v) val = hq[v];
+      if (v < V && n == V + v) val = lq[v];
+    }
+    qs[n][32 * u + lane] = (int8_t)val;
+  }
+  __syncthreads();
+  if (threadIdx.x < 4) {
+    const int v = threadIdx.x;
+    Z8Meta *const mt = meta + (size_t)p * G4 + grp;
+    const bool live = v < V;
+    mt->hs[v] = live ? wsum[0][0][v] + wsum[1][0][v] + wsum[2][0][v] + wsum[3][0][v] : 0;
+    mt->ls[v] = live ? wsum[0][1][v] + wsum[1][1][v] + wsum[2][1][v] + wsum[3][1][v] : 0;
+    if (!live) mt->s[v] = 0.f;
+    else if (nonfinite) mt->s[v] = __int_as_float(0x7fc00000);
+  }
+  const int qw = 4 * grp + u;
+  if (qw < QW) {
+    const int g = lane >> 2, q = lane & 3;
+    uint32_t b0 = 0, b1 = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      b0 |= (uint32_t)(uint8_t)qs[g][32 * u + q + 8 * e] << (8 * e);
+      b1 |= (uint32_t)(uint8_t)qs[g][32 * u + q + 4 + 8 * e] << (8 * e);
+    }
+    out[((size_t)p * QW + qw) * 32 + lane] = make_uint2(b0, b1);
+  }
+}
+
 // Pulls rows [row0, row0 + nrows) of a sign matrix toward L2.  Sign bits are weights, so this
 // may run before the wait on the preceding kernel; every address stays inside its row.
 __device__ __forceinline__ void prefetch_sign_rows(const uint8_t *S, size_t ld, int row0, int nrows, int rows) {
@@ -468,6 +595,25 @@ __global__ void __launch_bounds__(SP_WARPS * 32) mdbf_g_tile_kernel(Paths ps, co
   for (int e = threadIdx.x; e < NB * 32; e += blockDim.x)
     wpk[((size_t)p * QWr + qw) * NB * 32 + e] = pack_fragment(get, qw, e >> 5, e & 31, r, V);
 }
+
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+
+// fp32 scale and byte-sum correction of B column n for one group, from its Z8Meta at `mt`
+// (shared memory): high bytes weigh 256 s, low bytes s; columns past 2V are zero.
+__device__ __forceinline__ void z8_column(uint32_t mt, int n, int V, float &fac, int &corr) {
+  fac = 0.f;
+  corr = 0;
+  if (n < 2 * V) {
+    const int v = n < V ? n : n - V;
+    fac = __uint_as_float(lds32s(mt + 4 * v)) * (n < V ? 256.f : 1.f);
+    corr = (int)lds32s(mt + (n < V ? 16 : 32) + 4 * v);
+  }
+}
+
 
 // F stage: y[b][a] = sum_p sum_i A_amp[a][i] v_p[a][b*l+i], paths summed in p order
 template <int NB, int RT, bool VEC16>
@@ -902,9 +1048,10 @@ inline int nb1_rows(int S, int n) {
 // ------------------------------------------------------ G stage in split-K units (NB == 1) ----------
 // A unit is GS_ROWS = 128 rows of S_B of one path over one K slice, a run of 4-word groups.  Its
 // sign segments (one bulk copy per row, requested before the wait on pack z: signs are weights) and
-// the slice's z fragments (one bulk copy after the wait) sit in shared memory, where 16 warps (4 row
-// groups of 32 rows x 4 K-word groups) multiply them as the F stage does.  The K groups' sums are
-// added in group order.  With several slices per row block every unit writes its 128 x 8 partial
+// the slice's z fragments and Z8Meta entries (bulk copies after the wait) sit in shared memory,
+// where 16 warps (4 row groups of 32 rows x 4 runs of 4-word groups) multiply them on the s8 MMA
+// (see "Sign products on the s8 warp MMA"), scaling each group's int32 sums into fp32 once.  The
+// runs' sums are added in run order.  With several slices per row block every unit writes its 128 x 8 partial
 // sums to the workspace and counts itself in; the last unit of the row block to arrive adds the
 // slices' partials in slice order (so the result does not depend on which unit that is) and runs
 // the epilogue
@@ -920,7 +1067,9 @@ constexpr int GS_SMAX = 16;   // slices per row block at most (sizes the workspa
 struct GsLayout {
   int S;              // K slices per row block
   uint32_t sstride;   // bytes per sign row in shared memory (word count = 4 mod 8: conflict-free rows)
-  uint32_t frag_off;  // z fragments, then (after the products) the K groups' partial sums
+  uint32_t frag_off;  // z fragments (s8) and their groups' Z8Meta, then (after the products) the K groups'
+                      // partial sums
+  uint32_t meta_rel;  // the Z8Meta entries, relative to frag_off
   uint32_t bar_off;   // mbarriers and the last-unit flag (32 bytes)
   uint32_t q_off;     // the block's Q_V rows, then its Q_U rows: [2][GS_ROWS][l] fp16
   uint32_t total;
@@ -938,7 +1087,9 @@ inline GsLayout gs_layout(int S, int m, int l, int B) {
   // after the products the sign region holds the row sums D [128][8] and the w rows [128][V]
   const uint32_t sign_region = std::max(sign_bytes, (uint32_t)(GS_ROWS * 8 + GS_ROWS * l * B) * 4);
   L.frag_off = (sign_region + 127) / 128 * 128;
-  const uint32_t frag_region = std::max((uint32_t)(4 * gps) * 512, (uint32_t)(GS_KG * GS_ROWS * 8) * 4);
+  L.meta_rel = (uint32_t)(4 * gps) * 256;
+  const uint32_t frag_region =
+      std::max(L.meta_rel + (uint32_t)gps * (uint32_t)sizeof(Z8Meta), (uint32_t)(GS_KG * GS_ROWS * 8) * 4);
   L.bar_off = L.frag_off + frag_region;
   L.q_off = L.bar_off + 32;
   L.total = L.q_off + 2u * GS_ROWS * (uint32_t)l * 2u;
@@ -946,8 +1097,9 @@ inline GsLayout gs_layout(int S, int m, int l, int B) {
 }
 
 __global__ void __launch_bounds__(GS_KG * GS_NRG * 32, 1)
-    mdbf_g_split_kernel(Paths ps, const uint4 *__restrict__ zpk, uint4 *__restrict__ wpk, float *__restrict__ part,
-                        unsigned *__restrict__ cnt, int m, int r, int l, int B, GsLayout L) {
+    mdbf_g_split_kernel(Paths ps, const uint2 *__restrict__ zq, const Z8Meta *__restrict__ zmeta,
+                        uint4 *__restrict__ wpk, float *__restrict__ part, unsigned *__restrict__ cnt, int m, int r,
+                        int l, int B, GsLayout L) {
   constexpr int RT = GS_RT, NRG = GS_NRG, KG = GS_KG, ROWS = GS_ROWS;
   extern __shared__ __align__(128) unsigned char gsm[];
   const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(gsm));
@@ -981,14 +1133,17 @@ __global__ void __launch_bounds__(GS_KG * GS_NRG * 32, 1)
   }
   qld::pdl_trigger();
   qld::pdl_wait();
+  const int ng = g1 - g0;   // the slice's 4-word groups
   if (threadIdx.x == 0) {
-    sm100::mbar_arrive_expect_tx(frag_bar, (uint32_t)wn * 512);
-    sm100::bulk_g2s(base + L.frag_off, zpk + ((size_t)p * QWm + w0) * 32, (uint32_t)wn * 512, frag_bar);
+    sm100::mbar_arrive_expect_tx(frag_bar, (uint32_t)wn * 256 + (uint32_t)ng * (uint32_t)sizeof(Z8Meta));
+    sm100::bulk_g2s(base + L.frag_off, zq + ((size_t)p * QWm + w0) * 32, (uint32_t)wn * 256, frag_bar);
+    sm100::bulk_g2s(base + L.frag_off + L.meta_rel, zmeta + (size_t)p * G4 + g0, (uint32_t)ng * (uint32_t)sizeof(Z8Meta),
+                    frag_bar);
   }
 
   bool ok = true;
   const int rg = wid % NRG, kg = wid / NRG;
-  const int q0 = kg * wn / KG, q1 = (kg + 1) * wn / KG;
+  const int gq0 = kg * ng / KG, gq1 = (kg + 1) * ng / KG;   // this warp's groups of the slice
   const int rbase = 16 * RT * rg;
   float acc[RT][4];
 #pragma unroll
@@ -999,27 +1154,34 @@ __global__ void __launch_bounds__(GS_KG * GS_NRG * 32, 1)
     uint32_t r0[RT];
 #pragma unroll
     for (int t = 0; t < RT; ++t) r0[t] = base + (rbase + 16 * t + g) * L.sstride;
-    const uint32_t fb = base + L.frag_off + lane * 16;
+    const uint32_t fb = base + L.frag_off + lane * 8;
     const uint32_t l8 = 8 * L.sstride;
-#pragma unroll 2
-    for (int qw = q0; qw < q1; ++qw) {
-      const uint4 bf = lds128(fb + qw * 512);
-      uint32_t s0[RT], s1[RT];
+    for (int gq = gq0; gq < gq1; ++gq) {
+      float fac[2];
+      int corr[2];
 #pragma unroll
-      for (int t = 0; t < RT; ++t) {
-        s0[t] = lds32s(r0[t] + 4 * qw);
-        s1[t] = lds32s(r0[t] + l8 + 4 * qw);
-      }
+      for (int j = 0; j < 2; ++j)
+        z8_column(base + L.frag_off + L.meta_rel + gq * (uint32_t)sizeof(Z8Meta), 2 * q + j, V, fac[j], corr[j]);
+      int ia[RT][4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t ma = 1u << (15 - 8 * h - q), mb = 1u << (11 - 8 * h - q);
+      for (int t = 0; t < RT; ++t) ia[t][0] = ia[t][1] = ia[t][2] = ia[t][3] = 0;
+      const int nw = min(4, wn - 4 * gq);   // the last group of m may hold fewer words
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (u >= nw) break;
+        const int qw = 4 * gq + u;
+        const uint2 bz = lds64(fb + qw * 256);
 #pragma unroll
         for (int t = 0; t < RT; ++t) {
-          const uint32_t a0 = sign_pair_mul(s0[t], ma), a1 = sign_pair_mul(s1[t], ma),
-                         a2 = sign_pair_mul(s0[t], mb), a3 = sign_pair_mul(s1[t], mb);
-          mma16816(acc[t], a0, a1, a2, a3, h ? bf.z : bf.x, h ? bf.w : bf.y);
+          const uint32_t s0 = lds32s(r0[t] + 4 * qw), s1 = lds32s(r0[t] + l8 + 4 * qw);
+          mma_s8_16832(ia[t], (s0 >> q) & 0x01010101u, (s1 >> q) & 0x01010101u, (s0 >> (q + 4)) & 0x01010101u,
+                       (s1 >> (q + 4)) & 0x01010101u, bz.x, bz.y);
         }
       }
+#pragma unroll
+      for (int t = 0; t < RT; ++t)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[t][i] = fmaf(fac[i & 1], (float)(2 * ia[t][i] - corr[i & 1]), acc[t][i]);
     }
   }
   if (!ok) atomicExch(&g_mdbf_timeout, 1);
@@ -1239,39 +1401,53 @@ ql_status run_mma_stages(const Paths &ps, int S, int P, int n, int m, int r, int
       ql::set_max_smem(kf, (int)smf) != cudaSuccess)
     return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
   // G stage through per-warp cp.async rings when sign rows are 16-byte aligned and the vectors
-  // are narrow (decode batches); wider ones keep mdbf_g_mma_kernel
+  // are narrow (decode batches); wider ones keep mdbf_g_mma_kernel.
   constexpr bool g_ring = VEC16 && NB <= 2;
-  const bool g_ring3 = NB == 1 && (int64_t)((r + 31) / 32) * PT > 2LL * ql::sm_count();   // three CTAs per SM
-  const size_t smg_t = (size_t)SP_WARPS * (g_ring3 ? 3 : GR_STAGES) * g_ring_stage_bytes<NB>() + smg + (size_t)2 * 32 * l * 2;
-  if constexpr (g_ring) {
-    auto kg_ring = ring_g_kernel<NB>(g_ring3);
-    if (ql::set_max_smem(kg_ring, (int)smg_t) != cudaSuccess)
-      return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-  }
   // the split G stage for NB == 1 on long sign rows (m >= 8192: 256 words or more), when its shared
   // memory fits; shorter rows keep the ring kernel, which is faster there (27B-class gate/up,
   // m = 5120: 26.5 against 28.1 us per call; down, m = 17408: 33.4 against 35.4 us)
   GsPlan gsp{};
   if constexpr (VEC16 && NB == 1)
     if (m >= 8192) gsp = gs_plan(P, m, r, l, B);
-  {
-    const int64_t total = (int64_t)((m + 31) / 32) * NB * 32;
+  // The split G stage runs on the s8 MMA over z quantised by mdbf_pack_z8_kernel (27B-class down
+  // call: 28.9 -> 27.4 us).  The ring kernel keeps the bf16 form: an s8 ring measured slower on a
+  // single 27B-class gate or up call (27.4 against 26.8 us), its longer pack launch costing what
+  // its products saved.  Whether a layer takes the s8 form depends on its own sizes only, so
+  // mdbf_linear_multi gives each layer what mdbf_linear gives it, bit for bit.
+  const bool z8 = gsp.ok;
+  // three ring stages fit three CTAs per SM (NB = 1), four fit two: three when a launch has more
+  // blocks than two per SM (the gate and up projections in one multi call: 364 blocks)
+  const bool g_ring3 = NB == 1 && (int64_t)((r + 31) / 32) * PT > 2LL * ql::sm_count();
+  const size_t smg_t = (size_t)SP_WARPS * (g_ring3 ? 3 : GR_STAGES) * g_ring_stage_bytes<NB>() + smg +
+                       (size_t)2 * 32 * l * 2;
+  if constexpr (g_ring) {
+    if (ql::set_max_smem(ring_g_kernel<NB>(g_ring3), (int)smg_t) != cudaSuccess)
+      return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
+  }
+  const int QW = (m + 31) / 32;
+  uint2 *const zq = reinterpret_cast<uint2 *>(zpk);   // z8: [PT][QW][32] fragments, then [PT][G4] Z8Meta
+  Z8Meta *const zmeta = reinterpret_cast<Z8Meta *>(reinterpret_cast<char *>(zpk) + (size_t)PT * QW * 256);
+  const int ncnt = gsp.ok && gsp.L.S > 1 ? PT * ((r + GS_ROWS - 1) / GS_ROWS) : 0;
+  if (z8) {
+    const int G4 = (QW + 3) / 4;
+    ql::launch(mdbf_pack_z8_kernel, dim3(G4, PT), 128, 0, s, ps, x, zq, zmeta, m, l, B, cnt, ncnt);
+  } else {
+    const int64_t total = (int64_t)QW * NB * 32;
     const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)ql::sm_count() * 4);
-    ql::launch(mdbf_pack_z_kernel, dim3(grid, PT), 256, 0, s, ps, x, zpk, m, l, B, NB, cnt,
-               gsp.ok && gsp.L.S > 1 ? PT * ((r + GS_ROWS - 1) / GS_ROWS) : 0);
+    ql::launch(mdbf_pack_z_kernel, dim3(grid, PT), 256, 0, s, ps, x, zpk, m, l, B, NB, cnt, ncnt);
+  }
+  {
     ql_status st = ql::launch_status("mdbf_linear (pack z)");
     if (st != QL_OK) return st;
   }
   if (gsp.ok) {
-    if (ql::set_max_smem(mdbf_g_split_kernel, (int)gsp.L.total) !=
-        cudaSuccess)
+    if (ql::set_max_smem(mdbf_g_split_kernel, (int)gsp.L.total) != cudaSuccess)
       return ql::fail(QL_ERR_CUDA, "mdbf_linear: cannot reserve shared memory");
-    ql::launch(mdbf_g_split_kernel, S * gsp.units, GS_KG * GS_NRG * 32, gsp.L.total, s, ps, (const uint4 *)zpk, wpk, part,
-               cnt, m, r, l, B, gsp.L);
+    ql::launch(mdbf_g_split_kernel, S * gsp.units, GS_KG * GS_NRG * 32, gsp.L.total, s, ps, (const uint2 *)zq,
+               (const Z8Meta *)zmeta, wpk, part, cnt, m, r, l, B, gsp.L);
   } else if constexpr (g_ring) {
-    auto kg_ring = ring_g_kernel<NB>(g_ring3);
-    ql::launch(kg_ring, dim3((r + 31) / 32, PT), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk, wpk,
-               m, r, l, B);
+    ql::launch(ring_g_kernel<NB>(g_ring3), dim3((r + 31) / 32, PT), SP_WARPS * 32, smg_t, s, ps, (const uint4 *)zpk,
+               wpk, m, r, l, B);
   } else
     ql::launch(kg, dim3((r + 31) / 32, PT), SP_WARPS * 32, smg, s, ps, (const uint4 *)zpk, wpk, m, r, l, B);
   ql_status st = ql::launch_status("mdbf_linear (G stage)");

@@ -159,6 +159,23 @@ def test_linear_f_stage_row_blocks(ql, n, P, l, B):
     assert torch.equal(ys[0], y) and torch.equal(ys[1], y)
 
 
+@pytest.mark.parametrize("m,spread", [(8222, 3.0), (9000, 3.0), (8192, 0.0)])
+def test_linear_s8_g_stage_group_scales(ql, m, spread):
+    # the split G stage (m >= 8192) runs on the s8 MMA with z quantised per 128-column group and
+    # vector: activations whose magnitudes span 10^(+-spread) across columns, a last group of one
+    # partial word (8222 = 256 words + 30 columns), and an input with whole zero groups
+    n, r, l, P, B = 700, 300, 4, 2, 1
+    paths = synth.mdbf_paths(P, n, m, r, l, seed=5290 + m)
+    xf = synth.bf16_bits_to_f32(synth.activations(B, m, seed=5390 + m))
+    rng = np.random.default_rng(m)
+    xf = xf * (10.0 ** rng.uniform(-spread, spread, size=(1, m))).astype(np.float32)
+    if spread == 0.0:
+        xf[:, 256:1024] = 0.0
+    x = synth.f32_to_bf16_bits(xf.astype(np.float32))
+    y = _linear(ql, paths, n, m, r, l, x)
+    assert max_rel(y.cpu().numpy(), om.linear_factored(paths, n, m, r, x)) <= MDBF_TOL
+
+
 def test_linear_ring_g_three_stages(ql):
     # more than two 32-row G blocks per SM (4790 / 32 -> 150 per path, two paths) take the ring G
     # kernel with three stages (three CTAs per SM); its sums equal the four-stage kernel's
