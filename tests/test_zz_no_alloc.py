@@ -3,8 +3,9 @@
 Some callers may not call cudaMalloc (allocator-internal code, real-time threads that must not
 block in the driver, hosts with a memory budget fixed at start-up).  mdbf_linear_noalloc serves
 them from a fixed scratch array compiled into the library.  This test calls it through the C ABI
-on each of the paths its scratch feeds -- the batch decode kernels, the envelope chunks of l > 32,
-and the tensor-core GEMMs whose split counters live in the scratch -- twice in a row on different
+on each of the paths its scratch feeds -- the batch decode kernels, the split G stage on long sign
+rows, the envelope chunks of l > 32, and the tensor-core GEMMs whose split counters live in the
+scratch -- twice in a row on different
 inputs, so stale scratch from one call cannot leak into the next.  Each result is checked against
 the oracle (within the MDBF tolerance) and against mdbf_linear, the workspace entry point (bit for
 bit).  The file is collected last and passes alone or after the other tests.
@@ -19,11 +20,12 @@ from tests.qlhelpers import MDBF_TOL, bf16, max_rel, mdbf_dev_paths
 
 pytestmark = pytest.mark.gpu
 
-# (n, m, r, l, P, B, seed): decode kernels (l*B <= 64), envelope chunks (l > 32), and the tensor
+# (n, m, r, l, P, B, seed): decode kernels (l*B <= 64), envelope chunks (l > 32), the tensor
 # cores (l*B > 64 with n, m, r >= 64) on a layer small enough for the array whose two K blocks per
-# GEMM make both GEMMs split their last wave, so the split counters in the scratch are used
+# GEMM make both GEMMs split their last wave, so the split counters in the scratch are used, and
+# the split s8 G stage (m >= 8192: quantised z, slice partials and arrival counts in the scratch)
 PROBLEMS = [(1024, 768, 300, 4, 2, 3, 71), (640, 1280, 257, 2, 1, 16, 72),
-            (256, 256, 128, 40, 1, 2, 74), (300, 128, 64, 4, 2, 20, 73)]
+            (256, 256, 128, 40, 1, 2, 74), (300, 128, 64, 4, 2, 20, 73), (256, 8192, 128, 4, 1, 1, 75)]
 
 
 def _reference(ql, paths_c, n, m, r, l, x):
