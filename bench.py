@@ -357,6 +357,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------------------------- device inputs
 
+# per-step copy bytes (in + out) from which the end-to-end steps overlap their copies with compute
+E2E_OVERLAP_BYTES = 1 << 20
+
+
 def packed_offsets(sizes, align=256):
     """Byte offsets of consecutive segments of the given sizes, each start aligned, and the total."""
     offs, o = [], 0
@@ -391,6 +395,7 @@ class Inputs:
             nb = L["x_h"].size * 2
             xh[o:o + nb] = np.ascontiguousarray(L["x_h"]).view(np.uint8).reshape(-1)
             L["x"] = self.xbuf[o:o + nb].view(torch.bfloat16).view(L["x_h"].shape)
+            L["_xo"] = (o, nb)
         self.xbuf.copy_(torch.from_numpy(xh))
         self.x_host = xh
         odts = [torch.float32 if L["out"] == "f32" else torch.bfloat16 for L in layers]
@@ -400,6 +405,7 @@ class Inputs:
         for L, o, n, d in zip(layers, yoff, nouts, odts):
             nb = L["B"] * n * (4 if d == torch.float32 else 2)
             L["y"] = self.ybuf[o:o + nb].view(d).view(L["B"], n)
+            L["_yo"] = (o, nb)
         for L in layers:
             L["ws"] = None
             if L["kind"] == "benq":
@@ -413,6 +419,7 @@ class Inputs:
                 # one output buffer, a contiguous view per part (batch 1, parts of 4k rows: 16-byte aligned)
                 w0 = tuple(self.benq_device_weights(N, L["K"], sd, ql, torch) for N, sd, _ in L["parts"])
                 offs = np.cumsum([0] + [N for N, _, _ in L["parts"]])
+                L["_ys_offs"] = offs
                 L["ys"] = [L["y"][:, offs[i]:offs[i + 1]] for i in range(len(L["parts"]))]
             else:
                 paths = synth.mdbf_paths(L["P"], L["n"], L["m"], L["r"], L["l"], seed=L["seed"])
@@ -433,6 +440,30 @@ class Inputs:
                 L["group_members"] = members
                 L["ws"] = torch.empty(ql.mdbf_workspace_bytes(len(members) * L["P"], L["n"], L["m"], L["r"], L["l"],
                                                               L["B"]), dtype=torch.uint8, device=cuda)
+
+    def views(self, torch, xbuf, ybuf):
+        """Every layer's x, y (and ys) as views of the given activation and output buffers, at this
+        record's offsets; group members read their first member's x."""
+        vs = []
+        for L in self.layers:
+            o, nb = L["_yo"]
+            v = {"y": ybuf[o:o + nb].view(L["y"].dtype).view(L["y"].shape)}
+            if "_xo" in L:
+                o, nb = L["_xo"]
+                v["x"] = xbuf[o:o + nb].view(torch.bfloat16).view(L["x"].shape)
+            if "_ys_offs" in L:
+                offs = L["_ys_offs"]
+                v["ys"] = [v["y"][:, offs[i]:offs[i + 1]] for i in range(len(offs) - 1)]
+            vs.append(v)
+        index = {id(L): i for i, L in enumerate(self.layers)}
+        for L, v in zip(self.layers, vs):
+            for M in L.get("group_members", [])[1:]:
+                vs[index[id(M)]]["x"] = v["x"]
+        return vs
+
+    def use(self, vs):
+        for L, v in zip(self.layers, vs):
+            L.update(v)
 
     @classmethod
     def benq_device_weights(cls, N, K, seed, ql, torch):
@@ -590,23 +621,83 @@ class Timer:
         return max_over_ranks(a.elapsed_time(b), self.world)
 
     def time_e2e(self, inp, layers, steps):
-        """The same steps through the public API with the step's inputs copied in from pinned host
-        memory and its results copied back every step (eager calls, one copy each way: the layers'
-        activations and outputs are views of one buffer each); returns (ms, h2d bytes, d2h bytes)."""
+        """The same steps through the public API with every step's inputs copied in from pinned host
+        memory and its results copied back (eager calls; one copy each way, the layers' activations
+        and outputs being views of one buffer each); returns (ms, h2d bytes, d2h bytes) per run.
+
+        Steps whose copies reach E2E_OVERLAP_BYTES alternate between two sets of device buffers, so
+        that step i's copy in (on a copy stream) overlaps step i-1's kernels and its copy out (on
+        another) overlaps step i+1's: a buffer is refilled only after the kernels two steps back
+        have read it, and an output buffer is rewritten only after its previous copy out.  Smaller
+        steps run on one stream, where the events and stream switches would cost more host time
+        than the overlap saves.  The last step's copied-back outputs are checked against a plain
+        call of the same step."""
         torch, n = self.torch, inp.copies
+        if inp.xbuf.numel() + inp.ybuf.numel() < E2E_OVERLAP_BYTES:
+            x_h = torch.from_numpy(inp.x_host).pin_memory()
+            y_h = torch.empty(inp.ybuf.numel(), dtype=torch.uint8).pin_memory()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            self.sync_all()
+            a.record(self.stream)
+            for i in range(steps):
+                inp.xbuf.copy_(x_h, non_blocking=True)
+                for L in layers:
+                    inp.run(self.ql, L, i % n)
+                y_h.copy_(inp.ybuf, non_blocking=True)
+            b.record(self.stream)
+            self.sync_all()
+            self.check_e2e(inp, layers, y_h.clone())
+            return max_over_ranks(a.elapsed_time(b), self.world), x_h.numel(), y_h.numel()
+        xb = [inp.xbuf, torch.empty_like(inp.xbuf)]
+        yb = [inp.ybuf, torch.empty_like(inp.ybuf)]
+        sets = [inp.views(torch, xb[k], yb[k]) for k in range(2)]
         x_h = torch.from_numpy(inp.x_host).pin_memory()
-        y_h = torch.empty(inp.ybuf.numel(), dtype=torch.uint8).pin_memory()
+        y_h = [torch.empty(inp.ybuf.numel(), dtype=torch.uint8).pin_memory() for _ in range(2)]
+        main, cin, cout = self.stream, torch.cuda.Stream(), torch.cuda.Stream()
+        read = [None, None]       # the kernels that last read activation buffer k
+        back = [None, None]       # the last copy out of output buffer k
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         self.sync_all()
-        a.record(self.stream)
+        a.record(main)
+        cin.wait_event(a)
         for i in range(steps):
-            inp.xbuf.copy_(x_h, non_blocking=True)
+            k = i % 2
+            if read[k] is not None:
+                cin.wait_event(read[k])
+            with torch.cuda.stream(cin):
+                xb[k].copy_(x_h, non_blocking=True)
+            e_in = torch.cuda.Event()
+            e_in.record(cin)
+            main.wait_event(e_in)
+            if back[k] is not None:
+                main.wait_event(back[k])
+            inp.use(sets[k])
             for L in layers:
                 inp.run(self.ql, L, i % n)
-            y_h.copy_(inp.ybuf, non_blocking=True)
-        b.record(self.stream)
+            read[k] = torch.cuda.Event()
+            read[k].record(main)
+            cout.wait_event(read[k])
+            with torch.cuda.stream(cout):
+                y_h[k].copy_(yb[k], non_blocking=True)
+            back[k] = torch.cuda.Event()
+            back[k].record(cout)
+        for e in back:
+            if e is not None:
+                main.wait_event(e)
+        b.record(main)
         self.sync_all()
-        return max_over_ranks(a.elapsed_time(b), self.world), x_h.numel(), y_h.numel()
+        last = y_h[(steps - 1) % 2].clone()
+        inp.use(sets[0])
+        self.check_e2e(inp, layers, last)
+        return max_over_ranks(a.elapsed_time(b), self.world), x_h.numel(), y_h[0].numel()
+
+    def check_e2e(self, inp, layers, copied):
+        """The outputs an end-to-end step copied back equal those of a plain call of the step."""
+        for L in layers:
+            inp.run(self.ql, L, 0)
+        self.torch.cuda.synchronize()
+        if not self.torch.equal(copied, inp.ybuf.cpu()):
+            raise RuntimeError("end-to-end step: the copied-back outputs differ from a plain call's")
 
 
 # ---------------------------------------------------------------------------------------------- records
