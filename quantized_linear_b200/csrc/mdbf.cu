@@ -7,7 +7,8 @@
 //   (F t)_a = sum_i A_amp[a,i] * sum_k S_A[a,k] * (Q_U[k,i] t_k)
 // so each path is two products of a packed +-1 matrix with l*B dense vectors:
 //   prologue  z[p][j][b*l+i] = B_amp[j,i] * x[b,j]                (exact in fp32, packed as
-//             bf16 high + low MMA fragments)
+//             bf16 high + low MMA fragments, or for the split G stage quantised per
+//             128-column group to two signed bytes: "Sign products on the s8 warp MMA")
 //   G stage   u = S_B z;   t[k][b] = sum_i Q_V[k,i] u[k][b*l+i];
 //             w[p][k][b*l+i] = Q_U[k,i] * t[k][b]                  (epilogue, fused)
 //   F stage   v = S_A w;   y[b][a] = sum_p sum_i A_amp[a,i] v[a][b*l+i]   (epilogue, fused;
